@@ -1,0 +1,263 @@
+"""CPU oracle for quantized scaled-dot-product attention -- TEST INFRASTRUCTURE ONLY.
+
+Only the test suite, ``__graft_entry__.smoke()`` and ``bench.py``'s CPU-baseline leg may
+import this package.  The CUDA library never loads it and shares no code with it.
+
+The arithmetic lives in ``qattn_oracle.c`` (plain C, FP64/FP32, OpenMP over query rows); this
+module compiles it with gcc on first use and marshals numpy arrays.  The method is the one the
+NVIDIA developer blog "Optimizing FLUX.1 Kontext for Image Editing with Low-Precision
+Quantization" describes in "Workflow and quantization" (SDPA bullets and Fig. 4): FakeQuantize
+Q, K, V to per-tensor FP8 or per-block FP4, FP8 BMM1 with higher-precision accumulation, FP32
+softmax, per-tensor FP8 P, FP8 BMM2.
+
+``attention_fp64`` is the unquantized closed form softmax(Q K^T * sm_scale) V in FP64 (numpy
+matmul as a library primitive), used to pin the oracle's attention and to report the
+quantized path's error against unquantized attention.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "qattn_oracle.c")
+_LIB_PATH = os.path.join(_HERE, "_build", "liboracle.so")
+_lock = threading.Lock()
+_lib = None
+
+FP32 = 1          # round scores / probabilities / row sum to binary32 (the FP32 softmax)
+QUANT_P = 2       # quantize P to E4M3 with per-tensor scale 1/448 (before normalization)
+FIG4_LITERAL = 4  # quantize the normalized probability instead (reported, not gated)
+METHOD = FP32 | QUANT_P
+
+OK, ERR_INVALID, ERR_NONFINITE = 0, 1, 4
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle with gcc (-O2, OpenMP, no fast-math).  Returns the .so path."""
+    os.makedirs(os.path.dirname(_LIB_PATH), exist_ok=True)
+    stale = (not os.path.exists(_LIB_PATH)
+             or os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC))
+    if force or stale:
+        tmp = _LIB_PATH + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-std=c11",
+                               "-fno-fast-math", "-ffp-contract=off", "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is None:
+            lib = ctypes.CDLL(build())
+            P = ctypes.c_void_p
+            i64, f32, f64, i32 = ctypes.c_int64, ctypes.c_float, ctypes.c_double, ctypes.c_int
+            lib.orc_bf16_to_float.argtypes = [ctypes.c_uint16]
+            lib.orc_bf16_to_float.restype = f32
+            lib.orc_e4m3_to_float.argtypes = [ctypes.c_uint8]
+            lib.orc_e4m3_to_float.restype = f32
+            lib.orc_e4m3_from_float.argtypes = [f32]
+            lib.orc_e4m3_from_float.restype = ctypes.c_uint8
+            lib.orc_e2m1_to_float.argtypes = [ctypes.c_uint8]
+            lib.orc_e2m1_to_float.restype = f32
+            lib.orc_e2m1_from_float.argtypes = [f32]
+            lib.orc_e2m1_from_float.restype = ctypes.c_uint8
+            lib.orc_amax_bf16.argtypes = [P, i64, P]
+            lib.orc_amax_bf16.restype = i32
+            lib.orc_quantize_fp8.argtypes = [P, i64, f32, P, P]
+            lib.orc_quantize_fp8.restype = i32
+            lib.orc_quantize_fp4_block.argtypes = [P, i64, f32, P, P, P, P, P]
+            lib.orc_quantize_fp4_block.restype = i32
+            lib.orc_dequant_fp4_block.argtypes = [P, P, f32, i64, P]
+            lib.orc_dequant_fp4_block.restype = None
+            att = [P, P, P, i32, i32, i64, i32, P, i32, f64, f64, f64, f64, i32, P, i64, P]
+            lib.orc_attention_values.argtypes = att
+            lib.orc_attention_values.restype = i32
+            lib.orc_attention_e4m3.argtypes = att
+            lib.orc_attention_e4m3.restype = i32
+            lib.orc_num_threads.argtypes = []
+            lib.orc_num_threads.restype = i32
+            _lib = lib
+    return _lib
+
+
+def _ptr(a: np.ndarray):
+    assert a.flags["C_CONTIGUOUS"]
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _bits(x) -> np.ndarray:
+    """bf16 input as a contiguous uint16 array (accepts a CPU torch bf16 tensor or uint16)."""
+    if hasattr(x, "view") and hasattr(x, "dtype") and str(x.dtype) == "torch.bfloat16":
+        import torch
+        return x.contiguous().view(torch.int16).numpy().view(np.uint16).reshape(-1)
+    a = np.ascontiguousarray(x)
+    assert a.dtype == np.uint16
+    return a.reshape(-1)
+
+
+def num_threads() -> int:
+    return int(_load().orc_num_threads())
+
+
+# --- scalar codecs -------------------------------------------------------------------------
+def bf16_to_float(bits: int) -> float:
+    return float(_load().orc_bf16_to_float(bits))
+
+
+def e4m3_to_float(code: int) -> float:
+    return float(_load().orc_e4m3_to_float(code))
+
+
+def e4m3_from_float(x: float) -> int:
+    return int(_load().orc_e4m3_from_float(x))
+
+
+def e2m1_to_float(code: int) -> float:
+    return float(_load().orc_e2m1_to_float(code))
+
+
+def e2m1_from_float(x: float) -> int:
+    return int(_load().orc_e2m1_from_float(x))
+
+
+def e4m3_table() -> np.ndarray:
+    """Values of all 256 E4M3 codes (NaN for 0x7F / 0xFF)."""
+    return np.array([e4m3_to_float(c) for c in range(256)], dtype=np.float64)
+
+
+# --- tensor ops -----------------------------------------------------------------------------
+def amax(x) -> tuple[int, float]:
+    b = _bits(x)
+    out = np.zeros(1, dtype=np.float32)
+    rc = _load().orc_amax_bf16(_ptr(b), b.size, _ptr(out))
+    return rc, float(out[0])
+
+
+def quantize_fp8(x, amax_value: float):
+    """Returns (codes uint8 [n], scale float32)."""
+    b = _bits(x)
+    codes = np.empty(b.size, dtype=np.uint8)
+    s = np.zeros(1, dtype=np.float32)
+    rc = _load().orc_quantize_fp8(_ptr(b), b.size, np.float32(amax_value), _ptr(codes), _ptr(s))
+    if rc != OK:
+        raise ValueError(f"orc_quantize_fp8 failed with status {rc}")
+    return codes, np.float32(s[0])
+
+
+def quantize_fp4_block(x, amax_value: float, requant: bool = True):
+    """Returns (packed uint8 [n/2], block scales uint8 [n/16], s_g, codes8 uint8 [n], s8)."""
+    b = _bits(x)
+    n = b.size
+    packed = np.empty(n // 2, dtype=np.uint8)
+    bscale = np.empty(n // 16, dtype=np.uint8)
+    sg = np.zeros(1, dtype=np.float32)
+    codes8 = np.empty(n, dtype=np.uint8) if requant else None
+    s8 = np.zeros(1, dtype=np.float32)
+    rc = _load().orc_quantize_fp4_block(
+        _ptr(b), n, np.float32(amax_value), _ptr(packed), _ptr(bscale), _ptr(sg),
+        _ptr(codes8) if requant else None, _ptr(s8) if requant else None)
+    if rc != OK:
+        raise ValueError(f"orc_quantize_fp4_block failed with status {rc}")
+    return packed, bscale, np.float32(sg[0]), codes8, np.float32(s8[0])
+
+
+def dequant_fp4_block(packed, bscale, sg, n) -> np.ndarray:
+    out = np.empty(n, dtype=np.float32)
+    _load().orc_dequant_fp4_block(_ptr(np.ascontiguousarray(packed)),
+                                  _ptr(np.ascontiguousarray(bscale)), np.float32(sg), n, _ptr(out))
+    return out
+
+
+def _cu(cu_seqlens, T):
+    if cu_seqlens is None:
+        return np.array([0, T], dtype=np.int64)
+    return np.ascontiguousarray(np.asarray(cu_seqlens, dtype=np.int64))
+
+
+def attention_values(q, k, v, s_q=1.0, s_k=1.0, s_v=1.0, sm_scale=None, flags=METHOD,
+                     cu_seqlens=None, rows=None) -> np.ndarray:
+    """Oracle attention over values q, k, v: float arrays [B, H, T, D]."""
+    q = np.ascontiguousarray(q, dtype=np.float64)
+    k = np.ascontiguousarray(k, dtype=np.float64)
+    v = np.ascontiguousarray(v, dtype=np.float64)
+    B, H, T, D = q.shape
+    sm = 1.0 / np.sqrt(D) if sm_scale is None else sm_scale
+    cu = _cu(cu_seqlens, T)
+    r = None if rows is None else np.ascontiguousarray(np.asarray(rows, dtype=np.int64))
+    nrows = B * H * T if r is None else r.size
+    out = np.empty((nrows, D), dtype=np.float64)
+    rc = _load().orc_attention_values(_ptr(q), _ptr(k), _ptr(v), B, H, T, D, _ptr(cu),
+                                      cu.size - 1, s_q, s_k, s_v, sm, flags,
+                                      None if r is None else _ptr(r), nrows, _ptr(out))
+    if rc != OK:
+        raise ValueError(f"orc_attention_values failed with status {rc}")
+    return out if r is not None else out.reshape(B, H, T, D)
+
+
+def attention_e4m3(q8, k8, v8, shape, s_q, s_k, s_v, sm_scale=None, flags=METHOD,
+                   cu_seqlens=None, rows=None) -> np.ndarray:
+    """Oracle attention over E4M3 codes (uint8 arrays of B*H*T*D) with per-tensor scales."""
+    B, H, T, D = shape
+    sm = 1.0 / np.sqrt(D) if sm_scale is None else sm_scale
+    q8, k8, v8 = (np.ascontiguousarray(a, dtype=np.uint8).reshape(-1) for a in (q8, k8, v8))
+    assert q8.size == k8.size == v8.size == B * H * T * D
+    cu = _cu(cu_seqlens, T)
+    r = None if rows is None else np.ascontiguousarray(np.asarray(rows, dtype=np.int64))
+    nrows = B * H * T if r is None else r.size
+    out = np.empty((nrows, D), dtype=np.float64)
+    rc = _load().orc_attention_e4m3(_ptr(q8), _ptr(k8), _ptr(v8), B, H, T, D, _ptr(cu),
+                                    cu.size - 1, float(s_q), float(s_k), float(s_v), sm, flags,
+                                    None if r is None else _ptr(r), nrows, _ptr(out))
+    if rc != OK:
+        raise ValueError(f"orc_attention_e4m3 failed with status {rc}")
+    return out if r is not None else out.reshape(B, H, T, D)
+
+
+def attention_fp64(q, k, v, sm_scale=None, cu_seqlens=None) -> np.ndarray:
+    """Unquantized closed form softmax(q k^T * sm_scale) v per sequence, FP64 throughout."""
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    B, H, T, D = q.shape
+    sm = 1.0 / np.sqrt(D) if sm_scale is None else sm_scale
+    cu = _cu(cu_seqlens, T)
+    out = np.empty_like(q)
+    for s in range(cu.size - 1):
+        a, b = int(cu[s]), int(cu[s + 1])
+        logits = np.einsum("bhid,bhjd->bhij", q[:, :, a:b], k[:, :, a:b]) * sm
+        logits -= logits.max(axis=-1, keepdims=True)
+        w = np.exp(logits)
+        w /= w.sum(axis=-1, keepdims=True)
+        out[:, :, a:b] = np.einsum("bhij,bhjd->bhid", w, v[:, :, a:b])
+    return out
+
+
+# --- the whole method, from bf16 inputs --------------------------------------------------------
+def quantize_tensor(x, mode: str):
+    """FakeQuantize one bf16 tensor for BMM input: returns (e4m3 codes [n], scale, extras)."""
+    rc, a = amax(x)
+    if rc != OK:
+        raise ValueError("non-finite input")
+    if mode == "fp8":
+        codes, s = quantize_fp8(x, a)
+        return codes, s, {"amax": a}
+    if mode == "fp4":
+        packed, bscale, sg, codes8, s8 = quantize_fp4_block(x, a)
+        return codes8, s8, {"amax": a, "packed": packed, "bscale": bscale, "sg": sg}
+    raise ValueError(mode)
+
+
+def method_forward(q, k, v, mode="fp8", sm_scale=None, cu_seqlens=None, rows=None,
+                   flags=METHOD):
+    """The quantized SDPA from bf16 inputs [B, H, T, D] (CPU torch bf16 tensors)."""
+    shape = tuple(q.shape)
+    q8, sq, _ = quantize_tensor(q, mode)
+    k8, sk, _ = quantize_tensor(k, mode)
+    v8, sv, _ = quantize_tensor(v, mode)
+    return attention_e4m3(q8, k8, v8, shape, sq, sk, sv, sm_scale, flags, cu_seqlens, rows)
