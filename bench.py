@@ -1,0 +1,320 @@
+"""Benchmark of the quantized attention hot path on B200.
+
+One step = the whole path on one batch of the L=8704 FLUX.1 Kontext editing workload (512 text +
+4096 target + 4096 context tokens, H=24, D=128, FP8 mode, outlier channels in Q and K):
+amax x3 -> FP8 quantize x3 -> fused attention, inputs resident in HBM.  Metric: algorithmic
+FLOPs of BMM1 + BMM2 (4 * H * D * L^2) per second.  The L2 is flushed between steps (a
+256 MiB write outside the timed events).  ``e2e`` repeats the measurement through the same C ABI
+with the bf16 inputs in pinned host memory: every step copies Q, K, V to the device and the
+output back.  ``--impl reference`` times the CPU oracle instead (rank 0 only) on a bounded row
+sample of the same workload.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference] [--mode fp8|fp4]
+Multi-GPU (launched with torchrun): every rank runs its own replica of the workload (weak
+scaling, no data-path collective); time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads  # noqa: E402
+
+HBM_FALLBACK_GBS = 6650.0
+BF16_FALLBACK_TFLOPS = 1590.0
+FP8_PER_BF16 = 2.0          # nominal dense FP8 / BF16 tensor throughput ratio on B200
+L2_FLUSH_BYTES = 256 << 20
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), float(p["bf16_tflops"]), "measured"
+    except Exception:
+        return HBM_FALLBACK_GBS, BF16_FALLBACK_TFLOPS, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        import tempfile
+        fd, self.path = tempfile.mkstemp(prefix="qattn_clocks_", suffix=".csv")
+        os.close(fd)
+
+    def __enter__(self):
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"], stdout=self.f,
+                stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+            self.f.close()
+
+    def summary(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    rows.append((float(parts[1]), float(parts[2]), parts[5:9]))
+                except ValueError:
+                    continue
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for _, _, flags in rows for i, fl in enumerate(flags)
+                          if fl.lower() == "active"})
+        return {"sm_mhz": statistics.median(r[0] for r in rows), "sm_max_mhz": rows[0][1],
+                "reasons": reasons, "samples": len(rows)}
+
+
+def dist_setup(n_gpus: int):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    return rank, world, local
+
+
+def barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def run_gpu(args):
+    import precision_quantized_attention_b200 as qa
+    rank, world, local = dist_setup(args.gpus)
+    w = workloads.WORKLOADS["edit_fp8" if args.mode == "fp8" else "edit_fp4"]
+    if world > 1:   # each replica gets its own seeded problem
+        import dataclasses
+        w = dataclasses.replace(w, seed=w.seed + 100 * rank)
+    q, k, v = workloads.make_qkv(w)
+    qd, kd, vd = (t.cuda() for t in (q, k, v))
+    path = qa.QuantizedAttention(w.shape, w.mode, sm_scale=w.sm_scale)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    def step():
+        path.quantize(qd, kd, vd)
+        return path.attend()
+
+    for _ in range(args.warmup):
+        step()
+    status = qa.get_error()
+    if status != 0:
+        raise RuntimeError(f"device error {status} during warm-up")
+
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clocks:
+        for i in range(args.steps):
+            flush.zero_()
+            ev[i][0].record(stream)
+            path.quantize(qd, kd, vd)
+            ev[i][1].record(stream)
+            path.attend()
+            ev[i][2].record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+    step_ms = [e[0].elapsed_time(e[2]) for e in ev]
+    attn_ms = [e[1].elapsed_time(e[2]) for e in ev]
+    quant_ms = [e[0].elapsed_time(e[1]) for e in ev]
+    status = qa.get_error()
+    if status != 0:
+        raise RuntimeError(f"device error {status} during timing")
+    ms = max_over_ranks(sum(step_ms) / len(step_ms), world)
+    attn = max_over_ranks(sum(attn_ms) / len(attn_ms), world)
+    quant = max_over_ranks(sum(quant_ms) / len(quant_ms), world)
+
+    # end to end through the C ABI with host buffers (pinned), copies inside the timed region
+    qh, kh, vh = (t.pin_memory() for t in (q, k, v))
+    oh = torch.empty(w.shape, dtype=torch.bfloat16).pin_memory()
+    e2e_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
+    for _ in range(2):
+        qd.copy_(qh, non_blocking=True); kd.copy_(kh, non_blocking=True); vd.copy_(vh, non_blocking=True)
+        oh.copy_(step(), non_blocking=True)
+    torch.cuda.synchronize()
+    barrier(world)
+    for i in range(args.steps):
+        flush.zero_()
+        e2e_ev[i][0].record(stream)
+        qd.copy_(qh, non_blocking=True)
+        kd.copy_(kh, non_blocking=True)
+        vd.copy_(vh, non_blocking=True)
+        oh.copy_(step(), non_blocking=True)
+        e2e_ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    e2e_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in e2e_ev) / args.steps, world)
+
+    hbm_gbs, bf16_tf, peak_kind = load_peaks()
+    fp8_peak = bf16_tf * FP8_PER_BF16
+    flops = w.flops
+    achieved_tf = flops / (attn * 1e-3) / 1e12
+    in_bytes = 3 * q.numel() * 2
+    quant_bytes = 3 * q.numel() * (2 + 2 + 1)   # amax read 2 B, quantize read 2 B + write 1 B
+    clock = clocks.summary()
+    result = {
+        "metric": "quantized attention TFLOP/s @L=8704,H=24,D=128 and % of B200 FP8 peak",
+        "value": world * flops / (ms * 1e-3) / 1e12,
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": ms,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "e4m3",
+        "data": "synthetic: seeded N(0,1) bf16 Q/K/V, 4 of 128 Q/K channels per head x10",
+        "config": {"workload": f"{w.name}: B=1 H=24 L=8704 (512 text + 4096 target + 4096 "
+                               f"context) D=128 {w.mode.upper()} full attention",
+                   "mode": w.mode, "B": w.B, "H": w.H, "L": w.L, "D": w.D,
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                   "l2": "flushed between steps (256 MiB write outside the timed events)"},
+        "roofline": {"bound": "tensor", "achieved": achieved_tf, "peak": fp8_peak,
+                     "unit": "TFLOP/s", "frac": achieved_tf / fp8_peak, "traffic": None,
+                     "kernel": "k_attn_fp8_fwd<128>",
+                     "peak_source": f"{peak_kind} bf16 burst {bf16_tf} TFLOP/s x {FP8_PER_BF16} "
+                                    "(nominal FP8/BF16 ratio)",
+                     "kernel_ms": attn},
+        "quantize": {"ms": quant, "algorithmic_bytes": quant_bytes,
+                     "gbs": quant_bytes / (quant * 1e-3) / 1e9,
+                     "frac_hbm": quant_bytes / (quant * 1e-3) / 1e9 / hbm_gbs,
+                     "hbm_peak_gbs": hbm_gbs, "launches": 6},
+        "e2e": {"value": world * flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+                "ms_per_step": e2e_ms, "h2d_bytes_per_step": in_bytes,
+                "d2h_bytes_per_step": q.numel() * 2},
+        "gpu_launches": 7 * args.steps,
+        "clocks": clock,
+    }
+    if rank == 0:
+        result["cpu_baseline"] = cpu_baseline(w) if not args.no_cpu_baseline else None
+        print(json.dumps(result), flush=True)
+    barrier(world)
+    del path
+    if world > 1:
+        torch.distributed.destroy_process_group()
+
+
+def cpu_baseline(w, rows_per_head: int = 1024, seed: int = 0):
+    """The oracle as it stands, on the host cores: quantize all of Q, K, V, then attention for
+    a seeded sample of `rows_per_head` query rows of every head; throughput counts the sampled
+    rows' BMM1 + BMM2 FLOPs only (the full-tensor quantization is charged to the sample)."""
+    import oracle
+    q, k, v = workloads.make_qkv(w)
+    g = torch.Generator().manual_seed(seed)
+    rows = []
+    for h in range(w.H):
+        pick = torch.randperm(w.L, generator=g)[:rows_per_head]
+        rows.extend((h * w.L + pick).tolist())
+    rows = sorted(rows)
+    t0 = time.perf_counter()
+    oracle.method_forward(q, k, v, w.mode, sm_scale=w.sm_scale, rows=rows)
+    dt = time.perf_counter() - t0
+    flops = 4.0 * w.D * w.L * len(rows)
+    return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": oracle.num_threads(),
+            "kind": "oracle", "seconds": dt,
+            "sample": f"{rows_per_head} of {w.L} query rows per head x {w.H} heads "
+                      f"({len(rows)} rows, {flops:.3e} FLOP) of {w.name}, plus amax+quantize "
+                      "of the full Q, K, V"}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    w = workloads.WORKLOADS["edit_fp8" if args.mode == "fp8" else "edit_fp4"]
+    for _ in range(args.warmup):
+        cpu_baseline(w, rows_per_head=16)
+    times, flops = [], 0.0
+    for i in range(args.steps):
+        r = cpu_baseline(w, rows_per_head=128, seed=i + 1)
+        times.append(r["seconds"])
+        flops = r["value"] * r["seconds"] * 1e12
+    ms = 1e3 * sum(times) / len(times)
+    value = flops / (ms * 1e-3) / 1e12
+    cores = r["cores"]
+    print(json.dumps({
+        "impl": "reference",
+        "metric": "quantized attention TFLOP/s @L=8704,H=24,D=128 and % of B200 FP8 peak",
+        "value": value, "unit": "TFLOP/s", "n_gpus": 0, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": f"{w.name}: B=1 H=24 L=8704 D=128 {w.mode.upper()}",
+                   "mode": w.mode, "B": w.B, "H": w.H, "L": w.L, "D": w.D},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                         "sample": r["sample"].replace("128 of", "128 of")},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--mode", default="fp8", choices=["fp8", "fp4"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_gpu(args)
+
+
+if __name__ == "__main__":
+    main()

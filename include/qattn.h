@@ -1,0 +1,150 @@
+/*
+ * qattn.h -- C ABI of libqattn, quantized scaled-dot-product attention for NVIDIA B200 (sm_100a).
+ *
+ * The operation is the quantized SDPA of the FLUX.1 Kontext transformer as described in the
+ * NVIDIA developer blog "Optimizing FLUX.1 Kontext for Image Editing with Low-Precision
+ * Quantization", section "Workflow and quantization" (the four SDPA bullets and Fig. 4):
+ *   1. Q, K, V are FakeQuantized to per-tensor FP8 (E4M3), or to per-block FP4 (E2M1 values
+ *      with E4M3 block scales and an FP32 tensor scale) followed by an extra per-tensor FP8
+ *      quantize, because BMM1's inputs are FP8 in both modes;
+ *   2. BMM1 = Q K^T in FP8 with FP32 accumulation;
+ *   3. softmax in FP32, unquantized;
+ *   4. P requantized to per-tensor FP8 (scale 1/448), BMM2 = P V in FP8.
+ * Scales come from max-calibration of the tensor in hand (the blog's post-training
+ * calibration step reduced to one tensor).
+ *
+ * Conventions for every entry point:
+ *   - Pointers named *_dev or tensor data are DEVICE pointers on the current CUDA device; the
+ *     caller owns and allocates every buffer.  The library keeps no state besides one device
+ *     error word per device and cached kernel attributes.
+ *   - Work is enqueued on `stream` (0 = legacy default stream) and is asynchronous: scales and
+ *     amax stay in device memory, nothing synchronizes with the host.  qattn_get_error() is the
+ *     only call that synchronizes.
+ *   - Argument errors are detected on the host before anything is launched and returned as
+ *     QATTN_ERR_INVALID_ARG / QATTN_ERR_UNSUPPORTED; launch failures as QATTN_ERR_CUDA.  Errors
+ *     found on the device (non-finite input, a timed-out wait) are recorded in the device
+ *     error word and reported by qattn_get_error().
+ *   - Tensors are contiguous.  bf16 inputs are 16-byte aligned; E4M3 code buffers are 16-byte
+ *     aligned (the attention kernel reads them with TMA).
+ *   - Only sm_100 devices are supported (QATTN_ERR_UNSUPPORTED otherwise).
+ */
+#ifndef QATTN_H_
+#define QATTN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define QATTN_API __attribute__((visibility("default")))
+#else
+#define QATTN_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* qattn_stream_t; /* a cudaStream_t */
+
+typedef enum {
+  QATTN_OK = 0,
+  QATTN_ERR_INVALID_ARG = 1,
+  QATTN_ERR_UNSUPPORTED = 2,
+  QATTN_ERR_CUDA = 3,
+  QATTN_ERR_NONFINITE = 4,
+  QATTN_ERR_TIMEOUT = 5
+} qattn_status;
+
+typedef enum { QATTN_MODE_FP8 = 0, QATTN_MODE_FP4 = 1 } qattn_mode;
+
+/* Per-tensor dequantization multipliers of the E4M3 inputs of qattn_forward: value of an
+ * element = val(code) * (*s).  All three are device pointers to one float each, as written by
+ * qattn_quantize_fp8 (scale_dev) or qattn_quantize_fp4_block (scale8_dev). */
+typedef struct {
+  const float* s_q;
+  const float* s_k;
+  const float* s_v;
+} qattn_scales;
+
+/* Calibration: *amax_dev = max |x| over n bf16 elements, exactly.
+ * Blog, "Workflow and quantization", flow steps 3-4 (post-training calibration), applied to the
+ * tensor in hand.  x_bf16: device, n elements, 16-byte aligned.  amax_dev: device float, set to
+ * 0 and then reduced into (so it must not be shared by concurrent calls).  A non-finite element
+ * records QATTN_ERR_NONFINITE in the error word (amax is then inf or NaN). */
+QATTN_API qattn_status qattn_calibrate_amax(const void* x_bf16, size_t n, float* amax_dev,
+                                  qattn_stream_t stream);
+
+/* Per-tensor FP8 FakeQuantize (blog, "Workflow and quantization", first SDPA bullet, Fig. 4):
+ *   s = fl32(amax / 448) (s = 1 when amax == 0);  out[i] = e4m3(fl32(x[i] / s))
+ * with round-to-nearest-even, saturation to +-448 and the sign kept.  x_bf16: device [n],
+ * 16-byte aligned.  amax_dev: device float from qattn_calibrate_amax.  out_e4m3: device [n]
+ * bytes, 8-byte aligned.  scale_dev: device float, receives s (the dequantization multiplier).
+ * A non-finite amax records QATTN_ERR_NONFINITE and writes nothing. */
+QATTN_API qattn_status qattn_quantize_fp8(const void* x_bf16, size_t n, const float* amax_dev,
+                                uint8_t* out_e4m3, float* scale_dev, qattn_stream_t stream);
+
+/* Per-block FP4 FakeQuantize fused with the per-tensor FP8 quantize of the dequantized values
+ * (blog, "Workflow and quantization", first and second SDPA bullets; Fig. 4 "inputs quantized
+ * with per-block FP4").  Blocks are 16 consecutive elements (along D of a [.., D] tensor):
+ *   s_g  = fl32(amax / 2688)                        -> *gscale_dev
+ *   s_b  = e4m3(fl32(amax_b / fl32(6 * s_g)))       -> blk_scale_e4m3[n / 16]
+ *   c    = e2m1(fl32(x / fl32(val(s_b) * s_g)))     -> out_e2m1[n / 2] (element 2i in the low
+ *                                                      nibble of byte i); 0 if that scale is 0
+ *   xhat = fl32(fl32(val(c) * val(s_b)) * s_g)
+ *   s8   = fl32(max|xhat| / 448)                    -> *scale8_dev
+ *   c8   = e4m3(fl32(xhat / s8))                    -> out_e4m3_requant[n]
+ * x_bf16: device [n], n % 16 == 0, 16-byte aligned.  out_e2m1 8-byte aligned,
+ * out_e4m3_requant 16-byte aligned.  out_e4m3_requant and scale8_dev may both be NULL (FP4
+ * codes only).  Non-finite amax: QATTN_ERR_NONFINITE recorded, nothing written. */
+QATTN_API qattn_status qattn_quantize_fp4_block(const void* x_bf16, size_t n, const float* amax_dev,
+                                      uint8_t* out_e2m1, uint8_t* blk_scale_e4m3,
+                                      float* gscale_dev, uint8_t* out_e4m3_requant,
+                                      float* scale8_dev, qattn_stream_t stream);
+
+/* Quantized attention forward, full (non-causal) attention over [B, H, L, D] (blog, "Workflow
+ * and quantization", SDPA bullets 2-4 and Fig. 4):
+ *   S' = (Q8 K8^T) * s_q * s_k * sm_scale * log2(e)   FP8 MMA, FP32 accumulation
+ *   M  = ceil(running row max of S')                  power-of-two running max
+ *   p  = 2^(S' - M),  l = sum p                       FP32
+ *   P8 = e4m3(p * 448)                                per-tensor scale 1/448
+ *   O  = (P8 V8) * s_v / 448 / l                      FP8 MMA, FP32 accumulation -> bf16
+ * q8, k8, v8: device E4M3 codes [B, H, L, D] (row-major, 16-byte aligned).  out_bf16: device
+ * [B, H, L, D] bf16.  D must be 64 or 128; B, H, L >= 1.  mode records whether the codes came
+ * from the FP8 or the FP4 path (both feed BMM1 with E4M3 codes).  sm_scale > 0 (1/sqrt(D) in
+ * the model). */
+QATTN_API qattn_status qattn_forward(const uint8_t* q8, const uint8_t* k8, const uint8_t* v8,
+                           void* out_bf16, int B, int H, int L, int D,
+                           const qattn_scales* scales, float sm_scale, qattn_mode mode,
+                           qattn_stream_t stream);
+
+/* Same over a packed batch of variable-length sequences ([1, H, T, D] with sequence s at token
+ * rows [cu_seqlens[s], cu_seqlens[s+1]) of every head; attention stays inside a sequence).
+ * cu_seqlens_dev: device int32 [nseq + 1], non-decreasing from 0 to total_tokens; max_seqlen:
+ * the largest cu_seqlens[s+1] - cu_seqlens[s] (a larger value only costs idle CTAs; a smaller
+ * one leaves rows unwritten).  The host does not read cu_seqlens_dev. */
+QATTN_API qattn_status qattn_forward_varlen(const uint8_t* q8, const uint8_t* k8, const uint8_t* v8,
+                                  void* out_bf16, const int* cu_seqlens_dev, int nseq,
+                                  int max_seqlen, int total_tokens, int H, int D,
+                                  const qattn_scales* scales, float sm_scale, qattn_mode mode,
+                                  qattn_stream_t stream);
+
+/* Synchronizes `stream`, then returns and clears the current device's error word: QATTN_OK,
+ * QATTN_ERR_NONFINITE or QATTN_ERR_TIMEOUT (or QATTN_ERR_CUDA if the synchronization failed). */
+QATTN_API qattn_status qattn_get_error(qattn_stream_t stream);
+
+/* Human-readable name of a status code (static storage). */
+QATTN_API const char* qattn_status_str(qattn_status status);
+
+/* Test hooks, not part of the method.  qattn_debug_set_wait_timeout_ns sets the limit after
+ * which a wait inside the attention kernel gives up (default 2 s; 0 restores the default).
+ * qattn_debug_inject_missing_q(1) makes the next attention launches never load Q, so every
+ * wait of the kernel runs into that limit and the kernel reports QATTN_ERR_TIMEOUT instead of
+ * hanging. */
+QATTN_API void qattn_debug_set_wait_timeout_ns(uint64_t ns);
+QATTN_API void qattn_debug_inject_missing_q(int enable);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* QATTN_H_ */

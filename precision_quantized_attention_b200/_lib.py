@@ -1,0 +1,170 @@
+"""ctypes binding of libqattn (include/qattn.h): argument marshalling only.
+
+Every entry point has the C name without the ``qattn_`` prefix, takes torch CUDA tensors for
+the device buffers, enqueues on torch's current CUDA stream and raises ``QattnError`` on a
+non-OK status.  There is no fallback: if the shared library is missing, loading fails loudly.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libqattn.so")
+
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_NONFINITE, ERR_TIMEOUT = range(6)
+MODE_FP8, MODE_FP4 = 0, 1
+
+# every symbol the header declares
+EXPORTS = (
+    "qattn_calibrate_amax", "qattn_quantize_fp8", "qattn_quantize_fp4_block", "qattn_forward",
+    "qattn_forward_varlen", "qattn_get_error", "qattn_status_str",
+    "qattn_debug_set_wait_timeout_ns", "qattn_debug_inject_missing_q",
+)
+
+
+class QattnError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {status_str(status)} ({status})")
+
+
+class _Scales(ctypes.Structure):
+    _fields_ = [("s_q", ctypes.c_void_p), ("s_k", ctypes.c_void_p), ("s_v", ctypes.c_void_p)]
+
+
+_lib = None
+
+
+def load() -> ctypes.CDLL:
+    """Load libqattn.so (built in-tree by ``python -m precision_quantized_attention_b200.build``)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing: build it with "
+                          "`python -m precision_quantized_attention_b200.build`")
+    lib = ctypes.CDLL(LIB_PATH)
+    P, S, I, F = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int, ctypes.c_float
+    lib.qattn_calibrate_amax.argtypes = [P, S, P, P]
+    lib.qattn_quantize_fp8.argtypes = [P, S, P, P, P, P]
+    lib.qattn_quantize_fp4_block.argtypes = [P, S, P, P, P, P, P, P, P]
+    lib.qattn_forward.argtypes = [P, P, P, P, I, I, I, I, ctypes.POINTER(_Scales), F, I, P]
+    lib.qattn_forward_varlen.argtypes = [P, P, P, P, P, I, I, I, I, I, ctypes.POINTER(_Scales),
+                                         F, I, P]
+    lib.qattn_get_error.argtypes = [P]
+    lib.qattn_status_str.argtypes = [I]
+    lib.qattn_status_str.restype = ctypes.c_char_p
+    lib.qattn_debug_set_wait_timeout_ns.argtypes = [ctypes.c_uint64]
+    lib.qattn_debug_set_wait_timeout_ns.restype = None
+    lib.qattn_debug_inject_missing_q.argtypes = [I]
+    lib.qattn_debug_inject_missing_q.restype = None
+    for name in EXPORTS[:6]:
+        getattr(lib, name).restype = I
+    _lib = lib
+    return lib
+
+
+def status_str(status: int) -> str:
+    return load().qattn_status_str(int(status)).decode()
+
+
+def _check(status: int, what: str):
+    if status != OK:
+        raise QattnError(status, what)
+
+
+def _stream(stream=None):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _dev(t: torch.Tensor | None, dtype=None, what="tensor"):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError(f"{what} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{what} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{what} must be {dtype}, got {t.dtype}")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def calibrate_amax(x: torch.Tensor, amax: torch.Tensor, stream=None):
+    _check(load().qattn_calibrate_amax(_dev(x, torch.bfloat16, "x"), x.numel(),
+                                       _dev(amax, torch.float32, "amax"), _stream(stream)),
+           "qattn_calibrate_amax")
+
+
+def quantize_fp8(x: torch.Tensor, amax: torch.Tensor, out: torch.Tensor, scale: torch.Tensor,
+                 stream=None):
+    if out.numel() != x.numel():
+        raise ValueError("out must have x.numel() bytes")
+    _check(load().qattn_quantize_fp8(_dev(x, torch.bfloat16, "x"), x.numel(),
+                                     _dev(amax, torch.float32, "amax"),
+                                     _dev(out, torch.uint8, "out"),
+                                     _dev(scale, torch.float32, "scale"), _stream(stream)),
+           "qattn_quantize_fp8")
+
+
+def quantize_fp4_block(x: torch.Tensor, amax: torch.Tensor, out_e2m1: torch.Tensor,
+                       blk_scale: torch.Tensor, gscale: torch.Tensor,
+                       out_e4m3_requant: torch.Tensor | None = None,
+                       scale8: torch.Tensor | None = None, stream=None):
+    n = x.numel()
+    if out_e2m1.numel() != n // 2 or blk_scale.numel() != n // 16:
+        raise ValueError("out_e2m1 needs n/2 bytes and blk_scale n/16 bytes")
+    if out_e4m3_requant is not None and out_e4m3_requant.numel() != n:
+        raise ValueError("out_e4m3_requant needs n bytes")
+    _check(load().qattn_quantize_fp4_block(
+        _dev(x, torch.bfloat16, "x"), n, _dev(amax, torch.float32, "amax"),
+        _dev(out_e2m1, torch.uint8, "out_e2m1"), _dev(blk_scale, torch.uint8, "blk_scale"),
+        _dev(gscale, torch.float32, "gscale"),
+        _dev(out_e4m3_requant, torch.uint8, "out_e4m3_requant"),
+        _dev(scale8, torch.float32, "scale8"), _stream(stream)), "qattn_quantize_fp4_block")
+
+
+def _scales(s_q, s_k, s_v):
+    return _Scales(_dev(s_q, torch.float32, "s_q").value, _dev(s_k, torch.float32, "s_k").value,
+                   _dev(s_v, torch.float32, "s_v").value)
+
+
+def forward(q8, k8, v8, out, s_q, s_k, s_v, sm_scale: float, mode: int = MODE_FP8, stream=None):
+    """q8, k8, v8: uint8 E4M3 codes [B, H, L, D]; out: bf16 [B, H, L, D]."""
+    B, H, L, D = q8.shape
+    for t, nm in ((k8, "k8"), (v8, "v8"), (out, "out")):
+        if tuple(t.shape) != (B, H, L, D):
+            raise ValueError(f"{nm} shape {tuple(t.shape)} != {(B, H, L, D)}")
+    sc = _scales(s_q, s_k, s_v)
+    _check(load().qattn_forward(_dev(q8, torch.uint8, "q8"), _dev(k8, torch.uint8, "k8"),
+                                _dev(v8, torch.uint8, "v8"), _dev(out, torch.bfloat16, "out"),
+                                B, H, L, D, ctypes.byref(sc), float(sm_scale), int(mode),
+                                _stream(stream)), "qattn_forward")
+
+
+def forward_varlen(q8, k8, v8, out, cu_seqlens: torch.Tensor, max_seqlen: int, s_q, s_k, s_v,
+                   sm_scale: float, mode: int = MODE_FP4, stream=None):
+    """q8, k8, v8: uint8 [1, H, T, D]; cu_seqlens: int32 CUDA tensor [nseq + 1]."""
+    _, H, T, D = q8.shape
+    sc = _scales(s_q, s_k, s_v)
+    _check(load().qattn_forward_varlen(
+        _dev(q8, torch.uint8, "q8"), _dev(k8, torch.uint8, "k8"), _dev(v8, torch.uint8, "v8"),
+        _dev(out, torch.bfloat16, "out"), _dev(cu_seqlens, torch.int32, "cu_seqlens"),
+        cu_seqlens.numel() - 1, int(max_seqlen), T, H, D, ctypes.byref(sc), float(sm_scale),
+        int(mode), _stream(stream)), "qattn_forward_varlen")
+
+
+def get_error(stream=None) -> int:
+    """Synchronizes the stream; returns (and clears) the device error word as a status."""
+    return int(load().qattn_get_error(_stream(stream)))
+
+
+def debug_set_wait_timeout_ns(ns: int):
+    load().qattn_debug_set_wait_timeout_ns(int(ns))
+
+
+def debug_inject_missing_q(enable: bool):
+    load().qattn_debug_inject_missing_q(1 if enable else 0)

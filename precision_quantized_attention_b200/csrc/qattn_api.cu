@@ -1,0 +1,211 @@
+// qattn_api.cu -- the C ABI (include/qattn.h): argument checks, device checks, launches.
+#include <cuda_runtime.h>
+#include <cstdint>
+
+#include "../../include/qattn.h"
+#include "sm100_ptx.cuh"
+
+namespace qattn {
+cudaError_t launch_amax(const void* x, size_t n, float* amax, int* err, int num_sms,
+                        cudaStream_t stream);
+cudaError_t launch_quant_fp8(const void* x, size_t n, const float* amax, uint8_t* out,
+                             float* scale, int* err, int num_sms, cudaStream_t stream);
+cudaError_t launch_quant_fp4_block(const void* x, size_t n, const float* amax, uint8_t* packed,
+                                   uint8_t* bscale, float* gscale, uint8_t* codes8, float* scale8,
+                                   int* err, int num_sms, cudaStream_t stream);
+cudaError_t launch_attention(const uint8_t* q8, const uint8_t* k8, const uint8_t* v8, void* out,
+                             int B, int H, int L, int D, const int* cu_seqlens, int nseq,
+                             int max_seqlen, int total_tokens, const float* s_q, const float* s_k,
+                             const float* s_v, float sm_scale, int* err, uint64_t timeout_ns,
+                             int inject_missing_q, cudaStream_t stream);
+}  // namespace qattn
+
+// The device error word (one per device that loads the library).
+static __device__ int g_qattn_error = 0;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+constexpr uint64_t kDefaultTimeoutNs = 2000000000ull;
+
+struct DeviceInfo {
+  bool ready = false;
+  bool supported = false;
+  int num_sms = 0;
+  int* err = nullptr;
+};
+DeviceInfo g_dev[kMaxDevices];
+uint64_t g_timeout_ns = kDefaultTimeoutNs;
+int g_inject_missing_q = 0;
+
+// Per-device setup on first use: capability check, SM count, address of the error word.
+qattn_status device_info(DeviceInfo** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return QATTN_ERR_CUDA;
+  DeviceInfo& d = g_dev[dev];
+  if (!d.ready) {
+    int major = 0, minor = 0, sms = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return QATTN_ERR_CUDA;
+    d.supported = (major == 10 && minor == 0);
+    d.num_sms = sms;
+    if (d.supported) {
+      void* p = nullptr;
+      if (cudaGetSymbolAddress(&p, g_qattn_error) != cudaSuccess) return QATTN_ERR_CUDA;
+      d.err = static_cast<int*>(p);
+    }
+    d.ready = true;
+  }
+  if (!d.supported) return QATTN_ERR_UNSUPPORTED;
+  *out = &d;
+  return QATTN_OK;
+}
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+qattn_status from_cuda(cudaError_t e) { return e == cudaSuccess ? QATTN_OK : QATTN_ERR_CUDA; }
+
+qattn_status check_attention_common(const uint8_t* q8, const uint8_t* k8, const uint8_t* v8,
+                                    const void* out, int H, int D, const qattn_scales* sc,
+                                    float sm_scale, qattn_mode mode) {
+  if (!q8 || !k8 || !v8 || !out || !sc || !sc->s_q || !sc->s_k || !sc->s_v)
+    return QATTN_ERR_INVALID_ARG;
+  if (!aligned(q8, 16) || !aligned(k8, 16) || !aligned(v8, 16) || !aligned(out, 16))
+    return QATTN_ERR_INVALID_ARG;
+  if (H < 1 || !(sm_scale > 0.0f) || !(sm_scale < 3.0e38f)) return QATTN_ERR_INVALID_ARG;
+  if (D != 64 && D != 128) return QATTN_ERR_UNSUPPORTED;
+  if (mode != QATTN_MODE_FP8 && mode != QATTN_MODE_FP4) return QATTN_ERR_INVALID_ARG;
+  return QATTN_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+qattn_status qattn_calibrate_amax(const void* x_bf16, size_t n, float* amax_dev,
+                                  qattn_stream_t stream) {
+  if (!x_bf16 || !amax_dev || n == 0 || !aligned(x_bf16, 16) || !aligned(amax_dev, 4))
+    return QATTN_ERR_INVALID_ARG;
+  DeviceInfo* d = nullptr;
+  qattn_status st = device_info(&d);
+  if (st != QATTN_OK) return st;
+  return from_cuda(qattn::launch_amax(x_bf16, n, amax_dev, d->err, d->num_sms,
+                                      reinterpret_cast<cudaStream_t>(stream)));
+}
+
+qattn_status qattn_quantize_fp8(const void* x_bf16, size_t n, const float* amax_dev,
+                                uint8_t* out_e4m3, float* scale_dev, qattn_stream_t stream) {
+  if (!x_bf16 || !amax_dev || !out_e4m3 || !scale_dev || n == 0) return QATTN_ERR_INVALID_ARG;
+  if (!aligned(x_bf16, 16) || !aligned(out_e4m3, 8) || !aligned(amax_dev, 4) ||
+      !aligned(scale_dev, 4))
+    return QATTN_ERR_INVALID_ARG;
+  DeviceInfo* d = nullptr;
+  qattn_status st = device_info(&d);
+  if (st != QATTN_OK) return st;
+  return from_cuda(qattn::launch_quant_fp8(x_bf16, n, amax_dev, out_e4m3, scale_dev, d->err,
+                                           d->num_sms, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+qattn_status qattn_quantize_fp4_block(const void* x_bf16, size_t n, const float* amax_dev,
+                                      uint8_t* out_e2m1, uint8_t* blk_scale_e4m3,
+                                      float* gscale_dev, uint8_t* out_e4m3_requant,
+                                      float* scale8_dev, qattn_stream_t stream) {
+  if (!x_bf16 || !amax_dev || !out_e2m1 || !blk_scale_e4m3 || !gscale_dev || n == 0 ||
+      n % 16 != 0)
+    return QATTN_ERR_INVALID_ARG;
+  if ((out_e4m3_requant == nullptr) != (scale8_dev == nullptr)) return QATTN_ERR_INVALID_ARG;
+  if (!aligned(x_bf16, 16) || !aligned(out_e2m1, 8) || !aligned(amax_dev, 4) ||
+      !aligned(gscale_dev, 4) || (out_e4m3_requant && !aligned(out_e4m3_requant, 16)) ||
+      (scale8_dev && !aligned(scale8_dev, 4)))
+    return QATTN_ERR_INVALID_ARG;
+  DeviceInfo* d = nullptr;
+  qattn_status st = device_info(&d);
+  if (st != QATTN_OK) return st;
+  return from_cuda(qattn::launch_quant_fp4_block(x_bf16, n, amax_dev, out_e2m1, blk_scale_e4m3,
+                                                 gscale_dev, out_e4m3_requant, scale8_dev, d->err,
+                                                 d->num_sms,
+                                                 reinterpret_cast<cudaStream_t>(stream)));
+}
+
+qattn_status qattn_forward(const uint8_t* q8, const uint8_t* k8, const uint8_t* v8,
+                           void* out_bf16, int B, int H, int L, int D,
+                           const qattn_scales* scales, float sm_scale, qattn_mode mode,
+                           qattn_stream_t stream) {
+  qattn_status st = check_attention_common(q8, k8, v8, out_bf16, H, D, scales, sm_scale, mode);
+  if (st != QATTN_OK) return st;
+  if (B < 1 || L < 1) return QATTN_ERR_INVALID_ARG;
+  if (static_cast<int64_t>(B) * H > 65535 * 65535LL || B > 65535 || H > 65535)
+    return QATTN_ERR_UNSUPPORTED;
+  if (static_cast<int64_t>(B) * H * L * D >= (int64_t(1) << 40)) return QATTN_ERR_UNSUPPORTED;
+  DeviceInfo* d = nullptr;
+  st = device_info(&d);
+  if (st != QATTN_OK) return st;
+  return from_cuda(qattn::launch_attention(q8, k8, v8, out_bf16, B, H, L, D, nullptr, 0, L, L,
+                                           scales->s_q, scales->s_k, scales->s_v, sm_scale,
+                                           d->err, g_timeout_ns, g_inject_missing_q,
+                                           reinterpret_cast<cudaStream_t>(stream)));
+}
+
+qattn_status qattn_forward_varlen(const uint8_t* q8, const uint8_t* k8, const uint8_t* v8,
+                                  void* out_bf16, const int* cu_seqlens_dev, int nseq,
+                                  int max_seqlen, int total_tokens, int H, int D,
+                                  const qattn_scales* scales, float sm_scale, qattn_mode mode,
+                                  qattn_stream_t stream) {
+  qattn_status st = check_attention_common(q8, k8, v8, out_bf16, H, D, scales, sm_scale, mode);
+  if (st != QATTN_OK) return st;
+  if (!cu_seqlens_dev || !aligned(cu_seqlens_dev, 4) || nseq < 1 || max_seqlen < 1 ||
+      total_tokens < 1 || max_seqlen > total_tokens)
+    return QATTN_ERR_INVALID_ARG;
+  if (nseq > 65535 || H > 65535) return QATTN_ERR_UNSUPPORTED;
+  DeviceInfo* d = nullptr;
+  st = device_info(&d);
+  if (st != QATTN_OK) return st;
+  return from_cuda(qattn::launch_attention(q8, k8, v8, out_bf16, 1, H, 0, D, cu_seqlens_dev,
+                                           nseq, max_seqlen, total_tokens, scales->s_q,
+                                           scales->s_k, scales->s_v, sm_scale, d->err,
+                                           g_timeout_ns, g_inject_missing_q,
+                                           reinterpret_cast<cudaStream_t>(stream)));
+}
+
+qattn_status qattn_get_error(qattn_stream_t stream) {
+  DeviceInfo* d = nullptr;
+  qattn_status st = device_info(&d);
+  if (st != QATTN_OK) return st;
+  if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return QATTN_ERR_CUDA;
+  int word = 0;
+  if (cudaMemcpyFromSymbol(&word, g_qattn_error, sizeof(int)) != cudaSuccess) return QATTN_ERR_CUDA;
+  if (word != 0) {
+    const int zero = 0;
+    if (cudaMemcpyToSymbol(g_qattn_error, &zero, sizeof(int)) != cudaSuccess)
+      return QATTN_ERR_CUDA;
+  }
+  switch (word) {
+    case 0: return QATTN_OK;
+    case qattn::DEV_ERR_NONFINITE: return QATTN_ERR_NONFINITE;
+    case qattn::DEV_ERR_TIMEOUT: return QATTN_ERR_TIMEOUT;
+    default: return QATTN_ERR_CUDA;
+  }
+}
+
+const char* qattn_status_str(qattn_status status) {
+  switch (status) {
+    case QATTN_OK: return "QATTN_OK";
+    case QATTN_ERR_INVALID_ARG: return "QATTN_ERR_INVALID_ARG";
+    case QATTN_ERR_UNSUPPORTED: return "QATTN_ERR_UNSUPPORTED";
+    case QATTN_ERR_CUDA: return "QATTN_ERR_CUDA";
+    case QATTN_ERR_NONFINITE: return "QATTN_ERR_NONFINITE";
+    case QATTN_ERR_TIMEOUT: return "QATTN_ERR_TIMEOUT";
+  }
+  return "QATTN_ERR_UNKNOWN";
+}
+
+void qattn_debug_set_wait_timeout_ns(uint64_t ns) {
+  g_timeout_ns = ns ? ns : kDefaultTimeoutNs;
+}
+
+void qattn_debug_inject_missing_q(int enable) { g_inject_missing_q = enable ? 1 : 0; }
+
+}  // extern "C"

@@ -1,0 +1,230 @@
+// quant.cu -- HBM-bound calibration and FakeQuantize passes for Q, K and V.
+//
+// Method: NVIDIA developer blog "Optimizing FLUX.1 Kontext for Image Editing with Low-Precision
+// Quantization", section "Workflow and quantization": Q, K, V are quantized per tensor to FP8
+// or per block to FP4 (first SDPA bullet, Fig. 4), an extra FP8 quantize feeds BMM1 (second
+// bullet), and scales come from post-training calibration (steps 3-4 of the flow), reduced here
+// to max-calibration of the tensor in hand.
+//
+// Every kernel streams its input once with 16-byte loads over a grid sized to the SM count,
+// and applies scales with correctly rounded binary32 division, so the codes are bit-identical
+// to the definition (E4M3 / E2M1 round-to-nearest-even with saturation, the hardware cvt
+// forms).
+#include <cuda_runtime.h>
+#include <cstdint>
+
+#include "sm100_ptx.cuh"
+
+namespace qattn {
+
+// -------------------------------------------------------------------------------------------
+// amax = max |x| over a bf16 tensor.  |x| of a bf16 is its bit pattern with the sign cleared,
+// and for non-negative values (NaN and inf included) the integer order of those patterns is
+// the numeric order, so the reduction runs on 16-bit integers (two per 32-bit word).
+// The result is written as float bits with one atomicMax per CTA; the host zeroes it first.
+// -------------------------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t absmax_word(uint32_t m2, uint32_t w) {
+  return __vmaxu2(m2, w & 0x7FFF7FFFu);
+}
+
+__global__ void __launch_bounds__(256) k_amax_bf16(const uint4* __restrict__ xv, size_t nvec,
+                                                   const uint16_t* __restrict__ xtail, int ntail,
+                                                   unsigned* __restrict__ amax_bits,
+                                                   int* __restrict__ err) {
+  uint32_t m2 = 0;
+  const size_t stride = static_cast<size_t>(gridDim.x) * blockDim.x;
+  size_t i = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  for (; i + 3 * stride < nvec; i += 4 * stride) {
+    uint4 a = __ldcs(xv + i), b = __ldcs(xv + i + stride);
+    uint4 c = __ldcs(xv + i + 2 * stride), d = __ldcs(xv + i + 3 * stride);
+    m2 = absmax_word(m2, a.x); m2 = absmax_word(m2, a.y);
+    m2 = absmax_word(m2, a.z); m2 = absmax_word(m2, a.w);
+    m2 = absmax_word(m2, b.x); m2 = absmax_word(m2, b.y);
+    m2 = absmax_word(m2, b.z); m2 = absmax_word(m2, b.w);
+    m2 = absmax_word(m2, c.x); m2 = absmax_word(m2, c.y);
+    m2 = absmax_word(m2, c.z); m2 = absmax_word(m2, c.w);
+    m2 = absmax_word(m2, d.x); m2 = absmax_word(m2, d.y);
+    m2 = absmax_word(m2, d.z); m2 = absmax_word(m2, d.w);
+  }
+  for (; i < nvec; i += stride) {
+    uint4 a = __ldcs(xv + i);
+    m2 = absmax_word(m2, a.x); m2 = absmax_word(m2, a.y);
+    m2 = absmax_word(m2, a.z); m2 = absmax_word(m2, a.w);
+  }
+  uint32_t m = max(m2 & 0xFFFFu, m2 >> 16);
+  if (blockIdx.x == 0 && static_cast<int>(threadIdx.x) < ntail)
+    m = max(m, static_cast<uint32_t>(xtail[threadIdx.x]) & 0x7FFFu);
+  m = __reduce_max_sync(0xFFFFFFFFu, m);
+  __shared__ uint32_t warp_max[8];
+  if ((threadIdx.x & 31) == 0) warp_max[threadIdx.x >> 5] = m;
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    m = threadIdx.x < (blockDim.x >> 5) ? warp_max[threadIdx.x] : 0u;
+    m = __reduce_max_sync(0xFFFFFFFFu, m);
+    if (threadIdx.x == 0) {
+      if (m >= 0x7F80u) atomicExch(err, DEV_ERR_NONFINITE);
+      atomicMax(amax_bits, m << 16);
+    }
+  }
+}
+
+// -------------------------------------------------------------------------------------------
+// Per-tensor FP8: s = fl32(amax / 448), code = e4m3(fl32(x / s)); amax == 0 gives s = 1.
+// -------------------------------------------------------------------------------------------
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+__device__ __forceinline__ uint32_t quant4_e4m3(uint32_t w0, uint32_t w1, float s) {
+  const uint32_t lo = cvt_e4m3x2(__fdiv_rn(bf16_lo(w0), s), __fdiv_rn(bf16_hi(w0), s));
+  const uint32_t hi = cvt_e4m3x2(__fdiv_rn(bf16_lo(w1), s), __fdiv_rn(bf16_hi(w1), s));
+  return lo | (hi << 16);
+}
+
+__global__ void __launch_bounds__(256) k_quant_fp8(const uint4* __restrict__ xv, size_t nvec,
+                                                   const uint16_t* __restrict__ xtail, int ntail,
+                                                   const float* __restrict__ amax_p,
+                                                   uint2* __restrict__ outv,
+                                                   uint8_t* __restrict__ outtail,
+                                                   float* __restrict__ scale_out,
+                                                   int* __restrict__ err) {
+  const float amax = *amax_p;
+  if (!(amax <= 3.402823466e38f)) {  // inf or NaN: nothing is written
+    if (blockIdx.x == 0 && threadIdx.x == 0) atomicExch(err, DEV_ERR_NONFINITE);
+    return;
+  }
+  const float s = (amax == 0.0f) ? 1.0f : __fdiv_rn(amax, 448.0f);
+  if (blockIdx.x == 0 && threadIdx.x == 0) *scale_out = s;
+  const size_t stride = static_cast<size_t>(gridDim.x) * blockDim.x;
+  for (size_t i = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < nvec;
+       i += stride) {
+    const uint4 a = __ldcs(xv + i);
+    uint2 o;
+    o.x = quant4_e4m3(a.x, a.y, s);
+    o.y = quant4_e4m3(a.z, a.w, s);
+    __stcs(outv + i, o);
+  }
+  if (blockIdx.x == 0 && static_cast<int>(threadIdx.x) < ntail) {
+    const float x = __uint_as_float(static_cast<uint32_t>(xtail[threadIdx.x]) << 16);
+    outtail[threadIdx.x] = static_cast<uint8_t>(cvt_e4m3x2(__fdiv_rn(x, s), 0.0f) & 0xFFu);
+  }
+}
+
+// -------------------------------------------------------------------------------------------
+// Per-block FP4 (16 elements, E2M1 values, E4M3 block scale, FP32 tensor scale), fused with the
+// per-tensor FP8 requantization of the dequantized values that feeds BMM1:
+//   s_g = fl32(amax / 2688); s_b = e4m3(fl32(amax_b / fl32(6 s_g))); eff = fl32(val(s_b) s_g)
+//   c = e2m1(fl32(x / eff)) (eff == 0: c = 0);  xhat = fl32(fl32(val(c) val(s_b)) s_g)
+//   s8 = fl32(max|xhat| / 448), c8 = e4m3(fl32(xhat / s8)).
+// max|xhat| needs no second pass: the block that holds the tensor amax gets s_b = 448 and code
+// 6 (amax / fl32(6 s_g) rounds to 448 in E4M3 and amax / eff rounds to 6 in E2M1), and no
+// other |xhat| can exceed fl32(fl32(6 * 448) * s_g), so max|xhat| = fl32(2688 * s_g).
+// One thread per block: two 16-byte loads, an 8-byte packed store, the scale byte and a
+// 16-byte store of FP8 codes.
+// -------------------------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) k_quant_fp4_block(
+    const uint4* __restrict__ xv, size_t nblocks, const float* __restrict__ amax_p,
+    uint2* __restrict__ packed_out, uint8_t* __restrict__ bscale_out,
+    float* __restrict__ gscale_out, uint4* __restrict__ codes8_out,
+    float* __restrict__ scale8_out, int* __restrict__ err) {
+  const float amax = *amax_p;
+  if (!(amax <= 3.402823466e38f)) {
+    if (blockIdx.x == 0 && threadIdx.x == 0) atomicExch(err, DEV_ERR_NONFINITE);
+    return;
+  }
+  const float sg = (amax == 0.0f) ? 1.0f : __fdiv_rn(amax, 2688.0f);
+  const float six_sg = __fmul_rn(6.0f, sg);
+  const float s8 = (amax == 0.0f) ? 1.0f : __fdiv_rn(__fmul_rn(2688.0f, sg), 448.0f);
+  if (blockIdx.x == 0 && threadIdx.x == 0) {
+    *gscale_out = sg;
+    if (scale8_out) *scale8_out = s8;
+  }
+  const size_t stride = static_cast<size_t>(gridDim.x) * blockDim.x;
+  for (size_t b = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; b < nblocks;
+       b += stride) {
+    const uint4 a0 = __ldcs(xv + 2 * b), a1 = __ldcs(xv + 2 * b + 1);
+    const uint32_t w[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+    float x[16];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      x[2 * i] = bf16_lo(w[i]);
+      x[2 * i + 1] = bf16_hi(w[i]);
+    }
+    uint32_t am2 = 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) am2 = absmax_word(am2, w[i]);
+    const float amax_b = __uint_as_float(max(am2 & 0xFFFFu, am2 >> 16) << 16);
+    const uint32_t sb = cvt_e4m3x2(__fdiv_rn(amax_b, six_sg), 0.0f) & 0xFFu;
+    const float sbv = e4m3_to_f32(sb);
+    const float eff = __fmul_rn(sbv, sg);
+    uint32_t pk0 = 0, pk1 = 0;
+    uint32_t c8[4] = {0u, 0u, 0u, 0u};
+    if (eff != 0.0f) {
+      uint32_t nib[16];
+#pragma unroll
+      for (int i = 0; i < 16; i += 2) {
+        const uint32_t byte = cvt_e2m1x2(__fdiv_rn(x[i], eff), __fdiv_rn(x[i + 1], eff));
+        nib[i] = byte & 0xFu;
+        nib[i + 1] = byte >> 4;
+        if (i < 8) pk0 |= byte << (4 * i);
+        else pk1 |= byte << (4 * (i - 8));
+      }
+#pragma unroll
+      for (int i = 0; i < 16; i += 2) {
+        const float xh0 = __fmul_rn(__fmul_rn(e2m1_to_f32(nib[i]), sbv), sg);
+        const float xh1 = __fmul_rn(__fmul_rn(e2m1_to_f32(nib[i + 1]), sbv), sg);
+        const uint32_t pair = cvt_e4m3x2(__fdiv_rn(xh0, s8), __fdiv_rn(xh1, s8));
+        c8[i / 4] |= pair << (16 * ((i / 2) & 1));
+      }
+    }
+    __stcs(packed_out + b, make_uint2(pk0, pk1));
+    bscale_out[b] = static_cast<uint8_t>(sb);
+    if (codes8_out) __stcs(codes8_out + b, make_uint4(c8[0], c8[1], c8[2], c8[3]));
+  }
+}
+
+// -------------------------------------------------------------------------------------------
+// Host launchers (called from the C-ABI layer, which validates arguments).
+// -------------------------------------------------------------------------------------------
+static int grid_for(size_t work_items, int num_sms) {
+  const size_t per_cta = 256;
+  size_t need = (work_items + per_cta - 1) / per_cta;
+  size_t cap = static_cast<size_t>(num_sms) * 8;  // 8 CTAs of 256 threads fill an SM
+  if (need < 1) need = 1;
+  return static_cast<int>(need < cap ? need : cap);
+}
+
+cudaError_t launch_amax(const void* x, size_t n, float* amax, int* err, int num_sms,
+                        cudaStream_t stream) {
+  cudaError_t e = cudaMemsetAsync(amax, 0, sizeof(float), stream);
+  if (e != cudaSuccess) return e;
+  const size_t nvec = n / 8;
+  const int ntail = static_cast<int>(n - nvec * 8);
+  const uint16_t* xs = static_cast<const uint16_t*>(x);
+  k_amax_bf16<<<grid_for(nvec / 4 + 1, num_sms), 256, 0, stream>>>(
+      static_cast<const uint4*>(x), nvec, xs + nvec * 8, ntail, reinterpret_cast<unsigned*>(amax),
+      err);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_quant_fp8(const void* x, size_t n, const float* amax, uint8_t* out,
+                             float* scale, int* err, int num_sms, cudaStream_t stream) {
+  const size_t nvec = n / 8;
+  const int ntail = static_cast<int>(n - nvec * 8);
+  const uint16_t* xs = static_cast<const uint16_t*>(x);
+  k_quant_fp8<<<grid_for(nvec, num_sms), 256, 0, stream>>>(
+      static_cast<const uint4*>(x), nvec, xs + nvec * 8, ntail, amax,
+      reinterpret_cast<uint2*>(out), out + nvec * 8, scale, err);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_quant_fp4_block(const void* x, size_t n, const float* amax, uint8_t* packed,
+                                   uint8_t* bscale, float* gscale, uint8_t* codes8, float* scale8,
+                                   int* err, int num_sms, cudaStream_t stream) {
+  const size_t nblocks = n / 16;
+  k_quant_fp4_block<<<grid_for(nblocks, num_sms), 256, 0, stream>>>(
+      static_cast<const uint4*>(x), nblocks, amax, reinterpret_cast<uint2*>(packed), bscale,
+      gscale, reinterpret_cast<uint4*>(codes8), scale8, err);
+  return cudaGetLastError();
+}
+
+}  // namespace qattn

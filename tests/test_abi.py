@@ -1,0 +1,64 @@
+"""The C ABI without a GPU: the library loads, exports every symbol include/qattn.h declares,
+and rejects bad arguments on the host before touching the device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from precision_quantized_attention_b200 import _lib
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    with open(os.path.join(ROOT, "include", "qattn.h")) as f:
+        text = f.read()
+    return sorted(set(re.findall(r"QATTN_API\s+[\w\s\*]+?\b(qattn_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_exported_set():
+    assert _declared() == sorted(_lib.EXPORTS)
+
+
+def test_library_loads_and_exports_every_declared_symbol():
+    lib = _lib.load()
+    for name in _declared():
+        assert hasattr(lib, name), name
+    assert _lib.status_str(5) == "QATTN_ERR_TIMEOUT"
+    assert _lib.status_str(42) == "QATTN_ERR_UNKNOWN"
+
+
+def test_oracle_is_not_linked_into_the_product():
+    lib = _lib.load()
+    with pytest.raises(AttributeError):
+        getattr(lib, "orc_attention_e4m3")
+
+
+FAKE = ctypes.c_void_p(0x10000)       # aligned, never dereferenced: checks come first
+MISALIGNED = ctypes.c_void_p(0x10001)
+
+
+def test_host_side_argument_errors():
+    lib = _lib.load()
+    s0 = ctypes.c_void_p(0)
+    assert lib.qattn_calibrate_amax(None, 16, FAKE, s0) == _lib.ERR_INVALID_ARG
+    assert lib.qattn_calibrate_amax(MISALIGNED, 16, FAKE, s0) == _lib.ERR_INVALID_ARG
+    assert lib.qattn_calibrate_amax(FAKE, 0, FAKE, s0) == _lib.ERR_INVALID_ARG
+    assert lib.qattn_quantize_fp8(FAKE, 16, FAKE, None, FAKE, s0) == _lib.ERR_INVALID_ARG
+    # FP4 needs n % 16 == 0 and both-or-neither of the requant outputs
+    assert lib.qattn_quantize_fp4_block(FAKE, 24, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, s0) == _lib.ERR_INVALID_ARG
+    assert lib.qattn_quantize_fp4_block(FAKE, 32, FAKE, FAKE, FAKE, FAKE, FAKE, None, s0) == _lib.ERR_INVALID_ARG
+    sc = _lib._Scales(0x10000, 0x10000, 0x10000)
+    fwd = lib.qattn_forward
+    assert fwd(FAKE, FAKE, FAKE, FAKE, 1, 1, 16, 96, ctypes.byref(sc), 0.1, 0, s0) == _lib.ERR_UNSUPPORTED
+    assert fwd(FAKE, FAKE, FAKE, FAKE, 1, 1, 0, 64, ctypes.byref(sc), 0.1, 0, s0) == _lib.ERR_INVALID_ARG
+    assert fwd(FAKE, FAKE, FAKE, FAKE, 1, 1, 16, 64, ctypes.byref(sc), -1.0, 0, s0) == _lib.ERR_INVALID_ARG
+    assert fwd(FAKE, FAKE, FAKE, FAKE, 1, 1, 16, 64, ctypes.byref(sc), 0.1, 7, s0) == _lib.ERR_INVALID_ARG
+    assert fwd(MISALIGNED, FAKE, FAKE, FAKE, 1, 1, 16, 64, ctypes.byref(sc), 0.1, 0, s0) == _lib.ERR_INVALID_ARG
+    assert fwd(FAKE, FAKE, FAKE, FAKE, 1, 1, 16, 64, None, 0.1, 0, s0) == _lib.ERR_INVALID_ARG
+    bad = _lib._Scales(0x10000, 0, 0x10000)
+    assert fwd(FAKE, FAKE, FAKE, FAKE, 1, 1, 16, 64, ctypes.byref(bad), 0.1, 0, s0) == _lib.ERR_INVALID_ARG
+    vl = lib.qattn_forward_varlen
+    assert vl(FAKE, FAKE, FAKE, FAKE, None, 2, 8, 16, 1, 64, ctypes.byref(sc), 0.1, 1, s0) == _lib.ERR_INVALID_ARG
+    assert vl(FAKE, FAKE, FAKE, FAKE, FAKE, 2, 32, 16, 1, 64, ctypes.byref(sc), 0.1, 1, s0) == _lib.ERR_INVALID_ARG

@@ -1,0 +1,104 @@
+"""GPU calibration and quantize kernels vs the oracle: bit-exact codes, scales and amax."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import precision_quantized_attention_b200 as qa
+import workloads
+
+pytestmark = pytest.mark.gpu
+
+
+def _u8(t):
+    return t.cpu().numpy().reshape(-1)
+
+
+def _inputs():
+    g = torch.Generator().manual_seed(99)
+    cases = {
+        "tiny_tail": torch.randn(37, generator=g),
+        "tail_7": torch.randn(8 * 1000 + 7, generator=g) * 3.0,
+        "subnormal_heavy": torch.randn(16 * 4096, generator=g) * 1e-3,
+        "wide_range": torch.randn(16 * 5000, generator=g) * torch.exp(torch.randn(16 * 5000, generator=g) * 3),
+        "zeros": torch.zeros(16 * 64),
+        "neg_zero": -torch.zeros(16 * 64),
+    }
+    x = torch.randn(16 * 1024, generator=g)
+    x[:16] *= 1e-6          # a block whose E4M3 scale underflows
+    x[100] = -0.0
+    cases["mixed_blocks"] = x
+    return {k: v.to(torch.bfloat16) for k, v in cases.items()}
+
+
+@pytest.mark.parametrize("name", list(_inputs().keys()))
+def test_amax_and_fp8_bit_exact(name):
+    x = _inputs()[name]
+    xd = x.cuda()
+    amax = torch.zeros(1, device="cuda")
+    scale = torch.zeros(1, device="cuda")
+    codes = torch.empty(x.numel(), dtype=torch.uint8, device="cuda")
+    qa.calibrate_amax(xd, amax)
+    qa.quantize_fp8(xd, amax, codes, scale)
+    assert qa.get_error() == 0
+    rc, a = oracle.amax(x)
+    assert rc == 0 and float(amax.item()) == a
+    want, s = oracle.quantize_fp8(x, a)
+    assert np.float32(scale.item()) == s
+    assert np.array_equal(_u8(codes), want)
+
+
+@pytest.mark.parametrize("name", [k for k in _inputs() if k not in ("tiny_tail", "tail_7")])
+def test_fp4_block_bit_exact(name):
+    x = _inputs()[name]
+    n = x.numel()
+    xd = x.cuda()
+    amax = torch.zeros(1, device="cuda")
+    packed = torch.empty(n // 2, dtype=torch.uint8, device="cuda")
+    bscale = torch.empty(n // 16, dtype=torch.uint8, device="cuda")
+    gscale = torch.zeros(1, device="cuda")
+    c8 = torch.empty(n, dtype=torch.uint8, device="cuda")
+    s8 = torch.zeros(1, device="cuda")
+    qa.calibrate_amax(xd, amax)
+    qa.quantize_fp4_block(xd, amax, packed, bscale, gscale, c8, s8)
+    assert qa.get_error() == 0
+    _, a = oracle.amax(x)
+    w_packed, w_bscale, w_sg, w_c8, w_s8 = oracle.quantize_fp4_block(x, a)
+    assert np.float32(gscale.item()) == w_sg
+    assert np.float32(s8.item()) == w_s8
+    assert np.array_equal(_u8(bscale), w_bscale)
+    assert np.array_equal(_u8(packed), w_packed)
+    assert np.array_equal(_u8(c8), w_c8)
+
+
+@pytest.mark.parametrize("wname", ["small_fp8", "gen_fp8", "edit_fp8", "edit_fp4"])
+def test_workload_tensors_bit_exact(wname):
+    """Full-size workload tensors (the shapes the bench times): every code and scale matches."""
+    w = workloads.WORKLOADS[wname]
+    q, k, v = workloads.make_qkv(w)
+    path = qa.QuantizedAttention(w.shape, w.mode, sm_scale=w.sm_scale)
+    path.quantize(q.cuda(), k.cuda(), v.cuda())
+    assert qa.get_error() == 0
+    for i, x in enumerate((q, k, v)):
+        codes, s, extra = oracle.quantize_tensor(x, w.mode)
+        assert float(path.amax[i].item()) == extra["amax"]
+        assert np.float32(path.scale[i].item()) == s
+        assert np.array_equal(_u8(path.codes[i]), codes)
+        if w.mode == "fp4":
+            assert np.array_equal(_u8(path.e2m1[i]), extra["packed"])
+            assert np.array_equal(_u8(path.bscale[i]), extra["bscale"])
+            assert np.float32(path.gscale[i].item()) == extra["sg"]
+
+
+def test_nonfinite_input_is_reported():
+    x = torch.randn(4096).to(torch.bfloat16)
+    x[1234] = float("nan")
+    xd = x.cuda()
+    amax = torch.zeros(1, device="cuda")
+    scale = torch.full((1,), -1.0, device="cuda")
+    codes = torch.full((4096,), 0x55, dtype=torch.uint8, device="cuda")
+    qa.calibrate_amax(xd, amax)
+    qa.quantize_fp8(xd, amax, codes, scale)
+    assert qa.get_error() == qa._lib.ERR_NONFINITE
+    assert scale.item() == -1.0 and int(codes[0].item()) == 0x55     # nothing written
+    assert qa.get_error() == 0                                        # the word was cleared
