@@ -56,6 +56,7 @@ class ClockSampler:
     def __init__(self, gpu_index: int):
         self.gpu = gpu_index
         self.proc = None
+        self.skip = 0
         import tempfile
         fd, self.path = tempfile.mkstemp(prefix="qattn_clocks_", suffix=".csv")
         os.close(fd)
@@ -65,10 +66,16 @@ class ClockSampler:
             self.f = open(self.path, "w")
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "200"], stdout=self.f,
+                 "--format=csv,noheader,nounits", "-lms", "100"], stdout=self.f,
                 stderr=subprocess.DEVNULL)
         except Exception:
             self.proc = None
+            return self
+        deadline = time.time() + 5.0          # the first sample marks the sampler as running
+        while time.time() < deadline and os.path.getsize(self.path) == 0:
+            time.sleep(0.02)
+        with open(self.path) as f:
+            self.skip = len(f.readlines())
         return self
 
     def __exit__(self, *exc):
@@ -85,7 +92,7 @@ class ClockSampler:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
         rows = []
         with open(self.path) as f:
-            for line in f:
+            for line in f.readlines()[self.skip:]:
                 parts = [p.strip() for p in line.split(",")]
                 if len(parts) < 9:
                     continue
@@ -132,7 +139,9 @@ def max_over_ranks(x: float, world: int) -> float:
 def run_gpu(args):
     import precision_quantized_attention_b200 as qa
     rank, world, local = dist_setup(args.gpus)
-    w = workloads.WORKLOADS["edit_fp8" if args.mode == "fp8" else "edit_fp4"]
+    w = workloads.WORKLOADS[args.workload or ("edit_fp8" if args.mode == "fp8" else "edit_fp4")]
+    if w.varlen:
+        raise SystemExit("bench.py times dense workloads; varlen is covered by the parity tests")
     if world > 1:   # each replica gets its own seeded problem
         import dataclasses
         w = dataclasses.replace(w, seed=w.seed + 100 * rank)
@@ -175,7 +184,19 @@ def run_gpu(args):
     attn = max_over_ranks(sum(attn_ms) / len(attn_ms), world)
     quant = max_over_ranks(sum(quant_ms) / len(quant_ms), world)
 
-    # end to end through the C ABI with host buffers (pinned), copies inside the timed region
+    if args.no_e2e:
+        e2e_ms = float("nan")
+    else:
+        e2e_ms = e2e_time(args, w, q, k, v, qd, kd, vd, step, flush, stream, world)
+    report(args, w, q, rank, world, ms, attn, quant, e2e_ms, clocks)
+    barrier(world)
+    del path
+    if world > 1:
+        torch.distributed.destroy_process_group()
+
+
+def e2e_time(args, w, q, k, v, qd, kd, vd, step, flush, stream, world):
+    """Same step through the C ABI with pinned host buffers; copies inside the timed region."""
     qh, kh, vh = (t.pin_memory() for t in (q, k, v))
     oh = torch.empty(w.shape, dtype=torch.bfloat16).pin_memory()
     e2e_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
@@ -194,8 +215,10 @@ def run_gpu(args):
         e2e_ev[i][1].record(stream)
     torch.cuda.synchronize()
     barrier(world)
-    e2e_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in e2e_ev) / args.steps, world)
+    return max_over_ranks(sum(a.elapsed_time(b) for a, b in e2e_ev) / args.steps, world)
 
+
+def report(args, w, q, rank, world, ms, attn, quant, e2e_ms, clocks):
     hbm_gbs, bf16_tf, peak_kind = load_peaks()
     fp8_peak = bf16_tf * FP8_PER_BF16
     flops = w.flops
@@ -216,14 +239,16 @@ def run_gpu(args):
         "vs_baseline": None,
         "dtype": "e4m3",
         "data": "synthetic: seeded N(0,1) bf16 Q/K/V, 4 of 128 Q/K channels per head x10",
-        "config": {"workload": f"{w.name}: B=1 H=24 L=8704 (512 text + 4096 target + 4096 "
-                               f"context) D=128 {w.mode.upper()} full attention",
+        "config": {"workload": f"{w.name}: B={w.B} H={w.H} L={w.L} D={w.D} "
+                               f"{w.mode.upper()} full attention" + (
+                                   " (512 text + 4096 target + 4096 context tokens)"
+                                   if w.L == workloads.L_EDIT else ""),
                    "mode": w.mode, "B": w.B, "H": w.H, "L": w.L, "D": w.D,
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                    "l2": "flushed between steps (256 MiB write outside the timed events)"},
         "roofline": {"bound": "tensor", "achieved": achieved_tf, "peak": fp8_peak,
                      "unit": "TFLOP/s", "frac": achieved_tf / fp8_peak, "traffic": None,
-                     "kernel": "k_attn_fp8_fwd<128>",
+                     "kernel": f"k_attn_fp8_fwd<{w.D}>",
                      "peak_source": f"{peak_kind} bf16 burst {bf16_tf} TFLOP/s x {FP8_PER_BF16} "
                                     "(nominal FP8/BF16 ratio)",
                      "kernel_ms": attn},
@@ -240,10 +265,6 @@ def run_gpu(args):
     if rank == 0:
         result["cpu_baseline"] = cpu_baseline(w) if not args.no_cpu_baseline else None
         print(json.dumps(result), flush=True)
-    barrier(world)
-    del path
-    if world > 1:
-        torch.distributed.destroy_process_group()
 
 
 def cpu_baseline(w, rows_per_head: int = 1024, seed: int = 0):
@@ -302,11 +323,14 @@ def run_reference(args):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
-    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--steps", type=int, default=300)
+    ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--mode", default="fp8", choices=["fp8", "fp4"])
+    ap.add_argument("--workload", default=None, choices=sorted(workloads.WORKLOADS),
+                    help="time another dense workload (default: the L=8704 editing workload)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -75,7 +75,7 @@ def _load():
             lib.orc_quantize_fp4_block.restype = i32
             lib.orc_dequant_fp4_block.argtypes = [P, P, f32, i64, P]
             lib.orc_dequant_fp4_block.restype = None
-            att = [P, P, P, i32, i32, i64, i32, P, i32, f64, f64, f64, f64, i32, P, i64, P]
+            att = [P, P, P, i32, i32, i64, i32, P, i32, f64, f64, f64, f64, i32, P, i64, P, P]
             lib.orc_attention_values.argtypes = att
             lib.orc_attention_values.restype = i32
             lib.orc_attention_e4m3.argtypes = att
@@ -194,15 +194,19 @@ def attention_values(q, k, v, s_q=1.0, s_k=1.0, s_v=1.0, sm_scale=None, flags=ME
     out = np.empty((nrows, D), dtype=np.float64)
     rc = _load().orc_attention_values(_ptr(q), _ptr(k), _ptr(v), B, H, T, D, _ptr(cu),
                                       cu.size - 1, s_q, s_k, s_v, sm, flags,
-                                      None if r is None else _ptr(r), nrows, _ptr(out))
+                                      None if r is None else _ptr(r), nrows, _ptr(out), None)
     if rc != OK:
         raise ValueError(f"orc_attention_values failed with status {rc}")
     return out if r is not None else out.reshape(B, H, T, D)
 
 
 def attention_e4m3(q8, k8, v8, shape, s_q, s_k, s_v, sm_scale=None, flags=METHOD,
-                   cu_seqlens=None, rows=None) -> np.ndarray:
-    """Oracle attention over E4M3 codes (uint8 arrays of B*H*T*D) with per-tensor scales."""
+                   cu_seqlens=None, rows=None, with_ambiguity=False):
+    """Oracle attention over E4M3 codes (uint8 arrays of B*H*T*D) with per-tensor scales.
+
+    with_ambiguity=True also returns, per output, the largest change that choosing the other
+    code of an ambiguous P decision can make (P codes whose FP32 rounding boundary lies within
+    the accumulation-order uncertainty of the score; see the C source)."""
     B, H, T, D = shape
     sm = 1.0 / np.sqrt(D) if sm_scale is None else sm_scale
     q8, k8, v8 = (np.ascontiguousarray(a, dtype=np.uint8).reshape(-1) for a in (q8, k8, v8))
@@ -211,12 +215,17 @@ def attention_e4m3(q8, k8, v8, shape, s_q, s_k, s_v, sm_scale=None, flags=METHOD
     r = None if rows is None else np.ascontiguousarray(np.asarray(rows, dtype=np.int64))
     nrows = B * H * T if r is None else r.size
     out = np.empty((nrows, D), dtype=np.float64)
+    amb = np.empty((nrows, D), dtype=np.float64) if with_ambiguity else None
     rc = _load().orc_attention_e4m3(_ptr(q8), _ptr(k8), _ptr(v8), B, H, T, D, _ptr(cu),
                                     cu.size - 1, float(s_q), float(s_k), float(s_v), sm, flags,
-                                    None if r is None else _ptr(r), nrows, _ptr(out))
+                                    None if r is None else _ptr(r), nrows, _ptr(out),
+                                    _ptr(amb) if with_ambiguity else None)
     if rc != OK:
         raise ValueError(f"orc_attention_e4m3 failed with status {rc}")
-    return out if r is not None else out.reshape(B, H, T, D)
+    if r is None:
+        out = out.reshape(B, H, T, D)
+        amb = amb.reshape(B, H, T, D) if with_ambiguity else None
+    return (out, amb) if with_ambiguity else out
 
 
 def attention_fp64(q, k, v, sm_scale=None, cu_seqlens=None) -> np.ndarray:
@@ -254,10 +263,11 @@ def quantize_tensor(x, mode: str):
 
 
 def method_forward(q, k, v, mode="fp8", sm_scale=None, cu_seqlens=None, rows=None,
-                   flags=METHOD):
+                   flags=METHOD, with_ambiguity=False):
     """The quantized SDPA from bf16 inputs [B, H, T, D] (CPU torch bf16 tensors)."""
     shape = tuple(q.shape)
     q8, sq, _ = quantize_tensor(q, mode)
     k8, sk, _ = quantize_tensor(k, mode)
     v8, sv, _ = quantize_tensor(v, mode)
-    return attention_e4m3(q8, k8, v8, shape, sq, sk, sv, sm_scale, flags, cu_seqlens, rows)
+    return attention_e4m3(q8, k8, v8, shape, sq, sk, sv, sm_scale, flags, cu_seqlens, rows,
+                          with_ambiguity)

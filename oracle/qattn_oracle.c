@@ -231,22 +231,41 @@ void orc_dequant_fp4_block(const uint8_t *packed, const uint8_t *bscale, float s
  * units, so every p lies in (0, 1] and the result does not depend on how keys are tiled.
  *
  * rows: NULL for every row, else nrows row ids r = (b * H + h) * T + t.  out: [nrows, D].
+ * amb (optional, [nrows, D]): per output, the largest change of O that choosing the other code
+ * of an ambiguous P decision (see attend_row) can make, summed over keys.
  * ---------------------------------------------------------------------------------------- */
 #define ORC_FP32 1
 #define ORC_QUANT_P 2
 #define ORC_FIG4_LITERAL 4
 
+/* Ambiguity of a P code (flag ORC_QUANT_P with ORC_FP32, `amb` != NULL).  The blog fixes the
+ * accumulation of BMM1 only as "higher precision"; an FP32 accumulator that rounds in another
+ * order than this oracle's exact sum changes S' by up to about kappa * u * sum_d |q_d k_d| * c
+ * (u = 2^-24, kappa = 16 roundings), the FP32 steps of the softmax add a few ulps of S', and a
+ * hardware exp2 a few ulps of p.  When that interval of S' - M straddles an E4M3 rounding
+ * boundary of p * 448, both codes are correct results of the method; amb[j] records how far the
+ * other code's value lies from this one's (0 when the code is unique). */
+#define ORC_AMB_KAPPA 16.0
+
+static double e4m3_val_of(double p448) {
+    return (double)orc_e4m3_to_float(orc_e4m3_from_float((float)p448));
+}
+
 static void attend_row(const double *q, const double *K, const double *V, int64_t nkeys, int D,
                        double c64, float c32, double s_v, int flags, double *S, double *P,
-                       double *out) {
+                       double *W, double *out, double *amb_out) {
     /* scores */
     double smax = -INFINITY;
     for (int64_t j = 0; j < nkeys; ++j) {
         const double *k = K + j * D;
-        double acc = 0.0;
-        for (int d = 0; d < D; ++d) acc += q[d] * k[d];
+        double acc = 0.0, absacc = 0.0;
+        for (int d = 0; d < D; ++d) {
+            acc += q[d] * k[d];
+            absacc += fabs(q[d] * k[d]);
+        }
         double s = (flags & ORC_FP32) ? (double)(float)((float)acc * c32) : acc * c64;
         S[j] = s;
+        W[j] = absacc;
         if (s > smax) smax = s;
     }
     double M = ceil(smax);
@@ -269,8 +288,19 @@ static void attend_row(const double *q, const double *K, const double *V, int64_
         }
         post = s_v / 448.0;
     } else if (flags & ORC_QUANT_P) {
-        for (int64_t j = 0; j < nkeys; ++j)
-            P[j] = (double)orc_e4m3_to_float(orc_e4m3_from_float((float)P[j] * 448.0f));
+        for (int64_t j = 0; j < nkeys; ++j) {
+            double code_val = (double)orc_e4m3_to_float(orc_e4m3_from_float((float)P[j] * 448.0f));
+            if (amb_out) {
+                double x = S[j] - M;
+                double delta = ORC_AMB_KAPPA * ldexp(W[j] * c64, -24)
+                             + 4.0 * ldexp(fabs(S[j]) + fabs(M) + 1.0, -23) + ldexp(1.0, -20);
+                double lo = e4m3_val_of(exp2(x - delta) * 448.0);
+                double hi = e4m3_val_of(exp2(x + delta) * 448.0);
+                double a = fabs(lo - code_val), b = fabs(hi - code_val);
+                W[j] = a > b ? a : b;     /* W is reused as the ambiguity of code j */
+            }
+            P[j] = code_val;
+        }
         post = s_v / 448.0 / l;
     }
     /* BMM2 */
@@ -281,6 +311,16 @@ static void attend_row(const double *q, const double *K, const double *V, int64_
         for (int d = 0; d < D; ++d) out[d] += p * v[d];
     }
     for (int d = 0; d < D; ++d) out[d] *= post;
+    if (amb_out) {
+        for (int d = 0; d < D; ++d) amb_out[d] = 0.0;
+        if ((flags & ORC_QUANT_P) && !(flags & ORC_FIG4_LITERAL)) {
+            for (int64_t j = 0; j < nkeys; ++j) {
+                if (W[j] == 0.0) continue;
+                const double *v = V + j * D;
+                for (int d = 0; d < D; ++d) amb_out[d] += W[j] * fabs(v[d]) * post;
+            }
+        }
+    }
 }
 
 typedef struct { int64_t row; int64_t slot; } row_ref;
@@ -294,7 +334,7 @@ static int cmp_row_ref(const void *a, const void *b) {
 int orc_attention_values(const double *q, const double *k, const double *v, int B, int H,
                          int64_t T, int D, const int64_t *cu, int nseq, double s_q, double s_k,
                          double s_v, double sm_scale, int flags, const int64_t *rows,
-                         int64_t nrows, double *out) {
+                         int64_t nrows, double *out, double *amb) {
     if (B < 1 || H < 1 || T < 1 || D < 1 || nseq < 1) return ORC_ERR_INVALID;
     if (cu[0] != 0 || cu[nseq] != T) return ORC_ERR_INVALID;
     for (int s = 0; s < nseq; ++s) if (cu[s + 1] <= cu[s]) return ORC_ERR_INVALID;
@@ -323,13 +363,15 @@ int orc_attention_values(const double *q, const double *k, const double *v, int 
         {
             double *S = (double *)malloc(sizeof(double) * (size_t)nkeys);
             double *P = (double *)malloc(sizeof(double) * (size_t)nkeys);
+            double *W = (double *)malloc(sizeof(double) * (size_t)nkeys);
 #pragma omp for schedule(dynamic, 8)
             for (int64_t i = g0; i < g1; ++i) {
-                attend_row(q + refs[i].row * D, Kb, Vb, nkeys, D, c64, c32, s_v, flags, S, P,
-                           out + refs[i].slot * D);
+                attend_row(q + refs[i].row * D, Kb, Vb, nkeys, D, c64, c32, s_v, flags, S, P, W,
+                           out + refs[i].slot * D, amb ? amb + refs[i].slot * D : NULL);
             }
             free(S);
             free(P);
+            free(W);
         }
         g0 = g1;
     }
@@ -341,7 +383,7 @@ int orc_attention_values(const double *q, const double *k, const double *v, int 
 int orc_attention_e4m3(const uint8_t *q8, const uint8_t *k8, const uint8_t *v8, int B, int H,
                        int64_t T, int D, const int64_t *cu, int nseq, double s_q, double s_k,
                        double s_v, double sm_scale, int flags, const int64_t *rows,
-                       int64_t nrows, double *out) {
+                       int64_t nrows, double *out, double *amb) {
     int64_t n = (int64_t)B * H * T * D;
     double tbl[256];
     for (int c = 0; c < 256; ++c) tbl[c] = (double)orc_e4m3_to_float((uint8_t)c);
@@ -356,7 +398,7 @@ int orc_attention_e4m3(const uint8_t *q8, const uint8_t *k8, const uint8_t *v8, 
         v[i] = tbl[v8[i]];
     }
     int rc = orc_attention_values(q, k, v, B, H, T, D, cu, nseq, s_q, s_k, s_v, sm_scale, flags,
-                                  rows, nrows, out);
+                                  rows, nrows, out, amb);
     free(q);
     free(k);
     free(v);

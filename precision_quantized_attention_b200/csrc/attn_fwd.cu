@@ -16,16 +16,22 @@
 //     E4M3 rounding commutes with power-of-two scaling in the normal range, so the result does
 //     not depend on how keys are tiled.
 //
-// Kernel structure (one CTA per SM, persistent over nothing: one CTA per pair of 128-row Q tiles):
-//   warp 8      TMA producer: Q tiles once, then K and V tiles through separate rings.
-//   warp 9      MMA issuer (one thread) and TMEM owner: S_t = Q_t K_j^T for both tiles as
-//               soon as the softmax of tile j-1 has read S_t, then O_t += P_t V_j.
+// Kernel structure: one CTA (one per SM) per pair of 128-row Q tiles of one (sequence, head).
+//   warp 8      TMA producer: both Q tiles once, then K and V tiles through separate rings.
+//   warp 9      MMA issuer (one elected thread) and TMEM owner.  Per KV tile j and Q tile t it
+//               issues O_t += P_t(j) V_j (P read from tensor memory) and right behind it, in the
+//               same in-order tcgen05 stream, S_t = Q_t K_{j+1}^T into the columns P_t(j)
+//               occupied; one commit then tells softmax t that S_t(j+1) is ready and that O_t
+//               holds every P_t V up to tile j.
 //   warps 0-7   two softmax warpgroups, one per Q tile; thread = one query row = one TMEM lane.
-//               Each reads its 128 scores with tcgen05.ld, computes the row max, the exp2 and
-//               the row sum in FP32, converts p*448 to E4M3 and stores the row of P to shared
-//               memory in the 128-byte-swizzled K-major layout BMM2 reads; on a rise of M it
-//               rescales its O row in TMEM by 2^-(rise) first.
-// TMEM: S_0, S_1 (128 FP32 columns each), O_0, O_1 (D columns each).
+//               Each reads its 128 scores with tcgen05.ld, takes the row max (3-input maxima)
+//               and computes p*448 = 2^(S' - M + log2 448) in FP32 (hardware ex2 for most
+//               pairs, a degree-5 polynomial on the FMA pipe for the rest), sums p in packed
+//               f32x2 adds, converts to E4M3 and writes P_t(j) over S_t(j) with tcgen05.st.
+//               On a rise of M it first rescales its O row in TMEM by 2^-(rise).
+//   The two Q tiles alternate on the tensor pipe, so one tile's softmax overlaps the other
+//   tile's MMAs; K/V tiles are read by TMA once per CTA for both Q tiles.
+// TMEM: S_0/P_0, S_1/P_1 (128 FP32 columns each; P uses the first 32), O_0, O_1 (D columns).
 // All waits are bounded (a global-timer limit); on expiry the CTA records a timeout in the
 // library's error word, drains what it issued and exits.
 #include <cuda_runtime.h>
@@ -67,25 +73,23 @@ template <int D>
 struct Smem {
   static constexpr int TILE_Q = BLOCK_M * D;       // bytes (E4M3)
   static constexpr int TILE_KV = BLOCK_N * D;
-  static constexpr int TILE_P = BLOCK_M * BLOCK_N;
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_K = OFF_Q + NQ * TILE_Q;
   static constexpr int OFF_V = OFF_K + KSTAGES * TILE_KV;
-  static constexpr int OFF_P = OFF_V + VSTAGES * TILE_KV;
-  static constexpr int OFF_BAR = OFF_P + NQ * TILE_P;
+  static constexpr int OFF_BAR = OFF_V + VSTAGES * TILE_KV;
   // barriers: q_full, k_full[KS], k_empty[KS], v_full[VS], v_empty[VS], s_full[NQ],
-  // s_free[NQ], p_full[NQ], o_done[NQ], drain
-  static constexpr int NBARS = 1 + 2 * KSTAGES + 2 * VSTAGES + 4 * NQ + 1;
+  // p_full[NQ], o_final[NQ], drain
+  static constexpr int NBARS = 1 + 2 * KSTAGES + 2 * VSTAGES + 3 * NQ + 1;
   static constexpr int OFF_TMEM = OFF_BAR + 8 * NBARS;
   static constexpr int OFF_ABORT = OFF_TMEM + 4;
   static constexpr int BYTES = OFF_ABORT + 4;
   static constexpr int ALLOC = BYTES + 1024;       // slack for 1024-byte alignment
-  static_assert(TILE_Q % 1024 == 0 && TILE_KV % 1024 == 0 && TILE_P % 1024 == 0, "alignment");
+  static_assert(TILE_Q % 1024 == 0 && TILE_KV % 1024 == 0, "alignment");
 };
 
 template <int D>
 struct TmemCols {
-  static constexpr uint32_t S0 = 0;                      // S_t at t * BLOCK_N
+  static constexpr uint32_t S0 = 0;                      // S_t / P_t at t * BLOCK_N
   static constexpr uint32_t O0 = NQ * BLOCK_N;           // O_t at O0 + t * D
   static constexpr uint32_t USED = NQ * BLOCK_N + NQ * D;
   static constexpr uint32_t ALLOC = USED <= 256 ? 256 : 512;
@@ -99,6 +103,85 @@ __device__ __forceinline__ float fast_exp2(float x) {    // MUFU ex2, flush-to-z
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+__device__ __forceinline__ float max3f(float a, float b, float c) {   // sm_100 3-input max
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// (d0, d1) = (a0 * b + c, a1 * b + c) with one packed f32x2 FMA.
+__device__ __forceinline__ void ffma2_bc(float& d0, float& d1, float a0, float a1, float b, float c) {
+  asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %4};\n\tmov.b64 rc, {%5, %5};\n\t"
+      "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d0), "=f"(d1)
+      : "f"(a0), "f"(a1), "f"(b), "f"(c));
+}
+
+// (s0, s1) += (a0, a1) with one packed f32x2 add.
+__device__ __forceinline__ void fadd2_acc(float& s0, float& s1, float a0, float a1) {
+  asm("{\n\t.reg .b64 ra, rs;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rs, {%0, %1};\n\t"
+      "add.f32x2 rs, rs, ra;\n\tmov.b64 {%0, %1}, rs;\n\t}"
+      : "+f"(s0), "+f"(s1)
+      : "f"(a0), "f"(a1));
+}
+
+// 2^x on the FMA pipe for two values at once (packed f32x2), for x <= 9.  x is clamped at -125
+// (2^-125 is far below the smallest E4M3 code of p * 448), split as x = n + f with
+// n = round(x) (by adding and subtracting 1.5 * 2^23) and f in [-1/2, 1/2]; 2^f comes from a
+// degree-5 minimax polynomial (relative error 2.1e-7 in binary32, fitted by
+// csrc/fit_exp2_poly.py) and 2^n is added into the exponent field.
+#ifndef QATTN_POLY_PAIRS_PER_8
+#define QATTN_POLY_PAIRS_PER_8 2       // of every 8 pairs of scores, this many take the polynomial
+#endif
+__device__ __forceinline__ void poly_exp2_x2(float x0, float x1, float& y0, float& y1) {
+  x0 = fmaxf(x0, -125.0f);
+  x1 = fmaxf(x1, -125.0f);
+  float p0, p1, t0, t1;
+  asm("{\n\t.reg .b64 x, t, n, f, p, m, nm, neg1, k;\n\t"
+      "mov.b64 x, {%4, %5};\n\t"
+      "mov.b64 m, {0f4B400000, 0f4B400000};\n\t"       // 1.5 * 2^23
+      "mov.b64 nm, {0fCB400000, 0fCB400000};\n\t"
+      "mov.b64 neg1, {0fBF800000, 0fBF800000};\n\t"
+      "add.rn.f32x2 t, x, m;\n\t"                       // t = n + 1.5 * 2^23, n = round(x)
+      "add.rn.f32x2 n, t, nm;\n\t"                      // n (exact)
+      "fma.rn.f32x2 f, n, neg1, x;\n\t"                 // f = x - n (exact)
+      "mov.b64 p, {0f3AAE0473, 0f3AAE0473};\n\t"        // c5
+      "mov.b64 k, {0f3C1E8629, 0f3C1E8629};\n\t"        // c4
+      "fma.rn.f32x2 p, p, f, k;\n\t"
+      "mov.b64 k, {0f3D635B72, 0f3D635B72};\n\t"        // c3
+      "fma.rn.f32x2 p, p, f, k;\n\t"
+      "mov.b64 k, {0f3E75FC8C, 0f3E75FC8C};\n\t"        // c2
+      "fma.rn.f32x2 p, p, f, k;\n\t"
+      "mov.b64 k, {0f3F317214, 0f3F317214};\n\t"        // c1
+      "fma.rn.f32x2 p, p, f, k;\n\t"
+      "mov.b64 k, {0f3F800001, 0f3F800001};\n\t"        // c0
+      "fma.rn.f32x2 p, p, f, k;\n\t"
+      "mov.b64 {%0, %1}, p;\n\t"
+      "mov.b64 {%2, %3}, t;\n\t}"
+      : "=f"(p0), "=f"(p1), "=f"(t0), "=f"(t1)
+      : "f"(x0), "f"(x1));
+  // the low 9 bits of t hold n (two's complement); shifted into the exponent field they add n
+  y0 = __int_as_float(__float_as_int(p0) + (__float_as_int(t0) << 23));
+  y1 = __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23));
+}
+
+// Row max of 128 scores: 8 independent chains of 3-input maxima, then a short tree.
+__device__ __forceinline__ float rowmax128(const float (&s)[128]) {
+  float m[8];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) m[k] = max3f(s[k], s[k + 8], s[k + 16]);
+#pragma unroll
+  for (int i = 24; i < 120; i += 16) {
+#pragma unroll
+    for (int k = 0; k < 8; ++k) m[k] = max3f(m[k], s[i + k], s[i + 8 + k]);
+  }
+#pragma unroll
+  for (int k = 0; k < 8; ++k) m[k] = fmaxf(m[k], s[120 + k]);
+  return max3f(max3f(m[0], m[1], m[2]), max3f(m[3], m[4], m[5]), fmaxf(m[6], m[7]));
 }
 
 template <int D>
@@ -136,12 +219,11 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
   // ---- barriers --------------------------------------------------------------------------
   const uint32_t bar0 = base_u32 + SL::OFF_BAR;
   auto BAR = [&](int i) { return bar0 + 8u * static_cast<uint32_t>(i); };
-  const int B_QFULL = 0;
-  const int B_KFULL = 1, B_KEMPTY = B_KFULL + KSTAGES;
-  const int B_VFULL = B_KEMPTY + KSTAGES, B_VEMPTY = B_VFULL + VSTAGES;
-  const int B_SFULL = B_VEMPTY + VSTAGES, B_SFREE = B_SFULL + NQ;
-  const int B_PFULL = B_SFREE + NQ, B_ODONE = B_PFULL + NQ;
-  const int B_DRAIN = B_ODONE + NQ;
+  constexpr int B_QFULL = 0;
+  constexpr int B_KFULL = 1, B_KEMPTY = B_KFULL + KSTAGES;
+  constexpr int B_VFULL = B_KEMPTY + KSTAGES, B_VEMPTY = B_VFULL + VSTAGES;
+  constexpr int B_SFULL = B_VEMPTY + VSTAGES, B_PFULL = B_SFULL + NQ;
+  constexpr int B_OFINAL = B_PFULL + NQ, B_DRAIN = B_OFINAL + NQ;
   volatile int* abort_flag = reinterpret_cast<volatile int*>(base + SL::OFF_ABORT);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base + SL::OFF_TMEM);
 
@@ -151,9 +233,8 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
     for (int i = 0; i < VSTAGES; ++i) { mbar_init(BAR(B_VFULL + i), 1); mbar_init(BAR(B_VEMPTY + i), 1); }
     for (int t = 0; t < NQ; ++t) {
       mbar_init(BAR(B_SFULL + t), 1);
-      mbar_init(BAR(B_SFREE + t), BLOCK_M);
       mbar_init(BAR(B_PFULL + t), BLOCK_M);
-      mbar_init(BAR(B_ODONE + t), 1);
+      mbar_init(BAR(B_OFINAL + t), 1);
     }
     mbar_init(BAR(B_DRAIN), 1);
     *abort_flag = 0;
@@ -171,108 +252,114 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
 
   if (warp == WARP_LOAD) {
     // ======================= TMA producer =======================
-    if (lane == 0) {
+    if (lane == 0 && !args.inject_missing_q) {
       tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
-      bool ok = true;
       int nk = 0, nv = 0;                          // loads issued
-      if (!args.inject_missing_q) {
-        mbar_arrive_expect_tx(BAR(B_QFULL), NQ * SL::TILE_Q);
-        for (int t = 0; t < NQ; ++t)
-          tma_load_3d(base_u32 + SL::OFF_Q + t * SL::TILE_Q, &tm_q, BAR(B_QFULL), 0,
-                      seq_start + q_row0 + t * BLOCK_M, slab);
-        auto load_k = [&](int j) -> bool {
-          const int s = j % KSTAGES;
-          if (j >= KSTAGES &&
-              !mbar_wait(BAR(B_KEMPTY + s), ((j / KSTAGES) - 1) & 1, tlim, abort_flag, args.err))
-            return false;
-          mbar_arrive_expect_tx(BAR(B_KFULL + s), SL::TILE_KV);
-          tma_load_3d(base_u32 + SL::OFF_K + s * SL::TILE_KV, &tm_k, BAR(B_KFULL + s), 0,
-                      seq_start + j * BLOCK_N, slab);
-          ++nk;
-          return true;
-        };
-        auto load_v = [&](int j) -> bool {
-          const int s = j % VSTAGES;
-          if (j >= VSTAGES &&
-              !mbar_wait(BAR(B_VEMPTY + s), ((j / VSTAGES) - 1) & 1, tlim, abort_flag, args.err))
-            return false;
-          mbar_arrive_expect_tx(BAR(B_VFULL + s), SL::TILE_KV);
-          tma_load_3d(base_u32 + SL::OFF_V + s * SL::TILE_KV, &tm_v, BAR(B_VFULL + s), 0,
-                      seq_start + j * BLOCK_N, slab);
-          ++nv;
-          return true;
-        };
-        ok = load_k(0);
-        for (int j = 0; ok && j < nkv; ++j) {
-          if (j + 1 < nkv) ok = load_k(j + 1);
-          if (ok) ok = load_v(j);
-        }
-        // drain: every issued load has landed before the CTA may exit (instant when healthy)
-        mbar_drain(BAR(B_QFULL), 0, tlim);
-        for (int j = nk - 1; j >= 0 && j >= nk - KSTAGES; --j)
-          mbar_drain(BAR(B_KFULL + j % KSTAGES), (j / KSTAGES) & 1, tlim);
-        for (int j = nv - 1; j >= 0 && j >= nv - VSTAGES; --j)
-          mbar_drain(BAR(B_VFULL + j % VSTAGES), (j / VSTAGES) & 1, tlim);
+      mbar_arrive_expect_tx(BAR(B_QFULL), NQ * SL::TILE_Q);
+      for (int t = 0; t < NQ; ++t)
+        tma_load_3d(base_u32 + SL::OFF_Q + t * SL::TILE_Q, &tm_q, BAR(B_QFULL), 0,
+                    seq_start + q_row0 + t * BLOCK_M, slab);
+      auto load_k = [&](int j) -> bool {
+        const int s = j % KSTAGES;
+        if (j >= KSTAGES &&
+            !mbar_wait(BAR(B_KEMPTY + s), ((j / KSTAGES) - 1) & 1, tlim, abort_flag, args.err))
+          return false;
+        mbar_arrive_expect_tx(BAR(B_KFULL + s), SL::TILE_KV);
+        tma_load_3d(base_u32 + SL::OFF_K + s * SL::TILE_KV, &tm_k, BAR(B_KFULL + s), 0,
+                    seq_start + j * BLOCK_N, slab);
+        ++nk;
+        return true;
+      };
+      auto load_v = [&](int j) -> bool {
+        const int s = j % VSTAGES;
+        if (j >= VSTAGES &&
+            !mbar_wait(BAR(B_VEMPTY + s), ((j / VSTAGES) - 1) & 1, tlim, abort_flag, args.err))
+          return false;
+        mbar_arrive_expect_tx(BAR(B_VFULL + s), SL::TILE_KV);
+        tma_load_3d(base_u32 + SL::OFF_V + s * SL::TILE_KV, &tm_v, BAR(B_VFULL + s), 0,
+                    seq_start + j * BLOCK_N, slab);
+        ++nv;
+        return true;
+      };
+      // order of use on the tensor pipe: K0, V0, K1, V1, ...; K runs one tile ahead
+      bool ok = load_k(0);
+      for (int j = 0; ok && j < nkv; ++j) {
+        if (j + 1 < nkv) ok = load_k(j + 1);
+        if (ok) ok = load_v(j);
       }
-      (void)ok;
+      // drain: every issued load has landed before the CTA may exit (instant when healthy)
+      mbar_drain(BAR(B_QFULL), 0, tlim);
+      for (int j = nk - 1; j >= 0 && j >= nk - KSTAGES; --j)
+        mbar_drain(BAR(B_KFULL + j % KSTAGES), (j / KSTAGES) & 1, tlim);
+      for (int j = nv - 1; j >= 0 && j >= nv - VSTAGES; --j)
+        mbar_drain(BAR(B_VFULL + j % VSTAGES), (j / VSTAGES) & 1, tlim);
     }
   } else if (warp == WARP_MMA) {
     // ======================= MMA issuer =======================
     if (lane == 0) {
       constexpr uint32_t IDESC_S = idesc_e4m3_f32(BLOCK_M, BLOCK_N, false);
       constexpr uint32_t IDESC_O = idesc_e4m3_f32(BLOCK_M, D, true);
-      // Q, K: K-major rows of D bytes, swizzled in 8-row atoms (SBO = 8 rows).
+      // Q, K: K-major rows of D bytes, swizzled in 8-row atoms (SBO = 8 rows); 32-byte K steps.
       constexpr uint32_t QK_LAYOUT = (D == 128) ? 2u : 4u;   // 128B / 64B swizzle
       constexpr uint32_t QK_SBO = 8 * D;
-      // P: K-major rows of 128 bytes (128 keys), 128B swizzle.
-      // V: MN-major (D contiguous per key row), rows of D bytes, SBO = 8 key rows.
+      // V: MN-major (D contiguous per key row), rows of D bytes, SBO = 8 key rows; a K step
+      // of 32 keys advances 32 rows.
       constexpr uint32_t V_LAYOUT = QK_LAYOUT;
       constexpr uint32_t V_SBO = 8 * D;
-      bool ok = mbar_wait(BAR(B_QFULL), 0, tlim, abort_flag, args.err);
-      auto bmm1 = [&](int j) -> bool {
-        const int s = j % KSTAGES;
-        if (!mbar_wait(BAR(B_KFULL + s), (j / KSTAGES) & 1, tlim, abort_flag, args.err))
-          return false;
-        for (int t = 0; t < NQ; ++t) {
-          if (j > 0 && !mbar_wait(BAR(B_SFREE + t), (j - 1) & 1, tlim, abort_flag, args.err))
-            return false;
-          tc_fence_after();
-          const uint32_t qa = base_u32 + SL::OFF_Q + t * SL::TILE_Q;
-          const uint32_t kb = base_u32 + SL::OFF_K + s * SL::TILE_KV;
+      auto bmm1 = [&](int t, int ks) {
+        const uint32_t qa = base_u32 + SL::OFF_Q + t * SL::TILE_Q;
+        const uint32_t kb = base_u32 + SL::OFF_K + ks * SL::TILE_KV;
 #pragma unroll
-          for (int kk = 0; kk < D / 32; ++kk) {
-            const uint64_t da = smem_desc(qa + kk * 32, 16, QK_SBO, QK_LAYOUT);
-            const uint64_t db = smem_desc(kb + kk * 32, 16, QK_SBO, QK_LAYOUT);
-            mma_f8_ss(tmem + TC::S0 + t * BLOCK_N, da, db, IDESC_S, kk > 0 ? 1u : 0u);
-          }
+        for (int kk = 0; kk < D / 32; ++kk) {
+          const uint64_t da = smem_desc(qa + kk * 32, 16, QK_SBO, QK_LAYOUT);
+          const uint64_t db = smem_desc(kb + kk * 32, 16, QK_SBO, QK_LAYOUT);
+          mma_f8_ss(tmem + TC::S0 + t * BLOCK_N, da, db, IDESC_S, kk > 0 ? 1u : 0u);
+        }
+      };
+      auto bmm2 = [&](int t, int vs, bool first) {
+        const uint32_t vb = base_u32 + SL::OFF_V + vs * SL::TILE_KV;
+#pragma unroll
+        for (int kk = 0; kk < BLOCK_N / 32; ++kk) {
+          const uint64_t db = smem_desc(vb + kk * 32 * D, SL::TILE_KV, V_SBO, V_LAYOUT);
+          mma_f8_ts(tmem + TC::O0 + t * D, tmem + TC::S0 + t * BLOCK_N + kk * 8, db, IDESC_O,
+                    (!first || kk > 0) ? 1u : 0u);
+        }
+      };
+      bool ok = mbar_wait(BAR(B_QFULL), 0, tlim, abort_flag, args.err) &&
+                mbar_wait(BAR(B_KFULL + 0), 0, tlim, abort_flag, args.err);
+      if (ok) {
+        tc_fence_after();
+        for (int t = 0; t < NQ; ++t) {
+          bmm1(t, 0);
           mma_commit(BAR(B_SFULL + t));
         }
-        mma_commit(BAR(B_KEMPTY + s));
-        return true;
-      };
-      if (ok) ok = bmm1(0);
+        mma_commit(BAR(B_KEMPTY + 0));
+      }
       for (int j = 0; ok && j < nkv; ++j) {
-        if (j + 1 < nkv) ok = bmm1(j + 1);
-        if (!ok) break;
-        const int s = j % VSTAGES;
-        ok = mbar_wait(BAR(B_VFULL + s), (j / VSTAGES) & 1, tlim, abort_flag, args.err);
+        const int vs = j % VSTAGES;
+        const bool more = j + 1 < nkv;
+        const int ks = (j + 1) % KSTAGES;
+        ok = mbar_wait(BAR(B_VFULL + vs), (j / VSTAGES) & 1, tlim, abort_flag, args.err);
+        if (ok && more)
+          ok = mbar_wait(BAR(B_KFULL + ks), ((j + 1) / KSTAGES) & 1, tlim, abort_flag, args.err);
         for (int t = 0; ok && t < NQ; ++t) {
           ok = mbar_wait(BAR(B_PFULL + t), j & 1, tlim, abort_flag, args.err);
           if (!ok) break;
           tc_fence_after();
-          const uint32_t pa = base_u32 + SL::OFF_P + t * SL::TILE_P;
-          const uint32_t vb = base_u32 + SL::OFF_V + s * SL::TILE_KV;
-#pragma unroll
-          for (int kk = 0; kk < BLOCK_N / 32; ++kk) {
-            const uint64_t da = smem_desc(pa + kk * 32, 16, 1024, 2u);
-            const uint64_t db = smem_desc(vb + kk * 32 * D, SL::TILE_KV, V_SBO, V_LAYOUT);
-            mma_f8_ss(tmem + TC::O0 + t * D, da, db, IDESC_O, (j > 0 || kk > 0) ? 1u : 0u);
+          bmm2(t, vs, j == 0);                     // reads P_t(j) from TMEM
+          if (more) {
+            bmm1(t, ks);                           // overwrites S_t / P_t after bmm2 read it
+            mma_commit(BAR(B_SFULL + t));
+          } else {
+            mma_commit(BAR(B_OFINAL + t));
           }
-          mma_commit(BAR(B_ODONE + t));
         }
-        if (ok) mma_commit(BAR(B_VEMPTY + s));
+        if (ok) {
+          mma_commit(BAR(B_VEMPTY + vs));
+          if (more) mma_commit(BAR(B_KEMPTY + ks));
+        }
       }
       // drain: all issued MMAs complete before TMEM is released
       mma_commit(BAR(B_DRAIN));
@@ -286,53 +373,57 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
     const uint32_t tS = tmem + lane_off + TC::S0 + t * BLOCK_N;
     const uint32_t tO = tmem + lane_off + TC::O0 + t * D;
-    uint8_t* prow = base + SL::OFF_P + t * SL::TILE_P + r * BLOCK_N;
     const float c = __ldg(args.s_q) * __ldg(args.s_k) * args.sm_scale * LOG2E_F;
     float m_run = -INFINITY;                       // integer-valued running max (base 2)
     float l = 0.0f;                                // running sum of p * 448
     bool ok = true;
     for (int j = 0; j < nkv; ++j) {
+      // S_t(j) is in TMEM; BMM2 of tile j-1 has completed (it precedes in the MMA stream)
       ok = mbar_wait(BAR(B_SFULL + t), j & 1, tlim, abort_flag, args.err);
       if (!__all_sync(0xFFFFFFFFu, ok)) { ok = false; break; }
       tc_fence_after();
       float s[BLOCK_N];
+      {
+        uint32_t sv[BLOCK_N / 32][32];
 #pragma unroll
-      for (int c4 = 0; c4 < BLOCK_N / 32; ++c4) {
-        uint32_t v[32];
-        tmem_ld32(tS + c4 * 32, v);
+        for (int c4 = 0; c4 < BLOCK_N / 32; ++c4) tmem_ld32(tS + c4 * 32, sv[c4]);
         tmem_wait_ld();
 #pragma unroll
-        for (int i = 0; i < 32; ++i) s[c4 * 32 + i] = __uint_as_float(v[i]);
+        for (int i = 0; i < BLOCK_N; ++i) s[i] = __uint_as_float(sv[i / 32][i % 32]);
       }
-      tc_fence_before();
-      mbar_arrive(BAR(B_SFREE + t));               // S_t may now be overwritten
       const int kv_valid = seq_len - j * BLOCK_N;  // keys of this tile inside the sequence
       if (kv_valid < BLOCK_N) {
 #pragma unroll
         for (int i = 0; i < BLOCK_N; ++i)
           if (i >= kv_valid) s[i] = -INFINITY;
       }
-      float mx = s[0];
-#pragma unroll
-      for (int i = 1; i < BLOCK_N; ++i) mx = fmaxf(mx, s[i]);
-      const float m_new = fmaxf(m_run, ceilf(mx * c));
+      const float m_new = fmaxf(m_run, ceilf(rowmax128(s) * c));
       const float neg_off = LOG2_448 - m_new;
-      float rowsum = 0.0f;
+      float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
       uint32_t pk[BLOCK_N / 4];
 #pragma unroll
-      for (int i = 0; i < BLOCK_N; i += 4) {
-        const float p0 = fast_exp2(fmaf(s[i + 0], c, neg_off));
-        const float p1 = fast_exp2(fmaf(s[i + 1], c, neg_off));
-        const float p2 = fast_exp2(fmaf(s[i + 2], c, neg_off));
-        const float p3 = fast_exp2(fmaf(s[i + 3], c, neg_off));
-        rowsum += (p0 + p1) + (p2 + p3);
-        pk[i / 4] = cvt_e4m3x2(p0, p1) | (cvt_e4m3x2(p2, p3) << 16);
+      for (int i = 0; i < BLOCK_N; i += 16) {
+        float p[16];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          float x0, x1;
+          ffma2_bc(x0, x1, s[i + 2 * q], s[i + 2 * q + 1], c, neg_off);
+          if (q < QATTN_POLY_PAIRS_PER_8) {
+            poly_exp2_x2(x0, x1, p[2 * q], p[2 * q + 1]);
+          } else {
+            p[2 * q] = fast_exp2(x0);
+            p[2 * q + 1] = fast_exp2(x1);
+          }
+        }
+#pragma unroll
+        for (int q = 0; q < 8; ++q) fadd2_acc(acc[2 * (q & 3)], acc[2 * (q & 3) + 1], p[2 * q], p[2 * q + 1]);
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          pk[i / 4 + q] = cvt_e4m3x2(p[4 * q], p[4 * q + 1]) | (cvt_e4m3x2(p[4 * q + 2], p[4 * q + 3]) << 16);
       }
-      // BMM2 of the previous tile must be done: it reads the P buffer and accumulates O.
+      const float rowsum = ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
+      // A rise of the running max rescales this row of O (quiescent: its last BMM2 is done).
       if (j > 0) {
-        ok = mbar_wait(BAR(B_ODONE + t), (j - 1) & 1, tlim, abort_flag, args.err);
-        if (!__all_sync(0xFFFFFFFFu, ok)) { ok = false; break; }
-        tc_fence_after();
         const bool rise = m_new > m_run;
         if (__any_sync(0xFFFFFFFFu, rise)) {
           const float f = rise ? exp2_int(static_cast<int>(m_run - m_new)) : 1.0f;
@@ -345,24 +436,19 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
             for (int i = 0; i < 32; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) * f);
             tmem_st32(tO + c4 * 32, v);
           }
-          tmem_wait_st();
           l *= f;
         }
       }
       l += rowsum;
       m_run = m_new;
-      // row r of P: 8 chunks of 16 bytes, chunk index XOR (r mod 8) (128-byte swizzle)
-#pragma unroll
-      for (int ch = 0; ch < BLOCK_N / 16; ++ch) {
-        uint4* dst = reinterpret_cast<uint4*>(prow + ((ch ^ (r & 7)) << 4));
-        *dst = make_uint4(pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]);
-      }
-      fence_proxy_async_smem();
+      // P_t(j) over the first 32 columns of S_t: column c holds keys 4c..4c+3 (byte = key % 4)
+      tmem_st32(tS, pk);
+      tmem_wait_st();
       tc_fence_before();
       mbar_arrive(BAR(B_PFULL + t));
     }
     if (ok) {
-      ok = mbar_wait(BAR(B_ODONE + t), (nkv - 1) & 1, tlim, abort_flag, args.err);
+      ok = mbar_wait(BAR(B_OFINAL + t), 0, tlim, abort_flag, args.err);
       if (__all_sync(0xFFFFFFFFu, ok)) {
         tc_fence_after();
         const int row = q_row0 + t * BLOCK_M + r;

@@ -2,7 +2,7 @@
 #include <cuda_runtime.h>
 #include <cstdint>
 
-#include "../../include/qattn.h"
+#include "qattn.h"
 #include "sm100_ptx.cuh"
 
 namespace qattn {

@@ -25,9 +25,9 @@ def gpu_path(w: workloads.Workload, q, k, v):
     return qa_
 
 
-def oracle_path(w: workloads.Workload, q, k, v, rows=None):
+def oracle_path(w: workloads.Workload, q, k, v, rows=None, with_ambiguity=False):
     return oracle.method_forward(q, k, v, w.mode, sm_scale=w.sm_scale, cu_seqlens=w.cu_seqlens,
-                                 rows=rows)
+                                 rows=rows, with_ambiguity=with_ambiguity)
 
 
 def compare(gpu_out: np.ndarray, want: np.ndarray):
@@ -37,7 +37,16 @@ def compare(gpu_out: np.ndarray, want: np.ndarray):
     return rel, mx
 
 
-def assert_close(gpu_out, want, what=""):
+def assert_close(gpu_out, want, what="", amb=None):
+    """rel-L2 <= 1e-2 over everything; |diff| <= 3e-2 per output, beyond the oracle's
+    ambiguity bound `amb` when given (outputs whose P codes the method leaves undecided at
+    FP32 accumulation precision may move by that much, see oracle.attention_e4m3)."""
     rel, mx = compare(gpu_out, want)
-    assert rel <= REL_L2_TOL and mx <= MAX_ABS_TOL, f"{what}: rel-L2 {rel:.3e}, max-abs {mx:.3e}"
+    assert rel <= REL_L2_TOL, f"{what}: rel-L2 {rel:.3e}"
+    if amb is None:
+        assert mx <= MAX_ABS_TOL, f"{what}: max-abs {mx:.3e}"
+    else:
+        excess = np.abs(gpu_out.astype(np.float64) - want) - amb
+        worst = float(excess.max()) if excess.size else 0.0
+        assert worst <= MAX_ABS_TOL, f"{what}: max-abs beyond ambiguity {worst:.3e} (raw {mx:.3e})"
     return rel, mx

@@ -173,3 +173,64 @@ def test_invalid_arguments():
         oracle.attention_values(q, q, q, cu_seqlens=[0, 3])          # does not end at T
     with pytest.raises(ValueError):
         oracle.attention_values(q, q, q, cu_seqlens=[0, 2, 2, 4])    # empty sequence
+
+
+def _method_fp32_accumulation(q8, k8, v8, shape, sq, sk, sv, sm, order):
+    """The method with BMM1 accumulated in binary32 in a given order of the D terms (what a
+    tensor core with an FP32 accumulator may do), the rest as the oracle: used to check that
+    the oracle's ambiguity bound covers accumulation-order effects."""
+    import ml_dtypes
+    B, H, T, D = shape
+    val = lambda c: c.reshape(shape).view(ml_dtypes.float8_e4m3fn).astype(np.float32)
+    q, k, v = val(q8), val(k8), val(v8)
+    c32 = np.float32(float(sq) * float(sk) * sm * 1.4426950408889634)
+    out = np.empty(shape)
+    for b in range(B):
+        for h in range(H):
+            acc = np.zeros((T, T), dtype=np.float32)
+            for d in order:
+                acc = (acc + np.outer(q[b, h, :, d], k[b, h, :, d]).astype(np.float32)).astype(np.float32)
+            s = (acc * c32).astype(np.float32)
+            m = np.ceil(s.max(axis=1, keepdims=True).astype(np.float64))
+            p = np.exp2((s - m).astype(np.float32).astype(np.float64)).astype(np.float32)
+            l = p.astype(np.float64).sum(axis=1, keepdims=True).astype(np.float32)
+            p8 = (p * np.float32(448)).astype(np.float32)
+            p8 = np.clip(p8, 0, 448).astype(ml_dtypes.float8_e4m3fn).astype(np.float64)
+            out[b, h] = (p8 @ v[b, h].astype(np.float64)) * float(sv) / 448.0 / l.astype(np.float64)
+    return out
+
+
+def test_ambiguity_bound_covers_fp32_accumulation_orders():
+    """Outputs of the method with BMM1 accumulated in FP32 in several term orders stay within
+    the oracle's ambiguity bound (plus bf16-free float noise); the outlier structure makes rows
+    peaked, which is where ambiguous P codes matter."""
+    w = workloads.custom("amb", "fp8", 1, 2, 96, 64, seed=31, outliers=4)
+    q, k, v = workloads.make_qkv(w)
+    q8, sq, _ = oracle.quantize_tensor(q, "fp8")
+    k8, sk, _ = oracle.quantize_tensor(k, "fp8")
+    v8, sv, _ = oracle.quantize_tensor(v, "fp8")
+    want, amb = oracle.attention_e4m3(q8, k8, v8, w.shape, sq, sk, sv, w.sm_scale,
+                                      with_ambiguity=True)
+    assert amb.shape == want.shape and np.all(amb >= 0)
+    rng = np.random.default_rng(0)
+    worst, flips = 0.0, 0
+    for order in (range(64), range(63, -1, -1), rng.permutation(64), rng.permutation(64)):
+        got = _method_fp32_accumulation(q8, k8, v8, w.shape, sq, sk, sv, w.sm_scale, list(order))
+        # beyond the bound only FP32 noise of the unquantized row sum is left (~1e-5 relative
+        # for scores of magnitude ~60 in base-2 units)
+        excess = np.abs(got - want) - amb - 1e-4 * np.abs(want)
+        worst = max(worst, float(excess.max()))
+        flips += int(np.sum(np.abs(got - want) > 1e-3))
+    assert worst <= 1e-6
+    assert np.max(amb) > 0          # the peaked rows do contain undecided P codes
+
+
+def test_ambiguity_is_zero_without_p_quantization_and_small_otherwise():
+    w = workloads.custom("amb2", "fp8", 1, 2, 128, 64, seed=32)
+    q, k, v = workloads.make_qkv(w)
+    out, amb = oracle.method_forward(q, k, v, "fp8", with_ambiguity=True)
+    assert np.mean(amb) < 1e-3 * np.mean(np.abs(out))
+    q8, sq, _ = oracle.quantize_tensor(q, "fp8")
+    _, amb0 = oracle.attention_e4m3(q8, q8, q8, w.shape, sq, sq, sq, flags=oracle.FP32,
+                                    with_ambiguity=True)
+    assert np.all(amb0 == 0)
