@@ -7,9 +7,9 @@
 // to max-calibration of the tensor in hand.
 //
 // Every kernel streams its input once with 16-byte loads over a grid sized to the SM count,
-// and applies scales with correctly rounded binary32 division, so the codes are bit-identical
-// to the definition (E4M3 / E2M1 round-to-nearest-even with saturation, the hardware cvt
-// forms).
+// and applies scales as correctly rounded binary32 quotients (Markstein's multiply-and-correct
+// form for a shared divisor), so the codes are bit-identical to the definition (E4M3 / E2M1
+// round-to-nearest-even with saturation, the hardware cvt forms).
 #include <cuda_runtime.h>
 #include <cstdint>
 
@@ -69,14 +69,41 @@ __global__ void __launch_bounds__(256) k_amax_bf16(const uint4* __restrict__ xv,
 }
 
 // -------------------------------------------------------------------------------------------
+// Correctly rounded x / s for a divisor shared by many elements (Markstein's theorem: with
+// r = RN(1/s) and q0 = RN(x * r), which is within one ulp of x / s, the residual
+// x - q0 * s is exact in one FMA and RN(q0 + residual * r) = RN(x / s)).  Three FMA-pipe
+// instructions instead of a division; valid while s, r and the residual stay normal, which
+// `markstein_ok` checks once per divisor (callers use __fdiv_rn otherwise).  Quotients so small
+// that they leave the normal range map to a signed zero E4M3/E2M1 code either way.
+// -------------------------------------------------------------------------------------------
+__device__ __forceinline__ bool markstein_ok(float s) {
+  const float a = fabsf(s);
+  return a >= 0x1p-100f && a <= 0x1p+100f;
+}
+
+// s > 0, so RN(x / s) has the sign of x; copysign restores it where the correction step's
+// sum of zeros would not (x = -0, or a quotient that underflows).
+__device__ __forceinline__ float div_rn_by(float x, float s, float r) {
+  const float q0 = __fmul_rn(x, r);
+  const float e = __fmaf_rn(-q0, s, x);
+  return copysignf(__fmaf_rn(e, r, q0), x);
+}
+
+// -------------------------------------------------------------------------------------------
 // Per-tensor FP8: s = fl32(amax / 448), code = e4m3(fl32(x / s)); amax == 0 gives s = 1.
 // -------------------------------------------------------------------------------------------
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
-__device__ __forceinline__ uint32_t quant4_e4m3(uint32_t w0, uint32_t w1, float s) {
-  const uint32_t lo = cvt_e4m3x2(__fdiv_rn(bf16_lo(w0), s), __fdiv_rn(bf16_hi(w0), s));
-  const uint32_t hi = cvt_e4m3x2(__fdiv_rn(bf16_lo(w1), s), __fdiv_rn(bf16_hi(w1), s));
+template <bool FAST>
+__device__ __forceinline__ float div_s(float x, float s, float r) {
+  return FAST ? div_rn_by(x, s, r) : __fdiv_rn(x, s);
+}
+
+template <bool FAST>
+__device__ __forceinline__ uint32_t quant4_e4m3(uint32_t w0, uint32_t w1, float s, float r) {
+  const uint32_t lo = cvt_e4m3x2(div_s<FAST>(bf16_lo(w0), s, r), div_s<FAST>(bf16_hi(w0), s, r));
+  const uint32_t hi = cvt_e4m3x2(div_s<FAST>(bf16_lo(w1), s, r), div_s<FAST>(bf16_hi(w1), s, r));
   return lo | (hi << 16);
 }
 
@@ -94,14 +121,19 @@ __global__ void __launch_bounds__(256) k_quant_fp8(const uint4* __restrict__ xv,
   }
   const float s = (amax == 0.0f) ? 1.0f : __fdiv_rn(amax, 448.0f);
   if (blockIdx.x == 0 && threadIdx.x == 0) *scale_out = s;
+  const float r = __frcp_rn(s);
   const size_t stride = static_cast<size_t>(gridDim.x) * blockDim.x;
-  for (size_t i = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < nvec;
-       i += stride) {
-    const uint4 a = __ldcs(xv + i);
-    uint2 o;
-    o.x = quant4_e4m3(a.x, a.y, s);
-    o.y = quant4_e4m3(a.z, a.w, s);
-    __stcs(outv + i, o);
+  const size_t i0 = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (markstein_ok(s)) {
+    for (size_t i = i0; i < nvec; i += stride) {
+      const uint4 a = __ldcs(xv + i);
+      __stcs(outv + i, make_uint2(quant4_e4m3<true>(a.x, a.y, s, r), quant4_e4m3<true>(a.z, a.w, s, r)));
+    }
+  } else {
+    for (size_t i = i0; i < nvec; i += stride) {
+      const uint4 a = __ldcs(xv + i);
+      __stcs(outv + i, make_uint2(quant4_e4m3<false>(a.x, a.y, s, r), quant4_e4m3<false>(a.z, a.w, s, r)));
+    }
   }
   if (blockIdx.x == 0 && static_cast<int>(threadIdx.x) < ntail) {
     const float x = __uint_as_float(static_cast<uint32_t>(xtail[threadIdx.x]) << 16);
@@ -138,6 +170,8 @@ __global__ void __launch_bounds__(256) k_quant_fp4_block(
     *gscale_out = sg;
     if (scale8_out) *scale8_out = s8;
   }
+  const float r8 = __frcp_rn(s8);
+  const bool fast8 = markstein_ok(s8);
   const size_t stride = static_cast<size_t>(gridDim.x) * blockDim.x;
   for (size_t b = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; b < nblocks;
        b += stride) {
@@ -160,9 +194,13 @@ __global__ void __launch_bounds__(256) k_quant_fp4_block(
     uint32_t c8[4] = {0u, 0u, 0u, 0u};
     if (eff != 0.0f) {
       uint32_t nib[16];
+      const float r_eff = __frcp_rn(eff);
+      const bool fast_eff = markstein_ok(eff);
 #pragma unroll
       for (int i = 0; i < 16; i += 2) {
-        const uint32_t byte = cvt_e2m1x2(__fdiv_rn(x[i], eff), __fdiv_rn(x[i + 1], eff));
+        const float q0 = fast_eff ? div_rn_by(x[i], eff, r_eff) : __fdiv_rn(x[i], eff);
+        const float q1 = fast_eff ? div_rn_by(x[i + 1], eff, r_eff) : __fdiv_rn(x[i + 1], eff);
+        const uint32_t byte = cvt_e2m1x2(q0, q1);
         nib[i] = byte & 0xFu;
         nib[i + 1] = byte >> 4;
         if (i < 8) pk0 |= byte << (4 * i);
@@ -172,7 +210,9 @@ __global__ void __launch_bounds__(256) k_quant_fp4_block(
       for (int i = 0; i < 16; i += 2) {
         const float xh0 = __fmul_rn(__fmul_rn(e2m1_to_f32(nib[i]), sbv), sg);
         const float xh1 = __fmul_rn(__fmul_rn(e2m1_to_f32(nib[i + 1]), sbv), sg);
-        const uint32_t pair = cvt_e4m3x2(__fdiv_rn(xh0, s8), __fdiv_rn(xh1, s8));
+        const float d0 = fast8 ? div_rn_by(xh0, s8, r8) : __fdiv_rn(xh0, s8);
+        const float d1 = fast8 ? div_rn_by(xh1, s8, r8) : __fdiv_rn(xh1, s8);
+        const uint32_t pair = cvt_e4m3x2(d0, d1);
         c8[i / 4] |= pair << (16 * ((i / 2) & 1));
       }
     }

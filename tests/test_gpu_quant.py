@@ -28,6 +28,11 @@ def _inputs():
     x[:16] *= 1e-6          # a block whose E4M3 scale underflows
     x[100] = -0.0
     cases["mixed_blocks"] = x
+    # scales outside [2^-100, 2^100] take the division path, inside the multiply-and-correct one
+    cases["scale_tiny"] = torch.randn(16 * 2048, generator=g) * 1e-35
+    cases["scale_huge"] = torch.randn(16 * 2048, generator=g) * 1e33
+    cases["scale_large_fast"] = torch.randn(16 * 2048, generator=g) * 1e29
+    cases["uniform_grid"] = (torch.arange(16 * 4096, dtype=torch.float32) - 32768.0) / 97.0
     return {k: v.to(torch.bfloat16) for k, v in cases.items()}
 
 
