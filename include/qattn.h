@@ -101,6 +101,32 @@ QATTN_API qattn_status qattn_quantize_fp4_block(const void* x_bf16, size_t n, co
                                       float* gscale_dev, uint8_t* out_e4m3_requant,
                                       float* scale8_dev, qattn_stream_t stream);
 
+/* Bytes of device workspace the fused calibrate+quantize calls need (16-byte aligned). */
+#define QATTN_FUSED_WORKSPACE_BYTES 256
+
+/* Fused calibration + per-tensor FP8 FakeQuantize: the result of qattn_calibrate_amax followed by
+ * qattn_quantize_fp8 (same definitions, same codes), computed by one cooperative kernel that
+ * reads x from HBM once (the second pass reads it back from L2).  amax_dev receives the amax,
+ * scale_dev the dequantization multiplier s.  workspace_dev: caller-owned device scratch of at
+ * least QATTN_FUSED_WORKSPACE_BYTES bytes, 16-byte aligned, ZERO-FILLED before its first use;
+ * every call that completes leaves it zero-filled again (after a call reported
+ * QATTN_ERR_TIMEOUT, zero it again).  Calls that share a workspace must not overlap on the
+ * device (stream order is enough; concurrent streams race).  n >= 1, x_bf16 16-byte aligned,
+ * out_e4m3 8-byte aligned.  Non-finite input: QATTN_ERR_NONFINITE recorded, amax written, codes
+ * and scale not written. */
+QATTN_API qattn_status qattn_calibrate_quantize_fp8(const void* x_bf16, size_t n, float* amax_dev,
+                                                    uint8_t* out_e4m3, float* scale_dev,
+                                                    void* workspace_dev, size_t workspace_bytes,
+                                                    qattn_stream_t stream);
+
+/* Fused calibration + per-block FP4 FakeQuantize with the FP8 requant (the result of
+ * qattn_calibrate_amax followed by qattn_quantize_fp4_block), one cooperative kernel; workspace
+ * rules as for qattn_calibrate_quantize_fp8.  n % 16 == 0. */
+QATTN_API qattn_status qattn_calibrate_quantize_fp4_block(
+    const void* x_bf16, size_t n, float* amax_dev, uint8_t* out_e2m1, uint8_t* blk_scale_e4m3,
+    float* gscale_dev, uint8_t* out_e4m3_requant, float* scale8_dev, void* workspace_dev,
+    size_t workspace_bytes, qattn_stream_t stream);
+
 /* Quantized attention forward, full (non-causal) attention over [B, H, L, D] (blog, "Workflow
  * and quantization", SDPA bullets 2-4 and Fig. 4):
  *   S' = (Q8 K8^T) * s_q * s_k * sm_scale * log2(e)   FP8 MMA, FP32 accumulation

@@ -15,19 +15,23 @@ from __future__ import annotations
 import torch
 
 from . import _lib
-from ._lib import (MODE_FP4, MODE_FP8, QattnError, calibrate_amax, forward, forward_varlen,
-                   get_error, quantize_fp4_block, quantize_fp8)
+from ._lib import (MODE_FP4, MODE_FP8, QattnError, calibrate_amax, calibrate_quantize_fp4_block,
+                   calibrate_quantize_fp8, forward, forward_varlen, get_error, new_workspace,
+                   quantize_fp4_block, quantize_fp8)
 
 __all__ = ["QuantizedAttention", "calibrate_amax", "quantize_fp8", "quantize_fp4_block",
-           "forward", "forward_varlen", "get_error", "QattnError", "MODE_FP8", "MODE_FP4"]
+           "calibrate_quantize_fp8", "calibrate_quantize_fp4_block", "new_workspace", "forward",
+           "forward_varlen", "get_error", "QattnError", "MODE_FP8", "MODE_FP4"]
 
 
 class QuantizedAttention:
-    """The whole hot path for one shape: amax -> quantize (x3) -> fused attention.
+    """The whole hot path for one shape: fused calibrate+quantize (x3) -> fused attention.
 
-    Holds the device buffers (codes, scales, FP4 side outputs, output) so repeated calls
-    allocate nothing.  ``mode`` is "fp8" or "fp4".  For varlen, pass ``cu_seqlens`` (list of
-    ints) and q, k, v of shape [1, H, T, D].
+    Holds the device buffers (codes, scales, FP4 side outputs, output, the calibration
+    workspace) so repeated calls allocate nothing.  Calls on one object must not overlap on
+    the device (they share the buffers and the workspace); stream order is enough.  ``mode`` is
+    "fp8" or "fp4".  For varlen, pass ``cu_seqlens`` (list of ints) and q, k, v of shape
+    [1, H, T, D].
     """
 
     def __init__(self, shape, mode: str = "fp8", cu_seqlens=None, sm_scale: float | None = None,
@@ -52,6 +56,7 @@ class QuantizedAttention:
         elif mode != "fp8":
             raise ValueError(mode)
         self.out = torch.empty(shape, dtype=torch.bfloat16, device=dev)
+        self.workspace = new_workspace(dev)
         self.varlen = cu_seqlens is not None
         if self.varlen:
             if B != 1:
@@ -61,13 +66,13 @@ class QuantizedAttention:
 
     def quantize(self, q, k, v, stream=None):
         for i, x in enumerate((q, k, v)):
-            calibrate_amax(x, self.amax[i:i + 1], stream)
             if self.mode == "fp8":
-                quantize_fp8(x, self.amax[i:i + 1], self.codes[i], self.scale[i:i + 1], stream)
+                calibrate_quantize_fp8(x, self.amax[i:i + 1], self.codes[i], self.scale[i:i + 1],
+                                       self.workspace, stream)
             else:
-                quantize_fp4_block(x, self.amax[i:i + 1], self.e2m1[i], self.bscale[i],
-                                   self.gscale[i:i + 1], self.codes[i], self.scale[i:i + 1],
-                                   stream)
+                calibrate_quantize_fp4_block(x, self.amax[i:i + 1], self.e2m1[i], self.bscale[i],
+                                             self.gscale[i:i + 1], self.codes[i],
+                                             self.scale[i:i + 1], self.workspace, stream)
 
     def attend(self, stream=None):
         mode = MODE_FP8 if self.mode == "fp8" else MODE_FP4

@@ -20,9 +20,12 @@ MODE_FP8, MODE_FP4 = 0, 1
 # every symbol the header declares
 EXPORTS = (
     "qattn_calibrate_amax", "qattn_quantize_fp8", "qattn_quantize_fp4_block", "qattn_forward",
-    "qattn_forward_varlen", "qattn_get_error", "qattn_status_str",
+    "qattn_forward_varlen", "qattn_get_error", "qattn_calibrate_quantize_fp8",
+    "qattn_calibrate_quantize_fp4_block", "qattn_status_str",
     "qattn_debug_set_wait_timeout_ns", "qattn_debug_inject_missing_q",
 )
+_RETURNS_STATUS = EXPORTS[:8]
+FUSED_WORKSPACE_BYTES = 256     # QATTN_FUSED_WORKSPACE_BYTES
 
 
 class QattnError(RuntimeError):
@@ -51,6 +54,8 @@ def load() -> ctypes.CDLL:
     lib.qattn_calibrate_amax.argtypes = [P, S, P, P]
     lib.qattn_quantize_fp8.argtypes = [P, S, P, P, P, P]
     lib.qattn_quantize_fp4_block.argtypes = [P, S, P, P, P, P, P, P, P]
+    lib.qattn_calibrate_quantize_fp8.argtypes = [P, S, P, P, P, P, S, P]
+    lib.qattn_calibrate_quantize_fp4_block.argtypes = [P, S, P, P, P, P, P, P, P, S, P]
     lib.qattn_forward.argtypes = [P, P, P, P, I, I, I, I, ctypes.POINTER(_Scales), F, I, P]
     lib.qattn_forward_varlen.argtypes = [P, P, P, P, P, I, I, I, I, I, ctypes.POINTER(_Scales),
                                          F, I, P]
@@ -61,7 +66,7 @@ def load() -> ctypes.CDLL:
     lib.qattn_debug_set_wait_timeout_ns.restype = None
     lib.qattn_debug_inject_missing_q.argtypes = [I]
     lib.qattn_debug_inject_missing_q.restype = None
-    for name in EXPORTS[:6]:
+    for name in _RETURNS_STATUS:
         getattr(lib, name).restype = I
     _lib = lib
     return lib
@@ -125,6 +130,41 @@ def quantize_fp4_block(x: torch.Tensor, amax: torch.Tensor, out_e2m1: torch.Tens
         _dev(gscale, torch.float32, "gscale"),
         _dev(out_e4m3_requant, torch.uint8, "out_e4m3_requant"),
         _dev(scale8, torch.float32, "scale8"), _stream(stream)), "qattn_quantize_fp4_block")
+
+
+def new_workspace(device="cuda") -> torch.Tensor:
+    """A zero-filled workspace for the fused calibrate+quantize calls."""
+    return torch.zeros(FUSED_WORKSPACE_BYTES, dtype=torch.uint8, device=device)
+
+
+def calibrate_quantize_fp8(x: torch.Tensor, amax: torch.Tensor, out: torch.Tensor,
+                           scale: torch.Tensor, workspace: torch.Tensor, stream=None):
+    if out.numel() != x.numel():
+        raise ValueError("out must have x.numel() bytes")
+    _check(load().qattn_calibrate_quantize_fp8(
+        _dev(x, torch.bfloat16, "x"), x.numel(), _dev(amax, torch.float32, "amax"),
+        _dev(out, torch.uint8, "out"), _dev(scale, torch.float32, "scale"),
+        _dev(workspace, torch.uint8, "workspace"), workspace.numel(), _stream(stream)),
+        "qattn_calibrate_quantize_fp8")
+
+
+def calibrate_quantize_fp4_block(x: torch.Tensor, amax: torch.Tensor, out_e2m1: torch.Tensor,
+                                 blk_scale: torch.Tensor, gscale: torch.Tensor,
+                                 out_e4m3_requant: torch.Tensor | None,
+                                 scale8: torch.Tensor | None, workspace: torch.Tensor,
+                                 stream=None):
+    n = x.numel()
+    if out_e2m1.numel() != n // 2 or blk_scale.numel() != n // 16:
+        raise ValueError("out_e2m1 needs n/2 bytes and blk_scale n/16 bytes")
+    if out_e4m3_requant is not None and out_e4m3_requant.numel() != n:
+        raise ValueError("out_e4m3_requant needs n bytes")
+    _check(load().qattn_calibrate_quantize_fp4_block(
+        _dev(x, torch.bfloat16, "x"), n, _dev(amax, torch.float32, "amax"),
+        _dev(out_e2m1, torch.uint8, "out_e2m1"), _dev(blk_scale, torch.uint8, "blk_scale"),
+        _dev(gscale, torch.float32, "gscale"),
+        _dev(out_e4m3_requant, torch.uint8, "out_e4m3_requant"),
+        _dev(scale8, torch.float32, "scale8"), _dev(workspace, torch.uint8, "workspace"),
+        workspace.numel(), _stream(stream)), "qattn_calibrate_quantize_fp4_block")
 
 
 def _scales(s_q, s_k, s_v):

@@ -13,6 +13,13 @@ cudaError_t launch_quant_fp8(const void* x, size_t n, const float* amax, uint8_t
 cudaError_t launch_quant_fp4_block(const void* x, size_t n, const float* amax, uint8_t* packed,
                                    uint8_t* bscale, float* gscale, uint8_t* codes8, float* scale8,
                                    int* err, int num_sms, cudaStream_t stream);
+cudaError_t launch_calib_quant_fp8(const void* x, size_t n, float* amax, uint8_t* out,
+                                   float* scale, void* workspace, uint64_t limit_ns, int* err,
+                                   int num_sms, cudaStream_t stream);
+cudaError_t launch_calib_quant_fp4_block(const void* x, size_t n, float* amax, uint8_t* packed,
+                                         uint8_t* bscale, float* gscale, uint8_t* codes8,
+                                         float* scale8, void* workspace, uint64_t limit_ns,
+                                         int* err, int num_sms, cudaStream_t stream);
 cudaError_t launch_attention(const uint8_t* q8, const uint8_t* k8, const uint8_t* v8, void* out,
                              int B, int H, int L, int D, const int* cu_seqlens, int nseq,
                              int max_seqlen, int total_tokens, const float* s_q, const float* s_k,
@@ -127,6 +134,48 @@ qattn_status qattn_quantize_fp4_block(const void* x_bf16, size_t n, const float*
                                                  gscale_dev, out_e4m3_requant, scale8_dev, d->err,
                                                  d->num_sms,
                                                  reinterpret_cast<cudaStream_t>(stream)));
+}
+
+qattn_status qattn_calibrate_quantize_fp8(const void* x_bf16, size_t n, float* amax_dev,
+                                          uint8_t* out_e4m3, float* scale_dev,
+                                          void* workspace_dev, size_t workspace_bytes,
+                                          qattn_stream_t stream) {
+  if (!x_bf16 || !amax_dev || !out_e4m3 || !scale_dev || !workspace_dev || n == 0)
+    return QATTN_ERR_INVALID_ARG;
+  if (workspace_bytes < QATTN_FUSED_WORKSPACE_BYTES || !aligned(workspace_dev, 16))
+    return QATTN_ERR_INVALID_ARG;
+  if (!aligned(x_bf16, 16) || !aligned(out_e4m3, 8) || !aligned(amax_dev, 4) ||
+      !aligned(scale_dev, 4))
+    return QATTN_ERR_INVALID_ARG;
+  DeviceInfo* d = nullptr;
+  qattn_status st = device_info(&d);
+  if (st != QATTN_OK) return st;
+  return from_cuda(qattn::launch_calib_quant_fp8(x_bf16, n, amax_dev, out_e4m3, scale_dev,
+                                                 workspace_dev, g_timeout_ns, d->err, d->num_sms,
+                                                 reinterpret_cast<cudaStream_t>(stream)));
+}
+
+qattn_status qattn_calibrate_quantize_fp4_block(const void* x_bf16, size_t n, float* amax_dev,
+                                                uint8_t* out_e2m1, uint8_t* blk_scale_e4m3,
+                                                float* gscale_dev, uint8_t* out_e4m3_requant,
+                                                float* scale8_dev, void* workspace_dev,
+                                                size_t workspace_bytes, qattn_stream_t stream) {
+  if (!x_bf16 || !amax_dev || !out_e2m1 || !blk_scale_e4m3 || !gscale_dev || !workspace_dev ||
+      n == 0 || n % 16 != 0)
+    return QATTN_ERR_INVALID_ARG;
+  if ((out_e4m3_requant == nullptr) != (scale8_dev == nullptr)) return QATTN_ERR_INVALID_ARG;
+  if (workspace_bytes < QATTN_FUSED_WORKSPACE_BYTES || !aligned(workspace_dev, 16))
+    return QATTN_ERR_INVALID_ARG;
+  if (!aligned(x_bf16, 16) || !aligned(out_e2m1, 8) || !aligned(amax_dev, 4) ||
+      !aligned(gscale_dev, 4) || (out_e4m3_requant && !aligned(out_e4m3_requant, 16)) ||
+      (scale8_dev && !aligned(scale8_dev, 4)))
+    return QATTN_ERR_INVALID_ARG;
+  DeviceInfo* d = nullptr;
+  qattn_status st = device_info(&d);
+  if (st != QATTN_OK) return st;
+  return from_cuda(qattn::launch_calib_quant_fp4_block(
+      x_bf16, n, amax_dev, out_e2m1, blk_scale_e4m3, gscale_dev, out_e4m3_requant, scale8_dev,
+      workspace_dev, g_timeout_ns, d->err, d->num_sms, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 qattn_status qattn_forward(const uint8_t* q8, const uint8_t* k8, const uint8_t* v8,

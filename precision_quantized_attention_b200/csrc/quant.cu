@@ -153,6 +153,57 @@ __global__ void __launch_bounds__(256) k_quant_fp8(const uint4* __restrict__ xv,
 // One thread per block: two 16-byte loads, an 8-byte packed store, the scale byte and a
 // 16-byte store of FP8 codes.
 // -------------------------------------------------------------------------------------------
+// One 16-element block: E2M1 codes, E4M3 block scale and (optionally) the FP8 requant codes.
+__device__ __forceinline__ void fp4_block(uint4 a0, uint4 a1, size_t b, float sg, float six_sg,
+                                          float s8, float r8, bool fast8,
+                                          uint2* __restrict__ packed_out,
+                                          uint8_t* __restrict__ bscale_out,
+                                          uint4* __restrict__ codes8_out) {
+  const uint32_t w[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+  float x[16];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    x[2 * i] = bf16_lo(w[i]);
+    x[2 * i + 1] = bf16_hi(w[i]);
+  }
+  uint32_t am2 = 0;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) am2 = absmax_word(am2, w[i]);
+  const float amax_b = __uint_as_float(max(am2 & 0xFFFFu, am2 >> 16) << 16);
+  const uint32_t sb = cvt_e4m3x2(__fdiv_rn(amax_b, six_sg), 0.0f) & 0xFFu;
+  const float sbv = e4m3_to_f32(sb);
+  const float eff = __fmul_rn(sbv, sg);
+  uint32_t pk0 = 0, pk1 = 0;
+  uint32_t c8[4] = {0u, 0u, 0u, 0u};
+  if (eff != 0.0f) {
+    uint32_t nib[16];
+    const float r_eff = __frcp_rn(eff);
+    const bool fast_eff = markstein_ok(eff);
+#pragma unroll
+    for (int i = 0; i < 16; i += 2) {
+      const float q0 = fast_eff ? div_rn_by(x[i], eff, r_eff) : __fdiv_rn(x[i], eff);
+      const float q1 = fast_eff ? div_rn_by(x[i + 1], eff, r_eff) : __fdiv_rn(x[i + 1], eff);
+      const uint32_t byte = cvt_e2m1x2(q0, q1);
+      nib[i] = byte & 0xFu;
+      nib[i + 1] = byte >> 4;
+      if (i < 8) pk0 |= byte << (4 * i);
+      else pk1 |= byte << (4 * (i - 8));
+    }
+#pragma unroll
+    for (int i = 0; i < 16; i += 2) {
+      const float xh0 = __fmul_rn(__fmul_rn(e2m1_to_f32(nib[i]), sbv), sg);
+      const float xh1 = __fmul_rn(__fmul_rn(e2m1_to_f32(nib[i + 1]), sbv), sg);
+      const float d0 = fast8 ? div_rn_by(xh0, s8, r8) : __fdiv_rn(xh0, s8);
+      const float d1 = fast8 ? div_rn_by(xh1, s8, r8) : __fdiv_rn(xh1, s8);
+      const uint32_t pair = cvt_e4m3x2(d0, d1);
+      c8[i / 4] |= pair << (16 * ((i / 2) & 1));
+    }
+  }
+  __stcs(packed_out + b, make_uint2(pk0, pk1));
+  bscale_out[b] = static_cast<uint8_t>(sb);
+  if (codes8_out) __stcs(codes8_out + b, make_uint4(c8[0], c8[1], c8[2], c8[3]));
+}
+
 __global__ void __launch_bounds__(256) k_quant_fp4_block(
     const uint4* __restrict__ xv, size_t nblocks, const float* __restrict__ amax_p,
     uint2* __restrict__ packed_out, uint8_t* __restrict__ bscale_out,
@@ -174,52 +225,165 @@ __global__ void __launch_bounds__(256) k_quant_fp4_block(
   const bool fast8 = markstein_ok(s8);
   const size_t stride = static_cast<size_t>(gridDim.x) * blockDim.x;
   for (size_t b = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; b < nblocks;
-       b += stride) {
-    const uint4 a0 = __ldcs(xv + 2 * b), a1 = __ldcs(xv + 2 * b + 1);
-    const uint32_t w[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
-    float x[16];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      x[2 * i] = bf16_lo(w[i]);
-      x[2 * i + 1] = bf16_hi(w[i]);
-    }
-    uint32_t am2 = 0;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) am2 = absmax_word(am2, w[i]);
-    const float amax_b = __uint_as_float(max(am2 & 0xFFFFu, am2 >> 16) << 16);
-    const uint32_t sb = cvt_e4m3x2(__fdiv_rn(amax_b, six_sg), 0.0f) & 0xFFu;
-    const float sbv = e4m3_to_f32(sb);
-    const float eff = __fmul_rn(sbv, sg);
-    uint32_t pk0 = 0, pk1 = 0;
-    uint32_t c8[4] = {0u, 0u, 0u, 0u};
-    if (eff != 0.0f) {
-      uint32_t nib[16];
-      const float r_eff = __frcp_rn(eff);
-      const bool fast_eff = markstein_ok(eff);
-#pragma unroll
-      for (int i = 0; i < 16; i += 2) {
-        const float q0 = fast_eff ? div_rn_by(x[i], eff, r_eff) : __fdiv_rn(x[i], eff);
-        const float q1 = fast_eff ? div_rn_by(x[i + 1], eff, r_eff) : __fdiv_rn(x[i + 1], eff);
-        const uint32_t byte = cvt_e2m1x2(q0, q1);
-        nib[i] = byte & 0xFu;
-        nib[i + 1] = byte >> 4;
-        if (i < 8) pk0 |= byte << (4 * i);
-        else pk1 |= byte << (4 * (i - 8));
+       b += stride)
+    fp4_block(__ldcs(xv + 2 * b), __ldcs(xv + 2 * b + 1), b, sg, six_sg, s8, r8, fast8,
+              packed_out, bscale_out, codes8_out);
+}
+
+// -------------------------------------------------------------------------------------------
+// Fused calibrate + quantize (one cooperative launch per tensor).  Every CTA reduces the amax of
+// its contiguous chunk, publishes it with one atomicMax into the workspace and arrives on a
+// grid-wide counter; after the last arrival every CTA quantizes its chunk, which it just read
+// and which is still in L2, so HBM sees the input once.  The spin on the counter is bounded by
+// a global-timer limit (a launch that somehow is not co-resident records DEV_ERR_TIMEOUT and
+// writes nothing).  Once a CTA has read the result it departs on a second counter; the last
+// CTA to depart zeroes the workspace again, so it needs zeroing only before its first use and
+// no reset launch precedes a call.
+// -------------------------------------------------------------------------------------------
+struct FusedWorkspace {
+  unsigned amax_bits;
+  unsigned arrived;
+  unsigned departed;
+};
+
+__device__ __forceinline__ unsigned ld_acquire_gpu(const unsigned* p) {
+  unsigned v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+// Reduces m over the CTA, publishes it, waits for every CTA; returns the tensor amax (as float
+// bits) in every thread, or 0xFFFFFFFF after a timeout.
+__device__ __forceinline__ unsigned grid_amax(uint32_t m, FusedWorkspace* ws, uint64_t limit_ns,
+                                              int* err) {
+  __shared__ uint32_t warp_max[32];
+  __shared__ unsigned result;
+  m = __reduce_max_sync(0xFFFFFFFFu, m);
+  if ((threadIdx.x & 31) == 0) warp_max[threadIdx.x >> 5] = m;
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    m = threadIdx.x < (blockDim.x >> 5) ? warp_max[threadIdx.x] : 0u;
+    m = __reduce_max_sync(0xFFFFFFFFu, m);
+    if (threadIdx.x == 0) {
+      atomicMax(&ws->amax_bits, m << 16);
+      __threadfence();
+      atomicAdd(&ws->arrived, 1u);
+      const uint64_t t0 = global_timer_ns();
+      unsigned r = 0xFFFFFFFFu;
+      while (true) {
+        if (ld_acquire_gpu(&ws->arrived) >= gridDim.x) {
+          r = ld_acquire_gpu(&ws->amax_bits);
+          break;
+        }
+        if (global_timer_ns() - t0 > limit_ns) {
+          atomicExch(err, DEV_ERR_TIMEOUT);
+          break;
+        }
       }
-#pragma unroll
-      for (int i = 0; i < 16; i += 2) {
-        const float xh0 = __fmul_rn(__fmul_rn(e2m1_to_f32(nib[i]), sbv), sg);
-        const float xh1 = __fmul_rn(__fmul_rn(e2m1_to_f32(nib[i + 1]), sbv), sg);
-        const float d0 = fast8 ? div_rn_by(xh0, s8, r8) : __fdiv_rn(xh0, s8);
-        const float d1 = fast8 ? div_rn_by(xh1, s8, r8) : __fdiv_rn(xh1, s8);
-        const uint32_t pair = cvt_e4m3x2(d0, d1);
-        c8[i / 4] |= pair << (16 * ((i / 2) & 1));
+      result = r;
+      // depart; every CTA has left its wait when the last one arrives here
+      __threadfence();
+      if (atomicAdd(&ws->departed, 1u) == gridDim.x - 1) {
+        __threadfence();
+        ws->amax_bits = 0u;
+        ws->arrived = 0u;
+        ws->departed = 0u;
       }
     }
-    __stcs(packed_out + b, make_uint2(pk0, pk1));
-    bscale_out[b] = static_cast<uint8_t>(sb);
-    if (codes8_out) __stcs(codes8_out + b, make_uint4(c8[0], c8[1], c8[2], c8[3]));
   }
+  __syncthreads();
+  return result;
+}
+
+constexpr int FUSED_THREADS = 512;
+
+__global__ void __launch_bounds__(FUSED_THREADS) k_calib_quant_fp8(
+    const uint4* __restrict__ xv, size_t nvec, const uint16_t* __restrict__ xtail, int ntail,
+    float* __restrict__ amax_out, uint2* __restrict__ outv, uint8_t* __restrict__ outtail,
+    float* __restrict__ scale_out, FusedWorkspace* ws, uint64_t limit_ns, int* __restrict__ err) {
+  // contiguous chunk per CTA (in 16-byte vectors)
+  const size_t per = (nvec + gridDim.x - 1) / gridDim.x;
+  const size_t lo = static_cast<size_t>(blockIdx.x) * per;
+  const size_t hi = lo + per < nvec ? lo + per : nvec;
+  uint32_t m2 = 0;
+  for (size_t i = lo + threadIdx.x; i < hi; i += FUSED_THREADS) {
+    const uint4 a = __ldg(xv + i);               // keep it cached: read again below
+    m2 = absmax_word(m2, a.x); m2 = absmax_word(m2, a.y);
+    m2 = absmax_word(m2, a.z); m2 = absmax_word(m2, a.w);
+  }
+  uint32_t m = max(m2 & 0xFFFFu, m2 >> 16);
+  if (blockIdx.x == 0 && static_cast<int>(threadIdx.x) < ntail)
+    m = max(m, static_cast<uint32_t>(xtail[threadIdx.x]) & 0x7FFFu);
+  const unsigned bits = grid_amax(m, ws, limit_ns, err);
+  if (bits == 0xFFFFFFFFu) return;
+  const float amax = __uint_as_float(bits);
+  if (!(amax <= 3.402823466e38f)) {
+    if (blockIdx.x == 0 && threadIdx.x == 0) {
+      atomicExch(err, DEV_ERR_NONFINITE);
+      *amax_out = amax;
+    }
+    return;
+  }
+  const float s = (amax == 0.0f) ? 1.0f : __fdiv_rn(amax, 448.0f);
+  if (blockIdx.x == 0 && threadIdx.x == 0) {
+    *amax_out = amax;
+    *scale_out = s;
+  }
+  const float r = __frcp_rn(s);
+  if (markstein_ok(s)) {
+    for (size_t i = lo + threadIdx.x; i < hi; i += FUSED_THREADS) {
+      const uint4 a = __ldcs(xv + i);
+      __stcs(outv + i, make_uint2(quant4_e4m3<true>(a.x, a.y, s, r), quant4_e4m3<true>(a.z, a.w, s, r)));
+    }
+  } else {
+    for (size_t i = lo + threadIdx.x; i < hi; i += FUSED_THREADS) {
+      const uint4 a = __ldcs(xv + i);
+      __stcs(outv + i, make_uint2(quant4_e4m3<false>(a.x, a.y, s, r), quant4_e4m3<false>(a.z, a.w, s, r)));
+    }
+  }
+  if (blockIdx.x == 0 && static_cast<int>(threadIdx.x) < ntail) {
+    const float x = __uint_as_float(static_cast<uint32_t>(xtail[threadIdx.x]) << 16);
+    outtail[threadIdx.x] = static_cast<uint8_t>(cvt_e4m3x2(__fdiv_rn(x, s), 0.0f) & 0xFFu);
+  }
+}
+
+__global__ void __launch_bounds__(FUSED_THREADS) k_calib_quant_fp4_block(
+    const uint4* __restrict__ xv, size_t nblocks, float* __restrict__ amax_out,
+    uint2* __restrict__ packed_out, uint8_t* __restrict__ bscale_out,
+    float* __restrict__ gscale_out, uint4* __restrict__ codes8_out,
+    float* __restrict__ scale8_out, FusedWorkspace* ws, uint64_t limit_ns, int* __restrict__ err) {
+  const size_t per = (nblocks + gridDim.x - 1) / gridDim.x;   // contiguous chunk of blocks
+  const size_t lo = static_cast<size_t>(blockIdx.x) * per;
+  const size_t hi = lo + per < nblocks ? lo + per : nblocks;
+  uint32_t m2 = 0;
+  for (size_t i = 2 * lo + threadIdx.x; i < 2 * hi; i += FUSED_THREADS) {
+    const uint4 a = __ldg(xv + i);
+    m2 = absmax_word(m2, a.x); m2 = absmax_word(m2, a.y);
+    m2 = absmax_word(m2, a.z); m2 = absmax_word(m2, a.w);
+  }
+  const unsigned bits = grid_amax(max(m2 & 0xFFFFu, m2 >> 16), ws, limit_ns, err);
+  if (bits == 0xFFFFFFFFu) return;
+  const float amax = __uint_as_float(bits);
+  if (!(amax <= 3.402823466e38f)) {
+    if (blockIdx.x == 0 && threadIdx.x == 0) {
+      atomicExch(err, DEV_ERR_NONFINITE);
+      *amax_out = amax;
+    }
+    return;
+  }
+  const float sg = (amax == 0.0f) ? 1.0f : __fdiv_rn(amax, 2688.0f);
+  const float six_sg = __fmul_rn(6.0f, sg);
+  const float s8 = (amax == 0.0f) ? 1.0f : __fdiv_rn(__fmul_rn(2688.0f, sg), 448.0f);
+  if (blockIdx.x == 0 && threadIdx.x == 0) {
+    *amax_out = amax;
+    *gscale_out = sg;
+    if (scale8_out) *scale8_out = s8;
+  }
+  const float r8 = __frcp_rn(s8);
+  const bool fast8 = markstein_ok(s8);
+  for (size_t b = lo + threadIdx.x; b < hi; b += FUSED_THREADS)
+    fp4_block(__ldcs(xv + 2 * b), __ldcs(xv + 2 * b + 1), b, sg, six_sg, s8, r8, fast8,
+              packed_out, bscale_out, codes8_out);
 }
 
 // -------------------------------------------------------------------------------------------
@@ -265,6 +429,58 @@ cudaError_t launch_quant_fp4_block(const void* x, size_t n, const float* amax, u
       static_cast<const uint4*>(x), nblocks, amax, reinterpret_cast<uint2*>(packed), bscale,
       gscale, reinterpret_cast<uint4*>(codes8), scale8, err);
   return cudaGetLastError();
+}
+
+cudaError_t launch_calib_quant_fp8(const void* x, size_t n, float* amax, uint8_t* out,
+                                   float* scale, void* workspace, uint64_t limit_ns, int* err,
+                                   int num_sms, cudaStream_t stream) {
+  static int blocks_per_sm = 0;
+  if (blocks_per_sm == 0) {
+    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&blocks_per_sm,
+                                                                  k_calib_quant_fp8,
+                                                                  FUSED_THREADS, 0);
+    if (e != cudaSuccess || blocks_per_sm < 1) return e != cudaSuccess ? e : cudaErrorInvalidValue;
+  }
+  const size_t nvec = n / 8;
+  const int ntail = static_cast<int>(n - nvec * 8);
+  size_t want = (nvec + FUSED_THREADS * 4 - 1) / (FUSED_THREADS * 4);   // >= 4 vectors/thread
+  size_t cap = static_cast<size_t>(num_sms) * blocks_per_sm;
+  unsigned grid = static_cast<unsigned>(want < 1 ? 1 : (want < cap ? want : cap));
+  const uint4* xv = static_cast<const uint4*>(x);
+  const uint16_t* xtail = static_cast<const uint16_t*>(x) + nvec * 8;
+  uint2* outv = reinterpret_cast<uint2*>(out);
+  uint8_t* outtail = out + nvec * 8;
+  FusedWorkspace* ws = static_cast<FusedWorkspace*>(workspace);
+  void* args[] = {(void*)&xv, (void*)&nvec, (void*)&xtail, (void*)&ntail, (void*)&amax,
+                  (void*)&outv, (void*)&outtail, (void*)&scale, (void*)&ws, (void*)&limit_ns,
+                  (void*)&err};
+  return cudaLaunchCooperativeKernel((const void*)k_calib_quant_fp8, dim3(grid),
+                                     dim3(FUSED_THREADS), args, 0, stream);
+}
+
+cudaError_t launch_calib_quant_fp4_block(const void* x, size_t n, float* amax, uint8_t* packed,
+                                         uint8_t* bscale, float* gscale, uint8_t* codes8,
+                                         float* scale8, void* workspace, uint64_t limit_ns,
+                                         int* err, int num_sms, cudaStream_t stream) {
+  static int blocks_per_sm = 0;
+  if (blocks_per_sm == 0) {
+    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(
+        &blocks_per_sm, k_calib_quant_fp4_block, FUSED_THREADS, 0);
+    if (e != cudaSuccess || blocks_per_sm < 1) return e != cudaSuccess ? e : cudaErrorInvalidValue;
+  }
+  const size_t nblocks = n / 16;
+  size_t want = (nblocks + FUSED_THREADS * 2 - 1) / (FUSED_THREADS * 2);
+  size_t cap = static_cast<size_t>(num_sms) * blocks_per_sm;
+  unsigned grid = static_cast<unsigned>(want < 1 ? 1 : (want < cap ? want : cap));
+  const uint4* xv = static_cast<const uint4*>(x);
+  uint2* pk = reinterpret_cast<uint2*>(packed);
+  uint4* c8 = reinterpret_cast<uint4*>(codes8);
+  FusedWorkspace* ws = static_cast<FusedWorkspace*>(workspace);
+  void* args[] = {(void*)&xv, (void*)&nblocks, (void*)&amax, (void*)&pk, (void*)&bscale,
+                  (void*)&gscale, (void*)&c8, (void*)&scale8, (void*)&ws, (void*)&limit_ns,
+                  (void*)&err};
+  return cudaLaunchCooperativeKernel((const void*)k_calib_quant_fp4_block, dim3(grid),
+                                     dim3(FUSED_THREADS), args, 0, stream);
 }
 
 }  // namespace qattn

@@ -49,6 +49,18 @@ def test_host_side_argument_errors():
     # FP4 needs n % 16 == 0 and both-or-neither of the requant outputs
     assert lib.qattn_quantize_fp4_block(FAKE, 24, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, s0) == _lib.ERR_INVALID_ARG
     assert lib.qattn_quantize_fp4_block(FAKE, 32, FAKE, FAKE, FAKE, FAKE, FAKE, None, s0) == _lib.ERR_INVALID_ARG
+    # fused calibrate+quantize: workspace present, large enough and aligned
+    W = _lib.FUSED_WORKSPACE_BYTES
+    cq8 = lib.qattn_calibrate_quantize_fp8
+    assert cq8(FAKE, 16, FAKE, FAKE, FAKE, None, W, s0) == _lib.ERR_INVALID_ARG
+    assert cq8(FAKE, 16, FAKE, FAKE, FAKE, FAKE, W - 1, s0) == _lib.ERR_INVALID_ARG
+    assert cq8(FAKE, 16, FAKE, FAKE, FAKE, ctypes.c_void_p(0x10008), W, s0) == _lib.ERR_INVALID_ARG
+    assert cq8(FAKE, 0, FAKE, FAKE, FAKE, FAKE, W, s0) == _lib.ERR_INVALID_ARG
+    assert cq8(MISALIGNED, 16, FAKE, FAKE, FAKE, FAKE, W, s0) == _lib.ERR_INVALID_ARG
+    cq4 = lib.qattn_calibrate_quantize_fp4_block
+    assert cq4(FAKE, 24, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, W, s0) == _lib.ERR_INVALID_ARG
+    assert cq4(FAKE, 32, FAKE, FAKE, FAKE, FAKE, None, FAKE, FAKE, W, s0) == _lib.ERR_INVALID_ARG
+    assert cq4(FAKE, 32, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 16, s0) == _lib.ERR_INVALID_ARG
     sc = _lib._Scales(0x10000, 0x10000, 0x10000)
     fwd = lib.qattn_forward
     assert fwd(FAKE, FAKE, FAKE, FAKE, 1, 1, 16, 96, ctypes.byref(sc), 0.1, 0, s0) == _lib.ERR_UNSUPPORTED

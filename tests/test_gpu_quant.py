@@ -107,3 +107,90 @@ def test_nonfinite_input_is_reported():
     assert qa.get_error() == qa._lib.ERR_NONFINITE
     assert scale.item() == -1.0 and int(codes[0].item()) == 0x55     # nothing written
     assert qa.get_error() == 0                                        # the word was cleared
+
+
+@pytest.mark.parametrize("name", list(_inputs().keys()))
+def test_fused_calibrate_quantize_fp8_bit_exact(name):
+    """One cooperative launch gives the amax, scale and codes of calibrate + quantize; twice in a
+    row on one workspace, which each call leaves zero-filled."""
+    x = _inputs()[name]
+    xd = x.cuda()
+    ws = qa.new_workspace()
+    _, a = oracle.amax(x)
+    want, s = oracle.quantize_fp8(x, a)
+    for _ in range(2):
+        amax = torch.full((1,), -1.0, device="cuda")
+        scale = torch.zeros(1, device="cuda")
+        codes = torch.full((x.numel(),), 0x55, dtype=torch.uint8, device="cuda")
+        qa.calibrate_quantize_fp8(xd, amax, codes, scale, ws)
+        assert qa.get_error() == 0
+        assert float(amax.item()) == a
+        assert np.float32(scale.item()) == s
+        assert np.array_equal(_u8(codes), want)
+        assert int(ws.count_nonzero().item()) == 0
+
+
+@pytest.mark.parametrize("name", [k for k in _inputs() if k not in ("tiny_tail", "tail_7")])
+def test_fused_calibrate_quantize_fp4_block_bit_exact(name):
+    x = _inputs()[name]
+    n = x.numel()
+    xd = x.cuda()
+    ws = qa.new_workspace()
+    _, a = oracle.amax(x)
+    w_packed, w_bscale, w_sg, w_c8, w_s8 = oracle.quantize_fp4_block(x, a)
+    for requant in (True, False):
+        amax = torch.zeros(1, device="cuda")
+        packed = torch.empty(n // 2, dtype=torch.uint8, device="cuda")
+        bscale = torch.empty(n // 16, dtype=torch.uint8, device="cuda")
+        gscale = torch.zeros(1, device="cuda")
+        c8 = torch.empty(n, dtype=torch.uint8, device="cuda") if requant else None
+        s8 = torch.zeros(1, device="cuda") if requant else None
+        qa.calibrate_quantize_fp4_block(xd, amax, packed, bscale, gscale, c8, s8, ws)
+        assert qa.get_error() == 0
+        assert float(amax.item()) == a
+        assert np.float32(gscale.item()) == w_sg
+        assert np.array_equal(_u8(bscale), w_bscale)
+        assert np.array_equal(_u8(packed), w_packed)
+        if requant:
+            assert np.float32(s8.item()) == w_s8
+            assert np.array_equal(_u8(c8), w_c8)
+        assert int(ws.count_nonzero().item()) == 0
+
+
+def test_fused_matches_separate_calls_on_a_large_tensor():
+    """Many CTAs (grid at the co-residency cap), every code equal to the two-call path."""
+    g = torch.Generator().manual_seed(5)
+    x = (torch.randn(24 * 4096 * 128, generator=g) * 2.0).to(torch.bfloat16).cuda()
+    x[7_000_001] = -300.0                          # the amax sits in one CTA's chunk
+    ws = qa.new_workspace()
+    a1, s1, c1 = torch.zeros(1, device="cuda"), torch.zeros(1, device="cuda"), torch.empty_like(x, dtype=torch.uint8)
+    a2, s2, c2 = torch.zeros(1, device="cuda"), torch.zeros(1, device="cuda"), torch.empty_like(x, dtype=torch.uint8)
+    qa.calibrate_amax(x, a1)
+    qa.quantize_fp8(x, a1, c1, s1)
+    qa.calibrate_quantize_fp8(x, a2, c2, s2, ws)
+    assert qa.get_error() == 0
+    assert float(a2.item()) == 300.0 == float(a1.item())
+    assert float(s2.item()) == float(s1.item())
+    assert torch.equal(c1, c2)
+
+
+def test_fused_nonfinite_input_is_reported():
+    x = torch.randn(4096 * 16).to(torch.bfloat16)
+    x[40000] = float("inf")
+    xd = x.cuda()
+    ws = qa.new_workspace()
+    amax = torch.zeros(1, device="cuda")
+    scale = torch.full((1,), -1.0, device="cuda")
+    codes = torch.full((x.numel(),), 0x55, dtype=torch.uint8, device="cuda")
+    qa.calibrate_quantize_fp8(xd, amax, codes, scale, ws)
+    assert qa.get_error() == qa._lib.ERR_NONFINITE
+    assert float(amax.item()) == float("inf")
+    assert scale.item() == -1.0 and int(codes[0].item()) == 0x55     # nothing written
+    assert int(ws.count_nonzero().item()) == 0
+    # the workspace is usable again right away
+    x[40000] = 1.0
+    qa.calibrate_quantize_fp8(x.cuda(), amax, codes, scale, ws)
+    assert qa.get_error() == 0
+    _, a = oracle.amax(x)
+    want, s = oracle.quantize_fp8(x, a)
+    assert np.array_equal(_u8(codes), want) and np.float32(scale.item()) == s
