@@ -4,7 +4,7 @@ One step = the whole path on one batch of the L=8704 FLUX.1 Kontext editing work
 4096 target + 4096 context tokens, H=24, D=128, FP8 mode, outlier channels in Q and K):
 fused calibrate+quantize x3 -> fused attention, inputs resident in HBM.  Metric: algorithmic
 FLOPs of BMM1 + BMM2 (4 * H * D * L^2) per second.  The L2 is flushed between steps (a
-256 MiB write outside the timed events).  ``e2e`` repeats the measurement through the same C ABI
+256 MiB write, then a 256 MiB read of another buffer, outside the timed events).  ``e2e`` repeats the measurement through the same C ABI
 with the bf16 inputs in pinned host memory: every step copies Q, K, V to the device and the
 output back.  ``--impl reference`` times the CPU oracle instead (rank 0 only) on a bounded row
 sample of the same workload.
@@ -19,7 +19,6 @@ import argparse
 import json
 import os
 import statistics
-import subprocess
 import sys
 import time
 
@@ -47,66 +46,87 @@ def load_peaks():
 
 
 class ClockSampler:
-    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
+    """SM clock and clock-event reasons of this process's GPU, sampled through NVML every 5 ms
+    by a background thread while the timed region runs (reading only; no setting is changed).
+    The GPU is matched by PCI address, so CUDA_VISIBLE_DEVICES renumbering does not matter."""
 
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    PERIOD_S = 0.005
 
-    def __init__(self, gpu_index: int):
-        self.gpu = gpu_index
-        self.proc = None
-        self.skip = 0
-        import tempfile
-        fd, self.path = tempfile.mkstemp(prefix="qattn_clocks_", suffix=".csv")
-        os.close(fd)
+    def __init__(self, cuda_index: int):
+        self.cuda_index = cuda_index
+        self.samples = []
+        self.max_mhz = None
+        self.error = None
+        self._thread = None
+
+    def _handle(self, nv):
+        props = torch.cuda.get_device_properties(self.cuda_index)
+        bus = f"{props.pci_domain_id:08x}:{props.pci_bus_id:02x}:{props.pci_device_id:02x}.0"
+        try:
+            return nv.nvmlDeviceGetHandleByPciBusId(bus)
+        except Exception:
+            return nv.nvmlDeviceGetHandleByIndex(self.cuda_index)
 
     def __enter__(self):
+        import threading
         try:
-            self.f = open(self.path, "w")
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "100"], stdout=self.f,
-                stderr=subprocess.DEVNULL)
-        except Exception:
-            self.proc = None
+            import pynvml as nv
+            nv.nvmlInit()
+            h = self._handle(nv)
+            self.max_mhz = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
+        except Exception as e:          # no NVML: the line says so
+            self.error = f"nvml unavailable: {type(e).__name__}"
             return self
-        deadline = time.time() + 5.0          # the first sample marks the sampler as running
-        while time.time() < deadline and os.path.getsize(self.path) == 0:
-            time.sleep(0.02)
-        with open(self.path) as f:
-            self.skip = len(f.readlines())
+        self._stop = threading.Event()
+
+        def run():
+            while True:
+                try:
+                    self.samples.append((nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM),
+                                         nv.nvmlDeviceGetCurrentClocksEventReasons(h)))
+                except Exception as e:
+                    self.error = f"nvml query failed: {type(e).__name__}"
+                    return
+                if self._stop.wait(self.PERIOD_S):
+                    return
+
+        self._thread = threading.Thread(target=run, daemon=True)
+        self._thread.start()
         return self
 
     def __exit__(self, *exc):
-        if self.proc is not None:
-            self.proc.terminate()
-            try:
-                self.proc.wait(timeout=5)
-            except Exception:
-                self.proc.kill()
-            self.f.close()
+        if self._thread is not None:
+            self._stop.set()
+            self._thread.join()
 
     def summary(self):
-        if self.proc is None:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
-        rows = []
-        with open(self.path) as f:
-            for line in f.readlines()[self.skip:]:
-                parts = [p.strip() for p in line.split(",")]
-                if len(parts) < 9:
-                    continue
-                try:
-                    rows.append((float(parts[1]), float(parts[2]), parts[5:9]))
-                except ValueError:
-                    continue
-        if not rows:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for _, _, flags in rows for i, fl in enumerate(flags)
-                          if fl.lower() == "active"})
-        return {"sm_mhz": statistics.median(r[0] for r in rows), "sm_max_mhz": rows[0][1],
-                "reasons": reasons, "samples": len(rows)}
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz,
+                    "reasons": [self.error or "no samples"]}
+        import pynvml as nv
+        names = {nv.nvmlClocksEventReasonHwSlowdown: "hw_slowdown",
+                 nv.nvmlClocksEventReasonHwThermalSlowdown: "hw_thermal_slowdown",
+                 nv.nvmlClocksEventReasonSwThermalSlowdown: "sw_thermal_slowdown",
+                 nv.nvmlClocksEventReasonSwPowerCap: "sw_power_cap",
+                 nv.nvmlClocksEventReasonHwPowerBrakeSlowdown: "hw_power_brake_slowdown"}
+        reasons = sorted({nm for _, bits in self.samples for bit, nm in names.items() if bits & bit})
+        return {"sm_mhz": statistics.median(m for m, _ in self.samples),
+                "sm_max_mhz": self.max_mhz, "reasons": reasons, "samples": len(self.samples),
+                "source": "nvml every 5 ms during the timed steps"}
+
+
+class L2Flush:
+    """Leaves a cold, clean L2: writing a buffer larger than the L2 evicts every line; reading a
+    second one then evicts those dirty lines, so their write-back does not land in the next
+    timed step."""
+
+    def __init__(self):
+        self.w = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+        self.r = torch.zeros(L2_FLUSH_BYTES // 4, dtype=torch.float32, device="cuda")
+
+    def __call__(self):
+        self.w.zero_()
+        self.r.max()
 
 
 def dist_setup(n_gpus: int):
@@ -148,7 +168,7 @@ def run_gpu(args):
     q, k, v = workloads.make_qkv(w)
     qd, kd, vd = (t.cuda() for t in (q, k, v))
     path = qa.QuantizedAttention(w.shape, w.mode, sm_scale=w.sm_scale)
-    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    flush = L2Flush()
     stream = torch.cuda.current_stream()
 
     def step():
@@ -166,7 +186,7 @@ def run_gpu(args):
     torch.cuda.synchronize()
     with ClockSampler(local) as clocks:
         for i in range(args.steps):
-            flush.zero_()
+            flush()
             ev[i][0].record(stream)
             path.quantize(qd, kd, vd)
             ev[i][1].record(stream)
@@ -206,7 +226,7 @@ def e2e_time(args, w, q, k, v, qd, kd, vd, step, flush, stream, world):
     torch.cuda.synchronize()
     barrier(world)
     for i in range(args.steps):
-        flush.zero_()
+        flush()
         e2e_ev[i][0].record(stream)
         qd.copy_(qh, non_blocking=True)
         kd.copy_(kh, non_blocking=True)
@@ -249,7 +269,9 @@ def report(args, w, qkv, rank, world, ms, attn, quant, e2e_ms, clocks):
                                    if w.L == workloads.L_EDIT else ""),
                    "mode": w.mode, "B": w.B, "H": w.H, "L": w.L, "D": w.D,
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
-                   "l2": "flushed between steps (256 MiB write outside the timed events)"},
+                   "l2": "flushed between steps outside the timed events: a 256 MiB write, then a "
+                         "256 MiB read of another buffer so the write's dirty lines are "
+                         "written back before the step starts"},
         "roofline": {"bound": "tensor", "achieved": achieved_tf, "peak": fp8_peak,
                      "unit": "TFLOP/s", "frac": achieved_tf / fp8_peak, "traffic": None,
                      "kernel": f"k_attn_fp8_fwd<{w.D}>",
