@@ -127,6 +127,22 @@ QATTN_API qattn_status qattn_calibrate_quantize_fp4_block(
     float* gscale_dev, uint8_t* out_e4m3_requant, float* scale8_dev, void* workspace_dev,
     size_t workspace_bytes, qattn_stream_t stream);
 
+/* qattn_calibrate_quantize_fp8 without a caller workspace (the blog has no counterpart: this is
+ * a calling convention, not part of the method).  For callers that cannot supply a scratch
+ * buffer -- C code with no device allocator at the call site, or a runtime whose device memory
+ * is planned ahead and must not allocate on the hot path.  The call allocates nothing: the
+ * workspace is a static QATTN_FUSED_WORKSPACE_BYTES-byte device array inside the library (one
+ * per device), cleared with a memset on `stream` before the kernel.  The workspace need does not
+ * grow with n, so no size is rejected on its account; the argument rules and results are those
+ * of qattn_calibrate_quantize_fp8.  The FIRST call on each device looks the array's address up
+ * (cudaGetSymbolAddress, with that device current); make that first call before any stream
+ * capture.  All calls on one device share the array: calls that overlap on the device (other
+ * streams, other host threads without ordering) race and give wrong results. */
+QATTN_API qattn_status qattn_calibrate_quantize_fp8_noalloc(const void* x_bf16, size_t n,
+                                                            float* amax_dev, uint8_t* out_e4m3,
+                                                            float* scale_dev,
+                                                            qattn_stream_t stream);
+
 /* Quantized attention forward, full (non-causal) attention over [B, H, L, D] (blog, "Workflow
  * and quantization", SDPA bullets 2-4 and Fig. 4):
  *   S' = (Q8 K8^T) * s_q * s_k * sm_scale * log2(e)   FP8 MMA, FP32 accumulation

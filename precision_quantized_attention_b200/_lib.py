@@ -21,10 +21,11 @@ MODE_FP8, MODE_FP4 = 0, 1
 EXPORTS = (
     "qattn_calibrate_amax", "qattn_quantize_fp8", "qattn_quantize_fp4_block", "qattn_forward",
     "qattn_forward_varlen", "qattn_get_error", "qattn_calibrate_quantize_fp8",
-    "qattn_calibrate_quantize_fp4_block", "qattn_status_str",
+    "qattn_calibrate_quantize_fp4_block", "qattn_calibrate_quantize_fp8_noalloc",
+    "qattn_status_str",
     "qattn_debug_set_wait_timeout_ns", "qattn_debug_inject_missing_q",
 )
-_RETURNS_STATUS = EXPORTS[:8]
+_RETURNS_STATUS = EXPORTS[:9]
 FUSED_WORKSPACE_BYTES = 256     # QATTN_FUSED_WORKSPACE_BYTES
 
 
@@ -56,6 +57,7 @@ def load() -> ctypes.CDLL:
     lib.qattn_quantize_fp4_block.argtypes = [P, S, P, P, P, P, P, P, P]
     lib.qattn_calibrate_quantize_fp8.argtypes = [P, S, P, P, P, P, S, P]
     lib.qattn_calibrate_quantize_fp4_block.argtypes = [P, S, P, P, P, P, P, P, P, S, P]
+    lib.qattn_calibrate_quantize_fp8_noalloc.argtypes = [P, S, P, P, P, P]
     lib.qattn_forward.argtypes = [P, P, P, P, I, I, I, I, ctypes.POINTER(_Scales), F, I, P]
     lib.qattn_forward_varlen.argtypes = [P, P, P, P, P, I, I, I, I, I, ctypes.POINTER(_Scales),
                                          F, I, P]
@@ -146,6 +148,17 @@ def calibrate_quantize_fp8(x: torch.Tensor, amax: torch.Tensor, out: torch.Tenso
         _dev(out, torch.uint8, "out"), _dev(scale, torch.float32, "scale"),
         _dev(workspace, torch.uint8, "workspace"), workspace.numel(), _stream(stream)),
         "qattn_calibrate_quantize_fp8")
+
+
+def calibrate_quantize_fp8_noalloc(x: torch.Tensor, amax: torch.Tensor, out: torch.Tensor,
+                                   scale: torch.Tensor, stream=None):
+    """calibrate_quantize_fp8 with the library's static workspace (no caller buffer)."""
+    if out.numel() != x.numel():
+        raise ValueError("out must have x.numel() bytes")
+    _check(load().qattn_calibrate_quantize_fp8_noalloc(
+        _dev(x, torch.bfloat16, "x"), x.numel(), _dev(amax, torch.float32, "amax"),
+        _dev(out, torch.uint8, "out"), _dev(scale, torch.float32, "scale"), _stream(stream)),
+        "qattn_calibrate_quantize_fp8_noalloc")
 
 
 def calibrate_quantize_fp4_block(x: torch.Tensor, amax: torch.Tensor, out_e2m1: torch.Tensor,

@@ -61,6 +61,10 @@ def test_host_side_argument_errors():
     assert cq4(FAKE, 24, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, W, s0) == _lib.ERR_INVALID_ARG
     assert cq4(FAKE, 32, FAKE, FAKE, FAKE, FAKE, None, FAKE, FAKE, W, s0) == _lib.ERR_INVALID_ARG
     assert cq4(FAKE, 32, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 16, s0) == _lib.ERR_INVALID_ARG
+    na = lib.qattn_calibrate_quantize_fp8_noalloc
+    assert na(None, 16, FAKE, FAKE, FAKE, s0) == _lib.ERR_INVALID_ARG
+    assert na(FAKE, 0, FAKE, FAKE, FAKE, s0) == _lib.ERR_INVALID_ARG
+    assert na(MISALIGNED, 16, FAKE, FAKE, FAKE, s0) == _lib.ERR_INVALID_ARG
     sc = _lib._Scales(0x10000, 0x10000, 0x10000)
     fwd = lib.qattn_forward
     assert fwd(FAKE, FAKE, FAKE, FAKE, 1, 1, 16, 96, ctypes.byref(sc), 0.1, 0, s0) == _lib.ERR_UNSUPPORTED
