@@ -236,15 +236,20 @@ __global__ void __launch_bounds__(256) k_quant_fp4_block(
 // grid-wide counter; after the last arrival every CTA quantizes its chunk, which it just read
 // and which is still in L2, so HBM sees the input once.  The spin on the counter is bounded by
 // a global-timer limit (a launch that somehow is not co-resident records DEV_ERR_TIMEOUT and
-// writes nothing).  Once a CTA has read the result it departs on a second counter; the last
-// CTA to depart zeroes the workspace again, so it needs zeroing only before its first use and
-// no reset launch precedes a call.
+// writes nothing).  Each CTA departs on a second counter when it is done; the last CTA to
+// depart zeroes the workspace again, so it needs zeroing only before its first use and no reset
+// launch precedes a call.
 // -------------------------------------------------------------------------------------------
+// The arrival counter has a 128-byte line of its own: the pollers read it while the other CTAs
+// still publish their maxima into the first line.
 struct FusedWorkspace {
   unsigned amax_bits;
-  unsigned arrived;
   unsigned departed;
+  unsigned pad0[30];
+  unsigned arrived;
+  unsigned pad1[31];
 };
+static_assert(sizeof(FusedWorkspace) <= 256, "fits QATTN_FUSED_WORKSPACE_BYTES");
 
 __device__ __forceinline__ unsigned ld_acquire_gpu(const unsigned* p) {
   unsigned v;
@@ -253,7 +258,10 @@ __device__ __forceinline__ unsigned ld_acquire_gpu(const unsigned* p) {
 }
 
 // Reduces m over the CTA, publishes it, waits for every CTA; returns the tensor amax (as float
-// bits) in every thread, or 0xFFFFFFFF after a timeout.
+// bits) in every thread, or 0xFFFFFFFF after a timeout.  One thread per CTA publishes with a
+// fire-and-forget max reduction and a releasing add on the arrival counter, then polls the
+// counter with acquire loads and a short sleep between polls (444 pollers on one line would
+// otherwise slow the arrivals down).
 __device__ __forceinline__ unsigned grid_amax(uint32_t m, FusedWorkspace* ws, uint64_t limit_ns,
                                               int* err) {
   __shared__ uint32_t warp_max[32];
@@ -265,9 +273,9 @@ __device__ __forceinline__ unsigned grid_amax(uint32_t m, FusedWorkspace* ws, ui
     m = threadIdx.x < (blockDim.x >> 5) ? warp_max[threadIdx.x] : 0u;
     m = __reduce_max_sync(0xFFFFFFFFu, m);
     if (threadIdx.x == 0) {
-      atomicMax(&ws->amax_bits, m << 16);
-      __threadfence();
-      atomicAdd(&ws->arrived, 1u);
+      asm volatile("red.relaxed.gpu.global.max.u32 [%0], %1;" ::"l"(&ws->amax_bits), "r"(m << 16)
+                   : "memory");
+      asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(&ws->arrived) : "memory");
       const uint64_t t0 = global_timer_ns();
       unsigned r = 0xFFFFFFFFu;
       while (true) {
@@ -279,23 +287,104 @@ __device__ __forceinline__ unsigned grid_amax(uint32_t m, FusedWorkspace* ws, ui
           atomicExch(err, DEV_ERR_TIMEOUT);
           break;
         }
+        __nanosleep(32);
       }
       result = r;
-      // depart; every CTA has left its wait when the last one arrives here
-      __threadfence();
-      if (atomicAdd(&ws->departed, 1u) == gridDim.x - 1) {
-        __threadfence();
-        ws->amax_bits = 0u;
-        ws->arrived = 0u;
-        ws->departed = 0u;
-      }
     }
   }
   __syncthreads();
   return result;
 }
 
-constexpr int FUSED_THREADS = 512;
+// Called by every CTA once it no longer needs the workspace (at its end, off the critical path):
+// when the last CTA departs, every CTA has read the amax, so it zeroes the workspace for the
+// next call.
+__device__ __forceinline__ void grid_depart(FusedWorkspace* ws) {
+  if (threadIdx.x == 0) {
+    unsigned old;
+    asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;"
+                 : "=r"(old)
+                 : "l"(&ws->departed)
+                 : "memory");
+    if (old == gridDim.x - 1) {
+      ws->amax_bits = 0u;
+      ws->arrived = 0u;
+      ws->departed = 0u;
+    }
+  }
+}
+
+constexpr int FUSED_THREADS = 1024;    // one CTA per SM: fewer arrivals on the grid barrier
+constexpr int FUSED_UNROLL = 4;       // independent 16-byte loads in flight per thread
+
+// L2 eviction priorities: phase 1 marks the chunk evict-last so that it is still in L2 when
+// phase 2 reads it back (evict-first, it is not needed afterwards).  Without the hint the L2
+// does not keep a streamed tensor of tens of MB and phase 2 goes back to HBM.
+__device__ __forceinline__ uint64_t l2_policy_evict_last() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+__device__ __forceinline__ uint64_t l2_policy_evict_first() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+__device__ __forceinline__ uint4 ld_hint(const uint4* p, uint64_t pol) {
+  uint4 v;
+  asm volatile("ld.global.nc.L2::cache_hint.v4.u32 {%0, %1, %2, %3}, [%4], %5;"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p), "l"(pol));
+  return v;
+}
+
+// Packed bf16 |x| maximum over the vectors [lo, hi) of this CTA's chunk (phase 1).
+__device__ __forceinline__ uint32_t chunk_absmax(const uint4* __restrict__ xv, size_t lo,
+                                                 size_t hi) {
+  constexpr size_t T = FUSED_THREADS, U = FUSED_UNROLL;
+  const uint64_t pol = l2_policy_evict_last();
+  uint32_t m2 = 0;
+  size_t i = lo + threadIdx.x;
+  for (; i + (U - 1) * T < hi; i += U * T) {
+    uint4 a[U];
+#pragma unroll
+    for (size_t u = 0; u < U; ++u) a[u] = ld_hint(xv + i + u * T, pol);
+#pragma unroll
+    for (size_t u = 0; u < U; ++u) {
+      m2 = absmax_word(m2, a[u].x); m2 = absmax_word(m2, a[u].y);
+      m2 = absmax_word(m2, a[u].z); m2 = absmax_word(m2, a[u].w);
+    }
+  }
+  for (; i < hi; i += T) {
+    const uint4 a = ld_hint(xv + i, pol);
+    m2 = absmax_word(m2, a.x); m2 = absmax_word(m2, a.y);
+    m2 = absmax_word(m2, a.z); m2 = absmax_word(m2, a.w);
+  }
+  return m2;
+}
+
+// FP8 codes of the vectors [lo, hi) (phase 2): the chunk comes back from L2.
+template <bool FAST>
+__device__ __forceinline__ void chunk_quant_fp8(const uint4* __restrict__ xv,
+                                                uint2* __restrict__ outv, size_t lo, size_t hi,
+                                                float s, float r) {
+  constexpr size_t T = FUSED_THREADS, U = FUSED_UNROLL;
+  const uint64_t pol = l2_policy_evict_first();
+  size_t i = lo + threadIdx.x;
+  for (; i + (U - 1) * T < hi; i += U * T) {
+    uint4 a[U];
+#pragma unroll
+    for (size_t u = 0; u < U; ++u) a[u] = ld_hint(xv + i + u * T, pol);
+#pragma unroll
+    for (size_t u = 0; u < U; ++u)
+      __stcs(outv + i + u * T, make_uint2(quant4_e4m3<FAST>(a[u].x, a[u].y, s, r),
+                                          quant4_e4m3<FAST>(a[u].z, a[u].w, s, r)));
+  }
+  for (; i < hi; i += T) {
+    const uint4 a = ld_hint(xv + i, pol);
+    __stcs(outv + i, make_uint2(quant4_e4m3<FAST>(a.x, a.y, s, r), quant4_e4m3<FAST>(a.z, a.w, s, r)));
+  }
+}
 
 __global__ void __launch_bounds__(FUSED_THREADS) k_calib_quant_fp8(
     const uint4* __restrict__ xv, size_t nvec, const uint16_t* __restrict__ xtail, int ntail,
@@ -305,23 +394,22 @@ __global__ void __launch_bounds__(FUSED_THREADS) k_calib_quant_fp8(
   const size_t per = (nvec + gridDim.x - 1) / gridDim.x;
   const size_t lo = static_cast<size_t>(blockIdx.x) * per;
   const size_t hi = lo + per < nvec ? lo + per : nvec;
-  uint32_t m2 = 0;
-  for (size_t i = lo + threadIdx.x; i < hi; i += FUSED_THREADS) {
-    const uint4 a = __ldg(xv + i);               // keep it cached: read again below
-    m2 = absmax_word(m2, a.x); m2 = absmax_word(m2, a.y);
-    m2 = absmax_word(m2, a.z); m2 = absmax_word(m2, a.w);
-  }
+  const uint32_t m2 = chunk_absmax(xv, lo, hi);
   uint32_t m = max(m2 & 0xFFFFu, m2 >> 16);
   if (blockIdx.x == 0 && static_cast<int>(threadIdx.x) < ntail)
     m = max(m, static_cast<uint32_t>(xtail[threadIdx.x]) & 0x7FFFu);
   const unsigned bits = grid_amax(m, ws, limit_ns, err);
-  if (bits == 0xFFFFFFFFu) return;
+  if (bits == 0xFFFFFFFFu) {
+    grid_depart(ws);
+    return;
+  }
   const float amax = __uint_as_float(bits);
   if (!(amax <= 3.402823466e38f)) {
     if (blockIdx.x == 0 && threadIdx.x == 0) {
       atomicExch(err, DEV_ERR_NONFINITE);
       *amax_out = amax;
     }
+    grid_depart(ws);
     return;
   }
   const float s = (amax == 0.0f) ? 1.0f : __fdiv_rn(amax, 448.0f);
@@ -330,21 +418,15 @@ __global__ void __launch_bounds__(FUSED_THREADS) k_calib_quant_fp8(
     *scale_out = s;
   }
   const float r = __frcp_rn(s);
-  if (markstein_ok(s)) {
-    for (size_t i = lo + threadIdx.x; i < hi; i += FUSED_THREADS) {
-      const uint4 a = __ldcs(xv + i);
-      __stcs(outv + i, make_uint2(quant4_e4m3<true>(a.x, a.y, s, r), quant4_e4m3<true>(a.z, a.w, s, r)));
-    }
-  } else {
-    for (size_t i = lo + threadIdx.x; i < hi; i += FUSED_THREADS) {
-      const uint4 a = __ldcs(xv + i);
-      __stcs(outv + i, make_uint2(quant4_e4m3<false>(a.x, a.y, s, r), quant4_e4m3<false>(a.z, a.w, s, r)));
-    }
-  }
+  if (markstein_ok(s))
+    chunk_quant_fp8<true>(xv, outv, lo, hi, s, r);
+  else
+    chunk_quant_fp8<false>(xv, outv, lo, hi, s, r);
   if (blockIdx.x == 0 && static_cast<int>(threadIdx.x) < ntail) {
     const float x = __uint_as_float(static_cast<uint32_t>(xtail[threadIdx.x]) << 16);
     outtail[threadIdx.x] = static_cast<uint8_t>(cvt_e4m3x2(__fdiv_rn(x, s), 0.0f) & 0xFFu);
   }
+  grid_depart(ws);
 }
 
 __global__ void __launch_bounds__(FUSED_THREADS) k_calib_quant_fp4_block(
@@ -355,20 +437,19 @@ __global__ void __launch_bounds__(FUSED_THREADS) k_calib_quant_fp4_block(
   const size_t per = (nblocks + gridDim.x - 1) / gridDim.x;   // contiguous chunk of blocks
   const size_t lo = static_cast<size_t>(blockIdx.x) * per;
   const size_t hi = lo + per < nblocks ? lo + per : nblocks;
-  uint32_t m2 = 0;
-  for (size_t i = 2 * lo + threadIdx.x; i < 2 * hi; i += FUSED_THREADS) {
-    const uint4 a = __ldg(xv + i);
-    m2 = absmax_word(m2, a.x); m2 = absmax_word(m2, a.y);
-    m2 = absmax_word(m2, a.z); m2 = absmax_word(m2, a.w);
-  }
+  const uint32_t m2 = chunk_absmax(xv, 2 * lo, 2 * hi);
   const unsigned bits = grid_amax(max(m2 & 0xFFFFu, m2 >> 16), ws, limit_ns, err);
-  if (bits == 0xFFFFFFFFu) return;
+  if (bits == 0xFFFFFFFFu) {
+    grid_depart(ws);
+    return;
+  }
   const float amax = __uint_as_float(bits);
   if (!(amax <= 3.402823466e38f)) {
     if (blockIdx.x == 0 && threadIdx.x == 0) {
       atomicExch(err, DEV_ERR_NONFINITE);
       *amax_out = amax;
     }
+    grid_depart(ws);
     return;
   }
   const float sg = (amax == 0.0f) ? 1.0f : __fdiv_rn(amax, 2688.0f);
@@ -381,9 +462,20 @@ __global__ void __launch_bounds__(FUSED_THREADS) k_calib_quant_fp4_block(
   }
   const float r8 = __frcp_rn(s8);
   const bool fast8 = markstein_ok(s8);
-  for (size_t b = lo + threadIdx.x; b < hi; b += FUSED_THREADS)
-    fp4_block(__ldcs(xv + 2 * b), __ldcs(xv + 2 * b + 1), b, sg, six_sg, s8, r8, fast8,
-              packed_out, bscale_out, codes8_out);
+  const uint64_t pol = l2_policy_evict_first();
+  size_t b = lo + threadIdx.x;
+  for (; b + FUSED_THREADS < hi; b += 2 * FUSED_THREADS) {     // two blocks' loads in flight
+    const uint4 a0 = ld_hint(xv + 2 * b, pol), a1 = ld_hint(xv + 2 * b + 1, pol);
+    const uint4 c0 = ld_hint(xv + 2 * (b + FUSED_THREADS), pol);
+    const uint4 c1 = ld_hint(xv + 2 * (b + FUSED_THREADS) + 1, pol);
+    fp4_block(a0, a1, b, sg, six_sg, s8, r8, fast8, packed_out, bscale_out, codes8_out);
+    fp4_block(c0, c1, b + FUSED_THREADS, sg, six_sg, s8, r8, fast8, packed_out, bscale_out,
+              codes8_out);
+  }
+  for (; b < hi; b += FUSED_THREADS)
+    fp4_block(ld_hint(xv + 2 * b, pol), ld_hint(xv + 2 * b + 1, pol), b, sg, six_sg, s8, r8,
+              fast8, packed_out, bscale_out, codes8_out);
+  grid_depart(ws);
 }
 
 // -------------------------------------------------------------------------------------------
