@@ -16,25 +16,22 @@
 //     E4M3 rounding commutes with power-of-two scaling in the normal range, so the result does
 //     not depend on how keys are tiled.
 //
-// Kernel structure: one CTA (one per SM) per pair of 128-row Q tiles of one (sequence, head);
-// keys advance in steps of BN = 64.
-//   warp 1      TMA producer: both Q tiles once, then K and V tiles through separate rings.
-//   warp 0      MMA issuer (one elected lane) and TMEM owner.  Each Q tile has two S buffers:
-//               once P_t(j) is in TMEM (written over S_t(j)) it issues O_t += P_t(j) V_j (A
-//               operand read from TMEM) and right behind it, in the same in-order tcgen05
-//               stream, S_t(j+2) = Q_t K_{j+2}^T into that buffer, so the scores of the next
-//               step are always computed while the softmax works on the current one.
-//   warps 2-17  softmax, eight per Q tile: two threads per query row (TMEM lane), each with
-//               half of the row's BN scores (16x32bx2 TMEM shapes), so every SM sub-partition
-//               interleaves four softmax warps.  Each takes the row max (3-input maxima and
-//               one shuffle) and computes p*448 = 2^(S' - M + log2 448) in FP32 (hardware ex2
-//               for most pairs, a degree-5 polynomial on the FMA pipe for the rest), sums p in
-//               packed f32x2 adds and converts to E4M3.  Once the previous P V has completed
-//               it rescales its half of the O row on a rise of M, then writes its half of
-//               P_t(j) with tcgen05.st.
-//   K/V tiles are read by TMA once per CTA for both Q tiles.
-// TMEM per Q tile: two S buffers (BN FP32 columns each; P of a step, 4 E4M3 per column, is
-// written over its first BN/4 columns) and O (D columns).
+// Kernel structure: one CTA (one per SM) per pair of 128-row Q tiles of one (sequence, head).
+//   warp 8      TMA producer: both Q tiles once, then K and V tiles through separate rings.
+//   warp 9      MMA issuer (one elected thread) and TMEM owner.  Per KV tile j and Q tile t it
+//               issues O_t += P_t(j) V_j (P read from tensor memory) and right behind it, in the
+//               same in-order tcgen05 stream, S_t = Q_t K_{j+1}^T into the columns P_t(j)
+//               occupied; one commit then tells softmax t that S_t(j+1) is ready and that O_t
+//               holds every P_t V up to tile j.
+//   warps 0-7   two softmax warpgroups, one per Q tile; thread = one query row = one TMEM lane.
+//               Each reads its 128 scores with tcgen05.ld, takes the row max (3-input maxima)
+//               and computes p*448 = 2^(S' - M + log2 448) in FP32 (hardware ex2 for most
+//               pairs, a degree-5 polynomial on the FMA pipe for the rest), sums p in packed
+//               f32x2 adds, converts to E4M3 and writes P_t(j) over S_t(j) with tcgen05.st.
+//               On a rise of M it first rescales its O row in TMEM by 2^-(rise).
+//   The two Q tiles alternate on the tensor pipe, so one tile's softmax overlaps the other
+//   tile's MMAs; K/V tiles are read by TMA once per CTA for both Q tiles.
+// TMEM: S_0/P_0, S_1/P_1 (128 FP32 columns each; P uses the first 32), O_0, O_1 (D columns).
 // All waits are bounded (a global-timer limit); on expiry the CTA records a timeout in the
 // library's error word, drains what it issued and exits.
 #include <cuda_runtime.h>
@@ -46,26 +43,16 @@
 namespace qattn {
 
 constexpr int BLOCK_M = 128;                 // query rows per tile (= TMEM lanes)
+constexpr int BLOCK_N = 128;                 // keys per KV tile
 constexpr int NQ = 2;                        // query tiles per CTA
-constexpr int KSTAGES = 6;
-constexpr int VSTAGES = 6;
-constexpr int NUM_SOFTMAX_WARPS = 8 * NQ;       // two warps per 32-lane quarter of each tile
-// The MMA issuer and the TMA producer are the lowest-numbered warps: the warp schedulers favour
-// older warps, and these two must not starve behind the four softmax warps of their sub-partition.
-constexpr int WARP_MMA = 0;
-constexpr int WARP_LOAD = 1;
-constexpr int FIRST_SOFTMAX_WARP = 2;
+constexpr int KSTAGES = 3;
+constexpr int VSTAGES = 3;
+constexpr int NUM_SOFTMAX_WARPS = 4 * NQ;
+constexpr int WARP_LOAD = NUM_SOFTMAX_WARPS;
+constexpr int WARP_MMA = NUM_SOFTMAX_WARPS + 1;
 constexpr int ATTN_THREADS = (NUM_SOFTMAX_WARPS + 2) * 32;
 constexpr float LOG2E_F = 1.4426950408889634f;
 constexpr float LOG2_448 = 8.807354922057604f;   // log2(448): p * 448 = 2^(S' - M + log2 448)
-
-// Keys per step.  Per Q tile TMEM holds two S buffers (the scores of step j+1 are computed
-// while the softmax works on step j; P of a step is written over its own S buffer) and O:
-// 2 * 64 + 128 = 256 columns for D = 128, so both tiles fill the 512 columns.
-template <int D>
-struct KvStep {
-  static constexpr int N = 64;
-};
 
 struct AttnArgs {
   int rows_per_slab;        // rows of one (b, h) slab in the tensor maps: L (dense) or T (varlen)
@@ -84,32 +71,28 @@ struct AttnArgs {
 
 template <int D>
 struct Smem {
-  static constexpr int BN = KvStep<D>::N;
   static constexpr int TILE_Q = BLOCK_M * D;       // bytes (E4M3)
-  static constexpr int TILE_KV = BN * D;
+  static constexpr int TILE_KV = BLOCK_N * D;
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_K = OFF_Q + NQ * TILE_Q;
   static constexpr int OFF_V = OFF_K + KSTAGES * TILE_KV;
   static constexpr int OFF_BAR = OFF_V + VSTAGES * TILE_KV;
-  // barriers: q_full, k_full[KS], k_empty[KS], v_full[VS], v_empty[VS], s_full[NQ][2],
-  // p_full[NQ][2], o_done[NQ][2], drain
-  static constexpr int NBARS = 1 + 2 * KSTAGES + 2 * VSTAGES + 6 * NQ + 1;
+  // barriers: q_full, k_full[KS], k_empty[KS], v_full[VS], v_empty[VS], s_full[NQ],
+  // p_full[NQ], o_final[NQ], drain
+  static constexpr int NBARS = 1 + 2 * KSTAGES + 2 * VSTAGES + 3 * NQ + 1;
   static constexpr int OFF_TMEM = OFF_BAR + 8 * NBARS;
   static constexpr int OFF_ABORT = OFF_TMEM + 4;
   static constexpr int BYTES = OFF_ABORT + 4;
   static constexpr int ALLOC = BYTES + 1024;       // slack for 1024-byte alignment
-  static_assert(TILE_Q % 1024 == 0 && TILE_KV % 1024 == 0, "1024-byte aligned tiles");
+  static_assert(TILE_Q % 1024 == 0 && TILE_KV % 1024 == 0, "alignment");
 };
 
 template <int D>
 struct TmemCols {
-  static constexpr int BN = KvStep<D>::N;
-  static constexpr uint32_t PER_TILE = 256;              // tile t uses [t * 256, t * 256 + 256)
-  static constexpr uint32_t S = 0;                       // buffer b: [b * BN, b * BN + BN);
-                                                         // P of that step: its first BN / 4
-  static constexpr uint32_t O = 256 - D;                 // D columns, ending at the tile's end
-  static constexpr uint32_t ALLOC = 512;
-  static_assert(2 * BN <= O, "S buffers and O of one tile overlap");
+  static constexpr uint32_t S0 = 0;                      // S_t / P_t at t * BLOCK_N
+  static constexpr uint32_t O0 = NQ * BLOCK_N;           // O_t at O0 + t * D
+  static constexpr uint32_t USED = NQ * BLOCK_N + NQ * D;
+  static constexpr uint32_t ALLOC = USED <= 256 ? 256 : 512;
 };
 
 __device__ __forceinline__ float exp2_int(int k) {       // 2^k for k <= 0, exact (0 below 2^-126)
@@ -128,94 +111,76 @@ __device__ __forceinline__ float max3f(float a, float b, float c) {   // sm_100 
   return d;
 }
 
-// Packed f32x2 helpers.  Pairs live in 64-bit registers; constant pairs are built once per
-// step (pair_of) so the inner loop issues only the arithmetic.
-__device__ __forceinline__ uint64_t pair_of(float lo, float hi) {
-  uint64_t r;
-  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
-  return r;
-}
-__device__ __forceinline__ void unpair(uint64_t p, float& lo, float& hi) {
-  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(p));
-}
-__device__ __forceinline__ uint64_t ffma2(uint64_t a, uint64_t b, uint64_t c) {
-  uint64_t d;
-  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
-  return d;
-}
-__device__ __forceinline__ uint64_t fadd2(uint64_t a, uint64_t b) {
-  uint64_t d;
-  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-  return d;
+// (d0, d1) = (a0 * b + c, a1 * b + c) with one packed f32x2 FMA.
+__device__ __forceinline__ void ffma2_bc(float& d0, float& d1, float a0, float a1, float b, float c) {
+  asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %4};\n\tmov.b64 rc, {%5, %5};\n\t"
+      "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d0), "=f"(d1)
+      : "f"(a0), "f"(a1), "f"(b), "f"(c));
 }
 
-// Four E4M3 codes in one word from four floats (first float in the low byte).
-__device__ __forceinline__ uint32_t pack4_e4m3(float a, float b, float c, float d) {
-  uint32_t r;
-  asm("{\n\t.reg .b16 lo, hi;\n\t"
-      "cvt.rn.satfinite.e4m3x2.f32 lo, %2, %1;\n\t"
-      "cvt.rn.satfinite.e4m3x2.f32 hi, %4, %3;\n\t"
-      "mov.b32 %0, {lo, hi};\n\t}"
-      : "=r"(r)
-      : "f"(a), "f"(b), "f"(c), "f"(d));
-  return r;
+// (s0, s1) += (a0, a1) with one packed f32x2 add.
+__device__ __forceinline__ void fadd2_acc(float& s0, float& s1, float a0, float a1) {
+  asm("{\n\t.reg .b64 ra, rs;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rs, {%0, %1};\n\t"
+      "add.f32x2 rs, rs, ra;\n\tmov.b64 {%0, %1}, rs;\n\t}"
+      : "+f"(s0), "+f"(s1)
+      : "f"(a0), "f"(a1));
 }
 
-// 2^x on the FMA pipe for two values at once, for x <= 9.  x is clamped at -125 (2^-125 is
-// far below the smallest E4M3 code of p * 448), split as x = n + f with n = round(x) (by
-// adding and subtracting 1.5 * 2^23) and f in [-1/2, 1/2]; 2^f comes from a degree-5 minimax
-// polynomial (relative error 2.1e-7 in binary32, fitted by csrc/fit_exp2_poly.py) and 2^n is
-// added into the exponent field.
+// 2^x on the FMA pipe for two values at once (packed f32x2), for x <= 9.  x is clamped at -125
+// (2^-125 is far below the smallest E4M3 code of p * 448), split as x = n + f with
+// n = round(x) (by adding and subtracting 1.5 * 2^23) and f in [-1/2, 1/2]; 2^f comes from a
+// degree-5 minimax polynomial (relative error 2.1e-7 in binary32, fitted by
+// csrc/fit_exp2_poly.py) and 2^n is added into the exponent field.
 #ifndef QATTN_POLY_PAIRS_PER_8
-#define QATTN_POLY_PAIRS_PER_8 1       // of every 8 pairs of scores, this many take the polynomial
+#define QATTN_POLY_PAIRS_PER_8 2       // of every 8 pairs of scores, this many take the polynomial
 #endif
-struct PolyConsts {
-  uint64_t magic, neg_magic, neg_one, c5, c4, c3, c2, c1, c0;
-  __device__ __forceinline__ PolyConsts()
-      : magic(pair_of(12582912.0f, 12582912.0f)),      // 1.5 * 2^23
-        neg_magic(pair_of(-12582912.0f, -12582912.0f)),
-        neg_one(pair_of(-1.0f, -1.0f)),
-        c5(pair_of(0x1.5c08e6p-10f, 0x1.5c08e6p-10f)),   // coefficients of the fit
-        c4(pair_of(0x1.3d0c52p-7f, 0x1.3d0c52p-7f)),
-        c3(pair_of(0x1.c6b6e4p-5f, 0x1.c6b6e4p-5f)),
-        c2(pair_of(0x1.ebf918p-3f, 0x1.ebf918p-3f)),
-        c1(pair_of(0x1.62e428p-1f, 0x1.62e428p-1f)),
-        c0(pair_of(0x1.000002p+0f, 0x1.000002p+0f)) {}
-};
-
-__device__ __forceinline__ uint64_t poly_exp2_x2(uint64_t x, const PolyConsts& k) {
-  float x0, x1;
-  unpair(x, x0, x1);
-  x = pair_of(fmaxf(x0, -125.0f), fmaxf(x1, -125.0f));
-  const uint64_t t = fadd2(x, k.magic);                 // n + 1.5 * 2^23, n = round(x)
-  const uint64_t n = fadd2(t, k.neg_magic);             // n (exact)
-  const uint64_t f = ffma2(n, k.neg_one, x);            // x - n (exact)
-  uint64_t p = ffma2(k.c5, f, k.c4);
-  p = ffma2(p, f, k.c3);
-  p = ffma2(p, f, k.c2);
-  p = ffma2(p, f, k.c1);
-  p = ffma2(p, f, k.c0);
-  // the low 9 bits of each half of t hold n (two's complement): shifted into the exponent
-  // field they add n
+__device__ __forceinline__ void poly_exp2_x2(float x0, float x1, float& y0, float& y1) {
+  x0 = fmaxf(x0, -125.0f);
+  x1 = fmaxf(x1, -125.0f);
   float p0, p1, t0, t1;
-  unpair(p, p0, p1);
-  unpair(t, t0, t1);
-  return pair_of(__int_as_float(__float_as_int(p0) + (__float_as_int(t0) << 23)),
-                 __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23)));
+  asm("{\n\t.reg .b64 x, t, n, f, p, m, nm, neg1, k;\n\t"
+      "mov.b64 x, {%4, %5};\n\t"
+      "mov.b64 m, {0f4B400000, 0f4B400000};\n\t"       // 1.5 * 2^23
+      "mov.b64 nm, {0fCB400000, 0fCB400000};\n\t"
+      "mov.b64 neg1, {0fBF800000, 0fBF800000};\n\t"
+      "add.rn.f32x2 t, x, m;\n\t"                       // t = n + 1.5 * 2^23, n = round(x)
+      "add.rn.f32x2 n, t, nm;\n\t"                      // n (exact)
+      "fma.rn.f32x2 f, n, neg1, x;\n\t"                 // f = x - n (exact)
+      "mov.b64 p, {0f3AAE0473, 0f3AAE0473};\n\t"        // c5
+      "mov.b64 k, {0f3C1E8629, 0f3C1E8629};\n\t"        // c4
+      "fma.rn.f32x2 p, p, f, k;\n\t"
+      "mov.b64 k, {0f3D635B72, 0f3D635B72};\n\t"        // c3
+      "fma.rn.f32x2 p, p, f, k;\n\t"
+      "mov.b64 k, {0f3E75FC8C, 0f3E75FC8C};\n\t"        // c2
+      "fma.rn.f32x2 p, p, f, k;\n\t"
+      "mov.b64 k, {0f3F317214, 0f3F317214};\n\t"        // c1
+      "fma.rn.f32x2 p, p, f, k;\n\t"
+      "mov.b64 k, {0f3F800001, 0f3F800001};\n\t"        // c0
+      "fma.rn.f32x2 p, p, f, k;\n\t"
+      "mov.b64 {%0, %1}, p;\n\t"
+      "mov.b64 {%2, %3}, t;\n\t}"
+      : "=f"(p0), "=f"(p1), "=f"(t0), "=f"(t1)
+      : "f"(x0), "f"(x1));
+  // the low 9 bits of t hold n (two's complement); shifted into the exponent field they add n
+  y0 = __int_as_float(__float_as_int(p0) + (__float_as_int(t0) << 23));
+  y1 = __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23));
 }
 
-// Row max of N scores (N a multiple of 16): 8 independent chains of 3-input maxima, then a
-// short tree.
-template <int N>
-__device__ __forceinline__ float rowmax(const float (&s)[N]) {
+// Row max of 128 scores: 8 independent chains of 3-input maxima, then a short tree.
+__device__ __forceinline__ float rowmax128(const float (&s)[128]) {
   float m[8];
 #pragma unroll
-  for (int k = 0; k < 8; ++k) m[k] = fmaxf(s[k], s[k + 8]);
+  for (int k = 0; k < 8; ++k) m[k] = max3f(s[k], s[k + 8], s[k + 16]);
 #pragma unroll
-  for (int i = 16; i + 16 <= N; i += 16) {
+  for (int i = 24; i < 120; i += 16) {
 #pragma unroll
     for (int k = 0; k < 8; ++k) m[k] = max3f(m[k], s[i + k], s[i + 8 + k]);
   }
+#pragma unroll
+  for (int k = 0; k < 8; ++k) m[k] = fmaxf(m[k], s[120 + k]);
   return max3f(max3f(m[0], m[1], m[2]), max3f(m[3], m[4], m[5]), fmaxf(m[6], m[7]));
 }
 
@@ -225,7 +190,6 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
                    const __grid_constant__ CUtensorMap tm_v, const AttnArgs args) {
   using SL = Smem<D>;
   using TC = TmemCols<D>;
-  constexpr int BN = KvStep<D>::N;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_u32 = smem_u32(smem_raw);
   const uint32_t base_u32 = (raw_u32 + 1023u) & ~1023u;
@@ -250,7 +214,7 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
   }
   const int q_row0 = qblk * (NQ * BLOCK_M);
   if (q_row0 >= seq_len) return;                  // uniform over the CTA: nothing to do
-  const int nkv = (seq_len + BN - 1) / BN;
+  const int nkv = (seq_len + BLOCK_N - 1) / BLOCK_N;
 
   // ---- barriers --------------------------------------------------------------------------
   const uint32_t bar0 = base_u32 + SL::OFF_BAR;
@@ -258,15 +222,8 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
   constexpr int B_QFULL = 0;
   constexpr int B_KFULL = 1, B_KEMPTY = B_KFULL + KSTAGES;
   constexpr int B_VFULL = B_KEMPTY + KSTAGES, B_VEMPTY = B_VFULL + VSTAGES;
-  constexpr int B_SFULL = B_VEMPTY + VSTAGES;     // B_SFULL + 2 * t + buffer
-  // Every per-step barrier exists once per S buffer (step j uses buffer j % 2 and phase j / 2):
-  // the softmax may run up to one step ahead of the MMA issuer and waits on o_done only when
-  // it rescales O (and before the epilogue), so one barrier per buffer keeps each waiter within
-  // one phase of its barrier.
-  constexpr int B_PFULL = B_SFULL + 2 * NQ;       // B_PFULL + 2 * t + buf
-  constexpr int B_ODONE = B_PFULL + 2 * NQ;       // B_ODONE + 2 * t + buf
-  constexpr int B_DRAIN = B_ODONE + 2 * NQ;
-  constexpr int TILE_WARPS = NUM_SOFTMAX_WARPS / NQ;   // one arrive per softmax warp
+  constexpr int B_SFULL = B_VEMPTY + VSTAGES, B_PFULL = B_SFULL + NQ;
+  constexpr int B_OFINAL = B_PFULL + NQ, B_DRAIN = B_OFINAL + NQ;
   volatile int* abort_flag = reinterpret_cast<volatile int*>(base + SL::OFF_ABORT);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base + SL::OFF_TMEM);
 
@@ -275,12 +232,9 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
     for (int i = 0; i < KSTAGES; ++i) { mbar_init(BAR(B_KFULL + i), 1); mbar_init(BAR(B_KEMPTY + i), 1); }
     for (int i = 0; i < VSTAGES; ++i) { mbar_init(BAR(B_VFULL + i), 1); mbar_init(BAR(B_VEMPTY + i), 1); }
     for (int t = 0; t < NQ; ++t) {
-      mbar_init(BAR(B_SFULL + 2 * t), 1);
-      mbar_init(BAR(B_SFULL + 2 * t + 1), 1);
-      mbar_init(BAR(B_PFULL + 2 * t), TILE_WARPS);
-      mbar_init(BAR(B_PFULL + 2 * t + 1), TILE_WARPS);
-      mbar_init(BAR(B_ODONE + 2 * t), 1);
-      mbar_init(BAR(B_ODONE + 2 * t + 1), 1);
+      mbar_init(BAR(B_SFULL + t), 1);
+      mbar_init(BAR(B_PFULL + t), BLOCK_M);
+      mbar_init(BAR(B_OFINAL + t), 1);
     }
     mbar_init(BAR(B_DRAIN), 1);
     *abort_flag = 0;
@@ -297,27 +251,24 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
   const uint64_t tlim = args.timeout_ns;
 
   if (warp == WARP_LOAD) {
-    // ======================= TMA producer (warp-wide loop, one elected lane issues) ============
-    const uint32_t leader = elect_one();
-    if (!args.inject_missing_q) {
-      if (leader) {
-        tma_prefetch_desc(&tm_q);
-        tma_prefetch_desc(&tm_k);
-        tma_prefetch_desc(&tm_v);
-      }
+    // ======================= TMA producer =======================
+    if (lane == 0 && !args.inject_missing_q) {
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v);
       int nk = 0, nv = 0;                          // loads issued
-      mbar_arrive_expect_tx_if(leader, BAR(B_QFULL), NQ * SL::TILE_Q);
+      mbar_arrive_expect_tx(BAR(B_QFULL), NQ * SL::TILE_Q);
       for (int t = 0; t < NQ; ++t)
-        tma_load_3d_if(leader, base_u32 + SL::OFF_Q + t * SL::TILE_Q, &tm_q, BAR(B_QFULL), 0,
-                       seq_start + q_row0 + t * BLOCK_M, slab);
+        tma_load_3d(base_u32 + SL::OFF_Q + t * SL::TILE_Q, &tm_q, BAR(B_QFULL), 0,
+                    seq_start + q_row0 + t * BLOCK_M, slab);
       auto load_k = [&](int j) -> bool {
         const int s = j % KSTAGES;
         if (j >= KSTAGES &&
             !mbar_wait(BAR(B_KEMPTY + s), ((j / KSTAGES) - 1) & 1, tlim, abort_flag, args.err))
           return false;
-        mbar_arrive_expect_tx_if(leader, BAR(B_KFULL + s), SL::TILE_KV);
-        tma_load_3d_if(leader, base_u32 + SL::OFF_K + s * SL::TILE_KV, &tm_k, BAR(B_KFULL + s), 0,
-                       seq_start + j * BN, slab);
+        mbar_arrive_expect_tx(BAR(B_KFULL + s), SL::TILE_KV);
+        tma_load_3d(base_u32 + SL::OFF_K + s * SL::TILE_KV, &tm_k, BAR(B_KFULL + s), 0,
+                    seq_start + j * BLOCK_N, slab);
         ++nk;
         return true;
       };
@@ -326,19 +277,17 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
         if (j >= VSTAGES &&
             !mbar_wait(BAR(B_VEMPTY + s), ((j / VSTAGES) - 1) & 1, tlim, abort_flag, args.err))
           return false;
-        mbar_arrive_expect_tx_if(leader, BAR(B_VFULL + s), SL::TILE_KV);
-        tma_load_3d_if(leader, base_u32 + SL::OFF_V + s * SL::TILE_KV, &tm_v, BAR(B_VFULL + s), 0,
-                       seq_start + j * BN, slab);
+        mbar_arrive_expect_tx(BAR(B_VFULL + s), SL::TILE_KV);
+        tma_load_3d(base_u32 + SL::OFF_V + s * SL::TILE_KV, &tm_v, BAR(B_VFULL + s), 0,
+                    seq_start + j * BLOCK_N, slab);
         ++nv;
         return true;
       };
-      // order of use on the tensor pipe: K0, K1, V0, K2, V1, K3, ...: K runs two steps ahead
+      // order of use on the tensor pipe: K0, V0, K1, V1, ...; K runs one tile ahead
       bool ok = load_k(0);
-      if (ok && nkv > 1) ok = load_k(1);
       for (int j = 0; ok && j < nkv; ++j) {
-        ok = load_v(j);
-        if (ok && j + 2 < nkv) ok = load_k(j + 2);
-        ok = __all_sync(0xFFFFFFFFu, ok);
+        if (j + 1 < nkv) ok = load_k(j + 1);
+        if (ok) ok = load_v(j);
       }
       // drain: every issued load has landed before the CTA may exit (instant when healthy)
       mbar_drain(BAR(B_QFULL), 0, tlim);
@@ -348,225 +297,183 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
         mbar_drain(BAR(B_VFULL + j % VSTAGES), (j / VSTAGES) & 1, tlim);
     }
   } else if (warp == WARP_MMA) {
-    // ======================= MMA issuer (warp-wide loop, one elected lane issues) =============
-    const uint32_t leader = elect_one();
-    constexpr uint32_t IDESC_S = idesc_e4m3_f32(BLOCK_M, BN, false);
-    constexpr uint32_t IDESC_O = idesc_e4m3_f32(BLOCK_M, D, true);
-    // Q, K: K-major rows of D bytes, swizzled in 8-row atoms (SBO = 8 rows); 32-byte K steps.
-    constexpr uint32_t QK_LAYOUT = (D == 128) ? 2u : 4u;   // 128B / 64B swizzle
-    constexpr uint32_t QK_SBO = 8 * D;
-    // V: MN-major (D contiguous per key row), rows of D bytes, SBO = 8 key rows; a K step of
-    // 32 keys advances 32 rows.
-    constexpr uint32_t V_LAYOUT = QK_LAYOUT;
-    constexpr uint32_t V_SBO = 8 * D;
-    // Descriptors are built once; a step only adds (address >> 4) offsets to the low bits.
-    const uint64_t desc_q0 = smem_desc(base_u32 + SL::OFF_Q, 16, QK_SBO, QK_LAYOUT);
-    const uint64_t desc_k0 = smem_desc(base_u32 + SL::OFF_K, 16, QK_SBO, QK_LAYOUT);
-    const uint64_t desc_v0 = smem_desc(base_u32 + SL::OFF_V, SL::TILE_KV, V_SBO, V_LAYOUT);
-    auto bmm1 = [&](int t, int ks, int buf) {       // S_t(buffer) = Q_t K^T
-      const uint64_t da = desc_q0 + static_cast<uint64_t>((t * SL::TILE_Q) >> 4);
-      const uint64_t db = desc_k0 + static_cast<uint64_t>((ks * SL::TILE_KV) >> 4);
-      const uint32_t d_tmem = tmem + t * TC::PER_TILE + TC::S + buf * BN;
+    // ======================= MMA issuer =======================
+    if (lane == 0) {
+      constexpr uint32_t IDESC_S = idesc_e4m3_f32(BLOCK_M, BLOCK_N, false);
+      constexpr uint32_t IDESC_O = idesc_e4m3_f32(BLOCK_M, D, true);
+      // Q, K: K-major rows of D bytes, swizzled in 8-row atoms (SBO = 8 rows); 32-byte K steps.
+      constexpr uint32_t QK_LAYOUT = (D == 128) ? 2u : 4u;   // 128B / 64B swizzle
+      constexpr uint32_t QK_SBO = 8 * D;
+      // V: MN-major (D contiguous per key row), rows of D bytes, SBO = 8 key rows; a K step
+      // of 32 keys advances 32 rows.
+      constexpr uint32_t V_LAYOUT = QK_LAYOUT;
+      constexpr uint32_t V_SBO = 8 * D;
+      auto bmm1 = [&](int t, int ks) {
+        const uint32_t qa = base_u32 + SL::OFF_Q + t * SL::TILE_Q;
+        const uint32_t kb = base_u32 + SL::OFF_K + ks * SL::TILE_KV;
 #pragma unroll
-      for (int kk = 0; kk < D / 32; ++kk)
-        mma_f8_ss_if(leader, d_tmem, da + kk * 2, db + kk * 2, IDESC_S, kk > 0 ? 1u : 0u);
-    };
-    auto bmm2 = [&](int t, int vs, int buf, bool first) {   // O_t += P_t(buffer) V
-      const uint64_t db = desc_v0 + static_cast<uint64_t>((vs * SL::TILE_KV) >> 4);
-      const uint32_t d_tmem = tmem + t * TC::PER_TILE + TC::O;
-      const uint32_t a_tmem = tmem + t * TC::PER_TILE + TC::S + buf * BN;
+        for (int kk = 0; kk < D / 32; ++kk) {
+          const uint64_t da = smem_desc(qa + kk * 32, 16, QK_SBO, QK_LAYOUT);
+          const uint64_t db = smem_desc(kb + kk * 32, 16, QK_SBO, QK_LAYOUT);
+          mma_f8_ss(tmem + TC::S0 + t * BLOCK_N, da, db, IDESC_S, kk > 0 ? 1u : 0u);
+        }
+      };
+      auto bmm2 = [&](int t, int vs, bool first) {
+        const uint32_t vb = base_u32 + SL::OFF_V + vs * SL::TILE_KV;
 #pragma unroll
-      for (int kk = 0; kk < BN / 32; ++kk)
-        mma_f8_ts_if(leader, d_tmem, a_tmem + kk * 8, db + static_cast<uint64_t>((kk * 32 * D) >> 4),
-                     IDESC_O, (!first || kk > 0) ? 1u : 0u);
-    };
-    // S of steps 0 and 1 into the two buffers of each tile.
-    bool ok = mbar_wait(BAR(B_QFULL), 0, tlim, abort_flag, args.err);
-    for (int jj = 0; jj < 2 && jj < nkv; ++jj) {
-      ok = ok && mbar_wait(BAR(B_KFULL + jj), 0, tlim, abort_flag, args.err);
-      ok = __all_sync(0xFFFFFFFFu, ok);
-      if (!ok) break;
-      tc_fence_after();
-      for (int t = 0; t < NQ; ++t) {
-        bmm1(t, jj, jj);
-        mma_commit_if(leader, BAR(B_SFULL + 2 * t + jj));
-      }
-      mma_commit_if(leader, BAR(B_KEMPTY + jj));
-    }
-    // Step j: O_t += P_t(j) V_j, then S_t(j+2) into the buffer P_t(j) occupied (the in-order
-    // tcgen05 stream reads P before it is overwritten).
-    for (int j = 0; ok && j < nkv; ++j) {
-      const int vs = j % VSTAGES;
-      const int buf = j & 1;
-      const bool more = j + 2 < nkv;
-      const int ks = (j + 2) % KSTAGES;
-      ok = mbar_wait(BAR(B_VFULL + vs), (j / VSTAGES) & 1, tlim, abort_flag, args.err);
-      if (ok && more)
-        ok = mbar_wait(BAR(B_KFULL + ks), ((j + 2) / KSTAGES) & 1, tlim, abort_flag, args.err);
-      for (int t = 0; ok && t < NQ; ++t) {
-        ok = mbar_wait(BAR(B_PFULL + 2 * t + buf), (j >> 1) & 1, tlim, abort_flag, args.err);
-        if (!__all_sync(0xFFFFFFFFu, ok)) { ok = false; break; }
+        for (int kk = 0; kk < BLOCK_N / 32; ++kk) {
+          const uint64_t db = smem_desc(vb + kk * 32 * D, SL::TILE_KV, V_SBO, V_LAYOUT);
+          mma_f8_ts(tmem + TC::O0 + t * D, tmem + TC::S0 + t * BLOCK_N + kk * 8, db, IDESC_O,
+                    (!first || kk > 0) ? 1u : 0u);
+        }
+      };
+      bool ok = mbar_wait(BAR(B_QFULL), 0, tlim, abort_flag, args.err) &&
+                mbar_wait(BAR(B_KFULL + 0), 0, tlim, abort_flag, args.err);
+      if (ok) {
         tc_fence_after();
-        bmm2(t, vs, buf, j == 0);
-        mma_commit_if(leader, BAR(B_ODONE + 2 * t + buf));
-        if (more) {
-          bmm1(t, ks, buf);
-          mma_commit_if(leader, BAR(B_SFULL + 2 * t + buf));
+        for (int t = 0; t < NQ; ++t) {
+          bmm1(t, 0);
+          mma_commit(BAR(B_SFULL + t));
+        }
+        mma_commit(BAR(B_KEMPTY + 0));
+      }
+      for (int j = 0; ok && j < nkv; ++j) {
+        const int vs = j % VSTAGES;
+        const bool more = j + 1 < nkv;
+        const int ks = (j + 1) % KSTAGES;
+        ok = mbar_wait(BAR(B_VFULL + vs), (j / VSTAGES) & 1, tlim, abort_flag, args.err);
+        if (ok && more)
+          ok = mbar_wait(BAR(B_KFULL + ks), ((j + 1) / KSTAGES) & 1, tlim, abort_flag, args.err);
+        for (int t = 0; ok && t < NQ; ++t) {
+          ok = mbar_wait(BAR(B_PFULL + t), j & 1, tlim, abort_flag, args.err);
+          if (!ok) break;
+          tc_fence_after();
+          bmm2(t, vs, j == 0);                     // reads P_t(j) from TMEM
+          if (more) {
+            bmm1(t, ks);                           // overwrites S_t / P_t after bmm2 read it
+            mma_commit(BAR(B_SFULL + t));
+          } else {
+            mma_commit(BAR(B_OFINAL + t));
+          }
+        }
+        if (ok) {
+          mma_commit(BAR(B_VEMPTY + vs));
+          if (more) mma_commit(BAR(B_KEMPTY + ks));
         }
       }
-      ok = __all_sync(0xFFFFFFFFu, ok);
-      if (ok) {
-        mma_commit_if(leader, BAR(B_VEMPTY + vs));
-        if (more) mma_commit_if(leader, BAR(B_KEMPTY + ks));
-      }
+      // drain: all issued MMAs complete before TMEM is released
+      mma_commit(BAR(B_DRAIN));
+      mbar_drain(BAR(B_DRAIN), 0, tlim);
     }
-    // drain: all issued MMAs complete before TMEM is released
-    mma_commit_if(leader, BAR(B_DRAIN));
-    mbar_drain(BAR(B_DRAIN), 0, tlim);
   } else {
-    // ======================= softmax warps =======================
-    // Softmax warp w (index i = w - 2) handles tile t = (i / 4) % 2, TMEM lane quarter w % 4
-    // (the quarter its SM sub-partition may access) and, within it, 16 lanes (i / 8 selects
-    // which); with the
-    // 16x32bx2 TMEM shapes, lanes 0-15 of the warp take the first half of every row's columns
-    // and lanes 16-31 the second half, so a row's max and sum combine with one shuffle and
-    // each sub-partition runs four softmax warps.
-    constexpr int HN = BN / 2;                     // scores per thread and step
-    constexpr int HD = D / 2;                      // O columns per thread
-    const int si = warp - FIRST_SOFTMAX_WARP;      // 0..15; quarter, tile and half are unique
-    const int quarter = warp & 3;
-    const int t = (si >> 2) & 1;
-    const int hs = si >> 3;
-    const int ch = lane >> 4;                      // column half
-    const int r = quarter * 32 + hs * 16 + (lane & 15);   // row within the Q tile
-    const uint32_t trow = tmem + (static_cast<uint32_t>(quarter * 32 + hs * 16) << 16) +
-                          t * TC::PER_TILE;
-    const uint32_t tO = trow + TC::O;
+    // ======================= softmax warpgroups =======================
+    const int t = warp >> 2;                       // Q tile of this warpgroup
+    const int quarter = warp & 3;                  // TMEM lane quarter
+    const int r = quarter * 32 + lane;             // row within the Q tile
+    const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+    const uint32_t tS = tmem + lane_off + TC::S0 + t * BLOCK_N;
+    const uint32_t tO = tmem + lane_off + TC::O0 + t * D;
     const float c = __ldg(args.s_q) * __ldg(args.s_k) * args.sm_scale * LOG2E_F;
-    const PolyConsts pk_consts;
     float m_run = -INFINITY;                       // integer-valued running max (base 2)
-    float l = 0.0f;                                // this thread's share of the sum of p * 448
+    float l = 0.0f;                                // running sum of p * 448
     bool ok = true;
-    auto load_o = [&](uint32_t (&v)[HD]) {
-#pragma unroll
-      for (int c4 = 0; c4 < HD / 32; ++c4) tmem_ld16x2_x32<HD>(tO + c4 * 32, v + c4 * 32);
-      tmem_wait_ld();
-    };
     for (int j = 0; j < nkv; ++j) {
-      const uint32_t tS = trow + TC::S + (j & 1) * BN;   // S_t(j); later P_t(j)
-      ok = mbar_wait(BAR(B_SFULL + 2 * t + (j & 1)), (j >> 1) & 1, tlim, abort_flag, args.err);
+      // S_t(j) is in TMEM; BMM2 of tile j-1 has completed (it precedes in the MMA stream)
+      ok = mbar_wait(BAR(B_SFULL + t), j & 1, tlim, abort_flag, args.err);
       if (!__all_sync(0xFFFFFFFFu, ok)) { ok = false; break; }
       tc_fence_after();
-      float s[HN];
+      float s[BLOCK_N];
       {
-        uint32_t sv[HN];
-        if constexpr (HN % 32 == 0) {
+        uint32_t sv[BLOCK_N / 32][32];
 #pragma unroll
-          for (int c4 = 0; c4 < HN / 32; ++c4) tmem_ld16x2_x32<HN>(tS + c4 * 32, sv + c4 * 32);
-        } else {
-#pragma unroll
-          for (int c4 = 0; c4 < HN / 16; ++c4) tmem_ld16x2_x16<HN>(tS + c4 * 16, sv + c4 * 16);
-        }
+        for (int c4 = 0; c4 < BLOCK_N / 32; ++c4) tmem_ld32(tS + c4 * 32, sv[c4]);
         tmem_wait_ld();
 #pragma unroll
-        for (int i = 0; i < HN; ++i) s[i] = __uint_as_float(sv[i]);
+        for (int i = 0; i < BLOCK_N; ++i) s[i] = __uint_as_float(sv[i / 32][i % 32]);
       }
-      const int kv_valid = seq_len - j * BN - ch * HN;   // this thread's keys inside the sequence
-      if (kv_valid < HN) {
+      const int kv_valid = seq_len - j * BLOCK_N;  // keys of this tile inside the sequence
+      if (kv_valid < BLOCK_N) {
 #pragma unroll
-        for (int i = 0; i < HN; ++i)
+        for (int i = 0; i < BLOCK_N; ++i)
           if (i >= kv_valid) s[i] = -INFINITY;
       }
-      float mx = rowmax<HN>(s);
-      mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, 16));
-      const float m_new = fmaxf(m_run, ceilf(mx * c));
+      const float m_new = fmaxf(m_run, ceilf(rowmax128(s) * c));
       const float neg_off = LOG2_448 - m_new;
-      const uint64_t c2 = pair_of(c, c), off2 = pair_of(neg_off, neg_off);
-      uint64_t acc[4] = {0, 0, 0, 0};             // four pairs of partial sums (0.0f bits)
-      uint32_t pk[HN / 4];
+      float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      uint32_t pk[BLOCK_N / 4];
 #pragma unroll
-      for (int i = 0; i < HN; i += 16) {
+      for (int i = 0; i < BLOCK_N; i += 16) {
         float p[16];
 #pragma unroll
         for (int q = 0; q < 8; ++q) {
-          const uint64_t x = ffma2(pair_of(s[i + 2 * q], s[i + 2 * q + 1]), c2, off2);
-          uint64_t pp;
+          float x0, x1;
+          ffma2_bc(x0, x1, s[i + 2 * q], s[i + 2 * q + 1], c, neg_off);
           if (q < QATTN_POLY_PAIRS_PER_8) {
-            pp = poly_exp2_x2(x, pk_consts);
+            poly_exp2_x2(x0, x1, p[2 * q], p[2 * q + 1]);
           } else {
-            float x0, x1;
-            unpair(x, x0, x1);
-            pp = pair_of(fast_exp2(x0), fast_exp2(x1));
+            p[2 * q] = fast_exp2(x0);
+            p[2 * q + 1] = fast_exp2(x1);
           }
-          acc[q & 3] = fadd2(acc[q & 3], pp);
-          unpair(pp, p[2 * q], p[2 * q + 1]);
         }
 #pragma unroll
+        for (int q = 0; q < 8; ++q) fadd2_acc(acc[2 * (q & 3)], acc[2 * (q & 3) + 1], p[2 * q], p[2 * q + 1]);
+#pragma unroll
         for (int q = 0; q < 4; ++q)
-          pk[i / 4 + q] = pack4_e4m3(p[4 * q], p[4 * q + 1], p[4 * q + 2], p[4 * q + 3]);
+          pk[i / 4 + q] = cvt_e4m3x2(p[4 * q], p[4 * q + 1]) | (cvt_e4m3x2(p[4 * q + 2], p[4 * q + 3]) << 16);
       }
-      float r0, r1, r2, r3, r4, r5, r6, r7;
-      unpair(acc[0], r0, r1);
-      unpair(acc[1], r2, r3);
-      unpair(acc[2], r4, r5);
-      unpair(acc[3], r6, r7);
-      const float rowsum = ((r0 + r1) + (r2 + r3)) + ((r4 + r5) + (r6 + r7));
-      // A rise of the running max rescales this row of O by 2^-(rise); O must be quiescent, so
-      // that (rare) case first waits for the previous P V.  P_t(j) itself goes to the buffer
-      // that P V of step j-1 does not read, so the common case does not wait at all.
-      const bool rise = j > 0 && m_new > m_run;   // same value in both threads of a row
-      if (__any_sync(0xFFFFFFFFu, rise)) {
-        ok = mbar_wait(BAR(B_ODONE + 2 * t + ((j - 1) & 1)), ((j - 1) >> 1) & 1, tlim, abort_flag,
-                       args.err);
-        if (!__all_sync(0xFFFFFFFFu, ok)) { ok = false; break; }
-        tc_fence_after();
-        const float f = rise ? exp2_int(static_cast<int>(m_run - m_new)) : 1.0f;
-        uint32_t v[HD];
-        load_o(v);
+      const float rowsum = ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
+      // A rise of the running max rescales this row of O (quiescent: its last BMM2 is done).
+      if (j > 0) {
+        const bool rise = m_new > m_run;
+        if (__any_sync(0xFFFFFFFFu, rise)) {
+          const float f = rise ? exp2_int(static_cast<int>(m_run - m_new)) : 1.0f;
 #pragma unroll
-        for (int i = 0; i < HD; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) * f);
+          for (int c4 = 0; c4 < D / 32; ++c4) {
+            uint32_t v[32];
+            tmem_ld32(tO + c4 * 32, v);
+            tmem_wait_ld();
 #pragma unroll
-        for (int c4 = 0; c4 < HD / 32; ++c4) tmem_st16x2_x32<HD>(tO + c4 * 32, v + c4 * 32);
-        l *= f;
+            for (int i = 0; i < 32; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) * f);
+            tmem_st32(tO + c4 * 32, v);
+          }
+          l *= f;
+        }
       }
       l += rowsum;
       m_run = m_new;
-      // P_t(j) over the first BN/4 columns of its S buffer: column c holds keys 4c..4c+3
-      // (byte = key % 4); this thread's keys start at column ch * HN / 4
-      static_assert(HN == 32, "P store covers 32 keys per thread");
-      tmem_st16x2_x8<8>(tS, pk);
+      // P_t(j) over the first 32 columns of S_t: column c holds keys 4c..4c+3 (byte = key % 4)
+      tmem_st32(tS, pk);
       tmem_wait_st();
       tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(BAR(B_PFULL + 2 * t + (j & 1)));
+      mbar_arrive(BAR(B_PFULL + t));
     }
     if (ok) {
-      // P V of the last step completes after every earlier one (in-order tcgen05 stream)
-      ok = mbar_wait(BAR(B_ODONE + 2 * t + ((nkv - 1) & 1)), ((nkv - 1) >> 1) & 1, tlim,
-                     abort_flag, args.err);
-      const float l_row = l + __shfl_xor_sync(0xFFFFFFFFu, l, 16);
+      ok = mbar_wait(BAR(B_OFINAL + t), 0, tlim, abort_flag, args.err);
       if (__all_sync(0xFFFFFFFFu, ok)) {
         tc_fence_after();
         const int row = q_row0 + t * BLOCK_M + r;
         const bool valid = row < seq_len;
-        const float scale = __ldg(args.s_v) / l_row;   // O = acc * s_v / 448 / (l / 448)
-        uint32_t v[HD];
-        load_o(v);
-        __nv_bfloat16* orow = args.out +
-                              (static_cast<size_t>(slab) * args.rows_per_slab + seq_start + row) * D +
-                              ch * HD;
-        uint32_t packed[HD / 2];
+        const float scale = __ldg(args.s_v) / l;   // O = acc * s_v / 448 / (l / 448)
+        __nv_bfloat16* orow =
+            args.out + (static_cast<size_t>(slab) * args.rows_per_slab + seq_start + row) * D;
 #pragma unroll
-        for (int i = 0; i < HD / 2; ++i) {
-          const __nv_bfloat162 b2 = __floats2bfloat162_rn(__uint_as_float(v[2 * i]) * scale,
-                                                          __uint_as_float(v[2 * i + 1]) * scale);
-          packed[i] = *reinterpret_cast<const uint32_t*>(&b2);
-        }
-        if (valid) {
-          uint4* dst = reinterpret_cast<uint4*>(orow);
+        for (int c4 = 0; c4 < D / 32; ++c4) {
+          uint32_t v[32];
+          tmem_ld32(tO + c4 * 32, v);
+          tmem_wait_ld();
+          uint32_t packed[16];
 #pragma unroll
-          for (int i = 0; i < HD / 8; ++i)
-            dst[i] = make_uint4(packed[4 * i], packed[4 * i + 1], packed[4 * i + 2], packed[4 * i + 3]);
+          for (int i = 0; i < 16; ++i) {
+            const __nv_bfloat162 b2 = __floats2bfloat162_rn(__uint_as_float(v[2 * i]) * scale,
+                                                            __uint_as_float(v[2 * i + 1]) * scale);
+            packed[i] = *reinterpret_cast<const uint32_t*>(&b2);
+          }
+          if (valid) {
+            uint4* dst = reinterpret_cast<uint4*>(orow + c4 * 32);
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+              dst[i] = make_uint4(packed[4 * i], packed[4 * i + 1], packed[4 * i + 2], packed[4 * i + 3]);
+          }
         }
       }
     }
@@ -601,15 +508,15 @@ static EncodeTiledFn get_encode_fn() {
   return fn;
 }
 
-// 3-D map over an E4M3 tensor viewed as [slabs][rows][D]: box = `box_rows` rows of one slab.
-static bool make_map(CUtensorMap* map, const void* ptr, int D, int rows, int slabs, int box_rows) {
+// 3-D map over an E4M3 tensor viewed as [slabs][rows][D]: box = one 128-row tile of one slab.
+static bool make_map(CUtensorMap* map, const void* ptr, int D, int rows, int slabs) {
   EncodeTiledFn enc = get_encode_fn();
   if (!enc) return false;
   cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(rows),
                         static_cast<cuuint64_t>(slabs)};
   cuuint64_t strides[2] = {static_cast<cuuint64_t>(D),
                            static_cast<cuuint64_t>(D) * static_cast<cuuint64_t>(rows)};
-  cuuint32_t box[3] = {static_cast<cuuint32_t>(D), static_cast<cuuint32_t>(box_rows), 1u};
+  cuuint32_t box[3] = {static_cast<cuuint32_t>(D), 128u, 1u};
   cuuint32_t estr[3] = {1u, 1u, 1u};
   CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(ptr), dims, strides,
                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
@@ -622,10 +529,8 @@ template <int D>
 static cudaError_t launch_attn_d(const void* q8, const void* k8, const void* v8, const AttnArgs& a,
                                  int rows_per_slab, int slabs, dim3 grid, cudaStream_t stream) {
   CUtensorMap mq, mk, mv;
-  constexpr int BN = KvStep<D>::N;
-  if (!make_map(&mq, q8, D, rows_per_slab, slabs, BLOCK_M) ||
-      !make_map(&mk, k8, D, rows_per_slab, slabs, BN) ||
-      !make_map(&mv, v8, D, rows_per_slab, slabs, BN))
+  if (!make_map(&mq, q8, D, rows_per_slab, slabs) || !make_map(&mk, k8, D, rows_per_slab, slabs) ||
+      !make_map(&mv, v8, D, rows_per_slab, slabs))
     return cudaErrorInvalidValue;
   static int configured_dev_mask = 0;   // bit per device id < 31
   int dev = 0;
