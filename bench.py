@@ -33,6 +33,13 @@ HBM_FALLBACK_GBS = 6650.0
 BF16_FALLBACK_TFLOPS = 1590.0
 FP8_PER_BF16 = 2.0          # nominal dense FP8 / BF16 tensor throughput ratio on B200
 L2_FLUSH_BYTES = 256 << 20
+# DRAM bytes (read + write) of one attention launch, from ncu on this build's kernel:
+#   ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum --clock-control none \
+#       -k regex:k_attn -s 3 -c 1 python bench.py --steps 3 --warmup 3 --no-cpu-baseline --no-e2e
+# 80.57 MB read (Q8 + K8 + V8 = 80.22 MB algorithmic) + 16.40 MB written (the rest of the
+# 53.5 MB bf16 output is still in L2 when the kernel ends).  Re-capture when the kernel changes.
+ATTN_TRAFFIC_BYTES = {(8704, 24, 128): 80.57e6 + 16.40e6}
+ATTN_TRAFFIC_SOURCE = "ncu dram__bytes_read.sum + dram__bytes_write.sum, one launch, L=8704"
 
 
 def load_peaks():
@@ -216,26 +223,60 @@ def run_gpu(args):
 
 
 def e2e_time(args, w, q, k, v, qd, kd, vd, step, flush, stream, world):
-    """Same step through the C ABI with pinned host buffers; copies inside the timed region."""
+    """The whole path through the public API with the bf16 inputs in pinned host memory: every
+    step copies its Q, K, V host->device, runs calibrate+quantize and attention, and copies the
+    output back.  Steps are pipelined as a serving loop would run them: the host->device copies,
+    the compute and the device->host copy of consecutive steps run on three streams over two
+    sets of device buffers, so step i's upload overlaps step i-1's compute and download.  Timed
+    with events from the first upload to the last download; no L2 flush is needed since every
+    step writes 160 MB of fresh input (more than the L2) into HBM."""
+    import precision_quantized_attention_b200 as qa
     qh, kh, vh = (t.pin_memory() for t in (q, k, v))
-    oh = torch.empty(w.shape, dtype=torch.bfloat16).pin_memory()
-    e2e_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
-    for _ in range(2):
-        qd.copy_(qh, non_blocking=True); kd.copy_(kh, non_blocking=True); vd.copy_(vh, non_blocking=True)
-        oh.copy_(step(), non_blocking=True)
-    torch.cuda.synchronize()
+    ohs = [torch.empty(w.shape, dtype=torch.bfloat16).pin_memory() for _ in range(2)]
+    paths = [qa.QuantizedAttention(w.shape, w.mode, sm_scale=w.sm_scale) for _ in range(2)]
+    ins = [(qd, kd, vd), tuple(torch.empty_like(t) for t in (qd, kd, vd))]
+    h2d, d2h = torch.cuda.Stream(), torch.cuda.Stream()
+
+    def run(n):
+        ev = lambda: torch.cuda.Event(enable_timing=True)
+        start, end = ev(), ev()
+        quant_done, comp_done, down_done = [None] * n, [None] * n, [None] * n
+        start.record(h2d)
+        for i in range(n):
+            b = i % 2
+            with torch.cuda.stream(h2d):
+                if i >= 2:
+                    h2d.wait_event(quant_done[i - 2])      # slot b's inputs are consumed
+                for dst, src in zip(ins[b], (qh, kh, vh)):
+                    dst.copy_(src, non_blocking=True)
+                up = ev()
+                up.record(h2d)
+            stream.wait_event(up)
+            if i >= 2:
+                stream.wait_event(down_done[i - 2])       # slot b's output was downloaded
+            paths[b].quantize(*ins[b], stream)
+            quant_done[i] = ev()
+            quant_done[i].record(stream)
+            paths[b].attend(stream)
+            comp_done[i] = ev()
+            comp_done[i].record(stream)
+            with torch.cuda.stream(d2h):
+                d2h.wait_event(comp_done[i])
+                ohs[b].copy_(paths[b].out, non_blocking=True)
+                down_done[i] = ev()
+                down_done[i].record(d2h)
+        end.record(d2h)
+        torch.cuda.synchronize()
+        return start.elapsed_time(end) / n
+
+    run(max(2, args.warmup))
     barrier(world)
-    for i in range(args.steps):
-        flush()
-        e2e_ev[i][0].record(stream)
-        qd.copy_(qh, non_blocking=True)
-        kd.copy_(kh, non_blocking=True)
-        vd.copy_(vh, non_blocking=True)
-        oh.copy_(step(), non_blocking=True)
-        e2e_ev[i][1].record(stream)
-    torch.cuda.synchronize()
+    ms = run(args.steps)
+    status = qa.get_error()
+    if status != 0:
+        raise RuntimeError(f"device error {status} in the end-to-end run")
     barrier(world)
-    return max_over_ranks(sum(a.elapsed_time(b) for a, b in e2e_ev) / args.steps, world)
+    return max_over_ranks(ms, world)
 
 
 def report(args, w, qkv, rank, world, ms, attn, quant, e2e_ms, clocks):
@@ -273,7 +314,9 @@ def report(args, w, qkv, rank, world, ms, attn, quant, e2e_ms, clocks):
                          "256 MiB read of another buffer so the write's dirty lines are "
                          "written back before the step starts"},
         "roofline": {"bound": "tensor", "achieved": achieved_tf, "peak": fp8_peak,
-                     "unit": "TFLOP/s", "frac": achieved_tf / fp8_peak, "traffic": None,
+                     "unit": "TFLOP/s", "frac": achieved_tf / fp8_peak,
+                     "traffic": ATTN_TRAFFIC_BYTES.get((w.L, w.H, w.D)),
+                     "traffic_source": ATTN_TRAFFIC_SOURCE,
                      "kernel": f"k_attn_fp8_fwd<{w.D}>",
                      "peak_source": f"{peak_kind} bf16 burst {bf16_tf} TFLOP/s x {FP8_PER_BF16} "
                                     "(nominal FP8/BF16 ratio)",
@@ -284,7 +327,10 @@ def report(args, w, qkv, rank, world, ms, attn, quant, e2e_ms, clocks):
                      "hbm_peak_gbs": hbm_gbs, "launches": 3},
         "e2e": {"value": world * flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
                 "ms_per_step": e2e_ms, "h2d_bytes_per_step": in_bytes,
-                "d2h_bytes_per_step": q.numel() * 2},
+                "d2h_bytes_per_step": q.numel() * 2,
+                "schedule": "pinned host bf16 Q/K/V -> device, fused calibrate+quantize, attention, "
+                            "bf16 output -> host every step; uploads, compute and downloads on "
+                            "three streams over two buffer sets, so consecutive steps overlap"},
         "gpu_launches": 4 * args.steps,     # 3 fused calibrate+quantize, 1 attention
         "clocks": clock,
     }
