@@ -127,6 +127,33 @@ QATTN_API qattn_status qattn_calibrate_quantize_fp4_block(
     float* gscale_dev, uint8_t* out_e4m3_requant, float* scale8_dev, void* workspace_dev,
     size_t workspace_bytes, qattn_stream_t stream);
 
+/* Inputs and outputs of one tensor for qattn_calibrate_quantize_qkv (all device pointers).
+ * FP8 mode: out_e4m3 receives the codes and scale_dev the multiplier s (as qattn_quantize_fp8);
+ * out_e2m1, blk_scale_e4m3 and gscale_dev are ignored.  FP4 mode: the outputs of
+ * qattn_quantize_fp4_block, out_e4m3 / scale_dev being the FP8 requant codes and multiplier. */
+typedef struct {
+  const void* x_bf16;        /* n bf16, 16-byte aligned */
+  uint8_t* out_e4m3;         /* n bytes; 8-byte aligned (FP8) or 16-byte aligned (FP4) */
+  float* amax_dev;           /* 1 float */
+  float* scale_dev;          /* 1 float */
+  uint8_t* out_e2m1;         /* FP4: n / 2 bytes, 8-byte aligned */
+  uint8_t* blk_scale_e4m3;   /* FP4: n / 16 bytes */
+  float* gscale_dev;         /* FP4: 1 float */
+} qattn_quant_io;
+
+/* Calibration + FakeQuantize of Q, K and V (three tensors of n elements each; io is a HOST
+ * array of three descriptors, read during the call) in one cooperative kernel: each tensor gets
+ * exactly the results of qattn_calibrate_amax followed by qattn_quantize_fp8 (mode FP8) or
+ * qattn_quantize_fp4_block with the FP8 requant (mode FP4).  The kernel staggers the tensors:
+ * while it quantizes one (read back from L2) it reduces the next one's amax from HBM.
+ * Workspace rules as for qattn_calibrate_quantize_fp8 (QATTN_FUSED_WORKSPACE_BYTES, zero-filled
+ * before first use, left zero-filled).  FP4 mode needs n % 16 == 0.  A tensor with a non-finite
+ * element gets its amax written and nothing else; QATTN_ERR_NONFINITE is recorded; the other
+ * tensors are still quantized. */
+QATTN_API qattn_status qattn_calibrate_quantize_qkv(const qattn_quant_io* io, size_t n,
+                                                    qattn_mode mode, void* workspace_dev,
+                                                    size_t workspace_bytes, qattn_stream_t stream);
+
 /* qattn_calibrate_quantize_fp8 without a caller workspace (the blog has no counterpart: this is
  * a calling convention, not part of the method).  For callers that cannot supply a scratch
  * buffer -- C code with no device allocator at the call site, or a runtime whose device memory

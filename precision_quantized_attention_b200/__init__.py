@@ -16,16 +16,18 @@ import torch
 
 from . import _lib
 from ._lib import (MODE_FP4, MODE_FP8, QattnError, calibrate_amax, calibrate_quantize_fp4_block,
-                   calibrate_quantize_fp8, forward, forward_varlen, get_error, new_workspace,
-                   quantize_fp4_block, quantize_fp8)
+                   calibrate_quantize_fp8, calibrate_quantize_qkv, forward, forward_varlen,
+                   get_error, new_workspace, quantize_fp4_block, quantize_fp8)
 
 __all__ = ["QuantizedAttention", "calibrate_amax", "quantize_fp8", "quantize_fp4_block",
-           "calibrate_quantize_fp8", "calibrate_quantize_fp4_block", "new_workspace", "forward",
+           "calibrate_quantize_fp8", "calibrate_quantize_fp4_block", "calibrate_quantize_qkv",
+           "new_workspace", "forward",
            "forward_varlen", "get_error", "QattnError", "MODE_FP8", "MODE_FP4"]
 
 
 class QuantizedAttention:
-    """The whole hot path for one shape: fused calibrate+quantize (x3) -> fused attention.
+    """The whole hot path for one shape: calibrate+quantize of Q, K, V (one launch) -> fused
+    attention.
 
     Holds the device buffers (codes, scales, FP4 side outputs, output, the calibration
     workspace) so repeated calls allocate nothing.  Calls on one object must not overlap on
@@ -65,14 +67,13 @@ class QuantizedAttention:
             self.max_seqlen = max(b - a for a, b in zip(cu_seqlens[:-1], cu_seqlens[1:]))
 
     def quantize(self, q, k, v, stream=None):
-        for i, x in enumerate((q, k, v)):
-            if self.mode == "fp8":
-                calibrate_quantize_fp8(x, self.amax[i:i + 1], self.codes[i], self.scale[i:i + 1],
-                                       self.workspace, stream)
-            else:
-                calibrate_quantize_fp4_block(x, self.amax[i:i + 1], self.e2m1[i], self.bscale[i],
-                                             self.gscale[i:i + 1], self.codes[i],
-                                             self.scale[i:i + 1], self.workspace, stream)
+        """Calibrate and FakeQuantize Q, K and V in one launch."""
+        if self.mode == "fp8":
+            calibrate_quantize_qkv((q, k, v), self.amax, self.codes, self.scale, self.workspace,
+                                   MODE_FP8, stream=stream)
+        else:
+            calibrate_quantize_qkv((q, k, v), self.amax, self.codes, self.scale, self.workspace,
+                                   MODE_FP4, self.e2m1, self.bscale, self.gscale, stream=stream)
 
     def attend(self, stream=None):
         mode = MODE_FP8 if self.mode == "fp8" else MODE_FP4

@@ -22,10 +22,10 @@ EXPORTS = (
     "qattn_calibrate_amax", "qattn_quantize_fp8", "qattn_quantize_fp4_block", "qattn_forward",
     "qattn_forward_varlen", "qattn_get_error", "qattn_calibrate_quantize_fp8",
     "qattn_calibrate_quantize_fp4_block", "qattn_calibrate_quantize_fp8_noalloc",
-    "qattn_status_str",
+    "qattn_calibrate_quantize_qkv", "qattn_status_str",
     "qattn_debug_set_wait_timeout_ns", "qattn_debug_inject_missing_q",
 )
-_RETURNS_STATUS = EXPORTS[:9]
+_RETURNS_STATUS = EXPORTS[:10]
 FUSED_WORKSPACE_BYTES = 256     # QATTN_FUSED_WORKSPACE_BYTES
 
 
@@ -33,6 +33,14 @@ class QattnError(RuntimeError):
     def __init__(self, status: int, what: str):
         self.status = status
         super().__init__(f"{what}: {status_str(status)} ({status})")
+
+
+class QuantIO(ctypes.Structure):
+    """qattn_quant_io: one tensor's device buffers for calibrate_quantize_qkv."""
+    _fields_ = [("x_bf16", ctypes.c_void_p), ("out_e4m3", ctypes.c_void_p),
+                ("amax_dev", ctypes.c_void_p), ("scale_dev", ctypes.c_void_p),
+                ("out_e2m1", ctypes.c_void_p), ("blk_scale_e4m3", ctypes.c_void_p),
+                ("gscale_dev", ctypes.c_void_p)]
 
 
 class _Scales(ctypes.Structure):
@@ -58,6 +66,7 @@ def load() -> ctypes.CDLL:
     lib.qattn_calibrate_quantize_fp8.argtypes = [P, S, P, P, P, P, S, P]
     lib.qattn_calibrate_quantize_fp4_block.argtypes = [P, S, P, P, P, P, P, P, P, S, P]
     lib.qattn_calibrate_quantize_fp8_noalloc.argtypes = [P, S, P, P, P, P]
+    lib.qattn_calibrate_quantize_qkv.argtypes = [ctypes.POINTER(QuantIO), S, I, P, S, P]
     lib.qattn_forward.argtypes = [P, P, P, P, I, I, I, I, ctypes.POINTER(_Scales), F, I, P]
     lib.qattn_forward_varlen.argtypes = [P, P, P, P, P, I, I, I, I, I, ctypes.POINTER(_Scales),
                                          F, I, P]
@@ -178,6 +187,38 @@ def calibrate_quantize_fp4_block(x: torch.Tensor, amax: torch.Tensor, out_e2m1: 
         _dev(out_e4m3_requant, torch.uint8, "out_e4m3_requant"),
         _dev(scale8, torch.float32, "scale8"), _dev(workspace, torch.uint8, "workspace"),
         workspace.numel(), _stream(stream)), "qattn_calibrate_quantize_fp4_block")
+
+
+def calibrate_quantize_qkv(xs, amax, codes8, scale8, workspace, mode: int = MODE_FP8,
+                           e2m1=None, bscale=None, gscale=None, stream=None):
+    """Q, K, V in one launch.  xs: three bf16 tensors of n elements; amax, scale8 (and gscale
+    in FP4 mode): float32 tensors of 3 elements (one per tensor); codes8, e2m1, bscale: lists of
+    three uint8 tensors."""
+    n = xs[0].numel()
+    if any(x.numel() != n for x in xs):
+        raise ValueError("Q, K and V must have the same number of elements")
+    for t, nm in ((amax, "amax"), (scale8, "scale8")):
+        if t.numel() != 3 or t.dtype != torch.float32 or not t.is_contiguous():
+            raise ValueError(f"{nm} must be a contiguous float32 tensor of 3 elements")
+    if mode == MODE_FP4 and (e2m1 is None or bscale is None or gscale is None or gscale.numel() != 3):
+        raise ValueError("FP4 mode needs e2m1, bscale and a 3-element gscale")
+    io = (QuantIO * 3)()
+    for i in range(3):
+        if codes8[i].numel() != n:
+            raise ValueError("codes8 tensors need n bytes")
+        io[i].x_bf16 = _dev(xs[i], torch.bfloat16, "x").value
+        io[i].out_e4m3 = _dev(codes8[i], torch.uint8, "codes8").value
+        io[i].amax_dev = amax.data_ptr() + 4 * i
+        io[i].scale_dev = scale8.data_ptr() + 4 * i
+        if mode == MODE_FP4:
+            if e2m1[i].numel() != n // 2 or bscale[i].numel() != n // 16:
+                raise ValueError("e2m1 needs n/2 bytes and bscale n/16 bytes")
+            io[i].out_e2m1 = _dev(e2m1[i], torch.uint8, "e2m1").value
+            io[i].blk_scale_e4m3 = _dev(bscale[i], torch.uint8, "bscale").value
+            io[i].gscale_dev = gscale.data_ptr() + 4 * i
+    _check(load().qattn_calibrate_quantize_qkv(io, n, int(mode), _dev(workspace, torch.uint8, "workspace"),
+                                               workspace.numel(), _stream(stream)),
+           "qattn_calibrate_quantize_qkv")
 
 
 def _scales(s_q, s_k, s_v):

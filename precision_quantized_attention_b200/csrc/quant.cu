@@ -479,6 +479,237 @@ __global__ void __launch_bounds__(FUSED_THREADS) k_calib_quant_fp4_block(
 }
 
 // -------------------------------------------------------------------------------------------
+// Q, K and V in one cooperative launch.  Stage 0 reduces Q's amax; stage s = 1, 2 quantizes
+// tensor s - 1 (its chunk comes back from L2, evict-first) while it reduces tensor s's amax from
+// HBM (evict-last), so the L2-bound half of one tensor overlaps the HBM-bound half of the next;
+// stage 3 quantizes V.  The stages are separated by grid barriers on one monotonic arrival
+// counter.  No CTA leaves early: a tensor whose amax is not finite (or a barrier that timed
+// out) only suppresses that tensor's writes, so every CTA arrives at every barrier.
+// -------------------------------------------------------------------------------------------
+constexpr int QKV = 3;
+
+struct QkvWorkspace {
+  unsigned amax_bits[4];
+  unsigned departed;
+  unsigned pad0[27];
+  unsigned arrived;          // own 128-byte line
+  unsigned pad1[31];
+};
+static_assert(sizeof(QkvWorkspace) <= 256, "fits QATTN_FUSED_WORKSPACE_BYTES");
+
+struct QkvTensor {
+  const uint4* x;            // n bf16 as 16-byte vectors
+  uint8_t* codes8;           // n E4M3 codes (FP8 mode: the codes; FP4 mode: the requant codes)
+  float* amax;
+  float* scale8;             // dequantization multiplier of codes8
+  uint2* e2m1;               // FP4 mode: n / 2 bytes of packed codes
+  uint8_t* bscale;           // FP4 mode: n / 16 block scales
+  float* gscale;             // FP4 mode: the FP32 tensor scale
+};
+
+struct QkvArgs {
+  QkvTensor t[QKV];
+  size_t n;                  // elements per tensor
+  uint64_t limit_ns;
+  int* err;
+  QkvWorkspace* ws;
+};
+
+// CTA-reduce m, publish it into `slot`, arrive, wait until `target` arrivals; returns the
+// published maximum (float bits) or 0xFFFFFFFF after a timeout.
+__device__ __forceinline__ unsigned grid_stage(uint32_t m, unsigned* slot, unsigned* arrived,
+                                               unsigned target, uint64_t limit_ns, int* err) {
+  __shared__ uint32_t warp_max[32];
+  __shared__ unsigned result;
+  m = __reduce_max_sync(0xFFFFFFFFu, m);
+  if ((threadIdx.x & 31) == 0) warp_max[threadIdx.x >> 5] = m;
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    m = threadIdx.x < (blockDim.x >> 5) ? warp_max[threadIdx.x] : 0u;
+    m = __reduce_max_sync(0xFFFFFFFFu, m);
+    if (threadIdx.x == 0) {
+      asm volatile("red.relaxed.gpu.global.max.u32 [%0], %1;" ::"l"(slot), "r"(m << 16) : "memory");
+      asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(arrived) : "memory");
+      const uint64_t t0 = global_timer_ns();
+      unsigned r = 0xFFFFFFFFu;
+      while (true) {
+        if (ld_acquire_gpu(arrived) >= target) {
+          r = ld_acquire_gpu(slot);
+          break;
+        }
+        if (global_timer_ns() - t0 > limit_ns) {
+          atomicExch(err, DEV_ERR_TIMEOUT);
+          break;
+        }
+        __nanosleep(32);
+      }
+      result = r;
+    }
+  }
+  __syncthreads();
+  return result;
+}
+
+__device__ __forceinline__ uint32_t fold_max(uint32_t m2) { return max(m2 & 0xFFFFu, m2 >> 16); }
+
+// One FP8 stage over the vectors [lo, hi): quantize xp into op (when xp is set) and reduce the
+// packed |x| maximum of xc (when xc is set).
+template <bool FAST>
+__device__ __forceinline__ uint32_t qkv_stage_fp8(const uint4* __restrict__ xp,
+                                                  uint2* __restrict__ op, float s, float r,
+                                                  const uint4* __restrict__ xc, size_t lo,
+                                                  size_t hi) {
+  constexpr size_t T = FUSED_THREADS, U = FUSED_UNROLL;
+  const uint64_t pf = l2_policy_evict_first(), pl = l2_policy_evict_last();
+  uint32_t m2 = 0;
+  size_t i = lo + threadIdx.x;
+  for (; i + (U - 1) * T < hi; i += U * T) {
+    uint4 a[U], b[U];
+    if (xc) {
+#pragma unroll
+      for (size_t u = 0; u < U; ++u) b[u] = ld_hint(xc + i + u * T, pl);
+    }
+    if (xp) {
+#pragma unroll
+      for (size_t u = 0; u < U; ++u) a[u] = ld_hint(xp + i + u * T, pf);
+    }
+    if (xc) {
+#pragma unroll
+      for (size_t u = 0; u < U; ++u) {
+        m2 = absmax_word(m2, b[u].x); m2 = absmax_word(m2, b[u].y);
+        m2 = absmax_word(m2, b[u].z); m2 = absmax_word(m2, b[u].w);
+      }
+    }
+    if (xp) {
+#pragma unroll
+      for (size_t u = 0; u < U; ++u)
+        __stcs(op + i + u * T, make_uint2(quant4_e4m3<FAST>(a[u].x, a[u].y, s, r),
+                                          quant4_e4m3<FAST>(a[u].z, a[u].w, s, r)));
+    }
+  }
+  for (; i < hi; i += T) {
+    if (xc) {
+      const uint4 b = ld_hint(xc + i, pl);
+      m2 = absmax_word(m2, b.x); m2 = absmax_word(m2, b.y);
+      m2 = absmax_word(m2, b.z); m2 = absmax_word(m2, b.w);
+    }
+    if (xp) {
+      const uint4 a = ld_hint(xp + i, pf);
+      __stcs(op + i, make_uint2(quant4_e4m3<FAST>(a.x, a.y, s, r), quant4_e4m3<FAST>(a.z, a.w, s, r)));
+    }
+  }
+  return m2;
+}
+
+// One FP4 stage over the 16-element blocks [lo, hi): block-quantize tp (when set) and reduce
+// the packed |x| maximum of xc (when set).
+__device__ __forceinline__ uint32_t qkv_stage_fp4(const QkvTensor* tp, float sg, float six_sg,
+                                                  float s8, float r8, bool fast8,
+                                                  const uint4* __restrict__ xc, size_t lo,
+                                                  size_t hi) {
+  constexpr size_t T = FUSED_THREADS;
+  const uint64_t pf = l2_policy_evict_first(), pl = l2_policy_evict_last();
+  uint32_t m2 = 0;
+  for (size_t b = lo + threadIdx.x; b < hi; b += T) {
+    uint4 c0, c1, a0, a1;
+    if (xc) {
+      c0 = ld_hint(xc + 2 * b, pl);
+      c1 = ld_hint(xc + 2 * b + 1, pl);
+    }
+    if (tp) {
+      a0 = ld_hint(tp->x + 2 * b, pf);
+      a1 = ld_hint(tp->x + 2 * b + 1, pf);
+    }
+    if (xc) {
+      m2 = absmax_word(m2, c0.x); m2 = absmax_word(m2, c0.y);
+      m2 = absmax_word(m2, c0.z); m2 = absmax_word(m2, c0.w);
+      m2 = absmax_word(m2, c1.x); m2 = absmax_word(m2, c1.y);
+      m2 = absmax_word(m2, c1.z); m2 = absmax_word(m2, c1.w);
+    }
+    if (tp)
+      fp4_block(a0, a1, b, sg, six_sg, s8, r8, fast8, tp->e2m1, tp->bscale,
+                reinterpret_cast<uint4*>(tp->codes8));
+  }
+  return m2;
+}
+
+template <int MODE>   // 0: per-tensor FP8, 1: FP4 blocks + FP8 requant
+__global__ void __launch_bounds__(FUSED_THREADS) k_calib_quant_qkv(const QkvArgs a) {
+  QkvWorkspace* ws = a.ws;
+  // FP8 works on 16-byte vectors (a tail of n % 8 elements goes to CTA 0); FP4 on 16-element
+  // blocks (n % 16 == 0)
+  const size_t units = MODE == 0 ? a.n / 8 : a.n / 16;
+  const int ntail = MODE == 0 ? static_cast<int>(a.n - units * 8) : 0;
+  const size_t per = (units + gridDim.x - 1) / gridDim.x;
+  const size_t lo = static_cast<size_t>(blockIdx.x) * per;
+  const size_t hi = lo + per < units ? lo + per : units;
+  const bool tail_thread = blockIdx.x == 0 && static_cast<int>(threadIdx.x) < ntail;
+  auto tail_elem = [&](int i) {
+    return reinterpret_cast<const uint16_t*>(a.t[i].x)[units * 8 + threadIdx.x];
+  };
+
+  uint32_t m = fold_max(MODE == 0 ? chunk_absmax(a.t[0].x, lo, hi)
+                                  : chunk_absmax(a.t[0].x, 2 * lo, 2 * hi));
+  if (tail_thread) m = max(m, static_cast<uint32_t>(tail_elem(0)) & 0x7FFFu);
+  unsigned bits = grid_stage(m, &ws->amax_bits[0], &ws->arrived, gridDim.x, a.limit_ns, a.err);
+
+#pragma unroll
+  for (int st = 1; st <= QKV; ++st) {
+    const int ip = st - 1;                          // tensor quantized in this stage
+    const QkvTensor& tp = a.t[ip];
+    const bool ok = bits < 0x7F800000u;             // finite amax (and no timeout)
+    const float amax = __uint_as_float(bits);
+    if (blockIdx.x == 0 && threadIdx.x == 0 && bits != 0xFFFFFFFFu) {
+      *tp.amax = amax;
+      if (!ok) atomicExch(a.err, DEV_ERR_NONFINITE);
+    }
+    const uint4* xc = st < QKV ? a.t[st].x : nullptr;
+    uint32_t m2;
+    if (MODE == 0) {
+      const float s = (amax == 0.0f) ? 1.0f : __fdiv_rn(amax, 448.0f);
+      const float r = __frcp_rn(s);
+      if (ok && blockIdx.x == 0 && threadIdx.x == 0) *tp.scale8 = s;
+      const uint4* xp = ok ? tp.x : nullptr;
+      uint2* op = reinterpret_cast<uint2*>(tp.codes8);
+      m2 = markstein_ok(s) ? qkv_stage_fp8<true>(xp, op, s, r, xc, lo, hi)
+                           : qkv_stage_fp8<false>(xp, op, s, r, xc, lo, hi);
+      if (ok && tail_thread) {
+        const float x = __uint_as_float(static_cast<uint32_t>(tail_elem(ip)) << 16);
+        tp.codes8[units * 8 + threadIdx.x] =
+            static_cast<uint8_t>(cvt_e4m3x2(__fdiv_rn(x, s), 0.0f) & 0xFFu);
+      }
+    } else {
+      const float sg = (amax == 0.0f) ? 1.0f : __fdiv_rn(amax, 2688.0f);
+      const float six_sg = __fmul_rn(6.0f, sg);
+      const float s8 = (amax == 0.0f) ? 1.0f : __fdiv_rn(__fmul_rn(2688.0f, sg), 448.0f);
+      if (ok && blockIdx.x == 0 && threadIdx.x == 0) {
+        *tp.gscale = sg;
+        *tp.scale8 = s8;
+      }
+      m2 = qkv_stage_fp4(ok ? &tp : nullptr, sg, six_sg, s8, __frcp_rn(s8), markstein_ok(s8),
+                         xc, lo, hi);
+    }
+    if (st < QKV) {
+      m = fold_max(m2);
+      if (tail_thread) m = max(m, static_cast<uint32_t>(tail_elem(st)) & 0x7FFFu);
+      bits = grid_stage(m, &ws->amax_bits[st], &ws->arrived, (st + 1) * gridDim.x, a.limit_ns,
+                        a.err);
+    }
+  }
+  // depart: the last CTA zeroes the workspace for the next call
+  if (threadIdx.x == 0) {
+    unsigned old;
+    asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;" : "=r"(old) : "l"(&ws->departed)
+                 : "memory");
+    if (old == gridDim.x - 1) {
+      for (int i = 0; i < 4; ++i) ws->amax_bits[i] = 0u;
+      ws->arrived = 0u;
+      ws->departed = 0u;
+    }
+  }
+}
+
+// -------------------------------------------------------------------------------------------
 // Host launchers (called from the C-ABI layer, which validates arguments).
 // -------------------------------------------------------------------------------------------
 static int grid_for(size_t work_items, int num_sms) {
@@ -548,6 +779,41 @@ cudaError_t launch_calib_quant_fp8(const void* x, size_t n, float* amax, uint8_t
                   (void*)&err};
   return cudaLaunchCooperativeKernel((const void*)k_calib_quant_fp8, dim3(grid),
                                      dim3(FUSED_THREADS), args, 0, stream);
+}
+
+// tensors: x, codes8, amax, scale8, e2m1, bscale, gscale for each of Q, K, V (FP8 mode: the last
+// three null).
+cudaError_t launch_calib_quant_qkv(const void* const* x, uint8_t* const* codes8, float* const* amax,
+                                   float* const* scale8, uint8_t* const* e2m1,
+                                   uint8_t* const* bscale, float* const* gscale, size_t n, int mode,
+                                   void* workspace, uint64_t limit_ns, int* err, int num_sms,
+                                   cudaStream_t stream) {
+  static int bps[2] = {0, 0};
+  const void* fn = mode == 0 ? (const void*)k_calib_quant_qkv<0> : (const void*)k_calib_quant_qkv<1>;
+  if (bps[mode] == 0) {
+    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&bps[mode], fn, FUSED_THREADS, 0);
+    if (e != cudaSuccess || bps[mode] < 1) return e != cudaSuccess ? e : cudaErrorInvalidValue;
+  }
+  QkvArgs a;
+  for (int i = 0; i < QKV; ++i) {
+    a.t[i].x = static_cast<const uint4*>(x[i]);
+    a.t[i].codes8 = codes8[i];
+    a.t[i].amax = amax[i];
+    a.t[i].scale8 = scale8[i];
+    a.t[i].e2m1 = reinterpret_cast<uint2*>(e2m1[i]);
+    a.t[i].bscale = bscale[i];
+    a.t[i].gscale = gscale[i];
+  }
+  a.n = n;
+  a.limit_ns = limit_ns;
+  a.err = err;
+  a.ws = static_cast<QkvWorkspace*>(workspace);
+  const size_t units = mode == 0 ? n / 8 : n / 16;
+  const size_t want = (units + FUSED_THREADS * 4 - 1) / (FUSED_THREADS * 4);
+  const size_t cap = static_cast<size_t>(num_sms) * bps[mode];
+  const unsigned grid = static_cast<unsigned>(want < 1 ? 1 : (want < cap ? want : cap));
+  void* args[] = {(void*)&a};
+  return cudaLaunchCooperativeKernel(fn, dim3(grid), dim3(FUSED_THREADS), args, 0, stream);
 }
 
 cudaError_t launch_calib_quant_fp4_block(const void* x, size_t n, float* amax, uint8_t* packed,

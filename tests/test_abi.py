@@ -65,6 +65,19 @@ def test_host_side_argument_errors():
     assert na(None, 16, FAKE, FAKE, FAKE, s0) == _lib.ERR_INVALID_ARG
     assert na(FAKE, 0, FAKE, FAKE, FAKE, s0) == _lib.ERR_INVALID_ARG
     assert na(MISALIGNED, 16, FAKE, FAKE, FAKE, s0) == _lib.ERR_INVALID_ARG
+    qkv = lib.qattn_calibrate_quantize_qkv
+    io = (_lib.QuantIO * 3)(*[_lib.QuantIO(0x10000, 0x10000, 0x10000, 0x10000, 0x10000, 0x10000,
+                                           0x10000) for _ in range(3)])
+    assert qkv(None, 16, 0, FAKE, W, s0) == _lib.ERR_INVALID_ARG
+    assert qkv(io, 0, 0, FAKE, W, s0) == _lib.ERR_INVALID_ARG
+    assert qkv(io, 16, 2, FAKE, W, s0) == _lib.ERR_INVALID_ARG            # bad mode
+    assert qkv(io, 24, 1, FAKE, W, s0) == _lib.ERR_INVALID_ARG            # FP4 needs n % 16 == 0
+    assert qkv(io, 16, 0, FAKE, W - 1, s0) == _lib.ERR_INVALID_ARG
+    io[1].x_bf16 = 0x10001                                                # misaligned input
+    assert qkv(io, 16, 0, FAKE, W, s0) == _lib.ERR_INVALID_ARG
+    io[1].x_bf16 = 0x10000
+    io[2].out_e2m1 = None                                                 # FP4 output missing
+    assert qkv(io, 32, 1, FAKE, W, s0) == _lib.ERR_INVALID_ARG
     sc = _lib._Scales(0x10000, 0x10000, 0x10000)
     fwd = lib.qattn_forward
     assert fwd(FAKE, FAKE, FAKE, FAKE, 1, 1, 16, 96, ctypes.byref(sc), 0.1, 0, s0) == _lib.ERR_UNSUPPORTED

@@ -194,3 +194,91 @@ def test_fused_nonfinite_input_is_reported():
     _, a = oracle.amax(x)
     want, s = oracle.quantize_fp8(x, a)
     assert np.array_equal(_u8(codes), want) and np.float32(scale.item()) == s
+
+
+def _qkv_inputs(n, seed, scales=(1.0, 3.0, 1e-2)):
+    g = torch.Generator().manual_seed(seed)
+    return [(torch.randn(n, generator=g) * sc).to(torch.bfloat16) for sc in scales]
+
+
+@pytest.mark.parametrize("n", [37, 8 * 1000 + 7, 16 * 4096, 24 * 4096 * 128 + 3])
+def test_qkv_fp8_bit_exact(n):
+    """Q, K, V in one staggered launch: every tensor's amax, scale and codes are the oracle's;
+    twice in a row on one workspace."""
+    xs = _qkv_inputs(n, seed=n % 1000)
+    xd = [x.cuda() for x in xs]
+    ws = qa.new_workspace()
+    for _ in range(2):
+        amax = torch.full((3,), -1.0, device="cuda")
+        scale = torch.zeros(3, device="cuda")
+        codes = [torch.full((n,), 0x55, dtype=torch.uint8, device="cuda") for _ in range(3)]
+        qa.calibrate_quantize_qkv(xd, amax, codes, scale, ws)
+        assert qa.get_error() == 0
+        for i, x in enumerate(xs):
+            _, a = oracle.amax(x)
+            want, s = oracle.quantize_fp8(x, a)
+            assert float(amax[i].item()) == a
+            assert np.float32(scale[i].item()) == s
+            assert np.array_equal(_u8(codes[i]), want), i
+        assert int(ws.count_nonzero().item()) == 0
+
+
+@pytest.mark.parametrize("n", [16 * 64, 16 * 4097, 24 * 4096 * 128])
+def test_qkv_fp4_bit_exact(n):
+    xs = _qkv_inputs(n, seed=7 + n % 1000, scales=(1.0, 1e-3, 40.0))
+    xs[0][:16] = xs[0][:16] * 1e-6                  # a block whose E4M3 scale underflows
+    xd = [x.cuda() for x in xs]
+    ws = qa.new_workspace()
+    amax, scale, gscale = (torch.zeros(3, device="cuda") for _ in range(3))
+    codes = [torch.empty(n, dtype=torch.uint8, device="cuda") for _ in range(3)]
+    e2m1 = [torch.empty(n // 2, dtype=torch.uint8, device="cuda") for _ in range(3)]
+    bscale = [torch.empty(n // 16, dtype=torch.uint8, device="cuda") for _ in range(3)]
+    qa.calibrate_quantize_qkv(xd, amax, codes, scale, ws, qa.MODE_FP4, e2m1, bscale, gscale)
+    assert qa.get_error() == 0
+    for i, x in enumerate(xs):
+        _, a = oracle.amax(x)
+        w_packed, w_bscale, w_sg, w_c8, w_s8 = oracle.quantize_fp4_block(x, a)
+        assert float(amax[i].item()) == a
+        assert np.float32(gscale[i].item()) == w_sg
+        assert np.float32(scale[i].item()) == w_s8
+        assert np.array_equal(_u8(bscale[i]), w_bscale)
+        assert np.array_equal(_u8(e2m1[i]), w_packed)
+        assert np.array_equal(_u8(codes[i]), w_c8)
+    assert int(ws.count_nonzero().item()) == 0
+
+
+def test_qkv_matches_single_tensor_kernel():
+    n = 24 * 2048 * 128
+    xs = [x.cuda() for x in _qkv_inputs(n, seed=3)]
+    ws = qa.new_workspace()
+    amax, scale = torch.zeros(3, device="cuda"), torch.zeros(3, device="cuda")
+    codes = [torch.empty(n, dtype=torch.uint8, device="cuda") for _ in range(3)]
+    qa.calibrate_quantize_qkv(xs, amax, codes, scale, ws)
+    for i, x in enumerate(xs):
+        a1, s1 = torch.zeros(1, device="cuda"), torch.zeros(1, device="cuda")
+        c1 = torch.empty(n, dtype=torch.uint8, device="cuda")
+        qa.calibrate_quantize_fp8(x, a1, c1, s1, ws)
+        assert float(a1.item()) == float(amax[i].item())
+        assert float(s1.item()) == float(scale[i].item())
+        assert torch.equal(c1, codes[i])
+    assert qa.get_error() == 0
+
+
+def test_qkv_nonfinite_tensor_is_reported_and_the_others_are_quantized():
+    n = 16 * 4096
+    xs = _qkv_inputs(n, seed=11)
+    xs[1][777] = float("nan")
+    xd = [x.cuda() for x in xs]
+    ws = qa.new_workspace()
+    amax = torch.zeros(3, device="cuda")
+    scale = torch.full((3,), -1.0, device="cuda")
+    codes = [torch.full((n,), 0x55, dtype=torch.uint8, device="cuda") for _ in range(3)]
+    qa.calibrate_quantize_qkv(xd, amax, codes, scale, ws)
+    assert qa.get_error() == qa._lib.ERR_NONFINITE
+    assert np.isnan(amax[1].item()) and scale[1].item() == -1.0
+    assert int(codes[1][0].item()) == 0x55                        # K: nothing written
+    for i in (0, 2):
+        _, a = oracle.amax(xs[i])
+        want, s = oracle.quantize_fp8(xs[i], a)
+        assert np.array_equal(_u8(codes[i]), want) and np.float32(scale[i].item()) == s
+    assert int(ws.count_nonzero().item()) == 0
