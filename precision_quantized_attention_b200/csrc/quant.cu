@@ -153,50 +153,66 @@ __global__ void __launch_bounds__(256) k_quant_fp8(const uint4* __restrict__ xv,
 // One thread per block: two 16-byte loads, an 8-byte packed store, the scale byte and a
 // 16-byte store of FP8 codes.
 // -------------------------------------------------------------------------------------------
-// One 16-element block: E2M1 codes, E4M3 block scale and (optionally) the FP8 requant codes.
+// FP8 requant table of one tensor: for every E4M3 block-scale code b (0..127: block scales are
+// never negative) and E2M1 magnitude m (0..7) the E4M3 code of the dequantized value over s8,
+//   lut[8 b + m] = e4m3(fl32(fl32(fl32(val(m) * val(b)) * s_g) / s8)),
+// in the same product order as the element-wise definition.  A negative E2M1 code gives the
+// same code with the sign bit set: the products, the quotient and round-to-nearest-even are
+// sign-symmetric, and -0 becomes 0x80.  Built by the whole CTA (then synchronized).
+__device__ __forceinline__ void build_requant_lut(uint2* lut, float sg, float s8) {
+  const float r8 = __frcp_rn(s8);
+  const bool fast8 = markstein_ok(s8);
+  uint8_t* bytes = reinterpret_cast<uint8_t*>(lut);
+  for (int i = threadIdx.x; i < 1024; i += blockDim.x) {
+    const float xh = __fmul_rn(__fmul_rn(e2m1_to_f32(static_cast<uint32_t>(i & 7)),
+                                         e4m3_to_f32(static_cast<uint32_t>(i >> 3))), sg);
+    const float d = fast8 ? div_rn_by(xh, s8, r8) : __fdiv_rn(xh, s8);
+    bytes[i] = static_cast<uint8_t>(cvt_e4m3x2(d, 0.0f) & 0xFFu);
+  }
+}
+
+// Four requant codes from four E2M1 codes packed as nibbles (low 16 bits of `nib4`) and the
+// two bf16 words they came from: the magnitudes index the block's 8-entry table (one byte
+// permute), and each code takes the sign of its input (the E2M1 code keeps the input's sign,
+// -0 included).
+__device__ __forceinline__ uint32_t requant4(uint2 t, uint32_t nib4, uint32_t w0, uint32_t w1) {
+  return __byte_perm(t.x, t.y, nib4 & 0x7777u) | (__byte_perm(w0, w1, 0x7531u) & 0x80808080u);
+}
+
+// One 16-element block: E2M1 codes, E4M3 block scale and (optionally) the FP8 requant codes,
+// the latter looked up in the tensor's requant table.
 __device__ __forceinline__ void fp4_block(uint4 a0, uint4 a1, size_t b, float sg, float six_sg,
-                                          float s8, float r8, bool fast8,
+                                          const uint2* __restrict__ lut,
                                           uint2* __restrict__ packed_out,
                                           uint8_t* __restrict__ bscale_out,
                                           uint4* __restrict__ codes8_out) {
   const uint32_t w[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
-  float x[16];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    x[2 * i] = bf16_lo(w[i]);
-    x[2 * i + 1] = bf16_hi(w[i]);
-  }
   uint32_t am2 = 0;
 #pragma unroll
   for (int i = 0; i < 8; ++i) am2 = absmax_word(am2, w[i]);
   const float amax_b = __uint_as_float(max(am2 & 0xFFFFu, am2 >> 16) << 16);
   const uint32_t sb = cvt_e4m3x2(__fdiv_rn(amax_b, six_sg), 0.0f) & 0xFFu;
-  const float sbv = e4m3_to_f32(sb);
-  const float eff = __fmul_rn(sbv, sg);
+  const float eff = __fmul_rn(e4m3_to_f32(sb), sg);
   uint32_t pk0 = 0, pk1 = 0;
   uint32_t c8[4] = {0u, 0u, 0u, 0u};
   if (eff != 0.0f) {
-    uint32_t nib[16];
     const float r_eff = __frcp_rn(eff);
     const bool fast_eff = markstein_ok(eff);
 #pragma unroll
-    for (int i = 0; i < 16; i += 2) {
-      const float q0 = fast_eff ? div_rn_by(x[i], eff, r_eff) : __fdiv_rn(x[i], eff);
-      const float q1 = fast_eff ? div_rn_by(x[i + 1], eff, r_eff) : __fdiv_rn(x[i + 1], eff);
+    for (int i = 0; i < 8; ++i) {
+      const float x0 = bf16_lo(w[i]), x1 = bf16_hi(w[i]);
+      const float q0 = fast_eff ? div_rn_by(x0, eff, r_eff) : __fdiv_rn(x0, eff);
+      const float q1 = fast_eff ? div_rn_by(x1, eff, r_eff) : __fdiv_rn(x1, eff);
       const uint32_t byte = cvt_e2m1x2(q0, q1);
-      nib[i] = byte & 0xFu;
-      nib[i + 1] = byte >> 4;
-      if (i < 8) pk0 |= byte << (4 * i);
-      else pk1 |= byte << (4 * (i - 8));
+      if (i < 4) pk0 |= byte << (8 * i);
+      else pk1 |= byte << (8 * (i - 4));
     }
-#pragma unroll
-    for (int i = 0; i < 16; i += 2) {
-      const float xh0 = __fmul_rn(__fmul_rn(e2m1_to_f32(nib[i]), sbv), sg);
-      const float xh1 = __fmul_rn(__fmul_rn(e2m1_to_f32(nib[i + 1]), sbv), sg);
-      const float d0 = fast8 ? div_rn_by(xh0, s8, r8) : __fdiv_rn(xh0, s8);
-      const float d1 = fast8 ? div_rn_by(xh1, s8, r8) : __fdiv_rn(xh1, s8);
-      const uint32_t pair = cvt_e4m3x2(d0, d1);
-      c8[i / 4] |= pair << (16 * ((i / 2) & 1));
+    if (codes8_out) {
+      const uint2 t = lut[sb & 0x7Fu];
+      c8[0] = requant4(t, pk0, w[0], w[1]);
+      c8[1] = requant4(t, pk0 >> 16, w[2], w[3]);
+      c8[2] = requant4(t, pk1, w[4], w[5]);
+      c8[3] = requant4(t, pk1 >> 16, w[6], w[7]);
     }
   }
   __stcs(packed_out + b, make_uint2(pk0, pk1));
@@ -221,13 +237,14 @@ __global__ void __launch_bounds__(256) k_quant_fp4_block(
     *gscale_out = sg;
     if (scale8_out) *scale8_out = s8;
   }
-  const float r8 = __frcp_rn(s8);
-  const bool fast8 = markstein_ok(s8);
+  __shared__ uint2 lut[128];
+  build_requant_lut(lut, sg, s8);
+  __syncthreads();
   const size_t stride = static_cast<size_t>(gridDim.x) * blockDim.x;
   for (size_t b = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; b < nblocks;
        b += stride)
-    fp4_block(__ldcs(xv + 2 * b), __ldcs(xv + 2 * b + 1), b, sg, six_sg, s8, r8, fast8,
-              packed_out, bscale_out, codes8_out);
+    fp4_block(__ldcs(xv + 2 * b), __ldcs(xv + 2 * b + 1), b, sg, six_sg, lut, packed_out,
+              bscale_out, codes8_out);
 }
 
 // -------------------------------------------------------------------------------------------
@@ -460,21 +477,21 @@ __global__ void __launch_bounds__(FUSED_THREADS) k_calib_quant_fp4_block(
     *gscale_out = sg;
     if (scale8_out) *scale8_out = s8;
   }
-  const float r8 = __frcp_rn(s8);
-  const bool fast8 = markstein_ok(s8);
+  __shared__ uint2 lut[128];
+  build_requant_lut(lut, sg, s8);
+  __syncthreads();
   const uint64_t pol = l2_policy_evict_first();
   size_t b = lo + threadIdx.x;
   for (; b + FUSED_THREADS < hi; b += 2 * FUSED_THREADS) {     // two blocks' loads in flight
     const uint4 a0 = ld_hint(xv + 2 * b, pol), a1 = ld_hint(xv + 2 * b + 1, pol);
     const uint4 c0 = ld_hint(xv + 2 * (b + FUSED_THREADS), pol);
     const uint4 c1 = ld_hint(xv + 2 * (b + FUSED_THREADS) + 1, pol);
-    fp4_block(a0, a1, b, sg, six_sg, s8, r8, fast8, packed_out, bscale_out, codes8_out);
-    fp4_block(c0, c1, b + FUSED_THREADS, sg, six_sg, s8, r8, fast8, packed_out, bscale_out,
-              codes8_out);
+    fp4_block(a0, a1, b, sg, six_sg, lut, packed_out, bscale_out, codes8_out);
+    fp4_block(c0, c1, b + FUSED_THREADS, sg, six_sg, lut, packed_out, bscale_out, codes8_out);
   }
   for (; b < hi; b += FUSED_THREADS)
-    fp4_block(ld_hint(xv + 2 * b, pol), ld_hint(xv + 2 * b + 1, pol), b, sg, six_sg, s8, r8,
-              fast8, packed_out, bscale_out, codes8_out);
+    fp4_block(ld_hint(xv + 2 * b, pol), ld_hint(xv + 2 * b + 1, pol), b, sg, six_sg, lut,
+              packed_out, bscale_out, codes8_out);
   grid_depart(ws);
 }
 
@@ -601,10 +618,13 @@ __device__ __forceinline__ uint32_t qkv_stage_fp8(const uint4* __restrict__ xp,
   return m2;
 }
 
-// One FP4 stage over the 16-element blocks [lo, hi): block-quantize tp (when set) and reduce
-// the packed |x| maximum of xc (when set).
-__device__ __forceinline__ uint32_t qkv_stage_fp4(const QkvTensor* tp, float sg, float six_sg,
-                                                  float s8, float r8, bool fast8,
+// One FP4 stage over the 16-element blocks [lo, hi): block-quantize xp into e2m1 / bscale /
+// codes8 (when xp is set) and reduce the packed |x| maximum of xc (when xc is set).
+__device__ __forceinline__ uint32_t qkv_stage_fp4(const uint4* __restrict__ xp,
+                                                  uint2* __restrict__ e2m1,
+                                                  uint8_t* __restrict__ bscale,
+                                                  uint4* __restrict__ codes8, float sg,
+                                                  float six_sg, const uint2* __restrict__ lut,
                                                   const uint4* __restrict__ xc, size_t lo,
                                                   size_t hi) {
   constexpr size_t T = FUSED_THREADS;
@@ -616,9 +636,9 @@ __device__ __forceinline__ uint32_t qkv_stage_fp4(const QkvTensor* tp, float sg,
       c0 = ld_hint(xc + 2 * b, pl);
       c1 = ld_hint(xc + 2 * b + 1, pl);
     }
-    if (tp) {
-      a0 = ld_hint(tp->x + 2 * b, pf);
-      a1 = ld_hint(tp->x + 2 * b + 1, pf);
+    if (xp) {
+      a0 = ld_hint(xp + 2 * b, pf);
+      a1 = ld_hint(xp + 2 * b + 1, pf);
     }
     if (xc) {
       m2 = absmax_word(m2, c0.x); m2 = absmax_word(m2, c0.y);
@@ -626,9 +646,7 @@ __device__ __forceinline__ uint32_t qkv_stage_fp4(const QkvTensor* tp, float sg,
       m2 = absmax_word(m2, c1.x); m2 = absmax_word(m2, c1.y);
       m2 = absmax_word(m2, c1.z); m2 = absmax_word(m2, c1.w);
     }
-    if (tp)
-      fp4_block(a0, a1, b, sg, six_sg, s8, r8, fast8, tp->e2m1, tp->bscale,
-                reinterpret_cast<uint4*>(tp->codes8));
+    if (xp) fp4_block(a0, a1, b, sg, six_sg, lut, e2m1, bscale, codes8);
   }
   return m2;
 }
@@ -686,8 +704,13 @@ __global__ void __launch_bounds__(FUSED_THREADS) k_calib_quant_qkv(const QkvArgs
         *tp.gscale = sg;
         *tp.scale8 = s8;
       }
-      m2 = qkv_stage_fp4(ok ? &tp : nullptr, sg, six_sg, s8, __frcp_rn(s8), markstein_ok(s8),
-                         xc, lo, hi);
+      __shared__ uint2 lut[128];
+      if (ok) {                                     // uniform over the grid
+        build_requant_lut(lut, sg, s8);
+        __syncthreads();
+      }
+      m2 = qkv_stage_fp4(ok ? tp.x : nullptr, tp.e2m1, tp.bscale,
+                         reinterpret_cast<uint4*>(tp.codes8), sg, six_sg, lut, xc, lo, hi);
     }
     if (st < QKV) {
       m = fold_max(m2);
