@@ -279,6 +279,18 @@ def e2e_time(args, w, q, k, v, qd, kd, vd, step, flush, stream, world):
     return max_over_ranks(ms, world)
 
 
+def bench_config(w, world):
+    """The workload description both arms print."""
+    return {"workload": f"{w.name}: B={w.B} H={w.H} L={w.L} D={w.D} {w.mode.upper()} full attention"
+                        + (" (512 text + 4096 target + 4096 context tokens)"
+                           if w.L == workloads.L_EDIT else ""),
+            "mode": w.mode, "B": w.B, "H": w.H, "L": w.L, "D": w.D,
+            "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+            "l2": "flushed between steps outside the timed events: a 256 MiB write, then a "
+                  "256 MiB read of another buffer so the write's dirty lines are written back "
+                  "before the step starts"}
+
+
 def report(args, w, qkv, rank, world, ms, attn, quant, e2e_ms, clocks):
     q = qkv[0]
     hbm_gbs, bf16_tf, peak_kind = load_peaks()
@@ -304,15 +316,7 @@ def report(args, w, qkv, rank, world, ms, attn, quant, e2e_ms, clocks):
         "vs_baseline": None,
         "dtype": "e4m3",
         "data": "synthetic: seeded N(0,1) bf16 Q/K/V, 4 of 128 Q/K channels per head x10",
-        "config": {"workload": f"{w.name}: B={w.B} H={w.H} L={w.L} D={w.D} "
-                               f"{w.mode.upper()} full attention" + (
-                                   " (512 text + 4096 target + 4096 context tokens)"
-                                   if w.L == workloads.L_EDIT else ""),
-                   "mode": w.mode, "B": w.B, "H": w.H, "L": w.L, "D": w.D,
-                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
-                   "l2": "flushed between steps outside the timed events: a 256 MiB write, then a "
-                         "256 MiB read of another buffer so the write's dirty lines are "
-                         "written back before the step starts"},
+        "config": bench_config(w, world),
         "roofline": {"bound": "tensor", "achieved": achieved_tf, "peak": fp8_peak,
                      "unit": "TFLOP/s", "frac": achieved_tf / fp8_peak,
                      "traffic": ATTN_TRAFFIC_BYTES.get((w.L, w.H, w.D)),
@@ -382,11 +386,10 @@ def run_reference(args):
     print(json.dumps({
         "impl": "reference",
         "metric": "quantized attention TFLOP/s @L=8704,H=24,D=128 and % of B200 FP8 peak",
-        "value": value, "unit": "TFLOP/s", "n_gpus": 0, "steps": args.steps,
+        "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": f"{w.name}: B=1 H=24 L=8704 D=128 {w.mode.upper()}",
-                   "mode": w.mode, "B": w.B, "H": w.H, "L": w.L, "D": w.D},
+        "config": bench_config(w, args.gpus),
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
                          "sample": r["sample"]},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
