@@ -17,11 +17,12 @@ import torch
 from . import _lib
 from ._lib import (MODE_FP4, MODE_FP8, QattnError, calibrate_amax, calibrate_quantize_fp4_block,
                    calibrate_quantize_fp8, calibrate_quantize_qkv, forward, forward_varlen,
-                   get_error, new_workspace, quantize_fp4_block, quantize_fp8)
+                   forward_workspace_bytes, get_error, new_workspace, quantize_fp4_block,
+                   quantize_fp8)
 
 __all__ = ["QuantizedAttention", "calibrate_amax", "quantize_fp8", "quantize_fp4_block",
            "calibrate_quantize_fp8", "calibrate_quantize_fp4_block", "calibrate_quantize_qkv",
-           "new_workspace", "forward",
+           "new_workspace", "forward", "forward_workspace_bytes",
            "forward_varlen", "get_error", "QattnError", "MODE_FP8", "MODE_FP4"]
 
 
@@ -60,6 +61,9 @@ class QuantizedAttention:
         self.out = torch.empty(shape, dtype=torch.bfloat16, device=dev)
         self.workspace = new_workspace(dev)
         self.varlen = cu_seqlens is not None
+        # attention workspace: balances the last wave of a dense launch (none for varlen)
+        nbytes = 0 if self.varlen else forward_workspace_bytes(B, H, T, D)
+        self.attn_workspace = torch.empty(nbytes, dtype=torch.uint8, device=dev) if nbytes else None
         if self.varlen:
             if B != 1:
                 raise ValueError("varlen tensors are [1, H, T, D]")
@@ -83,7 +87,7 @@ class QuantizedAttention:
                            self.max_seqlen, *s, self.sm_scale, mode, stream)
         else:
             forward(self.codes[0], self.codes[1], self.codes[2], self.out, *s, self.sm_scale,
-                    mode, stream)
+                    mode, stream, workspace=self.attn_workspace)
         return self.out
 
     def __call__(self, q, k, v, stream=None):

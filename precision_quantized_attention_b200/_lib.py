@@ -22,10 +22,11 @@ EXPORTS = (
     "qattn_calibrate_amax", "qattn_quantize_fp8", "qattn_quantize_fp4_block", "qattn_forward",
     "qattn_forward_varlen", "qattn_get_error", "qattn_calibrate_quantize_fp8",
     "qattn_calibrate_quantize_fp4_block", "qattn_calibrate_quantize_fp8_noalloc",
-    "qattn_calibrate_quantize_qkv", "qattn_status_str",
+    "qattn_calibrate_quantize_qkv", "qattn_forward_ws", "qattn_status_str",
+    "qattn_forward_workspace_bytes",
     "qattn_debug_set_wait_timeout_ns", "qattn_debug_inject_missing_q",
 )
-_RETURNS_STATUS = EXPORTS[:10]
+_RETURNS_STATUS = EXPORTS[:11]
 FUSED_WORKSPACE_BYTES = 256     # QATTN_FUSED_WORKSPACE_BYTES
 
 
@@ -70,6 +71,9 @@ def load() -> ctypes.CDLL:
     lib.qattn_forward.argtypes = [P, P, P, P, I, I, I, I, ctypes.POINTER(_Scales), F, I, P]
     lib.qattn_forward_varlen.argtypes = [P, P, P, P, P, I, I, I, I, I, ctypes.POINTER(_Scales),
                                          F, I, P]
+    lib.qattn_forward_ws.argtypes = [P, P, P, P, I, I, I, I, ctypes.POINTER(_Scales), F, I, P, S, P]
+    lib.qattn_forward_workspace_bytes.argtypes = [I, I, I, I]
+    lib.qattn_forward_workspace_bytes.restype = S
     lib.qattn_get_error.argtypes = [P]
     lib.qattn_status_str.argtypes = [I]
     lib.qattn_status_str.restype = ctypes.c_char_p
@@ -226,17 +230,29 @@ def _scales(s_q, s_k, s_v):
                    _dev(s_v, torch.float32, "s_v").value)
 
 
-def forward(q8, k8, v8, out, s_q, s_k, s_v, sm_scale: float, mode: int = MODE_FP8, stream=None):
-    """q8, k8, v8: uint8 E4M3 codes [B, H, L, D]; out: bf16 [B, H, L, D]."""
+def forward_workspace_bytes(B: int, H: int, L: int, D: int) -> int:
+    """Bytes of the workspace forward() uses to balance its last wave (0: none needed)."""
+    return int(load().qattn_forward_workspace_bytes(int(B), int(H), int(L), int(D)))
+
+
+def forward(q8, k8, v8, out, s_q, s_k, s_v, sm_scale: float, mode: int = MODE_FP8, stream=None,
+            workspace: torch.Tensor | None = None):
+    """q8, k8, v8: uint8 E4M3 codes [B, H, L, D]; out: bf16 [B, H, L, D].  With a workspace of
+    forward_workspace_bytes(B, H, L, D) bytes (uint8 CUDA tensor) the last wave is balanced by
+    splitting it along the keys (qattn_forward_ws); without one, qattn_forward."""
     B, H, L, D = q8.shape
     for t, nm in ((k8, "k8"), (v8, "v8"), (out, "out")):
         if tuple(t.shape) != (B, H, L, D):
             raise ValueError(f"{nm} shape {tuple(t.shape)} != {(B, H, L, D)}")
     sc = _scales(s_q, s_k, s_v)
-    _check(load().qattn_forward(_dev(q8, torch.uint8, "q8"), _dev(k8, torch.uint8, "k8"),
-                                _dev(v8, torch.uint8, "v8"), _dev(out, torch.bfloat16, "out"),
-                                B, H, L, D, ctypes.byref(sc), float(sm_scale), int(mode),
-                                _stream(stream)), "qattn_forward")
+    args = (_dev(q8, torch.uint8, "q8"), _dev(k8, torch.uint8, "k8"), _dev(v8, torch.uint8, "v8"),
+            _dev(out, torch.bfloat16, "out"), B, H, L, D, ctypes.byref(sc), float(sm_scale),
+            int(mode))
+    if workspace is None:
+        _check(load().qattn_forward(*args, _stream(stream)), "qattn_forward")
+    else:
+        _check(load().qattn_forward_ws(*args, _dev(workspace, torch.uint8, "workspace"),
+                                       workspace.numel(), _stream(stream)), "qattn_forward_ws")
 
 
 def forward_varlen(q8, k8, v8, out, cu_seqlens: torch.Tensor, max_seqlen: int, s_q, s_k, s_v,

@@ -13,7 +13,7 @@ CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(os.path.dirname(HERE), "include")
 LIB = os.path.join(HERE, "libqattn.so")
 SOURCES = ["qattn_api.cu", "quant.cu", "attn_fwd.cu", "noalloc.cu"]
-HEADERS = ["sm100_ptx.cuh"]
+HEADERS = ["sm100_ptx.cuh", "launch.h"]
 
 
 def nvcc() -> str:

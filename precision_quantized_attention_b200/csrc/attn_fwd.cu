@@ -38,6 +38,7 @@
 #include <cuda_bf16.h>
 #include <cstdint>
 
+#include "launch.h"
 #include "sm100_ptx.cuh"
 
 namespace qattn {
@@ -67,6 +68,18 @@ struct AttnArgs {
   int* err;
   uint64_t timeout_ns;
   int inject_missing_q;     // fault injection for tests: the producer never loads Q
+  // Dense launches use a 1-D grid: CTAs [0, full_ctas) take one pair of Q tiles each; the pairs
+  // after them (the last, partial wave) are split into nsplit parts along the keys, one CTA per
+  // part, which writes unnormalised partial results for the combine kernel:
+  //   part_o[(((tp * nsplit + part) * NQ + t) * BLOCK_M + row) * D + c]  (FP32, row-major)
+  //   part_ml[((tp * nsplit + part) * NQ + t) * BLOCK_M + row] = (running max, row sum)
+  // with tp the index of the pair among the split ones.
+  int pairs_per_head;
+  int full_ctas;
+  int nsplit;
+  int combine_pairs;        // number of split pairs (the combine kernel's work)
+  float* part_o;
+  float2* part_ml;
 };
 
 template <int D>
@@ -199,9 +212,25 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
   const int lane = threadIdx.x & 31;
 
   // ---- which sequence and which rows -------------------------------------------------------
-  const int qblk = blockIdx.x;                    // pair of Q tiles
-  const int h = blockIdx.y;
-  const int bz = blockIdx.z;                      // batch row (dense) or sequence (varlen)
+  int qblk, h, bz;                                // pair of Q tiles, head, batch row / sequence
+  int part = 0, nparts = 1, split_pair = -1;
+  if (args.cu_seqlens) {
+    qblk = blockIdx.x;
+    h = blockIdx.y;
+    bz = blockIdx.z;
+  } else {
+    int pair = blockIdx.x;
+    if (pair >= args.full_ctas) {                 // a part of a split pair
+      const int u = pair - args.full_ctas;
+      split_pair = u / args.nsplit;
+      part = u % args.nsplit;
+      nparts = args.nsplit;
+      pair = args.full_ctas + split_pair;
+    }
+    qblk = pair % args.pairs_per_head;
+    h = (pair / args.pairs_per_head) % args.H;
+    bz = pair / (args.pairs_per_head * args.H);
+  }
   int seq_start, seq_len, slab;
   if (args.cu_seqlens) {
     seq_start = __ldg(args.cu_seqlens + bz);
@@ -214,7 +243,12 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
   }
   const int q_row0 = qblk * (NQ * BLOCK_M);
   if (q_row0 >= seq_len) return;                  // uniform over the CTA: nothing to do
-  const int nkv = (seq_len + BLOCK_N - 1) / BLOCK_N;
+  // key steps [kv0, kv0 + nkv) of this CTA (all of them unless the pair is split)
+  const int nkv_all = (seq_len + BLOCK_N - 1) / BLOCK_N;
+  const int steps_per_part = (nkv_all + nparts - 1) / nparts;
+  const int kv0 = part * steps_per_part;
+  const int nkv = min(nkv_all, kv0 + steps_per_part) - kv0;   // >= 1: the host keeps parts
+                                                               // shorter than the sequence
 
   // ---- barriers --------------------------------------------------------------------------
   const uint32_t bar0 = base_u32 + SL::OFF_BAR;
@@ -268,7 +302,7 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
           return false;
         mbar_arrive_expect_tx(BAR(B_KFULL + s), SL::TILE_KV);
         tma_load_3d(base_u32 + SL::OFF_K + s * SL::TILE_KV, &tm_k, BAR(B_KFULL + s), 0,
-                    seq_start + j * BLOCK_N, slab);
+                    seq_start + (kv0 + j) * BLOCK_N, slab);
         ++nk;
         return true;
       };
@@ -279,7 +313,7 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
           return false;
         mbar_arrive_expect_tx(BAR(B_VFULL + s), SL::TILE_KV);
         tma_load_3d(base_u32 + SL::OFF_V + s * SL::TILE_KV, &tm_v, BAR(B_VFULL + s), 0,
-                    seq_start + j * BLOCK_N, slab);
+                    seq_start + (kv0 + j) * BLOCK_N, slab);
         ++nv;
         return true;
       };
@@ -391,7 +425,7 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
 #pragma unroll
         for (int i = 0; i < BLOCK_N; ++i) s[i] = __uint_as_float(sv[i / 32][i % 32]);
       }
-      const int kv_valid = seq_len - j * BLOCK_N;  // keys of this tile inside the sequence
+      const int kv_valid = seq_len - (kv0 + j) * BLOCK_N;  // keys of this tile in the sequence
       if (kv_valid < BLOCK_N) {
 #pragma unroll
         for (int i = 0; i < BLOCK_N; ++i)
@@ -453,6 +487,22 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
         tc_fence_after();
         const int row = q_row0 + t * BLOCK_M + r;
         const bool valid = row < seq_len;
+        if (nparts > 1) {
+          // partial result of this part: raw O row, running max and row sum
+          const size_t slot = (static_cast<size_t>(split_pair) * nparts + part) * NQ + t;
+          float4* po = reinterpret_cast<float4*>(args.part_o + (slot * BLOCK_M + r) * D);
+#pragma unroll
+          for (int c4 = 0; c4 < D / 32; ++c4) {
+            uint32_t v[32];
+            tmem_ld32(tO + c4 * 32, v);
+            tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+              po[c4 * 8 + i] = make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
+                                           __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3]));
+          }
+          args.part_ml[slot * BLOCK_M + r] = make_float2(m_run, l);
+        } else {
         const float scale = __ldg(args.s_v) / l;   // O = acc * s_v / 448 / (l / 448)
         __nv_bfloat16* orow =
             args.out + (static_cast<size_t>(slab) * args.rows_per_slab + seq_start + row) * D;
@@ -475,6 +525,7 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
               dst[i] = make_uint4(packed[4 * i], packed[4 * i + 1], packed[4 * i + 2], packed[4 * i + 3]);
           }
         }
+        }
       }
     }
   }
@@ -485,6 +536,66 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
     tc_fence_after();
     tmem_dealloc(tmem, TC::ALLOC);
   }
+}
+
+// ---------------------------------------------------------------------------------------------
+// Combine of split pairs: one warp per output row (COMBINE_WARPS rows per CTA), each lane D / 32
+// columns.  The parts' running maxima are integers, so each part is brought to the common
+// maximum M by an exact power of two: O = sum_p 2^(m_p - M) O_p, l = sum_p 2^(m_p - M) l_p,
+// out = O * s_v / l.
+// ---------------------------------------------------------------------------------------------
+constexpr int COMBINE_WARPS = 8;
+
+template <int D>
+__global__ void __launch_bounds__(COMBINE_WARPS * 32) k_attn_combine(const AttnArgs args) {
+  constexpr int VEC = D / 32;                       // columns per lane: 4 or 2
+  const int lane = threadIdx.x & 31;
+  const int grow = blockIdx.x * COMBINE_WARPS + (threadIdx.x >> 5);   // row over all slots
+  const int tp = grow / (NQ * BLOCK_M);
+  const int t = (grow / BLOCK_M) % NQ;
+  const int r = grow % BLOCK_M;
+  if (tp >= args.combine_pairs) return;
+  const int pair = args.full_ctas + tp;
+  const int qblk = pair % args.pairs_per_head;
+  const int h = (pair / args.pairs_per_head) % args.H;
+  const int bz = pair / (args.pairs_per_head * args.H);
+  const int row = qblk * (NQ * BLOCK_M) + t * BLOCK_M + r;
+  if (row >= args.L) return;
+  const int S = args.nsplit;
+  auto slot = [&](int p) { return (static_cast<size_t>(tp) * S + p) * NQ + t; };
+  float M = -INFINITY;
+  for (int p = 0; p < S; ++p) M = fmaxf(M, args.part_ml[slot(p) * BLOCK_M + r].x);
+  float l = 0.0f;
+  float acc[VEC];
+#pragma unroll
+  for (int i = 0; i < VEC; ++i) acc[i] = 0.0f;
+  for (int p = 0; p < S; ++p) {
+    const float2 ml = args.part_ml[slot(p) * BLOCK_M + r];
+    const float w = exp2_int(static_cast<int>(ml.x - M));
+    l = fmaf(w, ml.y, l);
+    const float* po = args.part_o + (slot(p) * BLOCK_M + r) * D + lane * VEC;
+    if constexpr (VEC == 4) {
+      const float4 o = *reinterpret_cast<const float4*>(po);
+      acc[0] = fmaf(w, o.x, acc[0]); acc[1] = fmaf(w, o.y, acc[1]);
+      acc[2] = fmaf(w, o.z, acc[2]); acc[3] = fmaf(w, o.w, acc[3]);
+    } else {
+      const float2 o = *reinterpret_cast<const float2*>(po);
+      acc[0] = fmaf(w, o.x, acc[0]); acc[1] = fmaf(w, o.y, acc[1]);
+    }
+  }
+  const float scale = __ldg(args.s_v) / l;
+  __nv_bfloat16* orow =
+      args.out + (static_cast<size_t>(bz * args.H + h) * args.L + row) * D + lane * VEC;
+  uint32_t packed[VEC / 2];
+#pragma unroll
+  for (int i = 0; i < VEC / 2; ++i) {
+    const __nv_bfloat162 b2 = __floats2bfloat162_rn(acc[2 * i] * scale, acc[2 * i + 1] * scale);
+    packed[i] = *reinterpret_cast<const uint32_t*>(&b2);
+  }
+  if constexpr (VEC == 4)
+    *reinterpret_cast<uint2*>(orow) = make_uint2(packed[0], packed[1]);
+  else
+    *reinterpret_cast<uint32_t*>(orow) = packed[0];
 }
 
 // ---------------------------------------------------------------------------------------------
@@ -527,7 +638,8 @@ static bool make_map(CUtensorMap* map, const void* ptr, int D, int rows, int sla
 
 template <int D>
 static cudaError_t launch_attn_d(const void* q8, const void* k8, const void* v8, const AttnArgs& a,
-                                 int rows_per_slab, int slabs, dim3 grid, cudaStream_t stream) {
+                                 int rows_per_slab, int slabs, dim3 grid, int combine_ctas,
+                                 cudaStream_t stream) {
   CUtensorMap mq, mk, mv;
   if (!make_map(&mq, q8, D, rows_per_slab, slabs) || !make_map(&mk, k8, D, rows_per_slab, slabs) ||
       !make_map(&mv, v8, D, rows_per_slab, slabs))
@@ -542,14 +654,45 @@ static cudaError_t launch_attn_d(const void* q8, const void* k8, const void* v8,
     configured_dev_mask |= 1 << dev;
   }
   k_attn_fp8_fwd<D><<<grid, ATTN_THREADS, Smem<D>::ALLOC, stream>>>(mq, mk, mv, a);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess || combine_ctas == 0) return e;
+  k_attn_combine<D><<<combine_ctas, COMBINE_WARPS * 32, 0, stream>>>(a);
   return cudaGetLastError();
+}
+
+// Split plan of a dense launch: pairs beyond the last full wave of num_sms CTAs (one CTA per
+// SM) are split along the keys into the number of parts (2..4) that shortens that partial wave
+// the most, if it shortens it to at most 0.8 of a full CTA's time; each part keeps at least two
+// key steps.  bytes = the workspace the parts need (0: no split).
+AttnSplitPlan plan_attention_split(int B, int H, int L, int D, int num_sms) {
+  AttnSplitPlan p;
+  p.pairs_per_head = (L + NQ * BLOCK_M - 1) / (NQ * BLOCK_M);
+  const long long pairs = static_cast<long long>(p.pairs_per_head) * H * B;
+  const int nkv = (L + BLOCK_N - 1) / BLOCK_N;
+  const long long tail = num_sms > 0 ? pairs % num_sms : 0;
+  p.nsplit = 1;
+  double best = 1.0;
+  for (int S = 2; tail > 0 && S <= 4; ++S) {
+    if (nkv < 2 * S) break;
+    const double tt = static_cast<double>((tail * S + num_sms - 1) / num_sms) / S;
+    if (tt < best - 1e-9) {
+      best = tt;
+      p.nsplit = S;
+    }
+  }
+  if (best > 0.8) p.nsplit = 1;
+  p.tail = p.nsplit > 1 ? static_cast<int>(tail) : 0;
+  p.full_ctas = static_cast<int>(pairs - p.tail);
+  p.bytes = static_cast<size_t>(p.tail) * p.nsplit * NQ * BLOCK_M * (D + 2) * sizeof(float);
+  return p;
 }
 
 cudaError_t launch_attention(const uint8_t* q8, const uint8_t* k8, const uint8_t* v8, void* out,
                              int B, int H, int L, int D, const int* cu_seqlens, int nseq,
                              int max_seqlen, int total_tokens, const float* s_q, const float* s_k,
                              const float* s_v, float sm_scale, int* err, uint64_t timeout_ns,
-                             int inject_missing_q, cudaStream_t stream) {
+                             int inject_missing_q, void* workspace, size_t workspace_bytes,
+                             int num_sms, cudaStream_t stream) {
   AttnArgs a;
   const bool varlen = cu_seqlens != nullptr;
   a.rows_per_slab = varlen ? total_tokens : L;
@@ -564,11 +707,39 @@ cudaError_t launch_attention(const uint8_t* q8, const uint8_t* k8, const uint8_t
   a.err = err;
   a.timeout_ns = timeout_ns;
   a.inject_missing_q = inject_missing_q;
+  a.part_o = nullptr;
+  a.part_ml = nullptr;
+  a.combine_pairs = 0;
   const int slabs = varlen ? H : B * H;
-  const int lmax = varlen ? max_seqlen : L;
-  dim3 grid((lmax + NQ * BLOCK_M - 1) / (NQ * BLOCK_M), H, varlen ? nseq : B);
-  if (D == 128) return launch_attn_d<128>(q8, k8, v8, a, a.rows_per_slab, slabs, grid, stream);
-  return launch_attn_d<64>(q8, k8, v8, a, a.rows_per_slab, slabs, grid, stream);
+  dim3 grid;
+  int combine_ctas = 0;
+  if (varlen) {
+    a.pairs_per_head = 0;
+    a.full_ctas = 0;
+    a.nsplit = 1;
+    grid = dim3((max_seqlen + NQ * BLOCK_M - 1) / (NQ * BLOCK_M), H, nseq);
+  } else {
+    AttnSplitPlan p = plan_attention_split(B, H, L, D, num_sms);
+    if (workspace == nullptr || workspace_bytes < p.bytes) {   // no workspace: no split
+      p.nsplit = 1;
+      p.full_ctas += p.tail;
+      p.tail = 0;
+    }
+    a.pairs_per_head = p.pairs_per_head;
+    a.full_ctas = p.full_ctas;
+    a.nsplit = p.nsplit;
+    a.combine_pairs = p.tail;
+    if (p.tail > 0) {
+      const size_t o_elems = static_cast<size_t>(p.tail) * p.nsplit * NQ * BLOCK_M * D;
+      a.part_o = static_cast<float*>(workspace);
+      a.part_ml = reinterpret_cast<float2*>(a.part_o + o_elems);
+      combine_ctas = p.tail * NQ * BLOCK_M / COMBINE_WARPS;
+    }
+    grid = dim3(p.full_ctas + p.tail * p.nsplit, 1, 1);
+  }
+  if (D == 128)
+    return launch_attn_d<128>(q8, k8, v8, a, a.rows_per_slab, slabs, grid, combine_ctas, stream);
+  return launch_attn_d<64>(q8, k8, v8, a, a.rows_per_slab, slabs, grid, combine_ctas, stream);
 }
 
 }  // namespace qattn

@@ -1,0 +1,48 @@
+// launch.h -- host-side launchers of the kernels in quant.cu and attn_fwd.cu, called by the C ABI
+// layer (qattn_api.cu) after it has validated the arguments.  Internal to the library.
+#pragma once
+
+#include <cuda_runtime.h>
+
+#include <cstddef>
+#include <cstdint>
+
+namespace qattn {
+
+cudaError_t launch_amax(const void* x, size_t n, float* amax, int* err, int num_sms,
+                        cudaStream_t stream);
+cudaError_t launch_quant_fp8(const void* x, size_t n, const float* amax, uint8_t* out,
+                             float* scale, int* err, int num_sms, cudaStream_t stream);
+cudaError_t launch_quant_fp4_block(const void* x, size_t n, const float* amax, uint8_t* packed,
+                                   uint8_t* bscale, float* gscale, uint8_t* codes8, float* scale8,
+                                   int* err, int num_sms, cudaStream_t stream);
+cudaError_t launch_calib_quant_fp8(const void* x, size_t n, float* amax, uint8_t* out,
+                                   float* scale, void* workspace, uint64_t limit_ns, int* err,
+                                   int num_sms, cudaStream_t stream);
+cudaError_t launch_calib_quant_fp4_block(const void* x, size_t n, float* amax, uint8_t* packed,
+                                         uint8_t* bscale, float* gscale, uint8_t* codes8,
+                                         float* scale8, void* workspace, uint64_t limit_ns,
+                                         int* err, int num_sms, cudaStream_t stream);
+cudaError_t launch_calib_quant_qkv(const void* const* x, uint8_t* const* codes8, float* const* amax,
+                                   float* const* scale8, uint8_t* const* e2m1,
+                                   uint8_t* const* bscale, float* const* gscale, size_t n, int mode,
+                                   void* workspace, uint64_t limit_ns, int* err, int num_sms,
+                                   cudaStream_t stream);
+
+// How a dense attention launch splits its last, partial wave along the keys (see
+// plan_attention_split in attn_fwd.cu); bytes = workspace the split needs (0: no split).
+struct AttnSplitPlan {
+  int pairs_per_head, full_ctas, nsplit, tail;
+  size_t bytes;
+};
+AttnSplitPlan plan_attention_split(int B, int H, int L, int D, int num_sms);
+
+// workspace may be null (no split); it is used only when workspace_bytes covers the plan.
+cudaError_t launch_attention(const uint8_t* q8, const uint8_t* k8, const uint8_t* v8, void* out,
+                             int B, int H, int L, int D, const int* cu_seqlens, int nseq,
+                             int max_seqlen, int total_tokens, const float* s_q, const float* s_k,
+                             const float* s_v, float sm_scale, int* err, uint64_t timeout_ns,
+                             int inject_missing_q, void* workspace, size_t workspace_bytes,
+                             int num_sms, cudaStream_t stream);
+
+}  // namespace qattn

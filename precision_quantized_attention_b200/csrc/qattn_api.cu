@@ -2,35 +2,10 @@
 #include <cuda_runtime.h>
 #include <cstdint>
 
+#include "launch.h"
 #include "qattn.h"
 #include "sm100_ptx.cuh"
 
-namespace qattn {
-cudaError_t launch_amax(const void* x, size_t n, float* amax, int* err, int num_sms,
-                        cudaStream_t stream);
-cudaError_t launch_quant_fp8(const void* x, size_t n, const float* amax, uint8_t* out,
-                             float* scale, int* err, int num_sms, cudaStream_t stream);
-cudaError_t launch_quant_fp4_block(const void* x, size_t n, const float* amax, uint8_t* packed,
-                                   uint8_t* bscale, float* gscale, uint8_t* codes8, float* scale8,
-                                   int* err, int num_sms, cudaStream_t stream);
-cudaError_t launch_calib_quant_fp8(const void* x, size_t n, float* amax, uint8_t* out,
-                                   float* scale, void* workspace, uint64_t limit_ns, int* err,
-                                   int num_sms, cudaStream_t stream);
-cudaError_t launch_calib_quant_fp4_block(const void* x, size_t n, float* amax, uint8_t* packed,
-                                         uint8_t* bscale, float* gscale, uint8_t* codes8,
-                                         float* scale8, void* workspace, uint64_t limit_ns,
-                                         int* err, int num_sms, cudaStream_t stream);
-cudaError_t launch_calib_quant_qkv(const void* const* x, uint8_t* const* codes8, float* const* amax,
-                                   float* const* scale8, uint8_t* const* e2m1,
-                                   uint8_t* const* bscale, float* const* gscale, size_t n, int mode,
-                                   void* workspace, uint64_t limit_ns, int* err, int num_sms,
-                                   cudaStream_t stream);
-cudaError_t launch_attention(const uint8_t* q8, const uint8_t* k8, const uint8_t* v8, void* out,
-                             int B, int H, int L, int D, const int* cu_seqlens, int nseq,
-                             int max_seqlen, int total_tokens, const float* s_q, const float* s_k,
-                             const float* s_v, float sm_scale, int* err, uint64_t timeout_ns,
-                             int inject_missing_q, cudaStream_t stream);
-}  // namespace qattn
 
 // The device error word (one per device that loads the library).
 static __device__ int g_qattn_error = 0;
@@ -220,23 +195,42 @@ qattn_status qattn_calibrate_quantize_qkv(const qattn_quant_io* io, size_t n, qa
                                                  reinterpret_cast<cudaStream_t>(stream)));
 }
 
+qattn_status qattn_forward_ws(const uint8_t* q8, const uint8_t* k8, const uint8_t* v8,
+                              void* out_bf16, int B, int H, int L, int D,
+                              const qattn_scales* scales, float sm_scale, qattn_mode mode,
+                              void* workspace_dev, size_t workspace_bytes, qattn_stream_t stream) {
+  qattn_status st = check_attention_common(q8, k8, v8, out_bf16, H, D, scales, sm_scale, mode);
+  if (st != QATTN_OK) return st;
+  if (B < 1 || L < 1) return QATTN_ERR_INVALID_ARG;
+  if (B > 65535 || H > 65535) return QATTN_ERR_UNSUPPORTED;
+  if (static_cast<int64_t>(B) * H * L * D >= (int64_t(1) << 40)) return QATTN_ERR_UNSUPPORTED;
+  if (workspace_dev != nullptr && !aligned(workspace_dev, 16)) return QATTN_ERR_INVALID_ARG;
+  DeviceInfo* d = nullptr;
+  st = device_info(&d);
+  if (st != QATTN_OK) return st;
+  if (workspace_dev != nullptr &&
+      workspace_bytes < qattn::plan_attention_split(B, H, L, D, d->num_sms).bytes)
+    return QATTN_ERR_INVALID_ARG;
+  return from_cuda(qattn::launch_attention(q8, k8, v8, out_bf16, B, H, L, D, nullptr, 0, L, L,
+                                           scales->s_q, scales->s_k, scales->s_v, sm_scale,
+                                           d->err, g_timeout_ns, g_inject_missing_q,
+                                           workspace_dev, workspace_bytes, d->num_sms,
+                                           reinterpret_cast<cudaStream_t>(stream)));
+}
+
 qattn_status qattn_forward(const uint8_t* q8, const uint8_t* k8, const uint8_t* v8,
                            void* out_bf16, int B, int H, int L, int D,
                            const qattn_scales* scales, float sm_scale, qattn_mode mode,
                            qattn_stream_t stream) {
-  qattn_status st = check_attention_common(q8, k8, v8, out_bf16, H, D, scales, sm_scale, mode);
-  if (st != QATTN_OK) return st;
-  if (B < 1 || L < 1) return QATTN_ERR_INVALID_ARG;
-  if (static_cast<int64_t>(B) * H > 65535 * 65535LL || B > 65535 || H > 65535)
-    return QATTN_ERR_UNSUPPORTED;
-  if (static_cast<int64_t>(B) * H * L * D >= (int64_t(1) << 40)) return QATTN_ERR_UNSUPPORTED;
+  return qattn_forward_ws(q8, k8, v8, out_bf16, B, H, L, D, scales, sm_scale, mode, nullptr, 0,
+                          stream);
+}
+
+size_t qattn_forward_workspace_bytes(int B, int H, int L, int D) {
+  if (B < 1 || H < 1 || L < 1 || (D != 64 && D != 128)) return 0;
   DeviceInfo* d = nullptr;
-  st = device_info(&d);
-  if (st != QATTN_OK) return st;
-  return from_cuda(qattn::launch_attention(q8, k8, v8, out_bf16, B, H, L, D, nullptr, 0, L, L,
-                                           scales->s_q, scales->s_k, scales->s_v, sm_scale,
-                                           d->err, g_timeout_ns, g_inject_missing_q,
-                                           reinterpret_cast<cudaStream_t>(stream)));
+  if (device_info(&d) != QATTN_OK) return 0;
+  return qattn::plan_attention_split(B, H, L, D, d->num_sms).bytes;
 }
 
 qattn_status qattn_forward_varlen(const uint8_t* q8, const uint8_t* k8, const uint8_t* v8,
@@ -256,8 +250,8 @@ qattn_status qattn_forward_varlen(const uint8_t* q8, const uint8_t* k8, const ui
   return from_cuda(qattn::launch_attention(q8, k8, v8, out_bf16, 1, H, 0, D, cu_seqlens_dev,
                                            nseq, max_seqlen, total_tokens, scales->s_q,
                                            scales->s_k, scales->s_v, sm_scale, d->err,
-                                           g_timeout_ns, g_inject_missing_q,
-                                           reinterpret_cast<cudaStream_t>(stream)));
+                                           g_timeout_ns, g_inject_missing_q, nullptr, 0,
+                                           d->num_sms, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 qattn_status qattn_get_error(qattn_stream_t stream) {

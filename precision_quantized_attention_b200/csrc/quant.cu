@@ -13,6 +13,7 @@
 #include <cuda_runtime.h>
 #include <cstdint>
 
+#include "launch.h"
 #include "sm100_ptx.cuh"
 
 namespace qattn {

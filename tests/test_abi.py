@@ -79,6 +79,13 @@ def test_host_side_argument_errors():
     io[2].out_e2m1 = None                                                 # FP4 output missing
     assert qkv(io, 32, 1, FAKE, W, s0) == _lib.ERR_INVALID_ARG
     sc = _lib._Scales(0x10000, 0x10000, 0x10000)
+    fws = lib.qattn_forward_ws
+    assert fws(FAKE, FAKE, FAKE, FAKE, 1, 1, 16, 64, ctypes.byref(sc), 0.1, 0, MISALIGNED, 1 << 20,
+               s0) == _lib.ERR_INVALID_ARG                            # misaligned workspace
+    assert fws(FAKE, FAKE, FAKE, FAKE, 1, 1, 16, 96, ctypes.byref(sc), 0.1, 0, FAKE, 1 << 20,
+               s0) == _lib.ERR_UNSUPPORTED
+    assert lib.qattn_forward_workspace_bytes(1, 1, 16, 96) == 0          # D not supported
+    assert lib.qattn_forward_workspace_bytes(1, 0, 16, 64) == 0
     fwd = lib.qattn_forward
     assert fwd(FAKE, FAKE, FAKE, FAKE, 1, 1, 16, 96, ctypes.byref(sc), 0.1, 0, s0) == _lib.ERR_UNSUPPORTED
     assert fwd(FAKE, FAKE, FAKE, FAKE, 1, 1, 0, 64, ctypes.byref(sc), 0.1, 0, s0) == _lib.ERR_INVALID_ARG

@@ -106,3 +106,30 @@ def test_wait_timeout_reports_error_and_context_survives():
     assert status == qa._lib.ERR_TIMEOUT
     out = gpu_path(w, q, k, v).out.float().cpu().numpy()
     assert_close(out, oracle_path(w, q, k, v), "after timeout")
+
+
+@pytest.mark.parametrize("B,H,L,D", [(1, 2, 1000, 128), (2, 3, 777, 64), (1, 24, 8704, 128)])
+def test_split_last_wave_matches_unsplit_and_oracle(B, H, L, D):
+    """With a workspace the pairs after the last full wave are split along the keys and merged
+    by the combine kernel; the result equals the unsplit launch up to FP32 summation order and
+    meets the oracle bar."""
+    w = workloads.custom("split", "fp8", B, H, L, D, seed=40 + L)
+    q, k, v = workloads.make_qkv(w)
+    path = gpu_path(w, q, k, v)
+    nbytes = qa.forward_workspace_bytes(B, H, L, D)
+    assert nbytes > 0 and path.attn_workspace is not None        # these shapes do split
+    split = path.out.clone()
+    path.attend()                                                # same again: reusable workspace
+    assert torch.equal(path.out, split)
+    s = [path.scale[i:i + 1] for i in range(3)]
+    plain = torch.empty_like(path.out)
+    qa.forward(path.codes[0], path.codes[1], path.codes[2], plain, *s, w.sm_scale)
+    assert qa.get_error() == 0
+    # the two differ only by FP32 summation order: at most one bf16 rounding step apart
+    excess = ((split.float() - plain.float()).abs() - plain.float().abs() * 2.0 ** -7 - 1e-3)
+    assert excess.max().item() <= 0.0
+    rows = workloads.sample_rows(w, per_head=64).numpy() if L > 2000 else None
+    want = oracle_path(w, q, k, v, rows=rows)
+    got = split.float().reshape(-1, D)
+    got = (got[torch.as_tensor(rows, device=got.device)] if rows is not None else got).cpu().numpy()
+    assert_close(got.reshape(want.shape), want, f"split B{B} H{H} L{L} D{D}")
