@@ -461,13 +461,20 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
         const bool rise = m_new > m_run;
         if (__any_sync(0xFFFFFFFFu, rise)) {
           const float f = rise ? exp2_int(static_cast<int>(m_run - m_new)) : 1.0f;
+          uint64_t f2;                             // packed f32x2 multiplies
+          asm("mov.b64 %0, {%1, %1};" : "=l"(f2) : "f"(f));
 #pragma unroll
           for (int c4 = 0; c4 < D / 32; ++c4) {
             uint32_t v[32];
             tmem_ld32(tO + c4 * 32, v);
             tmem_wait_ld();
 #pragma unroll
-            for (int i = 0; i < 32; ++i) v[i] = __float_as_uint(__uint_as_float(v[i]) * f);
+            for (int i = 0; i < 32; i += 2) {
+              uint64_t pr;
+              asm("{\n\t.reg .b64 a;\n\tmov.b64 a, {%1, %2};\n\tmul.rn.f32x2 %0, a, %3;\n\t}"
+                  : "=l"(pr) : "r"(v[i]), "r"(v[i + 1]), "l"(f2));
+              asm("mov.b64 {%0, %1}, %2;" : "=r"(v[i]), "=r"(v[i + 1]) : "l"(pr));
+            }
             tmem_st32(tO + c4 * 32, v);
           }
           l *= f;
