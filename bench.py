@@ -158,25 +158,31 @@ def barrier(world):
 
 
 def max_over_ranks(x: float, world: int) -> float:
+    """Largest value over the ranks (time is reported as the slowest rank's)."""
     if world == 1:
         return x
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if torch.distributed.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
     return float(t.item())
+
+
+def replica_workload(w, rank: int, world: int):
+    """Weak scaling: every rank runs its own seeded problem of the same shape."""
+    if world == 1:
+        return w
+    import dataclasses
+    return dataclasses.replace(w, seed=w.seed + 100 * rank)
 
 
 def run_gpu(args):
     import precision_quantized_attention_b200 as qa
     rank, world, local = dist_setup(args.gpus)
     w = workloads.WORKLOADS[args.workload or ("edit_fp8" if args.mode == "fp8" else "edit_fp4")]
-    if w.varlen:
-        raise SystemExit("bench.py times dense workloads; varlen is covered by the parity tests")
-    if world > 1:   # each replica gets its own seeded problem
-        import dataclasses
-        w = dataclasses.replace(w, seed=w.seed + 100 * rank)
+    w = replica_workload(w, rank, world)
     q, k, v = workloads.make_qkv(w)
     qd, kd, vd = (t.cuda() for t in (q, k, v))
-    path = qa.QuantizedAttention(w.shape, w.mode, sm_scale=w.sm_scale)
+    path = qa.QuantizedAttention(w.shape, w.mode, cu_seqlens=w.cu_seqlens, sm_scale=w.sm_scale)
     flush = L2Flush()
     stream = torch.cuda.current_stream()
 
@@ -235,7 +241,8 @@ def e2e_time(args, w, q, k, v, qd, kd, vd, step, flush, stream, world):
     import precision_quantized_attention_b200 as qa
     qh, kh, vh = (t.pin_memory() for t in (q, k, v))
     ohs = [torch.empty(w.shape, dtype=torch.bfloat16).pin_memory() for _ in range(2)]
-    paths = [qa.QuantizedAttention(w.shape, w.mode, sm_scale=w.sm_scale) for _ in range(2)]
+    paths = [qa.QuantizedAttention(w.shape, w.mode, cu_seqlens=w.cu_seqlens, sm_scale=w.sm_scale)
+             for _ in range(2)]
     ins = [(qd, kd, vd), tuple(torch.empty_like(t) for t in (qd, kd, vd))]
     h2d, d2h = torch.cuda.Stream(), torch.cuda.Stream()
 
