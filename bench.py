@@ -288,6 +288,18 @@ def e2e_time(args, w, q, k, v, qd, kd, vd, step, flush, stream, world):
     return max_over_ranks(ms, world)
 
 
+def workload_data(w) -> str:
+    """How the synthetic inputs were made (same recipe as the tests)."""
+    parts = ["synthetic: seeded N(0,1) bf16 Q/K/V"]
+    if w.text_scale != 1.0:
+        parts.append(f"text rows x{w.text_scale:g}")
+    if w.outliers:
+        parts.append(f"{w.outliers} of {w.D} Q/K channels per head x{w.outlier_scale:g}")
+    if w.varlen:
+        parts.append("packed sequences " + "+".join(str(x) for x in w.seqlens))
+    return ", ".join(parts)
+
+
 def bench_config(w, world):
     """The workload description both arms print."""
     return {"workload": f"{w.name}: B={w.B} H={w.H} L={w.L} D={w.D} {w.mode.upper()} full attention"
@@ -324,7 +336,7 @@ def report(args, w, qkv, rank, world, ms, attn, quant, e2e_ms, clocks):
         "scaling": "weak",
         "vs_baseline": None,
         "dtype": "e4m3",
-        "data": "synthetic: seeded N(0,1) bf16 Q/K/V, 4 of 128 Q/K channels per head x10",
+        "data": workload_data(w),
         "config": bench_config(w, world),
         "roofline": {"bound": "tensor", "achieved": achieved_tf, "peak": fp8_peak,
                      "unit": "TFLOP/s", "frac": achieved_tf / fp8_peak,
@@ -397,7 +409,7 @@ def run_reference(args):
         "metric": "quantized attention TFLOP/s @L=8704,H=24,D=128 and % of B200 FP8 peak",
         "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "vs_baseline": None, "dtype": "f64", "data": workload_data(w),
         "config": bench_config(w, args.gpus),
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
                          "sample": r["sample"]},
