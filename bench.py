@@ -223,7 +223,10 @@ def run_gpu(args):
         e2e_ms = float("nan")
     else:
         e2e_ms = e2e_time(args, w, q, k, v, qd, kd, vd, step, flush, stream, world)
-    report(args, w, (q, k, v), rank, world, ms, attn, quant, e2e_ms, clocks)
+    # our kernels per step: the Q, K, V calibrate+quantize launch, the attention launch, and the
+    # combine launch when the last wave is split
+    launches = 2 + (1 if path.attn_workspace is not None else 0)
+    report(args, w, (q, k, v), rank, world, ms, attn, quant, e2e_ms, clocks, launches)
     barrier(world)
     del path
     if world > 1:
@@ -312,7 +315,7 @@ def bench_config(w, world):
                   "before the step starts"}
 
 
-def report(args, w, qkv, rank, world, ms, attn, quant, e2e_ms, clocks):
+def report(args, w, qkv, rank, world, ms, attn, quant, e2e_ms, clocks, launches):
     q = qkv[0]
     hbm_gbs, bf16_tf, peak_kind = load_peaks()
     fp8_peak = bf16_tf * FP8_PER_BF16
@@ -356,7 +359,7 @@ def report(args, w, qkv, rank, world, ms, attn, quant, e2e_ms, clocks):
                 "schedule": "pinned host bf16 Q/K/V -> device, fused calibrate+quantize, attention, "
                             "bf16 output -> host every step; uploads, compute and downloads on "
                             "three streams over two buffer sets, so consecutive steps overlap"},
-        "gpu_launches": 2 * args.steps,     # calibrate+quantize of Q, K, V; attention
+        "gpu_launches": launches * args.steps,
         "clocks": clock,
     }
     if rank == 0:

@@ -87,6 +87,11 @@ def test_host_side_argument_errors():
     assert lib.qattn_forward_workspace_bytes(1, 1, 16, 96) == 0          # D not supported
     assert lib.qattn_forward_workspace_bytes(1, 0, 16, 64) == 0
     fwd = lib.qattn_forward
+    # maximum sizes: B*H*L*D >= 2^40 elements and B or H > 65535 are refused on the host
+    assert fwd(FAKE, FAKE, FAKE, FAKE, 1, 65535, 1 << 20, 128, ctypes.byref(sc), 0.1, 0,
+               s0) == _lib.ERR_UNSUPPORTED
+    assert fwd(FAKE, FAKE, FAKE, FAKE, 70000, 1, 16, 64, ctypes.byref(sc), 0.1, 0,
+               s0) == _lib.ERR_UNSUPPORTED
     assert fwd(FAKE, FAKE, FAKE, FAKE, 1, 1, 16, 96, ctypes.byref(sc), 0.1, 0, s0) == _lib.ERR_UNSUPPORTED
     assert fwd(FAKE, FAKE, FAKE, FAKE, 1, 1, 0, 64, ctypes.byref(sc), 0.1, 0, s0) == _lib.ERR_INVALID_ARG
     assert fwd(FAKE, FAKE, FAKE, FAKE, 1, 1, 16, 64, ctypes.byref(sc), -1.0, 0, s0) == _lib.ERR_INVALID_ARG

@@ -133,3 +133,20 @@ def test_split_last_wave_matches_unsplit_and_oracle(B, H, L, D):
     got = split.float().reshape(-1, D)
     got = (got[torch.as_tensor(rows, device=got.device)] if rows is not None else got).cpu().numpy()
     assert_close(got.reshape(want.shape), want, f"split B{B} H{H} L{L} D{D}")
+
+
+@pytest.mark.parametrize("L,D", [(8704, 128), (1000, 64)])
+def test_zero_queries_give_the_mean_of_v(L, D):
+    """Degenerate case checked on every row at full size: Q = 0 makes every score 0, so every P
+    code is e4m3(448) = 448 exactly and each output row is the mean of the dequantized V rows of
+    its head (up to FP32 summation and the bf16 output rounding)."""
+    w = workloads.custom("zeroq", "fp8", 1, 24 if L > 2000 else 3, L, D, seed=21)
+    q, k, v = workloads.make_qkv(w)
+    q = torch.zeros_like(q)
+    path = gpu_path(w, q, k, v)
+    codes, s_v, _ = oracle.quantize_tensor(v, "fp8")
+    v_deq = torch.from_numpy(codes.reshape(v.shape)).view(torch.float8_e4m3fn).double() * s_v
+    want = v_deq.mean(dim=2, keepdim=True).expand_as(v_deq)             # [B, H, L, D]
+    got = path.out.double().cpu()
+    err = (got - want).abs() - want.abs() * 2.0 ** -8 - 1e-6            # bf16 rounding allowance
+    assert err.max().item() <= 0.0
