@@ -34,6 +34,12 @@
 // TMEM: S_0/P_0, S_1/P_1 (128 FP32 columns each; P uses the first 32), O_0, O_1 (D columns).
 // All waits are bounded (a global-timer limit); on expiry the CTA records a timeout in the
 // library's error word, drains what it issued and exits.
+//
+// Grid: dense launches are 1-D.  With a workspace, the pairs left after the last full wave of
+// one CTA per SM are split along the keys: each part CTA runs the same loop over its key range
+// and writes its unnormalised O rows, integer running max and row sum; k_attn_combine merges
+// the parts (exact power-of-two rescales) into the bf16 output.  Varlen launches keep a
+// (pair, head, sequence) grid without splitting.
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
 #include <cstdint>
