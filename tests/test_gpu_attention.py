@@ -150,3 +150,26 @@ def test_zero_queries_give_the_mean_of_v(L, D):
     got = path.out.double().cpu()
     err = (got - want).abs() - want.abs() * 2.0 ** -8 - 1e-6            # bf16 rounding allowance
     assert err.max().item() <= 0.0
+
+
+def test_power_of_two_scaling_of_v_scales_the_output_exactly():
+    """Full size: V * 2^3 has the same E4M3 codes and an 8x scale, so every bf16 output is
+    exactly 8x the unscaled one (bit-exact check of the whole path on every row)."""
+    w = workloads.WORKLOADS["edit_fp8"]
+    q, k, v = workloads.make_qkv(w)
+    a = gpu_path(w, q, k, v).out.clone()
+    b = gpu_path(w, q, k, (v.float() * 8.0).to(torch.bfloat16)).out
+    assert torch.equal(b, a * 8)
+
+
+def test_key_permutation_changes_only_the_summation_order():
+    """Permuting the keys (K and V rows together) leaves the method's result unchanged: with the
+    power-of-two running max the per-key P codes do not depend on the key order, so the GPU
+    outputs differ only by FP32 summation order (one bf16 step at most)."""
+    w = workloads.custom("perm", "fp8", 1, 4, 2000, 128, seed=31, outliers=4)
+    q, k, v = workloads.make_qkv(w)
+    perm = torch.randperm(w.L, generator=torch.Generator().manual_seed(5))
+    a = gpu_path(w, q, k, v).out.float()
+    b = gpu_path(w, q, k[:, :, perm], v[:, :, perm]).out.float()
+    excess = (a - b).abs() - a.abs() * 2.0 ** -7 - 1e-3
+    assert excess.max().item() <= 0.0
