@@ -250,7 +250,7 @@ __global__ void __launch_bounds__(256) k_quant_fp4_block(
 
 // -------------------------------------------------------------------------------------------
 // Fused calibrate + quantize (one cooperative launch per tensor).  Every CTA reduces the amax of
-// its contiguous chunk, publishes it with one atomicMax into the workspace and arrives on a
+// its contiguous chunk, publishes it with one max reduction into the workspace and arrives on a
 // grid-wide counter; after the last arrival every CTA quantizes its chunk, which it just read
 // and which is still in L2, so HBM sees the input once.  The spin on the counter is bounded by
 // a global-timer limit (a launch that somehow is not co-resident records DEV_ERR_TIMEOUT and
