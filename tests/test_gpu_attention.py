@@ -173,3 +173,50 @@ def test_key_permutation_changes_only_the_summation_order():
     b = gpu_path(w, q, k[:, :, perm], v[:, :, perm]).out.float()
     excess = (a - b).abs() - a.abs() * 2.0 ** -7 - 1e-3
     assert excess.max().item() <= 0.0
+
+
+def _dequantized(x, mode):
+    """The BMM operand the method feeds to BMM2: val(code) * scale, per element (oracle)."""
+    codes, s, _ = oracle.quantize_tensor(x, mode)
+    return (oracle.e4m3_table()[codes] * np.float64(s)).reshape(tuple(x.shape))
+
+
+def _p_code_bound(L):
+    """Relative bound on sum_j val(c_j)/448 / l - 1: E4M3 rounds each normal p*448 within
+    2^-4 of it (3 fraction bits); each subnormal code is off by at most 2^-10 absolute, against
+    l*448 >= 224 (the row maximum of p is above 1/2); plus bf16 output rounding and FP32 sums."""
+    return 2.0 ** -4 + L * 2.0 ** -10 / 224.0 + 2.0 ** -8
+
+
+@pytest.mark.parametrize("mode,D", [("fp8", 128), ("fp8", 64), ("fp4", 128)])
+def test_uniform_v_gives_v_within_the_p_code_bound(mode, D):
+    # every key of a head carries the same V row, so O = v8 * (sum_j val(c_j) / 448) / l
+    B, H, L = 1, 3, 700
+    w = workloads.custom(f"uniform_v_{mode}_{D}", mode, B, H, L, D, seed=31)
+    q, k, v = workloads.make_qkv(w)
+    v = v[:, :, :1, :].expand(B, H, L, D).contiguous()
+    path = gpu_path(w, q, k, v)
+    got = path.out.float().cpu().numpy()
+    assert_close(got, oracle_path(w, q, k, v), f"uniform V {mode} D={D}")
+    v8 = _dequantized(v, mode)[:, :, :1, :]
+    dev = np.abs(got - v8) / np.maximum(np.abs(v8), 1e-30)
+    bound = _p_code_bound(L)
+    assert float(dev[np.abs(np.broadcast_to(v8, got.shape)) > 0].max()) <= bound, dev.max()
+
+
+def test_dominant_key_gives_its_v_row():
+    # all queries point along (1, ..., 1); key j* = 3 * (1, ..., 1) scores ~48 binades above the
+    # rest, whose p * 448 then round to the zero code: every output row is v8[j*] * val(c)/448/p
+    B, H, L, D, jstar = 1, 2, 300, 128, 217
+    w = workloads.custom("dominant_key", "fp8", B, H, L, D, seed=32)
+    q, k, v = workloads.make_qkv(w)
+    q = (1.0 + 0.1 * q.float()).to(torch.bfloat16)
+    k = k.clone()
+    k[:, :, jstar, :] = 3.0
+    path = gpu_path(w, q, k, v)
+    got = path.out.float().cpu().numpy()
+    assert_close(got, oracle_path(w, q, k, v), "dominant key")
+    v8 = _dequantized(v, "fp8")[:, :, jstar:jstar + 1, :]
+    # per element: one code's rounding (<= 2^-4 relative) plus bf16 output rounding
+    excess = np.abs(got - v8) - (2.0 ** -4 + 2.0 ** -8) * np.abs(v8)
+    assert float(excess.max()) <= 1e-6, excess.max()
