@@ -359,11 +359,13 @@ def report(args, w, qkv, rank, world, ms, attn, quant, e2e_ms, clocks, launches)
                 "schedule": "pinned host bf16 Q/K/V -> device, fused calibrate+quantize, attention, "
                             "bf16 output -> host every step; uploads, compute and downloads on "
                             "three streams over two buffer sets, so consecutive steps overlap"},
-        "gpu_launches": launches * args.steps,
+        "gpu_launches": world * launches * args.steps,   # all ranks' launches in the timed steps
         "clocks": clock,
     }
     if rank == 0:
-        result["cpu_baseline"] = cpu_baseline(w, qkv=qkv) if not args.no_cpu_baseline else None
+        # the oracle is timed on the host cores at N=1 only
+        run_cpu = world == 1 and not args.no_cpu_baseline
+        result["cpu_baseline"] = cpu_baseline(w, qkv=qkv) if run_cpu else None
         print(json.dumps(result), flush=True)
 
 
