@@ -36,11 +36,11 @@ L2_FLUSH_BYTES = 256 << 20
 # DRAM bytes (read + write) of one launch of the attention kernel, from ncu on this build:
 #   ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum --clock-control none \
 #       -k regex:k_attn_fp8 -s 3 -c 1 python bench.py --steps 1 --warmup 3 --no-cpu-baseline --no-e2e
-# k_attn_fp8_fwd: 80.27 MB read (Q8 + K8 + V8 = 80.22 MB algorithmic) + 27.86 MB written (the
-# split pairs' partial results and part of the bf16 output; the rest of the output is still in
-# L2 when the kernel ends).  The combine kernel that follows reads the 30.4 MB of partials.
+# k_attn_fp8_fwd: 80.29 MB read (Q8 + K8 + V8 = 80.22 MB algorithmic) + 26.01 MB written (the
+# cut pairs' partial results and part of the bf16 output; the rest of the output is still in
+# L2 when the kernel ends).  The combine kernel that follows reads the partials back.
 # Re-capture when the kernel changes.
-ATTN_TRAFFIC_BYTES = {(8704, 24, 128): 80.27e6 + 27.86e6}
+ATTN_TRAFFIC_BYTES = {(8704, 24, 128): 80.29e6 + 26.01e6}
 ATTN_TRAFFIC_SOURCE = "ncu dram__bytes_read.sum + dram__bytes_write.sum, one launch, L=8704"
 
 
@@ -224,7 +224,7 @@ def run_gpu(args):
     else:
         e2e_ms = e2e_time(args, w, q, k, v, qd, kd, vd, step, flush, stream, world)
     # our kernels per step: the Q, K, V calibrate+quantize launch, the attention launch, and the
-    # combine launch when the last wave is split
+    # combine launch when tail pairs are cut
     launches = 2 + (1 if path.attn_workspace is not None else 0)
     report(args, w, (q, k, v), rank, world, ms, attn, quant, e2e_ms, clocks, launches)
     barrier(world)

@@ -186,22 +186,24 @@ QATTN_API qattn_status qattn_forward(const uint8_t* q8, const uint8_t* k8, const
                            const qattn_scales* scales, float sm_scale, qattn_mode mode,
                            qattn_stream_t stream);
 
-/* qattn_forward with a caller workspace that lets the kernel balance its last wave: the Q-tile
- * pairs left over after the last full wave of one CTA per SM are split along the keys into 2-4
- * parts; each part writes its unnormalised FP32 partial O, running row maximum and row sum to
- * the workspace, and a combine kernel merges them.  The maxima are integers (power-of-two
- * running max), so merging rescales by exact powers of two and the result equals the unsplit
- * one up to FP32 summation order.  workspace_dev: device, 16-byte aligned, at least
- * qattn_forward_workspace_bytes(B, H, L, D) bytes, no initial contents needed; NULL = no split
- * (exactly qattn_forward).  Calls sharing a workspace must not overlap on the device. */
+/* qattn_forward with a caller workspace that lets the kernel balance its work across SMs: the
+ * attention kernel is persistent (one CTA per SM); after an equal share of whole Q-tile pairs
+ * per CTA, the key steps of the remaining pairs are cut into equal contiguous ranges, one per
+ * CTA.  A range that covers part of a pair writes its unnormalised FP32 partial O, running row
+ * maximum and row sum to the workspace, and a combine kernel merges the parts.  The maxima are
+ * integers (power-of-two running max), so merging rescales by exact powers of two and the result
+ * equals the uncut one up to FP32 summation order.  workspace_dev: device, 16-byte aligned, at
+ * least qattn_forward_workspace_bytes(B, H, L, D) bytes, no initial contents needed; NULL = no
+ * pair is cut (exactly qattn_forward).  Calls sharing a workspace must not overlap on the
+ * device. */
 QATTN_API qattn_status qattn_forward_ws(const uint8_t* q8, const uint8_t* k8, const uint8_t* v8,
                                         void* out_bf16, int B, int H, int L, int D,
                                         const qattn_scales* scales, float sm_scale,
                                         qattn_mode mode, void* workspace_dev,
                                         size_t workspace_bytes, qattn_stream_t stream);
 
-/* Workspace bytes qattn_forward_ws uses for this shape on the current device (0: this shape
- * needs no split, or the arguments or device are not supported). */
+/* Workspace bytes qattn_forward_ws uses for this shape on the current device (0: no pair of
+ * this shape is cut, or the arguments or device are not supported). */
 QATTN_API size_t qattn_forward_workspace_bytes(int B, int H, int L, int D);
 
 /* Same over a packed batch of variable-length sequences ([1, H, T, D] with sequence s at token

@@ -61,7 +61,8 @@ class QuantizedAttention:
         self.out = torch.empty(shape, dtype=torch.bfloat16, device=dev)
         self.workspace = new_workspace(dev)
         self.varlen = cu_seqlens is not None
-        # attention workspace: balances the last wave of a dense launch (none for varlen)
+        # attention workspace: lets a dense launch cut its tail pairs so that every SM runs the
+        # same number of key steps (none for varlen)
         nbytes = 0 if self.varlen else forward_workspace_bytes(B, H, T, D)
         self.attn_workspace = torch.empty(nbytes, dtype=torch.uint8, device=dev) if nbytes else None
         if self.varlen:

@@ -231,15 +231,16 @@ def _scales(s_q, s_k, s_v):
 
 
 def forward_workspace_bytes(B: int, H: int, L: int, D: int) -> int:
-    """Bytes of the workspace forward() uses to balance its last wave (0: none needed)."""
+    """Bytes of the workspace forward() uses to cut its tail pairs (0: none needed)."""
     return int(load().qattn_forward_workspace_bytes(int(B), int(H), int(L), int(D)))
 
 
 def forward(q8, k8, v8, out, s_q, s_k, s_v, sm_scale: float, mode: int = MODE_FP8, stream=None,
             workspace: torch.Tensor | None = None):
     """q8, k8, v8: uint8 E4M3 codes [B, H, L, D]; out: bf16 [B, H, L, D].  With a workspace of
-    forward_workspace_bytes(B, H, L, D) bytes (uint8 CUDA tensor) the last wave is balanced by
-    splitting it along the keys (qattn_forward_ws); without one, qattn_forward."""
+    forward_workspace_bytes(B, H, L, D) bytes (uint8 CUDA tensor) the persistent kernel cuts the
+    pairs left after an equal share of whole pairs per SM along the keys (qattn_forward_ws);
+    without one, qattn_forward."""
     B, H, L, D = q8.shape
     for t, nm in ((k8, "k8"), (v8, "v8"), (out, "out")):
         if tuple(t.shape) != (B, H, L, D):

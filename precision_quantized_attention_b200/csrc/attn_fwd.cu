@@ -17,7 +17,8 @@
 //     not depend on how keys are tiled.
 //
 // Kernel structure: one CTA (one per SM) per pair of 128-row Q tiles of one (sequence, head).
-//   warp 8      TMA producer: both Q tiles once, then K and V tiles through separate rings.
+//   warp 8      TMA producer: per segment both Q tiles, then K and V tiles through separate
+//               rings.
 //   warp 9      MMA issuer (one elected thread) and TMEM owner.  Per KV tile j and Q tile t it
 //               issues O_t += P_t(j) V_j (P read from tensor memory) and right behind it, in the
 //               same in-order tcgen05 stream, S_t = Q_t K_{j+1}^T into the columns P_t(j)
@@ -35,11 +36,14 @@
 // All waits are bounded (a global-timer limit); on expiry the CTA records a timeout in the
 // library's error word, drains what it issued and exits.
 //
-// Grid: dense launches are 1-D.  With a workspace, the pairs left after the last full wave of
-// one CTA per SM are split along the keys: each part CTA runs the same loop over its key range
-// and writes its unnormalised O rows, integer running max and row sum; k_attn_combine merges
-// the parts (exact power-of-two rescales) into the bf16 output.  Varlen launches keep a
-// (pair, head, sequence) grid without splitting.
+// Grid: dense launches are persistent, one CTA per SM.  Each CTA runs a list of segments (key
+// ranges of one pair of Q tiles): an equal share of whole pairs, then, with a workspace, a
+// contiguous range of the remaining pairs' key steps laid end to end, so that every CTA runs
+// the same number of key steps.  A segment that covers part of a pair writes its unnormalised
+// O rows, integer running max and row sum; k_attn_combine merges the parts (exact power-of-two
+// rescales) into the bf16 output.  Between segments Q is double-buffered, and the first P V of
+// a segment waits until the softmax has read out the previous segment's O.  Varlen launches
+// keep a (pair, head, sequence) grid, one segment per CTA.
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
 #include <cstdint>
@@ -74,36 +78,94 @@ struct AttnArgs {
   int* err;
   uint64_t timeout_ns;
   int inject_missing_q;     // fault injection for tests: the producer never loads Q
-  // Dense launches use a 1-D grid: CTAs [0, full_ctas) take one pair of Q tiles each; the pairs
-  // after them (the last, partial wave) are split into nsplit parts along the keys, one CTA per
-  // part, which writes unnormalised partial results for the combine kernel:
-  //   part_o[(((tp * nsplit + part) * NQ + t) * BLOCK_M + row) * D + c]  (FP32, row-major)
-  //   part_ml[((tp * nsplit + part) * NQ + t) * BLOCK_M + row] = (running max, row sum)
-  // with tp the index of the pair among the split ones.
+  // Dense launches are persistent: G = ctas CTAs, at most one per SM.  CTA c runs, in order,
+  // the pairs of Q tiles c, c + G, ..., c + (whole - 1) G whole, and then the key steps
+  // [c * tail_w, (c + 1) * tail_w) of the tail: the pairs from whole * G on, their key steps
+  // laid end to end.  A tail range is at most one pair long, so a CTA has at most two tail
+  // segments; one that covers only part of a pair writes unnormalised partial results to slot
+  // 2c (the CTA's first tail segment) or 2c + 1 (its second), for the combine kernel:
+  //   part_o[((slot * NQ + t) * BLOCK_M + row) * D + c]   (FP32, row-major)
+  //   part_ml[(slot * NQ + t) * BLOCK_M + row] = (running max, row sum)
   int pairs_per_head;
-  int full_ctas;
-  int nsplit;
-  int combine_pairs;        // number of split pairs (the combine kernel's work)
+  int nkv;                  // key steps of a pair (dense)
+  int ctas;                 // G
+  int whole;                // whole pairs per CTA
+  int tail_pairs;
+  int tail_w;               // tail key steps per CTA, 1..nkv (nkv: no pair is cut)
   float* part_o;
   float2* part_ml;
 };
+
+// One unit of a CTA's work: key steps [kv0, kv1) of one pair of Q tiles.
+struct Seg {
+  int q_row0, seq_start, seq_len, slab;
+  int kv0, kv1;
+  int slot;                 // partial-result slot, or -1 when the segment covers the whole pair
+};
+
+// The i-th segment of this CTA (false when it has no more).  Varlen launches keep one pair per
+// CTA (grid = pairs x heads x sequences); dense ones follow the persistent schedule above.
+__device__ __forceinline__ bool get_segment(const AttnArgs& a, int i, Seg& s) {
+  int pair;
+  if (a.cu_seqlens) {
+    if (i > 0) return false;
+    const int bz = blockIdx.z;
+    s.seq_start = __ldg(a.cu_seqlens + bz);
+    s.seq_len = __ldg(a.cu_seqlens + bz + 1) - s.seq_start;
+    s.slab = blockIdx.y;
+    s.q_row0 = blockIdx.x * (NQ * BLOCK_M);
+    s.kv0 = 0;
+    s.kv1 = (s.seq_len + BLOCK_N - 1) / BLOCK_N;
+    s.slot = -1;
+    return s.q_row0 < s.seq_len;
+  }
+  const int c = blockIdx.x;
+  if (i < a.whole) {
+    pair = c + i * a.ctas;
+    s.kv0 = 0;
+    s.kv1 = a.nkv;
+    s.slot = -1;
+  } else {
+    const int k = i - a.whole;                   // tail segment 0 or 1
+    if (k > 1) return false;
+    const long long end = static_cast<long long>(a.tail_pairs) * a.nkv;
+    long long g0 = static_cast<long long>(c) * a.tail_w;
+    const long long g1 = min(g0 + a.tail_w, end);
+    if (k == 1) g0 = (g0 / a.nkv + 1) * a.nkv;   // the second segment starts at a pair start
+    if (g0 >= g1) return false;
+    const int tp = static_cast<int>(g0 / a.nkv);
+    s.kv0 = static_cast<int>(g0 - static_cast<long long>(tp) * a.nkv);
+    s.kv1 = static_cast<int>(min(static_cast<long long>(a.nkv), s.kv0 + (g1 - g0)));
+    s.slot = (s.kv0 == 0 && s.kv1 == a.nkv) ? -1 : 2 * c + k;
+    pair = a.whole * a.ctas + tp;
+  }
+  const int qblk = pair % a.pairs_per_head;
+  const int h = (pair / a.pairs_per_head) % a.H;
+  const int bz = pair / (a.pairs_per_head * a.H);
+  s.seq_start = 0;
+  s.seq_len = a.L;
+  s.slab = bz * a.H + h;
+  s.q_row0 = qblk * (NQ * BLOCK_M);
+  return true;
+}
 
 template <int D>
 struct Smem {
   static constexpr int TILE_Q = BLOCK_M * D;       // bytes (E4M3)
   static constexpr int TILE_KV = BLOCK_N * D;
-  static constexpr int OFF_Q = 0;
-  static constexpr int OFF_K = OFF_Q + NQ * TILE_Q;
+  static constexpr int OFF_Q = 0;                  // two buffers of NQ tiles (segment i: i % 2)
+  static constexpr int OFF_K = OFF_Q + 2 * NQ * TILE_Q;
   static constexpr int OFF_V = OFF_K + KSTAGES * TILE_KV;
   static constexpr int OFF_BAR = OFF_V + VSTAGES * TILE_KV;
-  // barriers: q_full, k_full[KS], k_empty[KS], v_full[VS], v_empty[VS], s_full[NQ],
-  // p_full[NQ], o_final[NQ], drain
-  static constexpr int NBARS = 1 + 2 * KSTAGES + 2 * VSTAGES + 3 * NQ + 1;
+  // barriers: q_full[2], q_empty[2], k_full[KS], k_empty[KS], v_full[VS], v_empty[VS],
+  // s_full[NQ], p_full[NQ], o_final[NQ], o_free[NQ], drain
+  static constexpr int NBARS = 4 + 2 * KSTAGES + 2 * VSTAGES + 4 * NQ + 1;
   static constexpr int OFF_TMEM = OFF_BAR + 8 * NBARS;
   static constexpr int OFF_ABORT = OFF_TMEM + 4;
   static constexpr int BYTES = OFF_ABORT + 4;
   static constexpr int ALLOC = BYTES + 1024;       // slack for 1024-byte alignment
   static_assert(TILE_Q % 1024 == 0 && TILE_KV % 1024 == 0, "alignment");
+  static_assert(ALLOC <= 227 * 1024, "shared memory per CTA");
 };
 
 template <int D>
@@ -207,7 +269,7 @@ __device__ __forceinline__ float rowmax128(const float (&s)[128]) {
 template <int D>
 __global__ void __launch_bounds__(ATTN_THREADS, 1)
     k_attn_fp8_fwd(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                   const __grid_constant__ CUtensorMap tm_v, const AttnArgs args) {
+                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ AttnArgs args) {
   using SL = Smem<D>;
   using TC = TmemCols<D>;
   extern __shared__ uint8_t smem_raw[];
@@ -217,65 +279,33 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-
-  // ---- which sequence and which rows -------------------------------------------------------
-  int qblk, h, bz;                                // pair of Q tiles, head, batch row / sequence
-  int part = 0, nparts = 1, split_pair = -1;
-  if (args.cu_seqlens) {
-    qblk = blockIdx.x;
-    h = blockIdx.y;
-    bz = blockIdx.z;
-  } else {
-    int pair = blockIdx.x;
-    if (pair >= args.full_ctas) {                 // a part of a split pair
-      const int u = pair - args.full_ctas;
-      split_pair = u / args.nsplit;
-      part = u % args.nsplit;
-      nparts = args.nsplit;
-      pair = args.full_ctas + split_pair;
-    }
-    qblk = pair % args.pairs_per_head;
-    h = (pair / args.pairs_per_head) % args.H;
-    bz = pair / (args.pairs_per_head * args.H);
+  {
+    Seg s0;
+    if (!get_segment(args, 0, s0)) return;        // uniform over the CTA: nothing to do
   }
-  int seq_start, seq_len, slab;
-  if (args.cu_seqlens) {
-    seq_start = __ldg(args.cu_seqlens + bz);
-    seq_len = __ldg(args.cu_seqlens + bz + 1) - seq_start;
-    slab = h;
-  } else {
-    seq_start = 0;
-    seq_len = args.L;
-    slab = bz * args.H + h;
-  }
-  const int q_row0 = qblk * (NQ * BLOCK_M);
-  if (q_row0 >= seq_len) return;                  // uniform over the CTA: nothing to do
-  // key steps [kv0, kv0 + nkv) of this CTA (all of them unless the pair is split)
-  const int nkv_all = (seq_len + BLOCK_N - 1) / BLOCK_N;
-  const int steps_per_part = (nkv_all + nparts - 1) / nparts;
-  const int kv0 = part * steps_per_part;
-  const int nkv = min(nkv_all, kv0 + steps_per_part) - kv0;   // >= 1: the host keeps parts
-                                                               // shorter than the sequence
 
   // ---- barriers --------------------------------------------------------------------------
+  // Phases run on across segments: the K/V rings count loads, s_full / p_full count key steps,
+  // o_final / o_free count segments, q_full / q_empty count the uses of each Q buffer.
   const uint32_t bar0 = base_u32 + SL::OFF_BAR;
   auto BAR = [&](int i) { return bar0 + 8u * static_cast<uint32_t>(i); };
-  constexpr int B_QFULL = 0;
-  constexpr int B_KFULL = 1, B_KEMPTY = B_KFULL + KSTAGES;
+  constexpr int B_QFULL = 0, B_QEMPTY = 2;
+  constexpr int B_KFULL = 4, B_KEMPTY = B_KFULL + KSTAGES;
   constexpr int B_VFULL = B_KEMPTY + KSTAGES, B_VEMPTY = B_VFULL + VSTAGES;
   constexpr int B_SFULL = B_VEMPTY + VSTAGES, B_PFULL = B_SFULL + NQ;
-  constexpr int B_OFINAL = B_PFULL + NQ, B_DRAIN = B_OFINAL + NQ;
+  constexpr int B_OFINAL = B_PFULL + NQ, B_OFREE = B_OFINAL + NQ, B_DRAIN = B_OFREE + NQ;
   volatile int* abort_flag = reinterpret_cast<volatile int*>(base + SL::OFF_ABORT);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base + SL::OFF_TMEM);
 
   if (threadIdx.x == 0) {
-    mbar_init(BAR(B_QFULL), 1);
+    for (int b = 0; b < 2; ++b) { mbar_init(BAR(B_QFULL + b), 1); mbar_init(BAR(B_QEMPTY + b), 1); }
     for (int i = 0; i < KSTAGES; ++i) { mbar_init(BAR(B_KFULL + i), 1); mbar_init(BAR(B_KEMPTY + i), 1); }
     for (int i = 0; i < VSTAGES; ++i) { mbar_init(BAR(B_VFULL + i), 1); mbar_init(BAR(B_VEMPTY + i), 1); }
     for (int t = 0; t < NQ; ++t) {
       mbar_init(BAR(B_SFULL + t), 1);
       mbar_init(BAR(B_PFULL + t), BLOCK_M);
       mbar_init(BAR(B_OFINAL + t), 1);
+      mbar_init(BAR(B_OFREE + t), BLOCK_M);
     }
     mbar_init(BAR(B_DRAIN), 1);
     *abort_flag = 0;
@@ -297,41 +327,52 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
       tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
-      int nk = 0, nv = 0;                          // loads issued
-      mbar_arrive_expect_tx(BAR(B_QFULL), NQ * SL::TILE_Q);
-      for (int t = 0; t < NQ; ++t)
-        tma_load_3d(base_u32 + SL::OFF_Q + t * SL::TILE_Q, &tm_q, BAR(B_QFULL), 0,
-                    seq_start + q_row0 + t * BLOCK_M, slab);
-      auto load_k = [&](int j) -> bool {
-        const int s = j % KSTAGES;
-        if (j >= KSTAGES &&
-            !mbar_wait(BAR(B_KEMPTY + s), ((j / KSTAGES) - 1) & 1, tlim, abort_flag, args.err))
+      int nk = 0, nv = 0, nseg = 0;                // loads issued (K, V tiles; Q buffers)
+      Seg sg{};
+      auto load_k = [&](int kv) -> bool {
+        const int s = nk % KSTAGES;
+        if (nk >= KSTAGES &&
+            !mbar_wait(BAR(B_KEMPTY + s), ((nk / KSTAGES) - 1) & 1, tlim, abort_flag, args.err))
           return false;
         mbar_arrive_expect_tx(BAR(B_KFULL + s), SL::TILE_KV);
         tma_load_3d(base_u32 + SL::OFF_K + s * SL::TILE_KV, &tm_k, BAR(B_KFULL + s), 0,
-                    seq_start + (kv0 + j) * BLOCK_N, slab);
+                    sg.seq_start + kv * BLOCK_N, sg.slab);
         ++nk;
         return true;
       };
-      auto load_v = [&](int j) -> bool {
-        const int s = j % VSTAGES;
-        if (j >= VSTAGES &&
-            !mbar_wait(BAR(B_VEMPTY + s), ((j / VSTAGES) - 1) & 1, tlim, abort_flag, args.err))
+      auto load_v = [&](int kv) -> bool {
+        const int s = nv % VSTAGES;
+        if (nv >= VSTAGES &&
+            !mbar_wait(BAR(B_VEMPTY + s), ((nv / VSTAGES) - 1) & 1, tlim, abort_flag, args.err))
           return false;
         mbar_arrive_expect_tx(BAR(B_VFULL + s), SL::TILE_KV);
         tma_load_3d(base_u32 + SL::OFF_V + s * SL::TILE_KV, &tm_v, BAR(B_VFULL + s), 0,
-                    seq_start + (kv0 + j) * BLOCK_N, slab);
+                    sg.seq_start + kv * BLOCK_N, sg.slab);
         ++nv;
         return true;
       };
-      // order of use on the tensor pipe: K0, V0, K1, V1, ...; K runs one tile ahead
-      bool ok = load_k(0);
-      for (int j = 0; ok && j < nkv; ++j) {
-        if (j + 1 < nkv) ok = load_k(j + 1);
-        if (ok) ok = load_v(j);
+      bool ok = true;
+      for (int i = 0; ok && get_segment(args, i, sg); ++i) {
+        // Q buffer i % 2: free once the MMAs of segment i - 2 that read it have completed
+        const int b = i & 1;
+        if (i >= 2 && !mbar_wait(BAR(B_QEMPTY + b), ((i >> 1) - 1) & 1, tlim, abort_flag, args.err))
+          break;
+        mbar_arrive_expect_tx(BAR(B_QFULL + b), NQ * SL::TILE_Q);
+        for (int t = 0; t < NQ; ++t)
+          tma_load_3d(base_u32 + SL::OFF_Q + (b * NQ + t) * SL::TILE_Q, &tm_q, BAR(B_QFULL + b), 0,
+                      sg.seq_start + sg.q_row0 + t * BLOCK_M, sg.slab);
+        ++nseg;
+        // order of use on the tensor pipe: K0, V0, K1, V1, ...; K runs one tile ahead
+        const int n = sg.kv1 - sg.kv0;
+        ok = load_k(sg.kv0);
+        for (int j = 0; ok && j < n; ++j) {
+          if (j + 1 < n) ok = load_k(sg.kv0 + j + 1);
+          if (ok) ok = load_v(sg.kv0 + j);
+        }
       }
       // drain: every issued load has landed before the CTA may exit (instant when healthy)
-      mbar_drain(BAR(B_QFULL), 0, tlim);
+      for (int i = nseg - 1; i >= 0 && i >= nseg - 2; --i)
+        mbar_drain(BAR(B_QFULL + (i & 1)), (i >> 1) & 1, tlim);
       for (int j = nk - 1; j >= 0 && j >= nk - KSTAGES; --j)
         mbar_drain(BAR(B_KFULL + j % KSTAGES), (j / KSTAGES) & 1, tlim);
       for (int j = nv - 1; j >= 0 && j >= nv - VSTAGES; --j)
@@ -349,8 +390,8 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
       // of 32 keys advances 32 rows.
       constexpr uint32_t V_LAYOUT = QK_LAYOUT;
       constexpr uint32_t V_SBO = 8 * D;
-      auto bmm1 = [&](int t, int ks) {
-        const uint32_t qa = base_u32 + SL::OFF_Q + t * SL::TILE_Q;
+      auto bmm1 = [&](int t, int qb, int ks) {
+        const uint32_t qa = base_u32 + SL::OFF_Q + (qb * NQ + t) * SL::TILE_Q;
         const uint32_t kb = base_u32 + SL::OFF_K + ks * SL::TILE_KV;
 #pragma unroll
         for (int kk = 0; kk < D / 32; ++kk) {
@@ -368,39 +409,58 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
                     (!first || kk > 0) ? 1u : 0u);
         }
       };
-      bool ok = mbar_wait(BAR(B_QFULL), 0, tlim, abort_flag, args.err) &&
-                mbar_wait(BAR(B_KFULL + 0), 0, tlim, abort_flag, args.err);
-      if (ok) {
+      int nk = 0, nv = 0, step = 0;               // K, V tiles consumed; key steps before this segment
+      bool ok = true;
+      Seg sg{};
+      for (int i = 0; ok && get_segment(args, i, sg); ++i) {
+        const int qb = i & 1;
+        const int n = sg.kv1 - sg.kv0;
+        // S_t of the segment's first key step (S_t is free: the last P V of the previous
+        // segment, which read P_t from it, precedes in the MMA stream)
+        ok = mbar_wait(BAR(B_QFULL + qb), (i >> 1) & 1, tlim, abort_flag, args.err) &&
+             mbar_wait(BAR(B_KFULL + nk % KSTAGES), (nk / KSTAGES) & 1, tlim, abort_flag, args.err);
+        if (!ok) break;
         tc_fence_after();
         for (int t = 0; t < NQ; ++t) {
-          bmm1(t, 0);
+          bmm1(t, qb, nk % KSTAGES);
           mma_commit(BAR(B_SFULL + t));
         }
-        mma_commit(BAR(B_KEMPTY + 0));
-      }
-      for (int j = 0; ok && j < nkv; ++j) {
-        const int vs = j % VSTAGES;
-        const bool more = j + 1 < nkv;
-        const int ks = (j + 1) % KSTAGES;
-        ok = mbar_wait(BAR(B_VFULL + vs), (j / VSTAGES) & 1, tlim, abort_flag, args.err);
-        if (ok && more)
-          ok = mbar_wait(BAR(B_KFULL + ks), ((j + 1) / KSTAGES) & 1, tlim, abort_flag, args.err);
-        for (int t = 0; ok && t < NQ; ++t) {
-          ok = mbar_wait(BAR(B_PFULL + t), j & 1, tlim, abort_flag, args.err);
-          if (!ok) break;
-          tc_fence_after();
-          bmm2(t, vs, j == 0);                     // reads P_t(j) from TMEM
-          if (more) {
-            bmm1(t, ks);                           // overwrites S_t / P_t after bmm2 read it
-            mma_commit(BAR(B_SFULL + t));
-          } else {
-            mma_commit(BAR(B_OFINAL + t));
+        mma_commit(BAR(B_KEMPTY + nk % KSTAGES));
+        ++nk;
+        // the first P V of this segment overwrites O_t: softmax t has read out the last one
+        for (int t = 0; ok && i > 0 && t < NQ; ++t)
+          ok = mbar_wait(BAR(B_OFREE + t), (i - 1) & 1, tlim, abort_flag, args.err);
+        const int pbase = step & 1;
+        for (int j = 0; ok && j < n; ++j) {
+          const int vs = nv % VSTAGES;
+          const bool more = j + 1 < n;
+          const int ks = nk % KSTAGES;
+          ok = mbar_wait(BAR(B_VFULL + vs), (nv / VSTAGES) & 1, tlim, abort_flag, args.err);
+          if (ok && more)
+            ok = mbar_wait(BAR(B_KFULL + ks), (nk / KSTAGES) & 1, tlim, abort_flag, args.err);
+          for (int t = 0; ok && t < NQ; ++t) {
+            ok = mbar_wait(BAR(B_PFULL + t), pbase ^ (j & 1), tlim, abort_flag, args.err);
+            if (!ok) break;
+            tc_fence_after();
+            bmm2(t, vs, j == 0);                   // reads P_t from TMEM
+            if (more) {
+              bmm1(t, qb, ks);                     // overwrites S_t / P_t after bmm2 read it
+              mma_commit(BAR(B_SFULL + t));
+            } else {
+              mma_commit(BAR(B_OFINAL + t));
+            }
+          }
+          if (ok) {
+            mma_commit(BAR(B_VEMPTY + vs));
+            ++nv;
+            if (more) {
+              mma_commit(BAR(B_KEMPTY + ks));
+              ++nk;
+            }
           }
         }
-        if (ok) {
-          mma_commit(BAR(B_VEMPTY + vs));
-          if (more) mma_commit(BAR(B_KEMPTY + ks));
-        }
+        if (ok) mma_commit(BAR(B_QEMPTY + qb));   // every MMA reading Q buffer qb is issued
+        step += n;
       }
       // drain: all issued MMAs complete before TMEM is released
       mma_commit(BAR(B_DRAIN));
@@ -415,12 +475,16 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
     const uint32_t tS = tmem + lane_off + TC::S0 + t * BLOCK_N;
     const uint32_t tO = tmem + lane_off + TC::O0 + t * D;
     const float c = __ldg(args.s_q) * __ldg(args.s_k) * args.sm_scale * LOG2E_F;
+    bool ok = true;
+    int step = 0;                                  // key steps of the earlier segments
+    Seg sg{};
+    for (int seg = 0; ok && get_segment(args, seg, sg); ++seg) {
+    const int n = sg.kv1 - sg.kv0;
     float m_run = -INFINITY;                       // integer-valued running max (base 2)
     float l = 0.0f;                                // running sum of p * 448
-    bool ok = true;
-    for (int j = 0; j < nkv; ++j) {
+    for (int j = 0; j < n; ++j) {
       // S_t(j) is in TMEM; BMM2 of tile j-1 has completed (it precedes in the MMA stream)
-      ok = mbar_wait(BAR(B_SFULL + t), j & 1, tlim, abort_flag, args.err);
+      ok = mbar_wait(BAR(B_SFULL + t), (step + j) & 1, tlim, abort_flag, args.err);
       if (!__all_sync(0xFFFFFFFFu, ok)) { ok = false; break; }
       tc_fence_after();
       float s[BLOCK_N];
@@ -432,7 +496,7 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
 #pragma unroll
         for (int i = 0; i < BLOCK_N; ++i) s[i] = __uint_as_float(sv[i / 32][i % 32]);
       }
-      const int kv_valid = seq_len - (kv0 + j) * BLOCK_N;  // keys of this tile in the sequence
+      const int kv_valid = sg.seq_len - (sg.kv0 + j) * BLOCK_N;  // keys of this tile in the sequence
       if (kv_valid < BLOCK_N) {
 #pragma unroll
         for (int i = 0; i < BLOCK_N; ++i)
@@ -495,15 +559,17 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
       tc_fence_before();
       mbar_arrive(BAR(B_PFULL + t));
     }
-    if (ok) {
-      ok = mbar_wait(BAR(B_OFINAL + t), 0, tlim, abort_flag, args.err);
-      if (__all_sync(0xFFFFFFFFu, ok)) {
+    if (!ok) break;
+    {
+      ok = mbar_wait(BAR(B_OFINAL + t), seg & 1, tlim, abort_flag, args.err);
+      if (!__all_sync(0xFFFFFFFFu, ok)) { ok = false; break; }
+      {
         tc_fence_after();
-        const int row = q_row0 + t * BLOCK_M + r;
-        const bool valid = row < seq_len;
-        if (nparts > 1) {
-          // partial result of this part: raw O row, running max and row sum
-          const size_t slot = (static_cast<size_t>(split_pair) * nparts + part) * NQ + t;
+        const int row = sg.q_row0 + t * BLOCK_M + r;
+        const bool valid = row < sg.seq_len;
+        if (sg.slot >= 0) {
+          // partial result of this segment: raw O row, running max and row sum
+          const size_t slot = static_cast<size_t>(sg.slot) * NQ + t;
           float4* po = reinterpret_cast<float4*>(args.part_o + (slot * BLOCK_M + r) * D);
 #pragma unroll
           for (int c4 = 0; c4 < D / 32; ++c4) {
@@ -519,7 +585,7 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
         } else {
         const float scale = __ldg(args.s_v) / l;   // O = acc * s_v / 448 / (l / 448)
         __nv_bfloat16* orow =
-            args.out + (static_cast<size_t>(slab) * args.rows_per_slab + seq_start + row) * D;
+            args.out + (static_cast<size_t>(sg.slab) * args.rows_per_slab + sg.seq_start + row) * D;
 #pragma unroll
         for (int c4 = 0; c4 < D / 32; ++c4) {
           uint32_t v[32];
@@ -542,6 +608,10 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
         }
       }
     }
+    tc_fence_before();
+    mbar_arrive(BAR(B_OFREE + t));                 // O_t is read out: the next segment may overwrite it
+    step += n;
+    }
   }
 
   tc_fence_before();
@@ -552,11 +622,15 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
   }
 }
 
+
 // ---------------------------------------------------------------------------------------------
-// Combine of split pairs: one warp per output row (COMBINE_WARPS rows per CTA), each lane D / 32
-// columns.  The parts' running maxima are integers, so each part is brought to the common
-// maximum M by an exact power of two: O = sum_p 2^(m_p - M) O_p, l = sum_p 2^(m_p - M) l_p,
-// out = O * s_v / l.
+// Combine of the tail pairs the persistent schedule cut: one warp per output row (COMBINE_WARPS
+// rows per CTA), each lane D / 32 columns.  Tail pair tp spans the key steps
+// [tp * nkv, (tp + 1) * nkv) of the tail, so its parts are those of CTAs
+// c_first = tp * nkv / tail_w .. c_last = ((tp + 1) * nkv - 1) / tail_w; CTA c's part sits in
+// slot 2c + 1 if the CTA started in an earlier pair, else in slot 2c.  The parts' running maxima
+// are integers, so each part is brought to the common maximum M by an exact power of two:
+// O = sum_p 2^(m_p - M) O_p, l = sum_p 2^(m_p - M) l_p, out = O * s_v / l.
 // ---------------------------------------------------------------------------------------------
 constexpr int COMBINE_WARPS = 8;
 
@@ -568,26 +642,31 @@ __global__ void __launch_bounds__(COMBINE_WARPS * 32) k_attn_combine(const AttnA
   const int tp = grow / (NQ * BLOCK_M);
   const int t = (grow / BLOCK_M) % NQ;
   const int r = grow % BLOCK_M;
-  if (tp >= args.combine_pairs) return;
-  const int pair = args.full_ctas + tp;
+  if (tp >= args.tail_pairs) return;
+  const long long W = args.tail_w, nkv = args.nkv, g0 = tp * nkv;
+  const int c_first = static_cast<int>(g0 / W);
+  const int c_last = static_cast<int>((g0 + nkv - 1) / W);
+  if (c_first == c_last) return;                  // one CTA ran the whole pair and wrote it
+  const int pair = args.whole * args.ctas + tp;
   const int qblk = pair % args.pairs_per_head;
   const int h = (pair / args.pairs_per_head) % args.H;
   const int bz = pair / (args.pairs_per_head * args.H);
   const int row = qblk * (NQ * BLOCK_M) + t * BLOCK_M + r;
   if (row >= args.L) return;
-  const int S = args.nsplit;
-  auto slot = [&](int p) { return (static_cast<size_t>(tp) * S + p) * NQ + t; };
+  auto slot = [&](int c) {
+    return static_cast<size_t>(2 * c + (c * W < g0 ? 1 : 0)) * NQ + t;
+  };
   float M = -INFINITY;
-  for (int p = 0; p < S; ++p) M = fmaxf(M, args.part_ml[slot(p) * BLOCK_M + r].x);
+  for (int c = c_first; c <= c_last; ++c) M = fmaxf(M, args.part_ml[slot(c) * BLOCK_M + r].x);
   float l = 0.0f;
   float acc[VEC];
 #pragma unroll
   for (int i = 0; i < VEC; ++i) acc[i] = 0.0f;
-  for (int p = 0; p < S; ++p) {
-    const float2 ml = args.part_ml[slot(p) * BLOCK_M + r];
+  for (int c = c_first; c <= c_last; ++c) {
+    const float2 ml = args.part_ml[slot(c) * BLOCK_M + r];
     const float w = exp2_int(static_cast<int>(ml.x - M));
     l = fmaf(w, ml.y, l);
-    const float* po = args.part_o + (slot(p) * BLOCK_M + r) * D + lane * VEC;
+    const float* po = args.part_o + (slot(c) * BLOCK_M + r) * D + lane * VEC;
     if constexpr (VEC == 4) {
       const float4 o = *reinterpret_cast<const float4*>(po);
       acc[0] = fmaf(w, o.x, acc[0]); acc[1] = fmaf(w, o.y, acc[1]);
@@ -674,30 +753,34 @@ static cudaError_t launch_attn_d(const void* q8, const void* k8, const void* v8,
   return cudaGetLastError();
 }
 
-// Split plan of a dense launch: pairs beyond the last full wave of num_sms CTAs (one CTA per
-// SM) are split along the keys into the number of parts (2..4) that shortens that partial wave
-// the most, if it shortens it to at most 0.8 of a full CTA's time; each part keeps at least two
-// key steps.  bytes = the workspace the parts need (0: no split).
+// Persistent plan of a dense launch: ctas = one CTA per SM (fewer when the work is small); each
+// CTA takes `whole` whole pairs, and the key steps of the remaining tail pairs, laid end to end,
+// are cut into equal contiguous ranges of tail_w steps, one per CTA, so every CTA runs the same
+// number of key steps to within one range.  A range is at least a quarter of a pair (a cut pair
+// has a handful of parts at most) and at most one pair; when the even share would be 0.8 of a
+// pair or more, the tail pairs stay whole (one per CTA).  bytes = the workspace the cut pairs'
+// partial results need (0: no pair is cut).
 AttnSplitPlan plan_attention_split(int B, int H, int L, int D, int num_sms) {
   AttnSplitPlan p;
   p.pairs_per_head = (L + NQ * BLOCK_M - 1) / (NQ * BLOCK_M);
   const long long pairs = static_cast<long long>(p.pairs_per_head) * H * B;
-  const int nkv = (L + BLOCK_N - 1) / BLOCK_N;
-  const long long tail = num_sms > 0 ? pairs % num_sms : 0;
-  p.nsplit = 1;
-  double best = 1.0;
-  for (int S = 2; tail > 0 && S <= 4; ++S) {
-    if (nkv < 2 * S) break;
-    const double tt = static_cast<double>((tail * S + num_sms - 1) / num_sms) / S;
-    if (tt < best - 1e-9) {
-      best = tt;
-      p.nsplit = S;
-    }
-  }
-  if (best > 0.8) p.nsplit = 1;
-  p.tail = p.nsplit > 1 ? static_cast<int>(tail) : 0;
-  p.full_ctas = static_cast<int>(pairs - p.tail);
-  p.bytes = static_cast<size_t>(p.tail) * p.nsplit * NQ * BLOCK_M * (D + 2) * sizeof(float);
+  p.nkv = (L + BLOCK_N - 1) / BLOCK_N;
+  const long long steps = pairs * p.nkv;
+  const int wmin = (p.nkv + 3) / 4;
+  const long long want = (steps + wmin - 1) / wmin;
+  p.ctas = static_cast<int>(want < num_sms ? want : num_sms);
+  if (p.ctas < 1) p.ctas = 1;
+  p.whole = static_cast<int>(pairs / p.ctas);
+  p.tail_pairs = static_cast<int>(pairs - static_cast<long long>(p.whole) * p.ctas);
+  const long long even =
+      (static_cast<long long>(p.tail_pairs) * p.nkv + p.ctas - 1) / p.ctas;
+  p.tail_w = p.tail_pairs > 0 ? static_cast<int>(even > wmin ? even : wmin) : p.nkv;
+  // cutting costs partial results and a combine: worth it only when it shortens the tail
+  // to less than 0.8 of a whole pair
+  if (p.tail_w * 5 >= p.nkv * 4) p.tail_w = p.nkv;
+  p.bytes = p.tail_w < p.nkv
+                ? static_cast<size_t>(2) * p.ctas * NQ * BLOCK_M * (D + 2) * sizeof(float)
+                : 0;
   return p;
 }
 
@@ -723,33 +806,36 @@ cudaError_t launch_attention(const uint8_t* q8, const uint8_t* k8, const uint8_t
   a.inject_missing_q = inject_missing_q;
   a.part_o = nullptr;
   a.part_ml = nullptr;
-  a.combine_pairs = 0;
+  a.pairs_per_head = 0;
+  a.nkv = 0;
+  a.ctas = 0;
+  a.whole = 0;
+  a.tail_pairs = 0;
+  a.tail_w = 1;
   const int slabs = varlen ? H : B * H;
   dim3 grid;
   int combine_ctas = 0;
   if (varlen) {
-    a.pairs_per_head = 0;
-    a.full_ctas = 0;
-    a.nsplit = 1;
     grid = dim3((max_seqlen + NQ * BLOCK_M - 1) / (NQ * BLOCK_M), H, nseq);
   } else {
     AttnSplitPlan p = plan_attention_split(B, H, L, D, num_sms);
-    if (workspace == nullptr || workspace_bytes < p.bytes) {   // no workspace: no split
-      p.nsplit = 1;
-      p.full_ctas += p.tail;
-      p.tail = 0;
+    if (workspace == nullptr || workspace_bytes < p.bytes) {   // no workspace: no pair is cut
+      p.tail_w = p.nkv;
+      p.bytes = 0;
     }
     a.pairs_per_head = p.pairs_per_head;
-    a.full_ctas = p.full_ctas;
-    a.nsplit = p.nsplit;
-    a.combine_pairs = p.tail;
-    if (p.tail > 0) {
-      const size_t o_elems = static_cast<size_t>(p.tail) * p.nsplit * NQ * BLOCK_M * D;
+    a.nkv = p.nkv;
+    a.ctas = p.ctas;
+    a.whole = p.whole;
+    a.tail_pairs = p.tail_pairs;
+    a.tail_w = p.tail_w;
+    if (p.bytes > 0) {
+      const size_t o_elems = static_cast<size_t>(2) * p.ctas * NQ * BLOCK_M * D;
       a.part_o = static_cast<float*>(workspace);
       a.part_ml = reinterpret_cast<float2*>(a.part_o + o_elems);
-      combine_ctas = p.tail * NQ * BLOCK_M / COMBINE_WARPS;
+      combine_ctas = p.tail_pairs * NQ * BLOCK_M / COMBINE_WARPS;
     }
-    grid = dim3(p.full_ctas + p.tail * p.nsplit, 1, 1);
+    grid = dim3(p.ctas, 1, 1);
   }
   if (D == 128)
     return launch_attn_d<128>(q8, k8, v8, a, a.rows_per_slab, slabs, grid, combine_ctas, stream);

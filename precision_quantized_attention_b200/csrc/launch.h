@@ -29,10 +29,11 @@ cudaError_t launch_calib_quant_qkv(const void* const* x, uint8_t* const* codes8,
                                    void* workspace, uint64_t limit_ns, int* err, int num_sms,
                                    cudaStream_t stream);
 
-// How a dense attention launch splits its last, partial wave along the keys (see
-// plan_attention_split in attn_fwd.cu); bytes = workspace the split needs (0: no split).
+// Persistent schedule of a dense attention launch (see plan_attention_split in attn_fwd.cu):
+// ctas CTAs, `whole` whole pairs each, then tail ranges of tail_w key steps; bytes = workspace
+// the cut tail pairs need (0: no pair is cut).
 struct AttnSplitPlan {
-  int pairs_per_head, full_ctas, nsplit, tail;
+  int pairs_per_head, nkv, ctas, whole, tail_pairs, tail_w;
   size_t bytes;
 };
 AttnSplitPlan plan_attention_split(int B, int H, int L, int D, int num_sms);

@@ -108,11 +108,14 @@ def test_wait_timeout_reports_error_and_context_survives():
     assert_close(out, oracle_path(w, q, k, v), "after timeout")
 
 
-@pytest.mark.parametrize("B,H,L,D", [(1, 2, 1000, 128), (2, 3, 777, 64), (1, 24, 8704, 128)])
+# (1, 300, 256, 64): two whole pairs per CTA, then a tail cut into single key steps
+@pytest.mark.parametrize("B,H,L,D", [(1, 2, 1000, 128), (2, 3, 777, 64), (1, 300, 256, 64),
+                                     (1, 24, 8704, 128)])
 def test_split_last_wave_matches_unsplit_and_oracle(B, H, L, D):
-    """With a workspace the pairs after the last full wave are split along the keys and merged
-    by the combine kernel; the result equals the unsplit launch up to FP32 summation order and
-    meets the oracle bar."""
+    """With a workspace the persistent schedule cuts the tail pairs (those left after an equal
+    share of whole pairs per CTA) along the keys and the combine kernel merges the parts; the
+    result equals the launch without a workspace (tail pairs whole) up to FP32 summation order
+    and meets the oracle bar."""
     w = workloads.custom("split", "fp8", B, H, L, D, seed=40 + L)
     q, k, v = workloads.make_qkv(w)
     path = gpu_path(w, q, k, v)
