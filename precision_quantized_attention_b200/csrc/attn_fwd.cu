@@ -758,8 +758,8 @@ static cudaError_t launch_attn_d(const void* q8, const void* k8, const void* v8,
 // are cut into equal contiguous ranges of tail_w steps, one per CTA, so every CTA runs the same
 // number of key steps to within one range.  A range is at least a quarter of a pair (a cut pair
 // has a handful of parts at most) and at most one pair; when the even share would be 0.8 of a
-// pair or more, the tail pairs stay whole (one per CTA).  bytes = the workspace the cut pairs'
-// partial results need (0: no pair is cut).
+// pair or more, or would save fewer than 4 key steps, the tail pairs stay whole (one per CTA).
+// bytes = the workspace the cut pairs' partial results need (0: no pair is cut).
 AttnSplitPlan plan_attention_split(int B, int H, int L, int D, int num_sms) {
   AttnSplitPlan p;
   p.pairs_per_head = (L + NQ * BLOCK_M - 1) / (NQ * BLOCK_M);
@@ -775,9 +775,14 @@ AttnSplitPlan plan_attention_split(int B, int H, int L, int D, int num_sms) {
   const long long even =
       (static_cast<long long>(p.tail_pairs) * p.nkv + p.ctas - 1) / p.ctas;
   p.tail_w = p.tail_pairs > 0 ? static_cast<int>(even > wmin ? even : wmin) : p.nkv;
-  // cutting costs partial results and a combine: worth it only when it shortens the tail
-  // to less than 0.8 of a whole pair
-  if (p.tail_w * 5 >= p.nkv * 4) p.tail_w = p.nkv;
+  // cutting costs partial results and a combine launch: worth it only when it shortens the
+  // tail to less than 0.8 of a whole pair and by at least 4 key steps
+  if (p.tail_w * 5 >= p.nkv * 4 || p.nkv - p.tail_w < 4) p.tail_w = p.nkv;
+  if (p.tail_w == p.nkv && p.whole == 0) {      // fewer pairs than CTAs: one CTA per pair
+    p.ctas = p.tail_pairs;
+    p.whole = 1;
+    p.tail_pairs = 0;
+  }
   p.bytes = p.tail_w < p.nkv
                 ? static_cast<size_t>(2) * p.ctas * NQ * BLOCK_M * (D + 2) * sizeof(float)
                 : 0;

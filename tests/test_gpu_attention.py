@@ -108,8 +108,9 @@ def test_wait_timeout_reports_error_and_context_survives():
     assert_close(out, oracle_path(w, q, k, v), "after timeout")
 
 
-# (1, 300, 256, 64): two whole pairs per CTA, then a tail cut into single key steps
-@pytest.mark.parametrize("B,H,L,D", [(1, 2, 1000, 128), (2, 3, 777, 64), (1, 300, 256, 64),
+# (1, 160, 1024, 64): four whole pairs per CTA (Q buffers reused), then a tail cut into
+# ranges of 3 key steps
+@pytest.mark.parametrize("B,H,L,D", [(1, 2, 1000, 128), (2, 3, 777, 64), (1, 160, 1024, 64),
                                      (1, 24, 8704, 128)])
 def test_split_last_wave_matches_unsplit_and_oracle(B, H, L, D):
     """With a workspace the persistent schedule cuts the tail pairs (those left after an equal
