@@ -156,19 +156,39 @@ __global__ void __launch_bounds__(256) k_quant_fp8(const uint4* __restrict__ xv,
 // -------------------------------------------------------------------------------------------
 // FP8 requant table of one tensor: for every E4M3 block-scale code b (0..127: block scales are
 // never negative) and E2M1 magnitude m (0..7) the E4M3 code of the dequantized value over s8,
-//   lut[8 b + m] = e4m3(fl32(fl32(fl32(val(m) * val(b)) * s_g) / s8)),
+//   requant[8 b + m] = e4m3(fl32(fl32(fl32(val(m) * val(b)) * s_g) / s8)),
 // in the same product order as the element-wise definition.  A negative E2M1 code gives the
 // same code with the sign bit set: the products, the quotient and round-to-nearest-even are
-// sign-symmetric, and -0 becomes 0x80.  Built by the whole CTA (then synchronized).
-__device__ __forceinline__ void build_requant_lut(uint2* lut, float sg, float s8) {
+// sign-symmetric, and -0 becomes 0x80.
+// Per block-scale code the divisor of the block's E2M1 quotients is tabulated too:
+//   er[b] = (eff, RN(1 / eff)), eff = fl32(val(b) * s_g),
+// and the quotient that picks the block scale, amax_b / fl32(6 s_g), uses the tensor's
+// RN(1 / fl32(6 s_g)) in Markstein's form (correctly rounded, as every quotient here).
+// Built by the whole CTA (then synchronized).
+struct Fp4Tables {
+  uint2 requant[128];        // 8 requant codes (one per E2M1 magnitude) per block-scale code
+  float2 er[128];            // (eff, RN(1 / eff)) per block-scale code
+  float r_six;               // RN(1 / fl32(6 s_g))
+  int fast_six;              // markstein_ok(fl32(6 s_g))
+};
+
+__device__ __forceinline__ void build_fp4_tables(Fp4Tables* tab, float sg, float six_sg, float s8) {
   const float r8 = __frcp_rn(s8);
   const bool fast8 = markstein_ok(s8);
-  uint8_t* bytes = reinterpret_cast<uint8_t*>(lut);
+  uint8_t* bytes = reinterpret_cast<uint8_t*>(tab->requant);
   for (int i = threadIdx.x; i < 1024; i += blockDim.x) {
     const float xh = __fmul_rn(__fmul_rn(e2m1_to_f32(static_cast<uint32_t>(i & 7)),
                                          e4m3_to_f32(static_cast<uint32_t>(i >> 3))), sg);
     const float d = fast8 ? div_rn_by(xh, s8, r8) : __fdiv_rn(xh, s8);
     bytes[i] = static_cast<uint8_t>(cvt_e4m3x2(d, 0.0f) & 0xFFu);
+  }
+  for (int b = threadIdx.x; b < 128; b += blockDim.x) {
+    const float eff = __fmul_rn(e4m3_to_f32(static_cast<uint32_t>(b)), sg);
+    tab->er[b] = make_float2(eff, eff != 0.0f ? __frcp_rn(eff) : 0.0f);
+  }
+  if (threadIdx.x == 0) {
+    tab->r_six = __frcp_rn(six_sg);
+    tab->fast_six = markstein_ok(six_sg) ? 1 : 0;
   }
 }
 
@@ -181,9 +201,9 @@ __device__ __forceinline__ uint32_t requant4(uint2 t, uint32_t nib4, uint32_t w0
 }
 
 // One 16-element block: E2M1 codes, E4M3 block scale and (optionally) the FP8 requant codes,
-// the latter looked up in the tensor's requant table.
-__device__ __forceinline__ void fp4_block(uint4 a0, uint4 a1, size_t b, float sg, float six_sg,
-                                          const uint2* __restrict__ lut,
+// the latter looked up in the tensor's tables.
+__device__ __forceinline__ void fp4_block(uint4 a0, uint4 a1, size_t b, float six_sg,
+                                          const Fp4Tables* __restrict__ tab,
                                           uint2* __restrict__ packed_out,
                                           uint8_t* __restrict__ bscale_out,
                                           uint4* __restrict__ codes8_out) {
@@ -192,12 +212,14 @@ __device__ __forceinline__ void fp4_block(uint4 a0, uint4 a1, size_t b, float sg
 #pragma unroll
   for (int i = 0; i < 8; ++i) am2 = absmax_word(am2, w[i]);
   const float amax_b = __uint_as_float(max(am2 & 0xFFFFu, am2 >> 16) << 16);
-  const uint32_t sb = cvt_e4m3x2(__fdiv_rn(amax_b, six_sg), 0.0f) & 0xFFu;
-  const float eff = __fmul_rn(e4m3_to_f32(sb), sg);
+  const float qb = tab->fast_six ? div_rn_by(amax_b, six_sg, tab->r_six) : __fdiv_rn(amax_b, six_sg);
+  const uint32_t sb = cvt_e4m3x2(qb, 0.0f) & 0xFFu;  // amax_b >= 0: sb < 128
+  const float2 er = tab->er[sb & 0x7Fu];
+  const float eff = er.x;
   uint32_t pk0 = 0, pk1 = 0;
   uint32_t c8[4] = {0u, 0u, 0u, 0u};
   if (eff != 0.0f) {
-    const float r_eff = __frcp_rn(eff);
+    const float r_eff = er.y;
     const bool fast_eff = markstein_ok(eff);
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
@@ -209,7 +231,7 @@ __device__ __forceinline__ void fp4_block(uint4 a0, uint4 a1, size_t b, float sg
       else pk1 |= byte << (8 * (i - 4));
     }
     if (codes8_out) {
-      const uint2 t = lut[sb & 0x7Fu];
+      const uint2 t = tab->requant[sb & 0x7Fu];
       c8[0] = requant4(t, pk0, w[0], w[1]);
       c8[1] = requant4(t, pk0 >> 16, w[2], w[3]);
       c8[2] = requant4(t, pk1, w[4], w[5]);
@@ -238,13 +260,13 @@ __global__ void __launch_bounds__(256) k_quant_fp4_block(
     *gscale_out = sg;
     if (scale8_out) *scale8_out = s8;
   }
-  __shared__ uint2 lut[128];
-  build_requant_lut(lut, sg, s8);
+  __shared__ Fp4Tables tab;
+  build_fp4_tables(&tab, sg, six_sg, s8);
   __syncthreads();
   const size_t stride = static_cast<size_t>(gridDim.x) * blockDim.x;
   for (size_t b = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; b < nblocks;
        b += stride)
-    fp4_block(__ldcs(xv + 2 * b), __ldcs(xv + 2 * b + 1), b, sg, six_sg, lut, packed_out,
+    fp4_block(__ldcs(xv + 2 * b), __ldcs(xv + 2 * b + 1), b, six_sg, &tab, packed_out,
               bscale_out, codes8_out);
 }
 
@@ -478,8 +500,8 @@ __global__ void __launch_bounds__(FUSED_THREADS) k_calib_quant_fp4_block(
     *gscale_out = sg;
     if (scale8_out) *scale8_out = s8;
   }
-  __shared__ uint2 lut[128];
-  build_requant_lut(lut, sg, s8);
+  __shared__ Fp4Tables tab;
+  build_fp4_tables(&tab, sg, six_sg, s8);
   __syncthreads();
   const uint64_t pol = l2_policy_evict_first();
   size_t b = lo + threadIdx.x;
@@ -487,11 +509,11 @@ __global__ void __launch_bounds__(FUSED_THREADS) k_calib_quant_fp4_block(
     const uint4 a0 = ld_hint(xv + 2 * b, pol), a1 = ld_hint(xv + 2 * b + 1, pol);
     const uint4 c0 = ld_hint(xv + 2 * (b + FUSED_THREADS), pol);
     const uint4 c1 = ld_hint(xv + 2 * (b + FUSED_THREADS) + 1, pol);
-    fp4_block(a0, a1, b, sg, six_sg, lut, packed_out, bscale_out, codes8_out);
-    fp4_block(c0, c1, b + FUSED_THREADS, sg, six_sg, lut, packed_out, bscale_out, codes8_out);
+    fp4_block(a0, a1, b, six_sg, &tab, packed_out, bscale_out, codes8_out);
+    fp4_block(c0, c1, b + FUSED_THREADS, six_sg, &tab, packed_out, bscale_out, codes8_out);
   }
   for (; b < hi; b += FUSED_THREADS)
-    fp4_block(ld_hint(xv + 2 * b, pol), ld_hint(xv + 2 * b + 1, pol), b, sg, six_sg, lut,
+    fp4_block(ld_hint(xv + 2 * b, pol), ld_hint(xv + 2 * b + 1, pol), b, six_sg, &tab,
               packed_out, bscale_out, codes8_out);
   grid_depart(ws);
 }
@@ -624,8 +646,8 @@ __device__ __forceinline__ uint32_t qkv_stage_fp8(const uint4* __restrict__ xp,
 __device__ __forceinline__ uint32_t qkv_stage_fp4(const uint4* __restrict__ xp,
                                                   uint2* __restrict__ e2m1,
                                                   uint8_t* __restrict__ bscale,
-                                                  uint4* __restrict__ codes8, float sg,
-                                                  float six_sg, const uint2* __restrict__ lut,
+                                                  uint4* __restrict__ codes8,
+                                                  float six_sg, const Fp4Tables* __restrict__ tab,
                                                   const uint4* __restrict__ xc, size_t lo,
                                                   size_t hi) {
   constexpr size_t T = FUSED_THREADS;
@@ -647,7 +669,7 @@ __device__ __forceinline__ uint32_t qkv_stage_fp4(const uint4* __restrict__ xp,
       m2 = absmax_word(m2, c1.x); m2 = absmax_word(m2, c1.y);
       m2 = absmax_word(m2, c1.z); m2 = absmax_word(m2, c1.w);
     }
-    if (xp) fp4_block(a0, a1, b, sg, six_sg, lut, e2m1, bscale, codes8);
+    if (xp) fp4_block(a0, a1, b, six_sg, tab, e2m1, bscale, codes8);
   }
   return m2;
 }
@@ -705,13 +727,13 @@ __global__ void __launch_bounds__(FUSED_THREADS) k_calib_quant_qkv(const QkvArgs
         *tp.gscale = sg;
         *tp.scale8 = s8;
       }
-      __shared__ uint2 lut[128];
+      __shared__ Fp4Tables tab;
       if (ok) {                                     // uniform over the grid
-        build_requant_lut(lut, sg, s8);
+        build_fp4_tables(&tab, sg, six_sg, s8);
         __syncthreads();
       }
       m2 = qkv_stage_fp4(ok ? tp.x : nullptr, tp.e2m1, tp.bscale,
-                         reinterpret_cast<uint4*>(tp.codes8), sg, six_sg, lut, xc, lo, hi);
+                         reinterpret_cast<uint4*>(tp.codes8), six_sg, &tab, xc, lo, hi);
     }
     if (st < QKV) {
       m = fold_max(m2);
