@@ -112,7 +112,7 @@ def test_wait_timeout_reports_error_and_context_survives():
 # ranges of 3 key steps
 @pytest.mark.parametrize("B,H,L,D", [(1, 2, 1000, 128), (2, 3, 777, 64), (1, 160, 1024, 64),
                                      (1, 24, 8704, 128)])
-def test_split_last_wave_matches_unsplit_and_oracle(B, H, L, D):
+def test_cut_tail_pairs_match_uncut_and_oracle(B, H, L, D):
     """With a workspace the persistent schedule cuts the tail pairs (those left after an equal
     share of whole pairs per CTA) along the keys and the combine kernel merges the parts; the
     result equals the launch without a workspace (tail pairs whole) up to FP32 summation order
