@@ -182,7 +182,14 @@ def run_gpu(args):
     w = replica_workload(w, rank, world)
     q, k, v = workloads.make_qkv(w)
     qd, kd, vd = (t.cuda() for t in (q, k, v))
-    path = qa.QuantizedAttention(w.shape, w.mode, cu_seqlens=w.cu_seqlens, sm_scale=w.sm_scale)
+    static_amax = None
+    if args.static_scales:                       # calibrate once, outside the timed region
+        cal = qa.QuantizedAttention(w.shape, w.mode, cu_seqlens=w.cu_seqlens, sm_scale=w.sm_scale)
+        cal.quantize(qd, kd, vd)
+        static_amax = cal.amax.tolist()
+        del cal
+    path = qa.QuantizedAttention(w.shape, w.mode, cu_seqlens=w.cu_seqlens, sm_scale=w.sm_scale,
+                                 static_amax=static_amax)
     flush = L2Flush()
     stream = torch.cuda.current_stream()
 
@@ -303,13 +310,15 @@ def workload_data(w) -> str:
     return ", ".join(parts)
 
 
-def bench_config(w, world):
+def bench_config(w, world, static_scales=False):
     """The workload description both arms print."""
     return {"workload": f"{w.name}: B={w.B} H={w.H} L={w.L} D={w.D} {w.mode.upper()} full attention"
                         + (" (512 text + 4096 target + 4096 context tokens)"
                            if w.L == workloads.L_EDIT else ""),
             "mode": w.mode, "B": w.B, "H": w.H, "L": w.L, "D": w.D,
             "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+            "scales": ("static: Q, K, V amax calibrated once before the timed steps"
+                       if static_scales else "calibrated every step (amax of Q, K and V)"),
             "l2": "flushed between steps outside the timed events: a 256 MiB write, then a "
                   "256 MiB read of another buffer so the write's dirty lines are written back "
                   "before the step starts"}
@@ -340,7 +349,7 @@ def report(args, w, qkv, rank, world, ms, attn, quant, e2e_ms, clocks, launches)
         "vs_baseline": None,
         "dtype": "e4m3",
         "data": workload_data(w),
-        "config": bench_config(w, world),
+        "config": bench_config(w, world, args.static_scales),
         "roofline": {"bound": "tensor", "achieved": achieved_tf, "peak": fp8_peak,
                      "unit": "TFLOP/s", "frac": achieved_tf / fp8_peak,
                      "traffic": ATTN_TRAFFIC_BYTES.get((w.L, w.H, w.D)),
@@ -434,6 +443,8 @@ def main():
                     help="time another dense workload (default: the L=8704 editing workload)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--static-scales", action="store_true",
+                    help="quantize with amax values calibrated once before timing (one pass)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -154,6 +154,17 @@ QATTN_API qattn_status qattn_calibrate_quantize_qkv(const qattn_quant_io* io, si
                                                     qattn_mode mode, void* workspace_dev,
                                                     size_t workspace_bytes, qattn_stream_t stream);
 
+/* FakeQuantize of Q, K and V with GIVEN scales, in one launch: io[i].amax_dev is an INPUT here
+ * (the amax of a calibration done earlier, as the blog's post-training quantization produces),
+ * and each tensor gets exactly the results of qattn_quantize_fp8 (mode FP8) or
+ * qattn_quantize_fp4_block with the FP8 requant (mode FP4) for that amax; the other io fields
+ * are as for qattn_calibrate_quantize_qkv (io: HOST array of three descriptors, read during the
+ * call).  No calibration pass and no workspace: one streaming read of each input.  FP4 mode
+ * needs n % 16 == 0.  A non-finite amax writes nothing for that tensor and records
+ * QATTN_ERR_NONFINITE. */
+QATTN_API qattn_status qattn_quantize_qkv(const qattn_quant_io* io, size_t n, qattn_mode mode,
+                                          qattn_stream_t stream);
+
 /* qattn_calibrate_quantize_fp8 without a caller workspace (the blog has no counterpart: this is
  * a calling convention, not part of the method).  For callers that cannot supply a scratch
  * buffer -- C code with no device allocator at the call site, or a runtime whose device memory

@@ -18,10 +18,11 @@ from . import _lib
 from ._lib import (MODE_FP4, MODE_FP8, QattnError, calibrate_amax, calibrate_quantize_fp4_block,
                    calibrate_quantize_fp8, calibrate_quantize_qkv, forward, forward_varlen,
                    forward_workspace_bytes, get_error, new_workspace, quantize_fp4_block,
-                   quantize_fp8)
+                   quantize_fp8, quantize_qkv)
 
 __all__ = ["QuantizedAttention", "calibrate_amax", "quantize_fp8", "quantize_fp4_block",
            "calibrate_quantize_fp8", "calibrate_quantize_fp4_block", "calibrate_quantize_qkv",
+           "quantize_qkv",
            "new_workspace", "forward", "forward_workspace_bytes",
            "forward_varlen", "get_error", "QattnError", "MODE_FP8", "MODE_FP4"]
 
@@ -34,11 +35,13 @@ class QuantizedAttention:
     workspace) so repeated calls allocate nothing.  Calls on one object must not overlap on
     the device (they share the buffers and the workspace); stream order is enough.  ``mode`` is
     "fp8" or "fp4".  For varlen, pass ``cu_seqlens`` (list of ints) and q, k, v of shape
-    [1, H, T, D].
+    [1, H, T, D].  With ``static_amax`` (three floats: the amax of Q, K and V from an earlier
+    calibration) the calls skip calibration and quantize with those scales in one streaming
+    pass; ``amax`` then holds them.
     """
 
     def __init__(self, shape, mode: str = "fp8", cu_seqlens=None, sm_scale: float | None = None,
-                 device="cuda"):
+                 device="cuda", static_amax=None):
         B, H, T, D = shape
         self.shape = tuple(shape)
         self.mode = mode
@@ -49,6 +52,12 @@ class QuantizedAttention:
         f32 = dict(dtype=torch.float32, device=dev)
         self.codes = [torch.empty(shape, **u8) for _ in range(3)]
         self.amax = torch.zeros(3, **f32)
+        self.static = static_amax is not None
+        if self.static:
+            vals = [float(a) for a in static_amax]
+            if len(vals) != 3:
+                raise ValueError("static_amax needs three values (Q, K, V)")
+            self.amax.copy_(torch.tensor(vals, dtype=torch.float32))
         self.scale = torch.zeros(3, **f32)          # per-tensor E4M3 dequant multipliers
         if mode == "fp4":
             if n % 16:
@@ -72,8 +81,13 @@ class QuantizedAttention:
             self.max_seqlen = max(b - a for a, b in zip(cu_seqlens[:-1], cu_seqlens[1:]))
 
     def quantize(self, q, k, v, stream=None):
-        """Calibrate and FakeQuantize Q, K and V in one launch."""
-        if self.mode == "fp8":
+        """Calibrate and FakeQuantize Q, K and V in one launch (with static scales: quantize
+        only)."""
+        if self.static:
+            extra = (self.e2m1, self.bscale, self.gscale) if self.mode == "fp4" else ()
+            quantize_qkv((q, k, v), self.amax, self.codes, self.scale,
+                         MODE_FP4 if self.mode == "fp4" else MODE_FP8, *extra, stream=stream)
+        elif self.mode == "fp8":
             calibrate_quantize_qkv((q, k, v), self.amax, self.codes, self.scale, self.workspace,
                                    MODE_FP8, stream=stream)
         else:

@@ -22,11 +22,11 @@ EXPORTS = (
     "qattn_calibrate_amax", "qattn_quantize_fp8", "qattn_quantize_fp4_block", "qattn_forward",
     "qattn_forward_varlen", "qattn_get_error", "qattn_calibrate_quantize_fp8",
     "qattn_calibrate_quantize_fp4_block", "qattn_calibrate_quantize_fp8_noalloc",
-    "qattn_calibrate_quantize_qkv", "qattn_forward_ws", "qattn_status_str",
+    "qattn_calibrate_quantize_qkv", "qattn_quantize_qkv", "qattn_forward_ws", "qattn_status_str",
     "qattn_forward_workspace_bytes",
     "qattn_debug_set_wait_timeout_ns", "qattn_debug_inject_missing_q",
 )
-_RETURNS_STATUS = EXPORTS[:11]
+_RETURNS_STATUS = EXPORTS[:12]
 FUSED_WORKSPACE_BYTES = 256     # QATTN_FUSED_WORKSPACE_BYTES
 
 
@@ -68,6 +68,7 @@ def load() -> ctypes.CDLL:
     lib.qattn_calibrate_quantize_fp4_block.argtypes = [P, S, P, P, P, P, P, P, P, S, P]
     lib.qattn_calibrate_quantize_fp8_noalloc.argtypes = [P, S, P, P, P, P]
     lib.qattn_calibrate_quantize_qkv.argtypes = [ctypes.POINTER(QuantIO), S, I, P, S, P]
+    lib.qattn_quantize_qkv.argtypes = [ctypes.POINTER(QuantIO), S, I, P]
     lib.qattn_forward.argtypes = [P, P, P, P, I, I, I, I, ctypes.POINTER(_Scales), F, I, P]
     lib.qattn_forward_varlen.argtypes = [P, P, P, P, P, I, I, I, I, I, ctypes.POINTER(_Scales),
                                          F, I, P]
@@ -193,11 +194,7 @@ def calibrate_quantize_fp4_block(x: torch.Tensor, amax: torch.Tensor, out_e2m1: 
         workspace.numel(), _stream(stream)), "qattn_calibrate_quantize_fp4_block")
 
 
-def calibrate_quantize_qkv(xs, amax, codes8, scale8, workspace, mode: int = MODE_FP8,
-                           e2m1=None, bscale=None, gscale=None, stream=None):
-    """Q, K, V in one launch.  xs: three bf16 tensors of n elements; amax, scale8 (and gscale
-    in FP4 mode): float32 tensors of 3 elements (one per tensor); codes8, e2m1, bscale: lists of
-    three uint8 tensors."""
+def _qkv_io(xs, amax, codes8, scale8, mode, e2m1, bscale, gscale):
     n = xs[0].numel()
     if any(x.numel() != n for x in xs):
         raise ValueError("Q, K and V must have the same number of elements")
@@ -220,9 +217,26 @@ def calibrate_quantize_qkv(xs, amax, codes8, scale8, workspace, mode: int = MODE
             io[i].out_e2m1 = _dev(e2m1[i], torch.uint8, "e2m1").value
             io[i].blk_scale_e4m3 = _dev(bscale[i], torch.uint8, "bscale").value
             io[i].gscale_dev = gscale.data_ptr() + 4 * i
+    return io, n
+
+
+def calibrate_quantize_qkv(xs, amax, codes8, scale8, workspace, mode: int = MODE_FP8,
+                           e2m1=None, bscale=None, gscale=None, stream=None):
+    """Q, K, V in one launch.  xs: three bf16 tensors of n elements; amax, scale8 (and gscale
+    in FP4 mode): float32 tensors of 3 elements (one per tensor); codes8, e2m1, bscale: lists of
+    three uint8 tensors."""
+    io, n = _qkv_io(xs, amax, codes8, scale8, mode, e2m1, bscale, gscale)
     _check(load().qattn_calibrate_quantize_qkv(io, n, int(mode), _dev(workspace, torch.uint8, "workspace"),
                                                workspace.numel(), _stream(stream)),
            "qattn_calibrate_quantize_qkv")
+
+
+def quantize_qkv(xs, amax, codes8, scale8, mode: int = MODE_FP8, e2m1=None, bscale=None,
+                 gscale=None, stream=None):
+    """Q, K, V with given scales in one launch: amax (float32, 3 elements) is an input, the
+    other arguments as for calibrate_quantize_qkv (no workspace)."""
+    io, n = _qkv_io(xs, amax, codes8, scale8, mode, e2m1, bscale, gscale)
+    _check(load().qattn_quantize_qkv(io, n, int(mode), _stream(stream)), "qattn_quantize_qkv")
 
 
 def _scales(s_q, s_k, s_v):

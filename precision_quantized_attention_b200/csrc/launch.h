@@ -29,6 +29,11 @@ cudaError_t launch_calib_quant_qkv(const void* const* x, uint8_t* const* codes8,
                                    void* workspace, uint64_t limit_ns, int* err, int num_sms,
                                    cudaStream_t stream);
 
+cudaError_t launch_quant_qkv(const void* const* x, uint8_t* const* codes8, float* const* amax,
+                             float* const* scale8, uint8_t* const* e2m1, uint8_t* const* bscale,
+                             float* const* gscale, size_t n, int mode, int* err, int num_sms,
+                             cudaStream_t stream);
+
 // Persistent schedule of a dense attention launch (see plan_attention_split in attn_fwd.cu):
 // ctas CTAs, `whole` whole pairs each, then tail ranges of tail_w key steps; bytes = workspace
 // the cut tail pairs need (0: no pair is cut).

@@ -195,6 +195,39 @@ qattn_status qattn_calibrate_quantize_qkv(const qattn_quant_io* io, size_t n, qa
                                                  reinterpret_cast<cudaStream_t>(stream)));
 }
 
+qattn_status qattn_quantize_qkv(const qattn_quant_io* io, size_t n, qattn_mode mode,
+                                qattn_stream_t stream) {
+  if (!io || n == 0) return QATTN_ERR_INVALID_ARG;
+  if (mode != QATTN_MODE_FP8 && mode != QATTN_MODE_FP4) return QATTN_ERR_INVALID_ARG;
+  if (mode == QATTN_MODE_FP4 && n % 16 != 0) return QATTN_ERR_INVALID_ARG;
+  const void* x[3];
+  uint8_t *c8[3], *e2m1[3], *bs[3];
+  float *am[3], *sc[3], *gs[3];
+  for (int i = 0; i < 3; ++i) {
+    const qattn_quant_io& t = io[i];
+    if (!t.x_bf16 || !t.out_e4m3 || !t.amax_dev || !t.scale_dev) return QATTN_ERR_INVALID_ARG;
+    if (!aligned(t.x_bf16, 16) || !aligned(t.amax_dev, 4) || !aligned(t.scale_dev, 4) ||
+        !aligned(t.out_e4m3, mode == QATTN_MODE_FP4 ? 16 : 8))
+      return QATTN_ERR_INVALID_ARG;
+    if (mode == QATTN_MODE_FP4 && (!t.out_e2m1 || !t.blk_scale_e4m3 || !t.gscale_dev ||
+                                   !aligned(t.out_e2m1, 8) || !aligned(t.gscale_dev, 4)))
+      return QATTN_ERR_INVALID_ARG;
+    x[i] = t.x_bf16;
+    c8[i] = t.out_e4m3;
+    am[i] = t.amax_dev;
+    sc[i] = t.scale_dev;
+    e2m1[i] = mode == QATTN_MODE_FP4 ? t.out_e2m1 : nullptr;
+    bs[i] = mode == QATTN_MODE_FP4 ? t.blk_scale_e4m3 : nullptr;
+    gs[i] = mode == QATTN_MODE_FP4 ? t.gscale_dev : nullptr;
+  }
+  DeviceInfo* d = nullptr;
+  qattn_status st = device_info(&d);
+  if (st != QATTN_OK) return st;
+  return from_cuda(qattn::launch_quant_qkv(x, c8, am, sc, e2m1, bs, gs, n,
+                                           mode == QATTN_MODE_FP4 ? 1 : 0, d->err, d->num_sms,
+                                           reinterpret_cast<cudaStream_t>(stream)));
+}
+
 qattn_status qattn_forward_ws(const uint8_t* q8, const uint8_t* k8, const uint8_t* v8,
                               void* out_bf16, int B, int H, int L, int D,
                               const qattn_scales* scales, float sm_scale, qattn_mode mode,

@@ -11,6 +11,7 @@
 // form for a shared divisor), so the codes are bit-identical to the definition (E4M3 / E2M1
 // round-to-nearest-even with saturation, the hardware cvt forms).
 #include <cuda_runtime.h>
+#include <type_traits>
 #include <cstdint>
 
 #include "launch.h"
@@ -756,6 +757,85 @@ __global__ void __launch_bounds__(FUSED_THREADS) k_calib_quant_qkv(const QkvArgs
 }
 
 // -------------------------------------------------------------------------------------------
+// Q, K and V with given (static) scales in one launch: blockIdx.y picks the tensor, whose amax is
+// an input (a calibration done earlier, as post-training quantization provides); each tensor
+// gets exactly the results of k_quant_fp8 (MODE 0) or k_quant_fp4_block with the FP8 requant
+// (MODE 1).  One streaming pass: read 2 B, write 1 B (FP8) or 1.5625 B (FP4) per element.
+// -------------------------------------------------------------------------------------------
+constexpr int STATIC_THREADS = 256;
+constexpr int STATIC_UNROLL = 4;           // 16-byte loads in flight per thread (FP8)
+
+template <int MODE>
+__global__ void __launch_bounds__(STATIC_THREADS) k_quant_qkv(const __grid_constant__ QkvArgs a) {
+  const int ti = blockIdx.y;
+  const QkvTensor tp = ti == 0 ? a.t[0] : (ti == 1 ? a.t[1] : a.t[2]);
+  const float amax = *tp.amax;
+  if (!(amax <= 3.402823466e38f)) {              // inf or NaN: nothing is written
+    if (blockIdx.x == 0 && threadIdx.x == 0) atomicExch(a.err, DEV_ERR_NONFINITE);
+    return;
+  }
+  const size_t T = static_cast<size_t>(gridDim.x) * STATIC_THREADS;
+  const size_t i0 = static_cast<size_t>(blockIdx.x) * STATIC_THREADS + threadIdx.x;
+  if (MODE == 0) {
+    const size_t nvec = a.n / 8;
+    const int ntail = static_cast<int>(a.n - nvec * 8);
+    const float s = (amax == 0.0f) ? 1.0f : __fdiv_rn(amax, 448.0f);
+    if (blockIdx.x == 0 && threadIdx.x == 0) *tp.scale8 = s;
+    const float r = __frcp_rn(s);
+    const uint4* xv = tp.x;
+    uint2* ov = reinterpret_cast<uint2*>(tp.codes8);
+    constexpr size_t U = STATIC_UNROLL;
+    auto sweep = [&](auto fast) {
+      constexpr bool FAST = decltype(fast)::value;
+      size_t i = i0;
+      for (; i + (U - 1) * T < nvec; i += U * T) {
+        uint4 x[U];
+#pragma unroll
+        for (size_t u = 0; u < U; ++u) x[u] = __ldcs(xv + i + u * T);
+#pragma unroll
+        for (size_t u = 0; u < U; ++u)
+          __stcs(ov + i + u * T, make_uint2(quant4_e4m3<FAST>(x[u].x, x[u].y, s, r),
+                                            quant4_e4m3<FAST>(x[u].z, x[u].w, s, r)));
+      }
+      for (; i < nvec; i += T) {
+        const uint4 x = __ldcs(xv + i);
+        __stcs(ov + i, make_uint2(quant4_e4m3<FAST>(x.x, x.y, s, r), quant4_e4m3<FAST>(x.z, x.w, s, r)));
+      }
+    };
+    if (markstein_ok(s)) sweep(std::true_type{});
+    else sweep(std::false_type{});
+    if (blockIdx.x == 0 && static_cast<int>(threadIdx.x) < ntail) {
+      const uint16_t xb = reinterpret_cast<const uint16_t*>(xv)[nvec * 8 + threadIdx.x];
+      const float x = __uint_as_float(static_cast<uint32_t>(xb) << 16);
+      tp.codes8[nvec * 8 + threadIdx.x] = static_cast<uint8_t>(cvt_e4m3x2(__fdiv_rn(x, s), 0.0f) & 0xFFu);
+    }
+  } else {
+    const size_t nblocks = a.n / 16;
+    const float sg = (amax == 0.0f) ? 1.0f : __fdiv_rn(amax, 2688.0f);
+    const float six_sg = __fmul_rn(6.0f, sg);
+    const float s8 = (amax == 0.0f) ? 1.0f : __fdiv_rn(__fmul_rn(2688.0f, sg), 448.0f);
+    if (blockIdx.x == 0 && threadIdx.x == 0) {
+      *tp.gscale = sg;
+      *tp.scale8 = s8;
+    }
+    __shared__ Fp4Tables tab;
+    build_fp4_tables(&tab, sg, six_sg, s8);
+    __syncthreads();
+    const uint4* xv = tp.x;
+    uint4* c8 = reinterpret_cast<uint4*>(tp.codes8);
+    size_t b = i0;
+    for (; b + T < nblocks; b += 2 * T) {         // two blocks' loads in flight
+      const uint4 a0 = __ldcs(xv + 2 * b), a1 = __ldcs(xv + 2 * b + 1);
+      const uint4 d0 = __ldcs(xv + 2 * (b + T)), d1 = __ldcs(xv + 2 * (b + T) + 1);
+      fp4_block(a0, a1, b, six_sg, &tab, tp.e2m1, tp.bscale, c8);
+      fp4_block(d0, d1, b + T, six_sg, &tab, tp.e2m1, tp.bscale, c8);
+    }
+    for (; b < nblocks; b += T)
+      fp4_block(__ldcs(xv + 2 * b), __ldcs(xv + 2 * b + 1), b, six_sg, &tab, tp.e2m1, tp.bscale, c8);
+  }
+}
+
+// -------------------------------------------------------------------------------------------
 // Host launchers (called from the C-ABI layer, which validates arguments).
 // -------------------------------------------------------------------------------------------
 static int grid_for(size_t work_items, int num_sms) {
@@ -860,6 +940,40 @@ cudaError_t launch_calib_quant_qkv(const void* const* x, uint8_t* const* codes8,
   const unsigned grid = static_cast<unsigned>(want < 1 ? 1 : (want < cap ? want : cap));
   void* args[] = {(void*)&a};
   return cudaLaunchCooperativeKernel(fn, dim3(grid), dim3(FUSED_THREADS), args, 0, stream);
+}
+
+// Q, K, V with given amax values (io amax pointers are inputs); tensors: as launch_calib_quant_qkv.
+cudaError_t launch_quant_qkv(const void* const* x, uint8_t* const* codes8, float* const* amax,
+                             float* const* scale8, uint8_t* const* e2m1, uint8_t* const* bscale,
+                             float* const* gscale, size_t n, int mode, int* err, int num_sms,
+                             cudaStream_t stream) {
+  QkvArgs a;
+  for (int i = 0; i < QKV; ++i) {
+    a.t[i].x = static_cast<const uint4*>(x[i]);
+    a.t[i].codes8 = codes8[i];
+    a.t[i].amax = amax[i];
+    a.t[i].scale8 = scale8[i];
+    a.t[i].e2m1 = reinterpret_cast<uint2*>(e2m1[i]);
+    a.t[i].bscale = bscale[i];
+    a.t[i].gscale = gscale[i];
+  }
+  a.n = n;
+  a.limit_ns = 0;
+  a.err = err;
+  a.ws = nullptr;
+  // per tensor: enough CTAs for four 16-byte vectors (FP8) or two blocks (FP4) per thread, at
+  // most 4 CTAs of 256 threads per SM (3 tensors: 12 per SM)
+  const size_t per_cta = mode == 0 ? static_cast<size_t>(STATIC_THREADS) * STATIC_UNROLL * 8
+                                   : static_cast<size_t>(STATIC_THREADS) * 2 * 16;
+  size_t want = (n + per_cta - 1) / per_cta;
+  const size_t cap = static_cast<size_t>(num_sms) * 4;
+  if (want < 1) want = 1;
+  const dim3 grid(static_cast<unsigned>(want < cap ? want : cap), QKV, 1);
+  if (mode == 0)
+    k_quant_qkv<0><<<grid, STATIC_THREADS, 0, stream>>>(a);
+  else
+    k_quant_qkv<1><<<grid, STATIC_THREADS, 0, stream>>>(a);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_calib_quant_fp4_block(const void* x, size_t n, float* amax, uint8_t* packed,

@@ -78,6 +78,17 @@ def test_host_side_argument_errors():
     io[1].x_bf16 = 0x10000
     io[2].out_e2m1 = None                                                 # FP4 output missing
     assert qkv(io, 32, 1, FAKE, W, s0) == _lib.ERR_INVALID_ARG
+    sq = lib.qattn_quantize_qkv                                           # given scales
+    io[2].out_e2m1 = 0x10000
+    assert sq(None, 16, 0, s0) == _lib.ERR_INVALID_ARG
+    assert sq(io, 0, 0, s0) == _lib.ERR_INVALID_ARG
+    assert sq(io, 16, 2, s0) == _lib.ERR_INVALID_ARG                      # bad mode
+    assert sq(io, 24, 1, s0) == _lib.ERR_INVALID_ARG                      # FP4 needs n % 16 == 0
+    io[0].amax_dev = None                                                 # the scales are inputs
+    assert sq(io, 16, 0, s0) == _lib.ERR_INVALID_ARG
+    io[0].amax_dev = 0x10000
+    io[1].out_e4m3 = 0x10004                                              # codes not 8-byte aligned
+    assert sq(io, 16, 0, s0) == _lib.ERR_INVALID_ARG
     sc = _lib._Scales(0x10000, 0x10000, 0x10000)
     fws = lib.qattn_forward_ws
     assert fws(FAKE, FAKE, FAKE, FAKE, 1, 1, 16, 64, ctypes.byref(sc), 0.1, 0, MISALIGNED, 1 << 20,

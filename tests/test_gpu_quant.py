@@ -282,3 +282,83 @@ def test_qkv_nonfinite_tensor_is_reported_and_the_others_are_quantized():
         want, s = oracle.quantize_fp8(xs[i], a)
         assert np.array_equal(_u8(codes[i]), want) and np.float32(scale[i].item()) == s
     assert int(ws.count_nonzero().item()) == 0
+
+
+# ---- given (static) scales: qattn_quantize_qkv ----------------------------------------------
+
+def _given(xs, factors):
+    """float32 amax values to quantize with: the data's amax times a factor."""
+    return [float(np.float32(oracle.amax(x)[1] * f)) for x, f in zip(xs, factors)]
+
+
+@pytest.mark.parametrize("n", [37, 8 * 1000 + 7, 24 * 4096 * 128 + 3])
+def test_static_qkv_fp8_bit_exact(n):
+    """Given scales below (codes saturate), at and above the data's amax: every tensor's scale
+    and codes are the oracle's quantize for that amax, and the amax is left as given."""
+    xs = _qkv_inputs(n, seed=20 + n % 1000)
+    given = _given(xs, (0.5, 1.0, 2.0))
+    amax = torch.tensor(given, dtype=torch.float32, device="cuda")
+    scale = torch.zeros(3, device="cuda")
+    codes = [torch.full((n,), 0x55, dtype=torch.uint8, device="cuda") for _ in range(3)]
+    qa.quantize_qkv([x.cuda() for x in xs], amax, codes, scale)
+    assert qa.get_error() == 0
+    for i, x in enumerate(xs):
+        want, s = oracle.quantize_fp8(x, given[i])
+        assert float(amax[i].item()) == given[i]
+        assert np.float32(scale[i].item()) == s
+        assert np.array_equal(_u8(codes[i]), want), i
+
+
+@pytest.mark.parametrize("n", [16 * 64, 24 * 4096 * 128])
+def test_static_qkv_fp4_bit_exact(n):
+    """FP4 blocks with given scales at and below the data's amax (there the requant scale's
+    closed form fl32(2688 s_g) / 448 is what the oracle finds by brute force: the block holding
+    the data's maximum saturates to scale 448 and code 6)."""
+    xs = _qkv_inputs(n, seed=30 + n % 1000, scales=(1.0, 1e-3, 40.0))
+    given = _given(xs, (1.0, 0.5, 0.25))
+    amax = torch.tensor(given, dtype=torch.float32, device="cuda")
+    scale, gscale = torch.zeros(3, device="cuda"), torch.zeros(3, device="cuda")
+    codes = [torch.empty(n, dtype=torch.uint8, device="cuda") for _ in range(3)]
+    e2m1 = [torch.empty(n // 2, dtype=torch.uint8, device="cuda") for _ in range(3)]
+    bscale = [torch.empty(n // 16, dtype=torch.uint8, device="cuda") for _ in range(3)]
+    qa.quantize_qkv([x.cuda() for x in xs], amax, codes, scale, qa.MODE_FP4, e2m1, bscale, gscale)
+    assert qa.get_error() == 0
+    for i, x in enumerate(xs):
+        w_packed, w_bscale, w_sg, w_c8, w_s8 = oracle.quantize_fp4_block(x, given[i])
+        assert np.float32(gscale[i].item()) == w_sg
+        assert np.float32(scale[i].item()) == w_s8
+        assert np.array_equal(_u8(bscale[i]), w_bscale)
+        assert np.array_equal(_u8(e2m1[i]), w_packed)
+        assert np.array_equal(_u8(codes[i]), w_c8)
+
+
+@pytest.mark.parametrize("mode", ["fp8", "fp4"])
+def test_static_path_with_the_calibrated_amax_equals_the_calibrated_path(mode):
+    w = workloads.custom("static", mode, 1, 3, 700, 128, seed=21)
+    q, k, v = (t.cuda() for t in workloads.make_qkv(w))
+    dyn = qa.QuantizedAttention(w.shape, mode)
+    dyn(q, k, v)
+    assert qa.get_error() == 0
+    stat = qa.QuantizedAttention(w.shape, mode, static_amax=dyn.amax.tolist())
+    stat(q, k, v)
+    assert qa.get_error() == 0
+    assert torch.equal(stat.scale, dyn.scale)
+    for i in range(3):
+        assert torch.equal(stat.codes[i], dyn.codes[i])
+    assert torch.equal(stat.out, dyn.out)
+
+
+def test_static_nonfinite_amax_writes_nothing_for_that_tensor():
+    n = 8 * 4096
+    xs = _qkv_inputs(n, seed=12)
+    given = _given(xs, (1.0, 1.0, 1.0))
+    amax = torch.tensor([given[0], float("inf"), given[2]], dtype=torch.float32, device="cuda")
+    scale = torch.full((3,), -1.0, device="cuda")
+    codes = [torch.full((n,), 0x55, dtype=torch.uint8, device="cuda") for _ in range(3)]
+    qa.quantize_qkv([x.cuda() for x in xs], amax, codes, scale)
+    assert qa.get_error() == qa._lib.ERR_NONFINITE
+    assert scale[1].item() == -1.0 and int(codes[1].count_nonzero().item()) == n
+    assert int((codes[1] == 0x55).sum().item()) == n
+    for i in (0, 2):
+        want, s = oracle.quantize_fp8(xs[i], given[i])
+        assert np.array_equal(_u8(codes[i]), want) and np.float32(scale[i].item()) == s
