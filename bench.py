@@ -365,9 +365,12 @@ def report(args, w, qkv, rank, world, ms, attn, quant, e2e_ms, clocks, launches)
         "e2e": {"value": world * flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
                 "ms_per_step": e2e_ms, "h2d_bytes_per_step": in_bytes,
                 "d2h_bytes_per_step": q.numel() * 2,
-                "schedule": "pinned host bf16 Q/K/V -> device, fused calibrate+quantize, attention, "
-                            "bf16 output -> host every step; uploads, compute and downloads on "
-                            "three streams over two buffer sets, so consecutive steps overlap"},
+                "schedule": "pinned host bf16 Q/K/V -> device, "
+                            + ("quantize with the static scales" if args.static_scales
+                               else "fused calibrate+quantize")
+                            + ", attention, bf16 output -> host every step; uploads, compute and "
+                            "downloads on three streams over two buffer sets, so consecutive "
+                            "steps overlap"},
         "gpu_launches": world * launches * args.steps,   # all ranks' launches in the timed steps
         "clocks": clock,
     }
