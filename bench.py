@@ -435,6 +435,93 @@ def run_reference(args):
     }), flush=True)
 
 
+# The transformer block's FP8 linear layers on the joint sequence (M = 512 + 4096 + 4096 tokens,
+# hidden 3072): the QKV projection and the two MLP GEMMs.
+GEMM_SHAPES = {"qkv_proj": (8704, 9216, 3072), "mlp_up": (8704, 12288, 3072),
+               "mlp_down": (8704, 3072, 12288)}
+
+
+def run_gemm(args):
+    """FP8 GEMM (qattn_gemm_fp8) on the block's linear-layer shapes: seeded random E4M3 codes
+    (every finite code, both signs), each launch after an L2 flush, CUDA events around each
+    launch; value = all shapes' FLOPs over their summed time."""
+    import oracle
+    import precision_quantized_attention_b200 as qa
+    torch.cuda.set_device(0)
+    _, bf16_tf, peak_kind = load_peaks()
+    # a long back-to-back loop of tensor-bound launches runs under the power cap: the sustained
+    # bf16 figure is its denominator when the peaks file has one
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            bf16_tf, peak_kind = float(json.load(f)["bf16_tflops_sustained"]), "measured sustained"
+    except Exception:
+        pass
+    fp8_peak = bf16_tf * FP8_PER_BF16
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(7)
+    flush = L2Flush()
+    per_shape, total_flops, total_ms, cpu = {}, 0.0, 0.0, None
+
+    def codes(rows, cols):
+        c = torch.randint(0, 256, (rows, cols), dtype=torch.uint8, device="cuda", generator=gen)
+        return torch.where((c & 0x7F) == 0x7F, c ^ 1, c)      # no NaN codes
+
+    with ClockSampler(0) as clocks:
+        for name, (M, N, K) in GEMM_SHAPES.items():
+            a8, b8 = codes(M, K), codes(N, K)
+            sa = torch.tensor([0.01], device="cuda")
+            sb = torch.tensor([0.002], device="cuda")
+            y = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
+            for _ in range(args.warmup):
+                qa.gemm_fp8(a8, b8, y, sa, sb)
+            ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                  for _ in range(args.steps)]
+            torch.cuda.synchronize()
+            for e0, e1 in ev:
+                flush()
+                e0.record()
+                qa.gemm_fp8(a8, b8, y, sa, sb)
+                e1.record()
+            torch.cuda.synchronize()
+            if qa.get_error() != 0:
+                raise RuntimeError("device error during the GEMM timing")
+            ms = sum(e0.elapsed_time(e1) for e0, e1 in ev) / len(ev)
+            flops = 2.0 * M * N * K
+            per_shape[name] = {"M": M, "N": N, "K": K, "ms": ms,
+                               "tflops": flops / (ms * 1e-3) / 1e12,
+                               "frac": flops / (ms * 1e-3) / 1e12 / fp8_peak}
+            total_flops += flops
+            total_ms += ms
+            if cpu is None and not args.no_cpu_baseline:
+                rows = list(range(0, M, M // 16))[:16]       # the oracle on 16 rows
+                a_rows, b_all = a8[rows].cpu().numpy(), b8.cpu().numpy()
+                t0 = time.perf_counter()
+                oracle.gemm_e4m3(a_rows, b_all, 0.01, 0.002)
+                dt = time.perf_counter() - t0
+                cpu = {"value": 2.0 * len(rows) * N * K / dt / 1e12, "unit": "TFLOP/s",
+                       "cores": os.cpu_count(), "kind": "oracle", "seconds": dt,
+                       "sample": f"16 of {M} rows of {name} (numpy FP64 matmul)"}
+    value = total_flops / (total_ms * 1e-3) / 1e12
+    print(json.dumps({
+        "metric": "FP8 GEMM TFLOP/s on the FLUX.1 Kontext block's linear layers "
+                  "(QKV projection and MLP, 8704 tokens, hidden 3072)",
+        "value": value, "unit": "TFLOP/s", "n_gpus": 1, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": total_ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "e4m3",
+        "data": "synthetic: seeded random E4M3 codes, per-tensor multipliers 0.01 and 0.002",
+        "config": {"workload": "qkv_proj 8704x9216x3072, mlp_up 8704x12288x3072, "
+                               "mlp_down 8704x3072x12288 (M x N x K)",
+                   "l2": "flushed before every launch, outside the timed events"},
+        "roofline": {"bound": "tensor", "achieved": value, "peak": fp8_peak, "unit": "TFLOP/s",
+                     "frac": value / fp8_peak, "traffic": None, "kernel": "k_gemm_fp8",
+                     "peak_source": f"{peak_kind} bf16 {bf16_tf} TFLOP/s x {FP8_PER_BF16} "
+                                    "(nominal FP8/BF16 ratio)", "per_shape": per_shape},
+        "gpu_launches": 3 * args.steps,
+        "clocks": clocks.summary(),
+        "cpu_baseline": cpu,
+    }), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -448,11 +535,15 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--static-scales", action="store_true",
                     help="quantize with amax values calibrated once before timing (one pass)")
+    ap.add_argument("--gemm", action="store_true",
+                    help="time the FP8 GEMM of the transformer block's linear layers instead")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     if args.impl == "reference":
         run_reference(args)
+    elif args.gemm:
+        run_gemm(args)
     else:
         run_gpu(args)
 

@@ -165,6 +165,17 @@ QATTN_API qattn_status qattn_calibrate_quantize_qkv(const qattn_quant_io* io, si
 QATTN_API qattn_status qattn_quantize_qkv(const qattn_quant_io* io, size_t n, qattn_mode mode,
                                           qattn_stream_t stream);
 
+/* FP8 GEMM of the transformer block's quantized linear layers (QKV and output projections,
+ * MLP; the blog quantizes them with the same per-tensor FP8 FakeQuantize, "Workflow and
+ * quantization"): Y = X W^T with X8 [M, K] and W8 [N, K] E4M3 codes (K contiguous, row-major),
+ *   y_bf16[m, n] = bf16( (sum_k val(a8[m, k]) * val(b8[n, k])) * fl32(s_a * s_b) ),
+ * products accumulated in FP32 on the tensor cores.  s_a_dev, s_b_dev: device floats (the
+ * dequantization multipliers, e.g. from qattn_quantize_fp8).  Needs K % 128 == 0 and
+ * N % 32 == 0 (M arbitrary); a8, b8, y_bf16 16-byte aligned; y_bf16 is [M, N] row-major. */
+QATTN_API qattn_status qattn_gemm_fp8(const uint8_t* a8, const uint8_t* b8, void* y_bf16, int M,
+                                      int N, int K, const float* s_a_dev, const float* s_b_dev,
+                                      qattn_stream_t stream);
+
 /* qattn_calibrate_quantize_fp8 without a caller workspace (the blog has no counterpart: this is
  * a calling convention, not part of the method).  For callers that cannot supply a scratch
  * buffer -- C code with no device allocator at the call site, or a runtime whose device memory

@@ -12,7 +12,9 @@ softmax, per-tensor FP8 P, FP8 BMM2.
 
 ``attention_fp64`` is the unquantized closed form softmax(Q K^T * sm_scale) V in FP64 (numpy
 matmul as a library primitive), used to pin the oracle's attention and to report the
-quantized path's error against unquantized attention.
+quantized path's error against unquantized attention.  ``gemm_e4m3`` is the plain definition of
+the block's FP8 linear layers (same blog, same section: the GEMMs are quantized like the
+attention inputs), also in FP64.
 """
 from __future__ import annotations
 
@@ -271,3 +273,19 @@ def method_forward(q, k, v, mode="fp8", sm_scale=None, cu_seqlens=None, rows=Non
     v8, sv, _ = quantize_tensor(v, mode)
     return attention_e4m3(q8, k8, v8, shape, sq, sk, sv, sm_scale, flags, cu_seqlens, rows,
                           with_ambiguity)
+
+
+def gemm_e4m3(a8, b8, s_a, s_b, rows=None):
+    """The FP8 linear layer, Y = X W^T, as its plain definition in FP64: a8 [M, K] and b8 [N, K]
+    E4M3 codes (uint8), s_a, s_b their per-tensor dequantization multipliers;
+    Y[m, n] = sum_k (val(a8[m, k]) s_a) (val(b8[n, k]) s_b).  numpy matmul as the library
+    primitive.  rows: optional row indices of Y to compute.  Returns (Y, bound) with
+    bound[m, n] = sum_k |val(a8[m, k]) s_a| |val(b8[n, k]) s_b|, the scale of the terms that an
+    FP32 accumulation error is relative to."""
+    tab = e4m3_table()
+    a8 = np.asarray(a8)
+    if rows is not None:
+        a8 = a8[np.asarray(rows)]
+    a = tab[a8] * float(s_a)
+    b = tab[np.asarray(b8)] * float(s_b)
+    return a @ b.T, np.abs(a) @ np.abs(b).T

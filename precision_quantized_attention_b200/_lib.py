@@ -22,11 +22,12 @@ EXPORTS = (
     "qattn_calibrate_amax", "qattn_quantize_fp8", "qattn_quantize_fp4_block", "qattn_forward",
     "qattn_forward_varlen", "qattn_get_error", "qattn_calibrate_quantize_fp8",
     "qattn_calibrate_quantize_fp4_block", "qattn_calibrate_quantize_fp8_noalloc",
-    "qattn_calibrate_quantize_qkv", "qattn_quantize_qkv", "qattn_forward_ws", "qattn_status_str",
+    "qattn_calibrate_quantize_qkv", "qattn_quantize_qkv", "qattn_forward_ws", "qattn_gemm_fp8",
+    "qattn_status_str",
     "qattn_forward_workspace_bytes",
     "qattn_debug_set_wait_timeout_ns", "qattn_debug_inject_missing_q",
 )
-_RETURNS_STATUS = EXPORTS[:12]
+_RETURNS_STATUS = EXPORTS[:13]
 FUSED_WORKSPACE_BYTES = 256     # QATTN_FUSED_WORKSPACE_BYTES
 
 
@@ -69,6 +70,7 @@ def load() -> ctypes.CDLL:
     lib.qattn_calibrate_quantize_fp8_noalloc.argtypes = [P, S, P, P, P, P]
     lib.qattn_calibrate_quantize_qkv.argtypes = [ctypes.POINTER(QuantIO), S, I, P, S, P]
     lib.qattn_quantize_qkv.argtypes = [ctypes.POINTER(QuantIO), S, I, P]
+    lib.qattn_gemm_fp8.argtypes = [P, P, P, I, I, I, P, P, P]
     lib.qattn_forward.argtypes = [P, P, P, P, I, I, I, I, ctypes.POINTER(_Scales), F, I, P]
     lib.qattn_forward_varlen.argtypes = [P, P, P, P, P, I, I, I, I, I, ctypes.POINTER(_Scales),
                                          F, I, P]
@@ -237,6 +239,21 @@ def quantize_qkv(xs, amax, codes8, scale8, mode: int = MODE_FP8, e2m1=None, bsca
     other arguments as for calibrate_quantize_qkv (no workspace)."""
     io, n = _qkv_io(xs, amax, codes8, scale8, mode, e2m1, bscale, gscale)
     _check(load().qattn_quantize_qkv(io, n, int(mode), _stream(stream)), "qattn_quantize_qkv")
+
+
+def gemm_fp8(a8, b8, y, s_a, s_b, stream=None):
+    """y [M, N] bf16 = (a8 [M, K] b8 [N, K]^T) * s_a * s_b (E4M3 codes, K contiguous; s_a, s_b
+    one-element float32 device tensors).  K % 128 == 0, N % 32 == 0."""
+    if a8.dim() != 2 or b8.dim() != 2 or a8.shape[1] != b8.shape[1]:
+        raise ValueError("a8 [M, K] and b8 [N, K] with the same K")
+    M, K = a8.shape
+    N = b8.shape[0]
+    if tuple(y.shape) != (M, N):
+        raise ValueError("y must be [M, N]")
+    _check(load().qattn_gemm_fp8(_dev(a8, torch.uint8, "a8"), _dev(b8, torch.uint8, "b8"),
+                                 _dev(y, torch.bfloat16, "y"), M, N, K,
+                                 _dev(s_a, torch.float32, "s_a"), _dev(s_b, torch.float32, "s_b"),
+                                 _stream(stream)), "qattn_gemm_fp8")
 
 
 def _scales(s_q, s_k, s_v):

@@ -12,7 +12,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(os.path.dirname(HERE), "include")
 LIB = os.path.join(HERE, "libqattn.so")
-SOURCES = ["qattn_api.cu", "quant.cu", "attn_fwd.cu", "noalloc.cu"]
+SOURCES = ["qattn_api.cu", "quant.cu", "attn_fwd.cu", "noalloc.cu", "gemm_fp8.cu"]
 HEADERS = ["sm100_ptx.cuh", "launch.h"]
 
 

@@ -1,0 +1,275 @@
+// gemm_fp8.cu -- FP8 (E4M3) GEMM with per-tensor scales for sm_100a (TMA + tcgen05 + TMEM).
+//
+// The transformer block around the quantized attention: the NVIDIA developer blog "Optimizing
+// FLUX.1 Kontext for Image Editing with Low-Precision Quantization" quantizes the block's
+// linear layers (QKV and output projections, MLP) to FP8 with the same per-tensor FakeQuantize
+// as the attention inputs ("Workflow and quantization"; Fig. 3 puts the GEMMs and the SDPA at
+// about 75 % of the transformer's time).  Computed here:
+//   Y[m, n] = bf16( (sum_k val(A8[m, k]) * val(B8[n, k])) * fl32(s_a * s_b) )
+// with A8 [M, K] the E4M3 activations and B8 [N, K] the E4M3 weights, both K-contiguous
+// (Y = X W^T), the products accumulated in FP32 on the tensor cores.
+//
+// Kernel structure: persistent, one CTA per SM, 192 threads.
+//   warp 0      TMA producer: per 128 x 256 output tile and per 128-byte K block, the A tile
+//               (128 rows) and the B tile (256 rows), 128-byte swizzle, into a 4-stage ring.
+//   warp 1      MMA issuer (one thread) and TMEM owner: tcgen05.mma.cta_group::1.kind::f8f6f4,
+//               M = 128, N = 256, four K = 32 steps per K block, into one of two 256-column
+//               FP32 accumulators in TMEM, so the next tile's MMAs overlap this tile's epilogue.
+//   warps 2-5   epilogue: thread = output row = TMEM lane; 32 columns at a time from TMEM,
+//               scaled, rounded to bf16 and stored (16-byte stores).
+// Output tiles are visited m-fastest (CTAs in flight share the weight tile, the activation
+// matrix stays in L2).  All waits are bounded (a global-timer limit).
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <cstdint>
+
+#include "launch.h"
+#include "sm100_ptx.cuh"
+
+namespace qattn {
+
+namespace gemm {
+constexpr int BM = 128;                  // output rows per tile (= TMEM lanes)
+constexpr int BN = 256;                  // output columns per tile (MMA N)
+constexpr int BK = 128;                  // K elements (bytes) per stage
+constexpr int STAGES = 4;
+constexpr int THREADS = 192;
+constexpr int WARP_LOAD = 0, WARP_MMA = 1;                  // warps 2-5: epilogue
+constexpr int TILE_A = BM * BK;          // 16 KB
+constexpr int TILE_B = BN * BK;          // 32 KB
+constexpr int OFF_A = 0;
+constexpr int OFF_B = OFF_A + STAGES * TILE_A;
+constexpr int OFF_BAR = OFF_B + STAGES * TILE_B;
+// barriers: full[STAGES], empty[STAGES], acc_full[2], acc_empty[2], drain
+constexpr int NBARS = 2 * STAGES + 4 + 1;
+constexpr int OFF_TMEM = OFF_BAR + 8 * NBARS;
+constexpr int OFF_ABORT = OFF_TMEM + 4;
+constexpr int BYTES = OFF_ABORT + 4;
+constexpr int ALLOC = BYTES + 1024;      // slack for 1024-byte alignment
+static_assert(TILE_A % 1024 == 0 && TILE_B % 1024 == 0, "alignment");
+static_assert(ALLOC <= 227 * 1024, "shared memory per CTA");
+constexpr uint32_t TMEM_COLS = 2 * BN;   // two accumulators
+}  // namespace gemm
+
+struct GemmArgs {
+  int M, N, K;
+  const float* s_a;
+  const float* s_b;
+  __nv_bfloat16* y;
+  int* err;
+  uint64_t timeout_ns;
+};
+
+__global__ void __launch_bounds__(gemm::THREADS, 1)
+    k_gemm_fp8(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
+               const __grid_constant__ GemmArgs args) {
+  using namespace gemm;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_u32 = smem_u32(smem_raw);
+  const uint32_t base_u32 = (raw_u32 + 1023u) & ~1023u;
+  uint8_t* base = smem_raw + (base_u32 - raw_u32);
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  const int tiles_m = (args.M + BM - 1) / BM;
+  const int tiles = tiles_m * ((args.N + BN - 1) / BN);
+  const int kblocks = args.K / BK;
+  if (static_cast<int>(blockIdx.x) >= tiles) return;   // uniform over the CTA
+
+  const uint32_t bar0 = base_u32 + OFF_BAR;
+  auto BAR = [&](int i) { return bar0 + 8u * static_cast<uint32_t>(i); };
+  constexpr int B_FULL = 0, B_EMPTY = STAGES, B_ACCF = 2 * STAGES, B_ACCE = B_ACCF + 2;
+  constexpr int B_DRAIN = B_ACCE + 2;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(base + OFF_ABORT);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base + OFF_TMEM);
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < STAGES; ++i) { mbar_init(BAR(B_FULL + i), 1); mbar_init(BAR(B_EMPTY + i), 1); }
+    for (int b = 0; b < 2; ++b) { mbar_init(BAR(B_ACCF + b), 1); mbar_init(BAR(B_ACCE + b), 128); }
+    mbar_init(BAR(B_DRAIN), 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == WARP_MMA) {
+    tmem_alloc(base_u32 + OFF_TMEM, TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint64_t tlim = args.timeout_ns;
+
+  if (warp == WARP_LOAD) {
+    // ======================= TMA producer =======================
+    if (lane == 0) {
+      tma_prefetch_desc(&tm_a);
+      tma_prefetch_desc(&tm_b);
+      int u = 0;                                   // K blocks issued (ring position)
+      bool ok = true;
+      for (int t = blockIdx.x; ok && t < tiles; t += gridDim.x) {
+        const int m0 = (t % tiles_m) * BM, n0 = (t / tiles_m) * BN;
+        for (int kb = 0; kb < kblocks; ++kb, ++u) {
+          const int s = u % STAGES;
+          if (u >= STAGES &&
+              !mbar_wait(BAR(B_EMPTY + s), ((u / STAGES) - 1) & 1, tlim, abort_flag, args.err)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(BAR(B_FULL + s), TILE_A + TILE_B);
+          tma_load_2d(base_u32 + OFF_A + s * TILE_A, &tm_a, BAR(B_FULL + s), kb * BK, m0);
+          tma_load_2d(base_u32 + OFF_B + s * TILE_B, &tm_b, BAR(B_FULL + s), kb * BK, n0);
+        }
+      }
+      // drain: every issued load has landed before the CTA may exit (instant when healthy)
+      for (int j = u - 1; j >= 0 && j >= u - STAGES; --j)
+        mbar_drain(BAR(B_FULL + j % STAGES), (j / STAGES) & 1, tlim);
+    }
+  } else if (warp == WARP_MMA) {
+    // ======================= MMA issuer =======================
+    if (lane == 0) {
+      constexpr uint32_t IDESC = idesc_e4m3_f32(BM, BN, false);
+      int u = 0, i = 0;                            // K blocks consumed; tiles of this CTA
+      bool ok = true;
+      for (int t = blockIdx.x; ok && t < tiles; t += gridDim.x, ++i) {
+        const int ab = i & 1;                      // accumulator of this tile
+        // the epilogue has read out the tile that used this accumulator two tiles ago
+        if (i >= 2)
+          ok = mbar_wait(BAR(B_ACCE + ab), ((i >> 1) - 1) & 1, tlim, abort_flag, args.err);
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t acc = tmem + static_cast<uint32_t>(ab * BN);
+        for (int kb = 0; kb < kblocks; ++kb, ++u) {
+          const int s = u % STAGES;
+          ok = mbar_wait(BAR(B_FULL + s), (u / STAGES) & 1, tlim, abort_flag, args.err);
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t a_s = base_u32 + OFF_A + s * TILE_A;
+          const uint32_t b_s = base_u32 + OFF_B + s * TILE_B;
+#pragma unroll
+          for (int kk = 0; kk < BK / 32; ++kk) {
+            // K-major rows of 128 bytes, 128-byte swizzle, 8-row atoms (SBO 1024); 32-byte K steps
+            const uint64_t da = smem_desc(a_s + kk * 32, 16, 1024, 2u);
+            const uint64_t db = smem_desc(b_s + kk * 32, 16, 1024, 2u);
+            mma_f8_ss(acc, da, db, IDESC, (kb > 0 || kk > 0) ? 1u : 0u);
+          }
+          mma_commit(BAR(B_EMPTY + s));           // stage free once these MMAs complete
+        }
+        if (ok) mma_commit(BAR(B_ACCF + ab));     // accumulator complete
+      }
+      mma_commit(BAR(B_DRAIN));
+      mbar_drain(BAR(B_DRAIN), 0, tlim);
+    }
+  } else {
+    // ======================= epilogue warps =======================
+    const int quarter = warp & 3;                  // TMEM lane quarter of this warp
+    const int r = quarter * 32 + lane;             // row within the tile
+    const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+    const float scale = __ldg(args.s_a) * __ldg(args.s_b);
+    int i = 0;
+    for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++i) {
+      const int ab = i & 1;
+      const bool ok = mbar_wait(BAR(B_ACCF + ab), (i >> 1) & 1, tlim, abort_flag, args.err);
+      if (!__all_sync(0xFFFFFFFFu, ok)) break;
+      tc_fence_after();
+      const int m = (t % tiles_m) * BM + r, n0 = (t / tiles_m) * BN;
+      __nv_bfloat16* yrow = args.y + static_cast<size_t>(m) * args.N + n0;
+      const uint32_t acc = tmem + lane_off + static_cast<uint32_t>(ab * BN);
+#pragma unroll 1
+      for (int c = 0; c < BN / 32; ++c) {
+        uint32_t v[32];
+        tmem_ld32(acc + c * 32, v);
+        tmem_wait_ld();
+        if (m < args.M && n0 + c * 32 < args.N) {   // N % 32 == 0: a chunk is all in or out
+          uint32_t packed[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const __nv_bfloat162 b2 = __floats2bfloat162_rn(__uint_as_float(v[2 * e]) * scale,
+                                                            __uint_as_float(v[2 * e + 1]) * scale);
+            packed[e] = *reinterpret_cast<const uint32_t*>(&b2);
+          }
+          uint4* dst = reinterpret_cast<uint4*>(yrow + c * 32);
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            dst[e] = make_uint4(packed[4 * e], packed[4 * e + 1], packed[4 * e + 2], packed[4 * e + 3]);
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(BAR(B_ACCE + ab));               // accumulator read out
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == WARP_MMA) {
+    tc_fence_after();
+    tmem_dealloc(tmem, gemm::TMEM_COLS);
+  }
+}
+
+// ---------------------------------------------------------------------------------------------
+// Host side
+// ---------------------------------------------------------------------------------------------
+using GemmEncodeFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static GemmEncodeFn gemm_encode_fn() {
+  static GemmEncodeFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<GemmEncodeFn>(p);
+  }
+  return fn;
+}
+
+// [rows, K] E4M3, K contiguous; box of `box_rows` rows x 128 bytes, 128-byte swizzle; reads past
+// the last row return zeros.
+static bool make_map_2d(CUtensorMap* map, const void* ptr, int rows, int K, int box_rows) {
+  GemmEncodeFn enc = gemm_encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(K)};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(gemm::BK), static_cast<cuuint32_t>(box_rows)};
+  cuuint32_t estr[2] = {1u, 1u};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(ptr), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+cudaError_t launch_gemm_fp8(const uint8_t* a8, const uint8_t* b8, void* y, int M, int N, int K,
+                            const float* s_a, const float* s_b, int* err, uint64_t timeout_ns,
+                            int num_sms, cudaStream_t stream) {
+  CUtensorMap ma, mb;
+  if (!make_map_2d(&ma, a8, M, K, gemm::BM) || !make_map_2d(&mb, b8, N, K, gemm::BN))
+    return cudaErrorInvalidValue;
+  static int configured_dev_mask = 0;   // bit per device id < 31
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev >= 31 || !(configured_dev_mask & (1 << dev))) {
+    cudaError_t e = cudaFuncSetAttribute(k_gemm_fp8, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         gemm::ALLOC);
+    if (e != cudaSuccess) return e;
+    if (dev < 31) configured_dev_mask |= 1 << dev;
+  }
+  GemmArgs a;
+  a.M = M;
+  a.N = N;
+  a.K = K;
+  a.s_a = s_a;
+  a.s_b = s_b;
+  a.y = static_cast<__nv_bfloat16*>(y);
+  a.err = err;
+  a.timeout_ns = timeout_ns;
+  const int tiles = ((M + gemm::BM - 1) / gemm::BM) * ((N + gemm::BN - 1) / gemm::BN);
+  const int grid = tiles < num_sms ? tiles : num_sms;
+  k_gemm_fp8<<<grid, gemm::THREADS, gemm::ALLOC, stream>>>(ma, mb, a);
+  return cudaGetLastError();
+}
+
+}  // namespace qattn

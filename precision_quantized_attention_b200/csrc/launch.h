@@ -34,6 +34,11 @@ cudaError_t launch_quant_qkv(const void* const* x, uint8_t* const* codes8, float
                              float* const* gscale, size_t n, int mode, int* err, int num_sms,
                              cudaStream_t stream);
 
+// Y[M, N] (bf16) = (A8[M, K] B8[N, K]^T) * s_a * s_b; K % 128 == 0, N % 32 == 0.
+cudaError_t launch_gemm_fp8(const uint8_t* a8, const uint8_t* b8, void* y, int M, int N, int K,
+                            const float* s_a, const float* s_b, int* err, uint64_t timeout_ns,
+                            int num_sms, cudaStream_t stream);
+
 // Persistent schedule of a dense attention launch (see plan_attention_split in attn_fwd.cu):
 // ctas CTAs, `whole` whole pairs each, then tail ranges of tail_w key steps; bytes = workspace
 // the cut tail pairs need (0: no pair is cut).

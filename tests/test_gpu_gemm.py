@@ -1,0 +1,67 @@
+"""GPU FP8 GEMM (the block's quantized linear layers) vs the oracle's FP64 definition.
+
+Inputs are seeded E4M3 codes drawn on the host (every finite code, both signs) with
+per-tensor multipliers; the bar follows from the arithmetic: the products are exact, their FP32
+accumulation is off by at most K * 2^-24 of the sum of |terms|, and the bf16 output rounding by
+2^-9 of the value (2^-8 allowed, covering the rounding of s_a * s_b)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import precision_quantized_attention_b200 as qa
+
+pytestmark = pytest.mark.gpu
+
+
+def _codes(rng, shape):
+    c = rng.integers(0, 256, size=shape, dtype=np.uint8)
+    c[(c & 0x7F) == 0x7F] ^= 0x01               # no NaN codes (0x7F -> 0x7E)
+    return c
+
+
+def _run(M, N, K, seed, s_a=0.01, s_b=0.002):
+    rng = np.random.default_rng(seed)
+    a8, b8 = _codes(rng, (M, K)), _codes(rng, (N, K))
+    sa = torch.tensor([s_a], dtype=torch.float32, device="cuda")
+    sb = torch.tensor([s_b], dtype=torch.float32, device="cuda")
+    y = torch.full((M, N), float("nan"), dtype=torch.bfloat16, device="cuda")
+    qa.gemm_fp8(torch.from_numpy(a8).cuda(), torch.from_numpy(b8).cuda(), y, sa, sb)
+    assert qa.get_error() == 0
+    return a8, b8, np.float32(s_a), np.float32(s_b), y
+
+
+def _check(got, want, bound, K):
+    excess = np.abs(got.astype(np.float64) - want) - (2.0 ** -8 * np.abs(want) + K * 2.0 ** -24 * bound)
+    assert np.isfinite(got).all()
+    assert excess.max() <= 0.0, f"worst excess {excess.max():.3e}"
+
+
+@pytest.mark.parametrize("M,N,K", [(1, 32, 128), (130, 288, 256), (300, 512, 384), (257, 96, 1024)])
+def test_small_shapes_all_elements(M, N, K):
+    """Ragged row tiles (M not a multiple of 128), a partial column tile (N not a multiple of
+    256) and several K blocks."""
+    a8, b8, sa, sb, y = _run(M, N, K, seed=M + N + K)
+    want, bound = oracle.gemm_e4m3(a8, b8, sa, sb)
+    _check(y.float().cpu().numpy(), want, bound, K)
+
+
+@pytest.mark.parametrize("M,N,K", [(8704, 9216, 3072), (8704, 12288, 3072), (8704, 3072, 12288)])
+def test_kontext_block_shapes_sampled_rows(M, N, K):
+    """The joint sequence (512 text + 4096 target + 4096 context tokens) through the block's QKV
+    projection (3072 -> 3 x 3072) and the MLP (3072 -> 12288 -> 3072): every column of 64
+    seeded rows, first and last row included."""
+    a8, b8, sa, sb, y = _run(M, N, K, seed=K)
+    rows = np.unique(np.concatenate([[0, M - 1], np.random.default_rng(1).integers(0, M, 62)]))
+    want, bound = oracle.gemm_e4m3(a8, b8, sa, sb, rows=rows)
+    got = y[torch.as_tensor(rows, device="cuda")].float().cpu().numpy()
+    _check(got, want, bound, K)
+
+
+def test_repeatable_and_scales_applied():
+    a8, b8, sa, sb, y = _run(384, 512, 512, seed=9)
+    y2 = torch.empty_like(y)
+    qa.gemm_fp8(torch.from_numpy(a8).cuda(), torch.from_numpy(b8).cuda(), y2,
+                torch.tensor([sa * 2], device="cuda"), torch.tensor([sb], device="cuda"))
+    assert qa.get_error() == 0
+    assert torch.equal(y2.float(), (y.float() * 2))   # a power of two: exact in bf16
