@@ -171,7 +171,10 @@ QATTN_API qattn_status qattn_quantize_qkv(const qattn_quant_io* io, size_t n, qa
  *   y_bf16[m, n] = bf16( (sum_k val(a8[m, k]) * val(b8[n, k])) * fl32(s_a * s_b) ),
  * products accumulated in FP32 on the tensor cores.  s_a_dev, s_b_dev: device floats (the
  * dequantization multipliers, e.g. from qattn_quantize_fp8).  Needs K % 128 == 0 and
- * N % 32 == 0 (M arbitrary); a8, b8, y_bf16 16-byte aligned; y_bf16 is [M, N] row-major. */
+ * N % 32 == 0 (M arbitrary); a8, b8, y_bf16 16-byte aligned; y_bf16 is [M, N] row-major.
+ * M > 128 runs on pairs of SMs (256 x 256 tiles, one MMA over both SMs), M <= 128 on one SM per
+ * 128 x 256 tile; both give the same result for every element (the same FP32 products are summed
+ * in the same K order). */
 QATTN_API qattn_status qattn_gemm_fp8(const uint8_t* a8, const uint8_t* b8, void* y_bf16, int M,
                                       int N, int K, const float* s_a_dev, const float* s_b_dev,
                                       qattn_stream_t stream);

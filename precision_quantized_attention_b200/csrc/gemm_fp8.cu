@@ -9,7 +9,9 @@
 // with A8 [M, K] the E4M3 activations and B8 [N, K] the E4M3 weights, both K-contiguous
 // (Y = X W^T), the products accumulated in FP32 on the tensor cores.
 //
-// Kernel structure: persistent, one CTA per SM, 192 threads.
+// Two persistent kernels, both 192 threads with the roles below: `k_gemm_fp8_pair` (M > 128)
+// pairs two SMs on each 256 x 256 tile (see its own comment); `k_gemm_fp8` (M <= 128) runs one
+// SM per 128 x 256 tile:
 //   warp 0      TMA producer: per 128 x 256 output tile and per 128-byte K block, the A tile
 //               (128 rows) and the B tile (256 rows), 128-byte swizzle, into a 4-stage ring.
 //   warp 1      MMA issuer (one thread) and TMEM owner: tcgen05.mma.cta_group::1.kind::f8f6f4,
@@ -208,6 +210,204 @@ __global__ void __launch_bounds__(gemm::THREADS, 1)
 }
 
 // ---------------------------------------------------------------------------------------------
+// Pair kernel: two SMs (a cluster of two CTAs) on one 256 x 256 output tile.
+//
+// One tcgen05.mma.cta_group::2 with M = 256, N = 256 reads 128 rows of A and 128 rows of B from
+// each CTA's shared memory and leaves 128 rows x 256 columns of the FP32 tile in each CTA's TMEM.
+// Per 128-byte K block an SM therefore stages 32 KB (not 48 KB as on one SM for the same MMA
+// work), so six stages fit and cover more of the TMA refill latency.
+//   warp 0 (both CTAs)  TMA producer for its own halves of A and B; completion is counted on the
+//                       leading CTA's `full` barrier (64 KB per stage); waits on its own `empty`.
+//   warp 1              TMEM owner in both CTAs; in the leading CTA, one thread issues the MMAs
+//                       and commits `empty` / `acc_full` to the barriers of both CTAs.
+//   warps 2-5 (both)    epilogue of the CTA's 128 rows; each warp arrives once per tile on the
+//                       leading CTA's `acc_empty` (8 arrivals release an accumulator).
+// Both CTAs reach the two cluster barriers (after set-up, before the TMEM free) on every path:
+// every wait in between is bounded.
+// ---------------------------------------------------------------------------------------------
+namespace gemm2 {
+constexpr int BM = 256;                  // output rows per tile pair (128 per CTA)
+constexpr int BN = 256;                  // output columns per tile (MMA N; 128 B rows per CTA)
+constexpr int BK = 128;
+constexpr int STAGES = 6;
+constexpr int THREADS = 192;
+constexpr int WARP_LOAD = 0, WARP_MMA = 1;
+constexpr int TILE_A = (BM / 2) * BK;    // 16 KB per CTA
+constexpr int TILE_B = (BN / 2) * BK;    // 16 KB per CTA
+constexpr int OFF_A = 0;
+constexpr int OFF_B = OFF_A + STAGES * TILE_A;
+constexpr int OFF_BAR = OFF_B + STAGES * TILE_B;
+// barriers: full[STAGES] (leader), empty[STAGES], acc_full[2], acc_empty[2] (leader), drain
+constexpr int NBARS = 2 * STAGES + 4 + 1;
+constexpr int OFF_TMEM = OFF_BAR + 8 * NBARS;
+constexpr int OFF_ABORT = OFF_TMEM + 4;
+constexpr int BYTES = OFF_ABORT + 4;
+constexpr int ALLOC = BYTES + 1024;
+static_assert(TILE_A % 1024 == 0 && TILE_B % 1024 == 0, "alignment");
+static_assert(ALLOC <= 227 * 1024, "shared memory per CTA");
+constexpr uint32_t TMEM_COLS = 2 * BN;
+constexpr uint32_t STAGE_TX = 2u * (TILE_A + TILE_B);   // bytes of both CTAs per stage
+}  // namespace gemm2
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(gemm2::THREADS, 1)
+    k_gemm_fp8_pair(const __grid_constant__ CUtensorMap tm_a,
+                    const __grid_constant__ CUtensorMap tm_b,
+                    const __grid_constant__ GemmArgs args) {
+  using namespace gemm2;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_u32 = smem_u32(smem_raw);
+  const uint32_t base_u32 = (raw_u32 + 1023u) & ~1023u;   // the same offset in both CTAs
+  uint8_t* base = smem_raw + (base_u32 - raw_u32);
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();                  // 0 leads the pair
+  const bool leader = rank == 0;
+  const int pair = static_cast<int>(blockIdx.x >> 1), npairs = static_cast<int>(gridDim.x >> 1);
+
+  const int tiles_m = (args.M + BM - 1) / BM;
+  const int tiles = tiles_m * ((args.N + BN - 1) / BN);   // the host launches <= tiles pairs
+  const int kblocks = args.K / BK;
+
+  const uint32_t bar0 = base_u32 + OFF_BAR;
+  auto BAR = [&](int i) { return bar0 + 8u * static_cast<uint32_t>(i); };
+  constexpr int B_FULL = 0, B_EMPTY = STAGES, B_ACCF = 2 * STAGES, B_ACCE = B_ACCF + 2;
+  constexpr int B_DRAIN = B_ACCE + 2;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(base + OFF_ABORT);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base + OFF_TMEM);
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < STAGES; ++i) { mbar_init(BAR(B_FULL + i), 1); mbar_init(BAR(B_EMPTY + i), 1); }
+    for (int b = 0; b < 2; ++b) { mbar_init(BAR(B_ACCF + b), 1); mbar_init(BAR(B_ACCE + b), 8); }
+    mbar_init(BAR(B_DRAIN), 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == WARP_MMA) {
+    tmem_alloc_pair(base_u32 + OFF_TMEM, TMEM_COLS);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  cluster_sync();                      // barriers of both CTAs initialised, TMEM allocated
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint64_t tlim = args.timeout_ns;
+
+  if (warp == WARP_LOAD) {
+    // ======================= TMA producer (both CTAs) =======================
+    if (lane == 0) {
+      tma_prefetch_desc(&tm_a);
+      tma_prefetch_desc(&tm_b);
+      int u = 0;
+      bool ok = true;
+      for (int t = pair; ok && t < tiles; t += npairs) {
+        const int m0 = (t % tiles_m) * BM + static_cast<int>(rank) * (BM / 2);
+        const int n0 = (t / tiles_m) * BN + static_cast<int>(rank) * (BN / 2);
+        for (int kb = 0; kb < kblocks; ++kb, ++u) {
+          const int s = u % STAGES;
+          if (u >= STAGES &&
+              !mbar_wait(BAR(B_EMPTY + s), ((u / STAGES) - 1) & 1, tlim, abort_flag, args.err)) {
+            ok = false;
+            break;
+          }
+          if (leader) mbar_arrive_expect_tx(BAR(B_FULL + s), STAGE_TX);
+          const uint32_t full_lead = mapa_shared(BAR(B_FULL + s), 0);
+          tma_load_2d_pair(base_u32 + OFF_A + s * TILE_A, &tm_a, full_lead, kb * BK, m0);
+          tma_load_2d_pair(base_u32 + OFF_B + s * TILE_B, &tm_b, full_lead, kb * BK, n0);
+        }
+      }
+      // the MMAs have released every stage this CTA filled: its loads have landed and no
+      // commit from the leading CTA is still on its way here (instant when healthy)
+      for (int j = u - 1; j >= 0 && j >= u - STAGES; --j)
+        mbar_drain(BAR(B_EMPTY + j % STAGES), (j / STAGES) & 1, tlim);
+    }
+  } else if (warp == WARP_MMA) {
+    // ======================= MMA issuer (leading CTA) =======================
+    if (leader && lane == 0) {
+      constexpr uint32_t IDESC = idesc_e4m3_f32(BM, BN, false);
+      const uint32_t peer = rank ^ 1u;
+      int u = 0, i = 0;
+      bool ok = true;
+      for (int t = pair; ok && t < tiles; t += npairs, ++i) {
+        const int ab = i & 1;
+        // both CTAs' epilogues have read out the tile that used this accumulator two tiles ago
+        if (i >= 2)
+          ok = mbar_wait(BAR(B_ACCE + ab), ((i >> 1) - 1) & 1, tlim, abort_flag, args.err);
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t acc = tmem + static_cast<uint32_t>(ab * BN);
+        for (int kb = 0; kb < kblocks; ++kb, ++u) {
+          const int s = u % STAGES;
+          ok = mbar_wait(BAR(B_FULL + s), (u / STAGES) & 1, tlim, abort_flag, args.err);
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t a_s = base_u32 + OFF_A + s * TILE_A;
+          const uint32_t b_s = base_u32 + OFF_B + s * TILE_B;
+#pragma unroll
+          for (int kk = 0; kk < BK / 32; ++kk) {
+            const uint64_t da = smem_desc(a_s + kk * 32, 16, 1024, 2u);
+            const uint64_t db = smem_desc(b_s + kk * 32, 16, 1024, 2u);
+            mma_f8_ss_pair(acc, da, db, IDESC, (kb > 0 || kk > 0) ? 1u : 0u);
+          }
+          mma_commit_pair(BAR(B_EMPTY + s));                      // stage free in both CTAs
+          mma_commit_pair(mapa_shared(BAR(B_EMPTY + s), peer));
+        }
+        if (ok) {
+          mma_commit_pair(BAR(B_ACCF + ab));                      // accumulator complete
+          mma_commit_pair(mapa_shared(BAR(B_ACCF + ab), peer));
+        }
+      }
+      mma_commit_pair(BAR(B_DRAIN));
+      mbar_drain(BAR(B_DRAIN), 0, tlim);
+    }
+  } else {
+    // ======================= epilogue warps (both CTAs) =======================
+    const int quarter = warp & 3;
+    const int r = quarter * 32 + lane;
+    const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+    const float scale = __ldg(args.s_a) * __ldg(args.s_b);
+    int i = 0;
+    for (int t = pair; t < tiles; t += npairs, ++i) {
+      const int ab = i & 1;
+      const bool ok = mbar_wait(BAR(B_ACCF + ab), (i >> 1) & 1, tlim, abort_flag, args.err);
+      if (!__all_sync(0xFFFFFFFFu, ok)) break;
+      tc_fence_after();
+      const int m = (t % tiles_m) * BM + static_cast<int>(rank) * (BM / 2) + r;
+      const int n0 = (t / tiles_m) * BN;
+      __nv_bfloat16* yrow = args.y + static_cast<size_t>(m) * args.N + n0;
+      const uint32_t acc = tmem + lane_off + static_cast<uint32_t>(ab * BN);
+#pragma unroll 1
+      for (int c = 0; c < BN / 32; ++c) {
+        uint32_t v[32];
+        tmem_ld32(acc + c * 32, v);
+        tmem_wait_ld();
+        if (m < args.M && n0 + c * 32 < args.N) {
+          uint32_t packed[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const __nv_bfloat162 b2 = __floats2bfloat162_rn(__uint_as_float(v[2 * e]) * scale,
+                                                            __uint_as_float(v[2 * e + 1]) * scale);
+            packed[e] = *reinterpret_cast<const uint32_t*>(&b2);
+          }
+          uint4* dst = reinterpret_cast<uint4*>(yrow + c * 32);
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            dst[e] = make_uint4(packed[4 * e], packed[4 * e + 1], packed[4 * e + 2], packed[4 * e + 3]);
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(mapa_shared(BAR(B_ACCE + ab), 0));   // read out
+    }
+  }
+
+  tc_fence_before();
+  cluster_sync();                      // no MMA, load or arrival of either CTA is outstanding
+  if (warp == WARP_MMA) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem, gemm2::TMEM_COLS);
+  }
+}
+
+// ---------------------------------------------------------------------------------------------
 // Host side
 // ---------------------------------------------------------------------------------------------
 using GemmEncodeFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
@@ -242,21 +442,39 @@ static bool make_map_2d(CUtensorMap* map, const void* ptr, int rows, int K, int 
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Largest number of pair clusters resident at once (one CTA per SM), per device.
+static int pair_clusters_resident(int num_sms) {
+  static int cached[32] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 32 && cached[dev] > 0) return cached[dev];
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(num_sms & ~1));
+  cfg.blockDim = dim3(gemm2::THREADS);
+  cfg.dynamicSmemBytes = gemm2::ALLOC;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, k_gemm_fp8_pair, &cfg) != cudaSuccess || n <= 0) {
+    cudaGetLastError();
+    n = num_sms / 2;
+  }
+  if (dev < 32) cached[dev] = n;
+  return n;
+}
+
+static bool set_smem_once(const void* fn, int bytes, int* mask) {
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 31 && (*mask & (1 << dev))) return true;
+  if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess)
+    return false;
+  if (dev < 31) *mask |= 1 << dev;
+  return true;
+}
+
+// M <= 128 (one row tile) keeps the one-SM kernel: a 256-row pair tile would be half empty.
 cudaError_t launch_gemm_fp8(const uint8_t* a8, const uint8_t* b8, void* y, int M, int N, int K,
                             const float* s_a, const float* s_b, int* err, uint64_t timeout_ns,
                             int num_sms, cudaStream_t stream) {
-  CUtensorMap ma, mb;
-  if (!make_map_2d(&ma, a8, M, K, gemm::BM) || !make_map_2d(&mb, b8, N, K, gemm::BN))
-    return cudaErrorInvalidValue;
-  static int configured_dev_mask = 0;   // bit per device id < 31
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev >= 31 || !(configured_dev_mask & (1 << dev))) {
-    cudaError_t e = cudaFuncSetAttribute(k_gemm_fp8, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         gemm::ALLOC);
-    if (e != cudaSuccess) return e;
-    if (dev < 31) configured_dev_mask |= 1 << dev;
-  }
   GemmArgs a;
   a.M = M;
   a.N = N;
@@ -266,6 +484,24 @@ cudaError_t launch_gemm_fp8(const uint8_t* a8, const uint8_t* b8, void* y, int M
   a.y = static_cast<__nv_bfloat16*>(y);
   a.err = err;
   a.timeout_ns = timeout_ns;
+  CUtensorMap ma, mb;
+  if (M > gemm::BM && num_sms >= 2) {
+    static int configured = 0;
+    if (!make_map_2d(&ma, a8, M, K, gemm2::BM / 2) || !make_map_2d(&mb, b8, N, K, gemm2::BN / 2))
+      return cudaErrorInvalidValue;
+    if (!set_smem_once(reinterpret_cast<const void*>(k_gemm_fp8_pair), gemm2::ALLOC, &configured))
+      return cudaGetLastError();
+    const int tiles = ((M + gemm2::BM - 1) / gemm2::BM) * ((N + gemm2::BN - 1) / gemm2::BN);
+    const int resident = pair_clusters_resident(num_sms);
+    const int pairs = tiles < resident ? tiles : resident;
+    k_gemm_fp8_pair<<<2 * pairs, gemm2::THREADS, gemm2::ALLOC, stream>>>(ma, mb, a);
+    return cudaGetLastError();
+  }
+  static int configured = 0;
+  if (!make_map_2d(&ma, a8, M, K, gemm::BM) || !make_map_2d(&mb, b8, N, K, gemm::BN))
+    return cudaErrorInvalidValue;
+  if (!set_smem_once(reinterpret_cast<const void*>(k_gemm_fp8), gemm::ALLOC, &configured))
+    return cudaGetLastError();
   const int tiles = ((M + gemm::BM - 1) / gemm::BM) * ((N + gemm::BN - 1) / gemm::BN);
   const int grid = tiles < num_sms ? tiles : num_sms;
   k_gemm_fp8<<<grid, gemm::THREADS, gemm::ALLOC, stream>>>(ma, mb, a);

@@ -37,10 +37,14 @@ def _check(got, want, bound, K):
     assert excess.max() <= 0.0, f"worst excess {excess.max():.3e}"
 
 
-@pytest.mark.parametrize("M,N,K", [(1, 32, 128), (130, 288, 256), (300, 512, 384), (257, 96, 1024)])
+@pytest.mark.parametrize("M,N,K", [(1, 32, 128), (128, 1056, 512),            # one-SM kernel
+                                   (129, 288, 256), (130, 288, 256), (300, 512, 384),
+                                   (257, 96, 1024), (2560, 2080, 256)])        # SM pairs
 def test_small_shapes_all_elements(M, N, K):
-    """Ragged row tiles (M not a multiple of 128), a partial column tile (N not a multiple of
-    256) and several K blocks."""
+    """Ragged row tiles, a partial column tile (N not a multiple of 256) and several K blocks.
+    M <= 128 runs on one SM per tile; larger M on pairs of SMs with 256-row tiles, where the
+    second CTA of a pair may hold a single valid row (M = 129) or no valid column of B
+    (N = 96), and where a pair runs more than one tile (2560 x 2080: 90 tiles of 256 x 256)."""
     a8, b8, sa, sb, y = _run(M, N, K, seed=M + N + K)
     want, bound = oracle.gemm_e4m3(a8, b8, sa, sb)
     _check(y.float().cpu().numpy(), want, bound, K)
