@@ -12,15 +12,16 @@
 //     value is e4m3(p * 448) with p = 2^(S' - M) in (0, 1]; the FP32 row sum l divides O after
 //     BMM2.  (A single-pass kernel never holds the normalized P.)
 //   * M is the running row max of the base-2 scores S' = S * s_q * s_k * sm_scale * log2(e),
-//     rounded UP to an integer.  A rise of M rescales O and l by an exact power of two, and
-//     E4M3 rounding commutes with power-of-two scaling in the normal range, so the result does
-//     not depend on how keys are tiled.
+//     rounded UP to an integer.  P of a key tile is relative to the M of that tile; all
+//     rescales are exact powers of two, and E4M3 rounding commutes with power-of-two scaling in
+//     the normal range, so the result does not depend on how keys are tiled.
 //
 // Kernel structure: one CTA (one per SM) per pair of 128-row Q tiles of one (sequence, head).
 //   warp 8      TMA producer: per segment both Q tiles, then K and V tiles through separate
 //               rings.
 //   warp 9      MMA issuer (one elected thread) and TMEM owner.  Per KV tile j and Q tile t it
-//               issues O_t += P_t(j) V_j (P read from tensor memory) and right behind it, in the
+//               issues O_t += P_t(j) V_j (P read from tensor memory; block-scaled MMA, see
+//               below) and right behind it, in the
 //               same in-order tcgen05 stream, S_t = Q_t K_{j+1}^T into the columns P_t(j)
 //               occupied; one commit then tells softmax t that S_t(j+1) is ready and that O_t
 //               holds every P_t V up to tile j.
@@ -29,10 +30,15 @@
 //               and computes p*448 = 2^(S' - M + log2 448) in FP32 (hardware ex2 for most
 //               pairs, a degree-5 polynomial on the FMA pipe for the rest), sums p in packed
 //               f32x2 adds, converts to E4M3 and writes P_t(j) over S_t(j) with tcgen05.st.
-//               On a rise of M it first rescales its O row in TMEM by 2^-(rise).
+//   O_t is kept relative to a reference max M_ref per row (the row's first M): BMM2 multiplies
+//   each row of P_t(j) by 2^(M - M_ref) as an E8M0 block scale factor (kind::mxf8f6f4), which
+//   the softmax writes next to P, so a rise of M costs no pass over O.  Only when M - M_ref
+//   would pass 64 (O could leave the FP32 range) does the softmax rescale its O row in TMEM and
+//   move M_ref up; the epilogue applies the last 2^(M_ref - M).
 //   The two Q tiles alternate on the tensor pipe, so one tile's softmax overlaps the other
 //   tile's MMAs; K/V tiles are read by TMA once per CTA for both Q tiles.
-// TMEM: S_0/P_0, S_1/P_1 (128 FP32 columns each; P uses the first 32), O_0, O_1 (D columns).
+// TMEM: S_0/P_0, S_1/P_1 (128 FP32 columns each; P uses the first 32, BMM2's scale factors
+// columns 64-67 and 96-99), O_0, O_1 (D columns).
 // All waits are bounded (a global-timer limit); on expiry the CTA records a timeout in the
 // library's error word, drains what it issued and exits.
 //
@@ -172,6 +178,9 @@ template <int D>
 struct TmemCols {
   static constexpr uint32_t S0 = 0;                      // S_t / P_t at t * BLOCK_N
   static constexpr uint32_t O0 = NQ * BLOCK_N;           // O_t at O0 + t * D
+  // BMM2's E8M0 scale factors (4 columns each), written with P_t inside S_t past P_t's 32
+  // columns (S_t is not read again before the next S_t = Q_t K^T overwrites it)
+  static constexpr uint32_t SFA = 64, SFB = 96;
   static constexpr uint32_t USED = NQ * BLOCK_N + NQ * D;
   static constexpr uint32_t ALLOC = USED <= 256 ? 256 : 512;
 };
@@ -382,7 +391,6 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
     // ======================= MMA issuer =======================
     if (lane == 0) {
       constexpr uint32_t IDESC_S = idesc_e4m3_f32(BLOCK_M, BLOCK_N, false);
-      constexpr uint32_t IDESC_O = idesc_e4m3_f32(BLOCK_M, D, true);
       // Q, K: K-major rows of D bytes, swizzled in 8-row atoms (SBO = 8 rows); 32-byte K steps.
       constexpr uint32_t QK_LAYOUT = (D == 128) ? 2u : 4u;   // 128B / 64B swizzle
       constexpr uint32_t QK_SBO = 8 * D;
@@ -400,13 +408,18 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
           mma_f8_ss(tmem + TC::S0 + t * BLOCK_N, da, db, IDESC_S, kk > 0 ? 1u : 0u);
         }
       };
+      // O_t += (P_t 2^(M - M_ref)) V: the per-row power of two rides on BMM2 as an E8M0 scale
+      // factor of P, written by the softmax with P; V's factors are all 2^0
       auto bmm2 = [&](int t, int vs, bool first) {
         const uint32_t vb = base_u32 + SL::OFF_V + vs * SL::TILE_KV;
+        const uint32_t sfa = tmem + TC::S0 + t * BLOCK_N + TC::SFA;
+        const uint32_t sfb = tmem + TC::S0 + t * BLOCK_N + TC::SFB;
 #pragma unroll
         for (int kk = 0; kk < BLOCK_N / 32; ++kk) {
           const uint64_t db = smem_desc(vb + kk * 32 * D, SL::TILE_KV, V_SBO, V_LAYOUT);
-          mma_f8_ts(tmem + TC::O0 + t * D, tmem + TC::S0 + t * BLOCK_N + kk * 8, db, IDESC_O,
-                    (!first || kk > 0) ? 1u : 0u);
+          mma_mxf8_ts(tmem + TC::O0 + t * D, tmem + TC::S0 + t * BLOCK_N + kk * 8, db,
+                      idesc_mxf8_e4m3(BLOCK_M, D, true, static_cast<uint32_t>(kk)), sfa, sfb,
+                      (!first || kk > 0) ? 1u : 0u);
         }
       };
       int nk = 0, nv = 0, step = 0;               // K, V tiles consumed; key steps before this segment
@@ -481,7 +494,8 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
     for (int seg = 0; ok && get_segment(args, seg, sg); ++seg) {
     const int n = sg.kv1 - sg.kv0;
     float m_run = -INFINITY;                       // integer-valued running max (base 2)
-    float l = 0.0f;                                // running sum of p * 448
+    float m_ref = 0.0f;                            // O_t holds sum_j P(j) V 2^(m_j - m_ref)
+    float l = 0.0f;                                // running sum of p * 448 (relative to m_run)
     for (int j = 0; j < n; ++j) {
       // S_t(j) is in TMEM; BMM2 of tile j-1 has completed (it precedes in the MMA stream)
       ok = mbar_wait(BAR(B_SFULL + t), (step + j) & 1, tlim, abort_flag, args.err);
@@ -527,11 +541,17 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
           pk[i / 4 + q] = cvt_e4m3x2(p[4 * q], p[4 * q + 1]) | (cvt_e4m3x2(p[4 * q + 2], p[4 * q + 3]) << 16);
       }
       const float rowsum = ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
-      // A rise of the running max rescales this row of O (quiescent: its last BMM2 is done).
-      if (j > 0) {
-        const bool rise = m_new > m_run;
-        if (__any_sync(0xFFFFFFFFu, rise)) {
-          const float f = rise ? exp2_int(static_cast<int>(m_run - m_new)) : 1.0f;
+      // P(j) is relative to m_new and enters O scaled by 2^(m_new - m_ref) (BMM2's scale factor),
+      // so a rise of the running max leaves O alone.  Only a gap beyond 2^64, which could carry
+      // O past the FP32 range, rescales this row of O (quiescent: its last BMM2 is done) and
+      // moves m_ref up.
+      if (j == 0) {
+        m_ref = m_new;
+      } else {
+        l *= exp2_int(static_cast<int>(m_run - m_new));
+        const bool far = m_new - m_ref > 64.0f;
+        if (__any_sync(0xFFFFFFFFu, far)) {
+          const float f = far ? exp2_int(static_cast<int>(m_ref - m_new)) : 1.0f;
           uint64_t f2;                             // packed f32x2 multiplies
           asm("mov.b64 %0, {%1, %1};" : "=l"(f2) : "f"(f));
 #pragma unroll
@@ -548,13 +568,18 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
             }
             tmem_st32(tO + c4 * 32, v);
           }
-          l *= f;
+          if (far) m_ref = m_new;
         }
       }
       l += rowsum;
       m_run = m_new;
-      // P_t(j) over the first 32 columns of S_t: column c holds keys 4c..4c+3 (byte = key % 4)
+      // P_t(j) over the first 32 columns of S_t: column c holds keys 4c..4c+3 (byte = key % 4).
+      // BMM2's scale factors: the MMA reads row r's factor of P from lane r (column r / 32 of
+      // the 4-column block, one byte per 32 keys), so each thread fills its own lane's block
+      // with its row's 2^(m_new - m_ref) (E8M0 code 127 + gap), and V's block with 2^0.
       tmem_st32(tS, pk);
+      tmem_st4_same(tS + TC::SFA, (127u + static_cast<uint32_t>(m_new - m_ref)) * 0x01010101u);
+      tmem_st4_same(tS + TC::SFB, 0x7F7F7F7Fu);
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(BAR(B_PFULL + t));
@@ -567,6 +592,7 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
         tc_fence_after();
         const int row = sg.q_row0 + t * BLOCK_M + r;
         const bool valid = row < sg.seq_len;
+        const float f_ref = exp2_int(static_cast<int>(m_ref - m_run));   // O relative to m_run
         if (sg.slot >= 0) {
           // partial result of this segment: raw O row, running max and row sum
           const size_t slot = static_cast<size_t>(sg.slot) * NQ + t;
@@ -578,12 +604,12 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
             tmem_wait_ld();
 #pragma unroll
             for (int i = 0; i < 8; ++i)
-              po[c4 * 8 + i] = make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]),
-                                           __uint_as_float(v[4 * i + 2]), __uint_as_float(v[4 * i + 3]));
+              po[c4 * 8 + i] = make_float4(__uint_as_float(v[4 * i]) * f_ref, __uint_as_float(v[4 * i + 1]) * f_ref,
+                                           __uint_as_float(v[4 * i + 2]) * f_ref, __uint_as_float(v[4 * i + 3]) * f_ref);
           }
           args.part_ml[slot * BLOCK_M + r] = make_float2(m_run, l);
         } else {
-        const float scale = __ldg(args.s_v) / l;   // O = acc * s_v / 448 / (l / 448)
+        const float scale = __ldg(args.s_v) / l * f_ref;   // O = acc * s_v / 448 / (l / 448)
         __nv_bfloat16* orow =
             args.out + (static_cast<size_t>(sg.slab) * args.rows_per_slab + sg.seq_start + row) * D;
 #pragma unroll

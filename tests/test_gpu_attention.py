@@ -224,3 +224,21 @@ def test_dominant_key_gives_its_v_row():
     # per element: one code's rounding (<= 2^-4 relative) plus bf16 output rounding
     excess = np.abs(got - v8) - (2.0 ** -4 + 2.0 ** -8) * np.abs(v8)
     assert float(excess.max()) <= 1e-6, excess.max()
+
+
+def test_large_and_staggered_rises_of_the_row_max():
+    """Rows whose max jumps by 50-85 binades at the second key tile and then rises a few
+    binades per tile, the jump differing from row to row: rows past 64 binades rescale O in
+    tensor memory, the others carry the gap in BMM2's per-row scale factor, and neighbouring
+    rows (same lane quarter) carry different factors."""
+    B, H, L, D = 1, 2, 640, 128
+    w = workloads.custom("rises", "fp8", B, H, L, D, seed=41)
+    q, k, v = workloads.make_qkv(w)
+    a = torch.tensor([1.0, 1.2, 0.8, 1.1, 0.9, 1.3, 0.7, 1.05])[torch.arange(L) % 8]
+    q = (a[None, None, :, None] * (1.0 + 0.05 * q.float())).to(torch.bfloat16)
+    b = torch.tensor([0.0, 4.0, 4.2, 4.5, 4.8])[torch.arange(L) // 128]   # per key tile
+    k = (b[None, None, :, None] + 0.1 * k.float()).to(torch.bfloat16)
+    path = gpu_path(w, q, k, v)
+    got = path.out.float().cpu().numpy()
+    rel, mx = assert_close(got, oracle_path(w, q, k, v), "staggered rises")
+    print(f"staggered rises: rel-L2 {rel:.2e} max-abs {mx:.2e}")
