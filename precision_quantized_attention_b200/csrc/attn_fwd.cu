@@ -574,11 +574,12 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
       l += rowsum;
       m_run = m_new;
       // P_t(j) over the first 32 columns of S_t: column c holds keys 4c..4c+3 (byte = key % 4).
-      // BMM2's scale factors: the MMA reads row r's factor of P from lane r (column r / 32 of
-      // the 4-column block, one byte per 32 keys), so each thread fills its own lane's block
-      // with its row's 2^(m_new - m_ref) (E8M0 code 127 + gap), and V's block with 2^0.
+      // BMM2's scale factors: the MMA reads row r's factor of P from lane r, column r / 32 of
+      // the SFA block (one byte per 32 keys), so each thread writes only that column of its own
+      // lane: its row's 2^(m_new - m_ref) (E8M0 code 127 + gap) in all four bytes.  V's block
+      // (2^0, code 127) is read by every lane quarter for all D columns: four columns per lane.
       tmem_st32(tS, pk);
-      tmem_st4_same(tS + TC::SFA, (127u + static_cast<uint32_t>(m_new - m_ref)) * 0x01010101u);
+      tmem_st1(tS + TC::SFA + quarter, (127u + static_cast<uint32_t>(m_new - m_ref)) * 0x01010101u);
       tmem_st4_same(tS + TC::SFB, 0x7F7F7F7Fu);
       tmem_wait_st();
       tc_fence_before();

@@ -234,8 +234,9 @@ __device__ __forceinline__ void mma_f8_ts(uint32_t d_tmem, uint32_t a_tmem, uint
 
 // Block-scaled form (kind::mxf8f6f4, E8M0 scale factors, one per 32 K elements):
 // D[tmem] (+)= (A[tmem] * SFA) * (B[smem desc] * SFB).  sfa_tmem / sfb_tmem address 4-column
-// blocks of scale factors in tensor memory; the factor of row r of A (column n of B) for K
-// block k is byte 4 * (r / 32) + k of lane r % 32 in r's own lane quarter.
+// blocks of scale factors in tensor memory: the factor of row r of A for K block k is byte k
+// of column r / 32 in lane r; that of column n of B is byte k of column n / 32 in lane n % 32
+// of every lane quarter (each quarter computes its own 32 rows against all of B).
 __device__ __forceinline__ void mma_mxf8_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
                                             uint32_t idesc, uint32_t sfa_tmem, uint32_t sfb_tmem,
                                             uint32_t accumulate) {
@@ -275,6 +276,11 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
         "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
         "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
       : "r"(taddr));
+}
+
+// One 32-bit value into one column of this thread's lane.
+__device__ __forceinline__ void tmem_st1(uint32_t taddr, uint32_t v) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x1.b32 [%0], {%1};" ::"r"(taddr), "r"(v) : "memory");
 }
 
 // The same 32-bit value into 4 consecutive columns of this thread's lane.
