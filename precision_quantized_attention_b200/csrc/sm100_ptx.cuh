@@ -220,19 +220,8 @@ __device__ __forceinline__ void mma_f8_ss(uint32_t d_tmem, uint64_t a_desc, uint
       : "memory");
 }
 
-// D[tmem] (+)= A[tmem] * B[smem desc], kind::f8f6f4: A is read from tensor memory (row m in
-// lane m, element k in column k/4, byte k%4), issued by a single thread.
-__device__ __forceinline__ void mma_f8_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
-                                          uint32_t idesc, uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-
-// Block-scaled form (kind::mxf8f6f4, E8M0 scale factors, one per 32 K elements):
+// Block-scaled, A from tensor memory (kind::mxf8f6f4, E8M0 scale factors, one per 32 K
+// elements; A's row m in lane m, element k in column k/4, byte k%4), one issuing thread:
 // D[tmem] (+)= (A[tmem] * SFA) * (B[smem desc] * SFB).  sfa_tmem / sfb_tmem address 4-column
 // blocks of scale factors in tensor memory: the factor of row r of A for K block k is byte k
 // of column r / 32 in lane r; that of column n of B is byte k of column n / 32 in lane n % 32
