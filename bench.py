@@ -33,10 +33,10 @@ HBM_FALLBACK_GBS = 6650.0
 BF16_FALLBACK_TFLOPS = 1590.0
 FP8_PER_BF16 = 2.0          # nominal dense FP8 / BF16 tensor throughput ratio on B200
 L2_FLUSH_BYTES = 256 << 20
-# DRAM bytes (read + write) of one launch of the attention kernel, from ncu on this build:
+# DRAM bytes (read + write) of one launch of the attention kernel, from ncu on the current kernel:
 #   ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum --clock-control none \
 #       -k regex:k_attn_fp8 -s 3 -c 1 python bench.py --steps 1 --warmup 3 --no-cpu-baseline --no-e2e
-# k_attn_fp8_fwd: 80.29 MB read (Q8 + K8 + V8 = 80.22 MB algorithmic) + 26.01 MB written (the
+# k_attn_fp8_fwd: 80.53 MB read (Q8 + K8 + V8 = 80.22 MB algorithmic) + 26.75 MB written (the
 # cut pairs' partial results and part of the bf16 output; the rest of the output is still in
 # L2 when the kernel ends).  The combine kernel that follows reads the partials back.
 # Re-capture when the kernel changes.
