@@ -257,6 +257,15 @@ QATTN_API const char* qattn_status_str(qattn_status status);
 QATTN_API void qattn_debug_set_wait_timeout_ns(uint64_t ns);
 QATTN_API void qattn_debug_inject_missing_q(int enable);
 
+/* Host-only view of the persistent schedule qattn_forward_ws runs for a dense (B, H, L, D) on a
+ * GPU with num_sms SMs (no device needed): plan[0..5] = pairs of Q tiles per head, key steps
+ * per pair, CTAs, whole pairs per CTA, tail pairs, tail key steps per CTA (== key steps per pair
+ * when no pair is cut); *workspace_bytes = qattn_forward_workspace_bytes on such a GPU.  CTA c
+ * runs pairs c, c + CTAs, ... (the whole ones), then tail key steps [c * tail_w, (c + 1) * tail_w)
+ * of the tail pairs laid end to end.  QATTN_ERR_INVALID_ARG for a shape the forward rejects. */
+QATTN_API qattn_status qattn_debug_attention_plan(int B, int H, int L, int D, int num_sms,
+                                                  int* plan, size_t* workspace_bytes);
+
 #ifdef __cplusplus
 }
 #endif

@@ -26,6 +26,7 @@ EXPORTS = (
     "qattn_status_str",
     "qattn_forward_workspace_bytes",
     "qattn_debug_set_wait_timeout_ns", "qattn_debug_inject_missing_q",
+    "qattn_debug_attention_plan",
 )
 _RETURNS_STATUS = EXPORTS[:13]
 FUSED_WORKSPACE_BYTES = 256     # QATTN_FUSED_WORKSPACE_BYTES
@@ -84,6 +85,9 @@ def load() -> ctypes.CDLL:
     lib.qattn_debug_set_wait_timeout_ns.restype = None
     lib.qattn_debug_inject_missing_q.argtypes = [I]
     lib.qattn_debug_inject_missing_q.restype = None
+    lib.qattn_debug_attention_plan.argtypes = [I, I, I, I, I, ctypes.POINTER(I),
+                                              ctypes.POINTER(S)]
+    lib.qattn_debug_attention_plan.restype = I
     for name in _RETURNS_STATUS:
         getattr(lib, name).restype = I
     _lib = lib
@@ -310,3 +314,13 @@ def debug_set_wait_timeout_ns(ns: int):
 
 def debug_inject_missing_q(enable: bool):
     load().qattn_debug_inject_missing_q(1 if enable else 0)
+
+
+def debug_attention_plan(B: int, H: int, L: int, D: int, num_sms: int) -> dict:
+    """The persistent schedule of a dense forward on a GPU with num_sms SMs (host only)."""
+    plan = (ctypes.c_int * 6)()
+    nbytes = ctypes.c_size_t(0)
+    _check(load().qattn_debug_attention_plan(int(B), int(H), int(L), int(D), int(num_sms), plan,
+                                             ctypes.byref(nbytes)), "qattn_debug_attention_plan")
+    keys = ("pairs_per_head", "nkv", "ctas", "whole", "tail_pairs", "tail_w")
+    return dict(zip(keys, list(plan)), workspace_bytes=int(nbytes.value))

@@ -342,4 +342,20 @@ void qattn_debug_set_wait_timeout_ns(uint64_t ns) {
 
 void qattn_debug_inject_missing_q(int enable) { g_inject_missing_q = enable ? 1 : 0; }
 
+qattn_status qattn_debug_attention_plan(int B, int H, int L, int D, int num_sms, int* plan,
+                                        size_t* workspace_bytes) {
+  if (B < 1 || H < 1 || L < 1 || (D != 64 && D != 128) || num_sms < 1 || !plan ||
+      !workspace_bytes)
+    return QATTN_ERR_INVALID_ARG;
+  const qattn::AttnSplitPlan p = qattn::plan_attention_split(B, H, L, D, num_sms);
+  plan[0] = p.pairs_per_head;
+  plan[1] = p.nkv;
+  plan[2] = p.ctas;
+  plan[3] = p.whole;
+  plan[4] = p.tail_pairs;
+  plan[5] = p.tail_w;
+  *workspace_bytes = p.bytes;
+  return QATTN_OK;
+}
+
 }  // extern "C"
