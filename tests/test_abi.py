@@ -114,3 +114,25 @@ def test_host_side_argument_errors():
     vl = lib.qattn_forward_varlen
     assert vl(FAKE, FAKE, FAKE, FAKE, None, 2, 8, 16, 1, 64, ctypes.byref(sc), 0.1, 1, s0) == _lib.ERR_INVALID_ARG
     assert vl(FAKE, FAKE, FAKE, FAKE, FAKE, 2, 32, 16, 1, 64, ctypes.byref(sc), 0.1, 1, s0) == _lib.ERR_INVALID_ARG
+
+
+def test_gemm_argument_errors():
+    """qattn_gemm_fp8 refuses on the host, before any launch: null or misaligned buffers, K not
+    a multiple of the 128-byte K block, N not a multiple of the 32-column epilogue chunk."""
+    lib = _lib.load()
+    g = lib.qattn_gemm_fp8
+    s0 = ctypes.c_void_p(0)
+    ok = (FAKE, FAKE, FAKE, 256, 256, 256, FAKE, FAKE, s0)
+
+    def call(**kw):
+        a = list(ok)
+        for i, name in enumerate(("a8", "b8", "y", "M", "N", "K", "s_a", "s_b")):
+            if name in kw:
+                a[i] = kw[name]
+        return g(*a)
+
+    for kw in ({"a8": None}, {"b8": None}, {"y": None}, {"s_a": None}, {"s_b": None},
+               {"a8": MISALIGNED}, {"b8": MISALIGNED}, {"y": MISALIGNED},
+               {"s_a": ctypes.c_void_p(0x10002)}, {"M": 0}, {"N": 16}, {"N": 48}, {"K": 64},
+               {"K": 200}):
+        assert call(**kw) == _lib.ERR_INVALID_ARG, kw
