@@ -249,6 +249,11 @@ QATTN_API qattn_status qattn_get_error(qattn_stream_t stream);
 /* Human-readable name of a status code (static storage). */
 QATTN_API const char* qattn_status_str(qattn_status status);
 
+/* The CUDA runtime error (a cudaError_t value) behind the last QATTN_ERR_CUDA that a call of
+ * this library returned on the calling host thread, or 0 if none has.  Argument checks and
+ * device error words do not change it.  Lets a caller report which CUDA call failed. */
+QATTN_API int qattn_last_cuda_error(void);
+
 /* Test hooks, not part of the method.  qattn_debug_set_wait_timeout_ns sets the limit after
  * which a wait inside the attention kernel gives up (default 2 s; 0 restores the default).
  * qattn_debug_inject_missing_q(1) makes the next attention launches never load Q, so every

@@ -23,7 +23,7 @@ EXPORTS = (
     "qattn_forward_varlen", "qattn_get_error", "qattn_calibrate_quantize_fp8",
     "qattn_calibrate_quantize_fp4_block", "qattn_calibrate_quantize_fp8_noalloc",
     "qattn_calibrate_quantize_qkv", "qattn_quantize_qkv", "qattn_forward_ws", "qattn_gemm_fp8",
-    "qattn_status_str",
+    "qattn_status_str", "qattn_last_cuda_error",
     "qattn_forward_workspace_bytes",
     "qattn_debug_set_wait_timeout_ns", "qattn_debug_inject_missing_q",
     "qattn_debug_attention_plan",
@@ -35,7 +35,10 @@ FUSED_WORKSPACE_BYTES = 256     # QATTN_FUSED_WORKSPACE_BYTES
 class QattnError(RuntimeError):
     def __init__(self, status: int, what: str):
         self.status = status
-        super().__init__(f"{what}: {status_str(status)} ({status})")
+        msg = f"{what}: {status_str(status)} ({status})"
+        if status == ERR_CUDA:
+            msg += f", cudaError_t {load().qattn_last_cuda_error()}"
+        super().__init__(msg)
 
 
 class QuantIO(ctypes.Structure):
@@ -81,6 +84,8 @@ def load() -> ctypes.CDLL:
     lib.qattn_get_error.argtypes = [P]
     lib.qattn_status_str.argtypes = [I]
     lib.qattn_status_str.restype = ctypes.c_char_p
+    lib.qattn_last_cuda_error.argtypes = []
+    lib.qattn_last_cuda_error.restype = I
     lib.qattn_debug_set_wait_timeout_ns.argtypes = [ctypes.c_uint64]
     lib.qattn_debug_set_wait_timeout_ns.restype = None
     lib.qattn_debug_inject_missing_q.argtypes = [I]

@@ -48,6 +48,20 @@ struct AttnSplitPlan {
 };
 AttnSplitPlan plan_attention_split(int B, int H, int L, int D, int num_sms);
 
+// Units of the persistent dense grid on the current device: SMs for D = 64 (one-SM kernel),
+// resident pair clusters for D = 128 (pair kernel); and the plan the launch uses for them.
+int attention_pair_units(int num_sms);
+AttnSplitPlan attention_plan(int B, int H, int L, int D, int num_sms);
+
+// The D = 128 pair kernel (attn_pair.cu): dense with `plan` (workspace may be null when the plan
+// cuts no pair), or varlen with plan == nullptr.
+cudaError_t launch_attention_pair(const uint8_t* q8, const uint8_t* k8, const uint8_t* v8, void* out,
+                                  int H, int L, const int* cu_seqlens, int nseq, int max_seqlen,
+                                  int rows_per_slab, int slabs, const float* s_q, const float* s_k,
+                                  const float* s_v, float sm_scale, int* err, uint64_t timeout_ns,
+                                  int inject_missing_q, const AttnSplitPlan* plan, void* workspace,
+                                  cudaStream_t stream);
+
 // workspace may be null (no split); it is used only when workspace_bytes covers the plan.
 cudaError_t launch_attention(const uint8_t* q8, const uint8_t* k8, const uint8_t* v8, void* out,
                              int B, int H, int L, int D, const int* cu_seqlens, int nseq,

@@ -25,10 +25,20 @@ DeviceInfo g_dev[kMaxDevices];
 uint64_t g_timeout_ns = kDefaultTimeoutNs;
 int g_inject_missing_q = 0;
 
+thread_local int t_last_cuda_error = 0;   // qattn_last_cuda_error: per calling host thread
+
+qattn_status from_cuda(cudaError_t e) {
+  if (e == cudaSuccess) return QATTN_OK;
+  t_last_cuda_error = static_cast<int>(e);
+  return QATTN_ERR_CUDA;
+}
+
 // Per-device setup on first use: capability check, SM count, address of the error word.
 qattn_status device_info(DeviceInfo** out) {
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return QATTN_ERR_CUDA;
+  const cudaError_t ge = cudaGetDevice(&dev);
+  if (ge != cudaSuccess) return from_cuda(ge);
+  if (dev < 0 || dev >= kMaxDevices) return QATTN_ERR_CUDA;
   DeviceInfo& d = g_dev[dev];
   if (!d.ready) {
     int major = 0, minor = 0, sms = 0;
@@ -52,7 +62,6 @@ qattn_status device_info(DeviceInfo** out) {
 
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
-qattn_status from_cuda(cudaError_t e) { return e == cudaSuccess ? QATTN_OK : QATTN_ERR_CUDA; }
 
 qattn_status check_attention_common(const uint8_t* q8, const uint8_t* k8, const uint8_t* v8,
                                     const void* out, int H, int D, const qattn_scales* sc,
@@ -258,7 +267,7 @@ qattn_status qattn_forward_ws(const uint8_t* q8, const uint8_t* k8, const uint8_
   st = device_info(&d);
   if (st != QATTN_OK) return st;
   if (workspace_dev != nullptr &&
-      workspace_bytes < qattn::plan_attention_split(B, H, L, D, d->num_sms).bytes)
+      workspace_bytes < qattn::attention_plan(B, H, L, D, d->num_sms).bytes)
     return QATTN_ERR_INVALID_ARG;
   return from_cuda(qattn::launch_attention(q8, k8, v8, out_bf16, B, H, L, D, nullptr, 0, L, L,
                                            scales->s_q, scales->s_k, scales->s_v, sm_scale,
@@ -279,7 +288,7 @@ size_t qattn_forward_workspace_bytes(int B, int H, int L, int D) {
   if (B < 1 || H < 1 || L < 1 || (D != 64 && D != 128)) return 0;
   DeviceInfo* d = nullptr;
   if (device_info(&d) != QATTN_OK) return 0;
-  return qattn::plan_attention_split(B, H, L, D, d->num_sms).bytes;
+  return qattn::attention_plan(B, H, L, D, d->num_sms).bytes;
 }
 
 qattn_status qattn_forward_varlen(const uint8_t* q8, const uint8_t* k8, const uint8_t* v8,
@@ -323,6 +332,8 @@ qattn_status qattn_get_error(qattn_stream_t stream) {
     default: return QATTN_ERR_CUDA;
   }
 }
+
+int qattn_last_cuda_error(void) { return t_last_cuda_error; }
 
 const char* qattn_status_str(qattn_status status) {
   switch (status) {
