@@ -33,15 +33,28 @@ HBM_FALLBACK_GBS = 6650.0
 BF16_FALLBACK_TFLOPS = 1590.0
 FP8_PER_BF16 = 2.0          # nominal dense FP8 / BF16 tensor throughput ratio on B200
 L2_FLUSH_BYTES = 256 << 20
-# DRAM bytes (read + write) of one launch of the attention kernel, from ncu on the current kernel:
+# DRAM bytes (read + write) of one launch of the attention kernel at L=8704 (B=1, H=24, D=128),
+# from ncu on the current kernel:
 #   ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum --clock-control none \
 #       -k regex:k_attn_fp8 -s 3 -c 1 python bench.py --steps 1 --warmup 3 --no-cpu-baseline --no-e2e
-# k_attn_fp8_fwd: 80.53 MB read (Q8 + K8 + V8 = 80.22 MB algorithmic) + 26.75 MB written (the
-# cut pairs' partial results and part of the bf16 output; the rest of the output is still in
-# L2 when the kernel ends).  The combine kernel that follows reads the partials back.
-# Re-capture when the kernel changes.
-ATTN_TRAFFIC_BYTES = {(8704, 24, 128): 80.53e6 + 26.75e6}
+# None until captured for this kernel (re-capture whenever the kernel changes).  Other shapes of
+# the same kernel: scaled by their algorithmic bytes (Q8 + K8 + V8 + bf16 output), and so marked.
+ATTN_TRAFFIC_L8704 = None
 ATTN_TRAFFIC_SOURCE = "ncu dram__bytes_read.sum + dram__bytes_write.sum, one launch, L=8704"
+ATTN_KERNEL = {128: "k_attn_fp8_pair (cluster of two CTAs per pair of Q tiles)", 64: "k_attn_fp8_fwd<64>"}
+
+
+def attn_traffic(w):
+    """(bytes per launch, how it was obtained) for the attention kernel on workload w."""
+    if ATTN_TRAFFIC_L8704 is None or w.D != 128:
+        return None, "not captured for this kernel"
+    tokens = sum(w.seqlens) if w.varlen else w.B * w.L
+    algo = tokens * w.H * w.D * (3 + 2)            # Q8, K8, V8 read; bf16 output written
+    algo_ref = 8704 * 24 * 128 * (3 + 2)
+    if not w.varlen and (w.L, w.H, w.B) == (8704, 24, 1):
+        return ATTN_TRAFFIC_L8704, ATTN_TRAFFIC_SOURCE
+    return ATTN_TRAFFIC_L8704 * algo / algo_ref, (ATTN_TRAFFIC_SOURCE +
+                                                  ", scaled by this workload's algorithmic bytes")
 
 
 def load_peaks():
@@ -233,11 +246,116 @@ def run_gpu(args):
     # our kernels per step: the Q, K, V calibrate+quantize launch, the attention launch, and the
     # combine launch when tail pairs are cut
     launches = 2 + (1 if path.attn_workspace is not None else 0)
-    report(args, w, (q, k, v), rank, world, ms, attn, quant, e2e_ms, clocks, launches)
+    extra = {}
+    if not args.no_extras:
+        # the quantize launch with static scales (the amax just calibrated, as post-training
+        # calibration would give): one streaming pass, no grid barrier
+        if not args.static_scales:
+            extra["quant_static_ms"] = time_quantize(w, qd, kd, vd, path.amax.tolist(), flush,
+                                                     min(args.steps, 100))
+        # FP4 mode on the same L=8704 shape, timed the same way in the same run
+        if w.name == "edit_fp8" and world == 1:
+            extra["fp4"] = run_mode_extra(workloads.WORKLOADS["edit_fp4"], flush, min(args.steps, 100),
+                                          args.warmup)
+        extra["fp8_measured"] = measured_fp8_rates(flush)
+    report(args, w, (q, k, v), rank, world, ms, attn, quant, e2e_ms, clocks, launches, extra)
     barrier(world)
     del path
     if world > 1:
         torch.distributed.destroy_process_group()
+
+
+def time_quantize(w, qd, kd, vd, amax, flush, steps):
+    """Mean ms of the Q, K, V quantize launch with the given (static) amax values."""
+    import precision_quantized_attention_b200 as qa
+    sp = qa.QuantizedAttention(w.shape, w.mode, cu_seqlens=w.cu_seqlens, sm_scale=w.sm_scale,
+                               static_amax=amax)
+    for _ in range(3):
+        sp.quantize(qd, kd, vd)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(steps)]
+    for e0, e1 in ev:
+        flush()
+        e0.record()
+        sp.quantize(qd, kd, vd)
+        e1.record()
+    torch.cuda.synchronize()
+    if qa.get_error() != 0:
+        raise RuntimeError("device error in the static-scale quantize timing")
+    return sum(e0.elapsed_time(e1) for e0, e1 in ev) / len(ev)
+
+
+def run_mode_extra(w, flush, steps, warmup):
+    """Step, attention and quantize (calibrated and static) times of workload w, timed like the
+    main line (inputs resident, L2 flushed between steps, CUDA events)."""
+    import precision_quantized_attention_b200 as qa
+    q, k, v = workloads.make_qkv(w)
+    qd, kd, vd = (t.cuda() for t in (q, k, v))
+    path = qa.QuantizedAttention(w.shape, w.mode, cu_seqlens=w.cu_seqlens, sm_scale=w.sm_scale)
+    for _ in range(warmup):
+        path.quantize(qd, kd, vd)
+        path.attend()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+    torch.cuda.synchronize()
+    for e in ev:
+        flush()
+        e[0].record()
+        path.quantize(qd, kd, vd)
+        e[1].record()
+        path.attend()
+        e[2].record()
+    torch.cuda.synchronize()
+    if qa.get_error() != 0:
+        raise RuntimeError(f"device error in the {w.name} timing")
+    step = sum(e[0].elapsed_time(e[2]) for e in ev) / steps
+    attn = sum(e[1].elapsed_time(e[2]) for e in ev) / steps
+    quant = sum(e[0].elapsed_time(e[1]) for e in ev) / steps
+    quant_static = time_quantize(w, qd, kd, vd, path.amax.tolist(), flush, steps)
+    return {"workload": w.name, "steps": steps, "step_ms": step, "attn_ms": attn,
+            "quant_ms": quant, "quant_static_ms": quant_static, "flops": w.flops,
+            "numel": q.numel(), "w": w}
+
+
+def measured_fp8_rates(flush, reps=5):
+    """Measured dense FP8 rates on this GPU beside the derived peak: this library's FP8 GEMM
+    and torch._scaled_mm (cuBLASLt) on the block's QKV projection shape, L2 flushed."""
+    import precision_quantized_attention_b200 as qa
+    M, N, K = GEMM_SHAPES["qkv_proj"]
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(3)
+    a8 = torch.randint(0, 256, (M, K), dtype=torch.uint8, device="cuda", generator=gen)
+    b8 = torch.randint(0, 256, (N, K), dtype=torch.uint8, device="cuda", generator=gen)
+    a8 = torch.where((a8 & 0x7F) == 0x7F, a8 ^ 1, a8)
+    b8 = torch.where((b8 & 0x7F) == 0x7F, b8 ^ 1, b8)
+    sa, sb = torch.tensor([0.01], device="cuda"), torch.tensor([0.002], device="cuda")
+    y = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
+    out = {"shape": f"{M}x{N}x{K}"}
+
+    def rate(fn):
+        for _ in range(2):
+            fn()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(reps)]
+        for e0, e1 in ev:
+            flush()
+            e0.record()
+            fn()
+            e1.record()
+        torch.cuda.synchronize()
+        ms = min(e0.elapsed_time(e1) for e0, e1 in ev)
+        return 2.0 * M * N * K / (ms * 1e-3) / 1e12
+
+    out["k_gemm_fp8_pair_tflops"] = rate(lambda: qa.gemm_fp8(a8, b8, y, sa, sb))
+    if qa.get_error() != 0:
+        raise RuntimeError("device error in the FP8 GEMM rate")
+    try:
+        af, bf = a8.view(torch.float8_e4m3fn), b8.view(torch.float8_e4m3fn)
+        out["torch_scaled_mm_tflops"] = rate(
+            lambda: torch._scaled_mm(af, bf.t(), scale_a=sa, scale_b=sb, out_dtype=torch.bfloat16))
+    except Exception as e:                       # not every torch build has it
+        out["torch_scaled_mm_tflops"] = None
+        out["torch_scaled_mm_error"] = type(e).__name__
+    return out
 
 
 def e2e_time(args, w, q, k, v, qd, kd, vd, step, flush, stream, world):
@@ -324,18 +442,55 @@ def bench_config(w, world, static_scales=False):
                   "before the step starts"}
 
 
-def report(args, w, qkv, rank, world, ms, attn, quant, e2e_ms, clocks, launches):
+def quantize_bytes(w, numel):
+    """Algorithmic bytes of the Q, K, V quantize launch: bf16 read once (2 B), E4M3 codes
+    written (1 B); FP4 mode also writes the packed E2M1 codes (0.5 B) and one block-scale byte
+    per 16 elements."""
+    per_elem = 3.0 if w.mode == "fp8" else 3.0 + 0.5 + 1.0 / 16
+    return 3 * numel * per_elem
+
+
+def report(args, w, qkv, rank, world, ms, attn, quant, e2e_ms, clocks, launches, extra=None):
     q = qkv[0]
     hbm_gbs, bf16_tf, peak_kind = load_peaks()
     fp8_peak = bf16_tf * FP8_PER_BF16
     flops = w.flops
     achieved_tf = flops / (attn * 1e-3) / 1e12
+    extra = extra or {}
     in_bytes = 3 * q.numel() * 2
-    # fused calibrate+quantize: bf16 read once (2 B), E4M3 codes written (1 B); FP4 mode also
-    # writes the packed E2M1 codes (0.5 B) and one block-scale byte per 16 elements
-    per_elem = 3.0 if w.mode == "fp8" else 3.0 + 0.5 + 1.0 / 16
-    quant_bytes = 3 * q.numel() * per_elem
+    quant_bytes = quantize_bytes(w, q.numel())
+    traffic, traffic_src = attn_traffic(w)
     clock = clocks.summary()
+    quantize = {"ms": quant, "algorithmic_bytes": quant_bytes,
+                "gbs": quant_bytes / (quant * 1e-3) / 1e9,
+                "frac_hbm": quant_bytes / (quant * 1e-3) / 1e9 / hbm_gbs,
+                "hbm_peak_gbs": hbm_gbs, "launches": 1,
+                "path": ("static scales (qattn_quantize_qkv, one pass)" if args.static_scales
+                         else "calibrated every step (qattn_calibrate_quantize_qkv: amax, grid "
+                              "barrier, quantize)")}
+    if "quant_static_ms" in extra:
+        qs = extra["quant_static_ms"]
+        quantize["static"] = {"ms": qs, "gbs": quant_bytes / (qs * 1e-3) / 1e9,
+                              "frac_hbm": quant_bytes / (qs * 1e-3) / 1e9 / hbm_gbs,
+                              "path": "static scales (qattn_quantize_qkv, one pass), the amax "
+                                      "calibrated in the timed steps"}
+    fp4 = None
+    if "fp4" in extra:
+        x = extra["fp4"]
+        w4 = x.pop("w")
+        qb4 = quantize_bytes(w4, x["numel"])
+        t4, t4_src = attn_traffic(w4)
+        a_tf = x["flops"] / (x["attn_ms"] * 1e-3) / 1e12
+        fp4 = {"workload": bench_config(w4, world)["workload"], "steps": x["steps"],
+               "ms_per_step": x["step_ms"], "value": x["flops"] / (x["step_ms"] * 1e-3) / 1e12,
+               "roofline": {"bound": "tensor", "achieved": a_tf, "peak": fp8_peak,
+                            "unit": "TFLOP/s", "frac": a_tf / fp8_peak, "traffic": t4,
+                            "traffic_source": t4_src, "kernel_ms": x["attn_ms"],
+                            "kernel": ATTN_KERNEL[w4.D]},
+               "quantize": {"ms": x["quant_ms"], "algorithmic_bytes": qb4,
+                            "frac_hbm": qb4 / (x["quant_ms"] * 1e-3) / 1e9 / hbm_gbs,
+                            "static": {"ms": x["quant_static_ms"],
+                                       "frac_hbm": qb4 / (x["quant_static_ms"] * 1e-3) / 1e9 / hbm_gbs}}}
     result = {
         "metric": "quantized attention TFLOP/s @L=8704,H=24,D=128 and % of B200 FP8 peak",
         "value": world * flops / (ms * 1e-3) / 1e12,
@@ -352,16 +507,14 @@ def report(args, w, qkv, rank, world, ms, attn, quant, e2e_ms, clocks, launches)
         "config": bench_config(w, world, args.static_scales),
         "roofline": {"bound": "tensor", "achieved": achieved_tf, "peak": fp8_peak,
                      "unit": "TFLOP/s", "frac": achieved_tf / fp8_peak,
-                     "traffic": ATTN_TRAFFIC_BYTES.get((w.L, w.H, w.D)),
-                     "traffic_source": ATTN_TRAFFIC_SOURCE,
-                     "kernel": f"k_attn_fp8_fwd<{w.D}>",
+                     "traffic": traffic, "traffic_source": traffic_src,
+                     "kernel": ATTN_KERNEL[w.D],
                      "peak_source": f"{peak_kind} bf16 burst {bf16_tf} TFLOP/s x {FP8_PER_BF16} "
                                     "(nominal FP8/BF16 ratio)",
+                     "fp8_measured_tflops": extra.get("fp8_measured"),
                      "kernel_ms": attn},
-        "quantize": {"ms": quant, "algorithmic_bytes": quant_bytes,
-                     "gbs": quant_bytes / (quant * 1e-3) / 1e9,
-                     "frac_hbm": quant_bytes / (quant * 1e-3) / 1e9 / hbm_gbs,
-                     "hbm_peak_gbs": hbm_gbs, "launches": 1},
+        "quantize": quantize,
+        "fp4": fp4,
         "e2e": {"value": world * flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
                 "ms_per_step": e2e_ms, "h2d_bytes_per_step": in_bytes,
                 "d2h_bytes_per_step": q.numel() * 2,
@@ -539,6 +692,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--static-scales", action="store_true",
                     help="quantize with amax values calibrated once before timing (one pass)")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="skip the static-scale quantize, FP4-mode and measured FP8 rate timings")
     ap.add_argument("--gemm", action="store_true",
                     help="time the FP8 GEMM of the transformer block's linear layers instead")
     args = ap.parse_args()

@@ -262,6 +262,18 @@ QATTN_API int qattn_last_cuda_error(void);
 QATTN_API void qattn_debug_set_wait_timeout_ns(uint64_t ns);
 QATTN_API void qattn_debug_inject_missing_q(int enable);
 
+/* Test hook, not part of the method: with enable != 0 the next D = 128 attention launches copy,
+ * for query row `row` (row index within the slab's rows: the token index for dense launches,
+ * the packed token index for varlen) of slab `slab` (b * H + h; the head for varlen), the E4M3
+ * codes of P of every key step s into codes_dev[s * 128 + key] (key within the step) and the
+ * step's integer tile maximum (base-2 units; P(s) = e4m3(2^(S' - max) * 448)) into maxima_dev[s].
+ * codes_dev: device, 16-byte aligned, ceil(L / 128) * 128 bytes; maxima_dev: device int32,
+ * ceil(L / 128) entries; both caller-owned and written only by launches made while enabled.
+ * enable = 0 turns it off (the pointers are forgotten); with it off nothing of the launches
+ * changes.  QATTN_ERR_INVALID_ARG for null or misaligned buffers or negative indices. */
+QATTN_API qattn_status qattn_debug_capture_p_row(int enable, int slab, int row, uint8_t* codes_dev,
+                                                 int* maxima_dev);
+
 /* Host-only view of the persistent schedule qattn_forward_ws runs for a dense (B, H, L, D) on a
  * GPU with num_sms SMs (no device needed): plan[0..5] = pairs of Q tiles per head, key steps
  * per pair, CTAs, whole pairs per CTA, tail pairs, tail key steps per CTA (== key steps per pair

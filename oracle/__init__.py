@@ -82,6 +82,9 @@ def _load():
             lib.orc_attention_values.restype = i32
             lib.orc_attention_e4m3.argtypes = att
             lib.orc_attention_e4m3.restype = i32
+            lib.orc_p_row_detail.argtypes = [P, P, i32, i32, i64, i32, P, i32, f64, f64, f64, i64,
+                                             P, P, P, P, P, P, P]
+            lib.orc_p_row_detail.restype = i64
             lib.orc_num_threads.argtypes = []
             lib.orc_num_threads.restype = i32
             _lib = lib
@@ -228,6 +231,32 @@ def attention_e4m3(q8, k8, v8, shape, s_q, s_k, s_v, sm_scale=None, flags=METHOD
         out = out.reshape(B, H, T, D)
         amb = amb.reshape(B, H, T, D) if with_ambiguity else None
     return (out, amb) if with_ambiguity else out
+
+
+def p_row_detail(q8, k8, shape, s_q, s_k, row, sm_scale=None, cu_seqlens=None):
+    """The method's P decisions for one query row (row = (b * H + h) * T + t) over E4M3 codes:
+    per key of its sequence the E4M3 code of p * 448, x = S' - M (base-2 score minus the integer
+    row max), the accumulation-order radius delta of S' and the codes lo, hi of
+    2^(x -+ delta) * 448 (the range of codes another FP32 summation order may give; see
+    orc_p_row_detail in the C source); and M and the FP32 row sum l of the unquantized p.
+    Returns (codes, x, delta, lo, hi, M, l)."""
+    B, H, T, D = shape
+    sm = 1.0 / np.sqrt(D) if sm_scale is None else sm_scale
+    q8, k8 = (np.ascontiguousarray(a, dtype=np.uint8).reshape(-1) for a in (q8, k8))
+    cu = _cu(cu_seqlens, T)
+    code = np.empty(T, dtype=np.uint8)
+    x = np.empty(T, dtype=np.float64)
+    delta = np.empty(T, dtype=np.float64)
+    lo = np.empty(T, dtype=np.uint8)
+    hi = np.empty(T, dtype=np.uint8)
+    M = ctypes.c_double()
+    l = ctypes.c_double()
+    n = _load().orc_p_row_detail(_ptr(q8), _ptr(k8), B, H, T, D, _ptr(cu), cu.size - 1, float(s_q),
+                                 float(s_k), sm, int(row), _ptr(code), _ptr(x), _ptr(delta),
+                                 _ptr(lo), _ptr(hi), ctypes.byref(M), ctypes.byref(l))
+    if n < 0:
+        raise ValueError(f"orc_p_row_detail failed with status {n}")
+    return code[:n], x[:n], delta[:n], lo[:n], hi[:n], M.value, l.value
 
 
 def attention_fp64(q, k, v, sm_scale=None, cu_seqlens=None) -> np.ndarray:

@@ -405,6 +405,64 @@ int orc_attention_e4m3(const uint8_t *q8, const uint8_t *k8, const uint8_t *v8, 
     return rc;
 }
 
+/* One query row's P decisions, for comparing the P codes of an implementation key by key
+ * (flags ORC_FP32 | ORC_QUANT_P, the method's steps as in attend_row).  row = (b * H + h) * T + t.
+ * For each key j of the row's sequence: code[j] = e4m3(fl32(2^fl32(S'_j - M)) * 448), x[j] = S'_j - M
+ * (S'_j the FP32 base-2 score), delta[j] = the accumulation-order radius of S'_j defined above
+ * (ORC_AMB_KAPPA), and lo[j], hi[j] = the E4M3 codes of 2^(x[j] - delta[j]) * 448 and
+ * 2^(x[j] + delta[j]) * 448: a method with another FP32 summation order may produce any code from
+ * lo[j] to hi[j] for key j.  *M_out = M, *l_out = the FP32 row sum of the unquantized p.
+ * Returns the number of keys, or a negative status. */
+int64_t orc_p_row_detail(const uint8_t *q8, const uint8_t *k8, int B, int H, int64_t T, int D,
+                         const int64_t *cu, int nseq, double s_q, double s_k, double sm_scale,
+                         int64_t row, uint8_t *code, double *x, double *delta, uint8_t *lo,
+                         uint8_t *hi, double *M_out, double *l_out) {
+    if (B < 1 || H < 1 || T < 1 || D < 1 || nseq < 1 || row < 0 || row >= (int64_t)B * H * T)
+        return ORC_ERR_INVALID;
+    if (cu[0] != 0 || cu[nseq] != T) return ORC_ERR_INVALID;
+    const int64_t bh = row / T, t = row % T;
+    int s = 0;
+    while (!(cu[s] <= t && t < cu[s + 1])) ++s;
+    const int64_t nkeys = cu[s + 1] - cu[s], base = bh * T + cu[s];
+    const double log2e = 1.4426950408889634;
+    const double c64 = s_q * s_k * sm_scale * log2e;
+    const float c32 = (float)c64;
+    double *S = (double *)malloc(sizeof(double) * (size_t)nkeys);
+    double *W = (double *)malloc(sizeof(double) * (size_t)nkeys);
+    if (!S || !W) { free(S); free(W); return ORC_ERR_INVALID; }
+    const uint8_t *q = q8 + row * D;
+    double smax = -INFINITY;
+    for (int64_t j = 0; j < nkeys; ++j) {
+        const uint8_t *k = k8 + (base + j) * D;
+        double acc = 0.0, absacc = 0.0;
+        for (int d = 0; d < D; ++d) {
+            const double prod = (double)orc_e4m3_to_float(q[d]) * (double)orc_e4m3_to_float(k[d]);
+            acc += prod;
+            absacc += fabs(prod);
+        }
+        S[j] = (double)(float)((float)acc * c32);
+        W[j] = absacc;
+        if (S[j] > smax) smax = S[j];
+    }
+    const double M = ceil(smax);
+    double lsum = 0.0;
+    for (int64_t j = 0; j < nkeys; ++j) {
+        const double p = (double)(float)exp2((double)(float)(S[j] - M));
+        lsum += p;
+        code[j] = orc_e4m3_from_float((float)p * 448.0f);
+        x[j] = S[j] - M;
+        delta[j] = ORC_AMB_KAPPA * ldexp(W[j] * c64, -24) + 4.0 * ldexp(fabs(S[j]) + fabs(M) + 1.0, -23) +
+                   ldexp(1.0, -20);
+        lo[j] = orc_e4m3_from_float((float)(exp2(x[j] - delta[j]) * 448.0));
+        hi[j] = orc_e4m3_from_float((float)(exp2(x[j] + delta[j]) * 448.0));
+    }
+    *M_out = M;
+    *l_out = (double)(float)lsum;
+    free(S);
+    free(W);
+    return nkeys;
+}
+
 int orc_num_threads(void) {
 #ifdef _OPENMP
     return omp_get_max_threads();

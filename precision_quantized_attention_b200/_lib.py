@@ -25,7 +25,7 @@ EXPORTS = (
     "qattn_calibrate_quantize_qkv", "qattn_quantize_qkv", "qattn_forward_ws", "qattn_gemm_fp8",
     "qattn_status_str", "qattn_last_cuda_error",
     "qattn_forward_workspace_bytes",
-    "qattn_debug_set_wait_timeout_ns", "qattn_debug_inject_missing_q",
+    "qattn_debug_set_wait_timeout_ns", "qattn_debug_inject_missing_q", "qattn_debug_capture_p_row",
     "qattn_debug_attention_plan",
 )
 _RETURNS_STATUS = EXPORTS[:13]
@@ -90,6 +90,8 @@ def load() -> ctypes.CDLL:
     lib.qattn_debug_set_wait_timeout_ns.restype = None
     lib.qattn_debug_inject_missing_q.argtypes = [I]
     lib.qattn_debug_inject_missing_q.restype = None
+    lib.qattn_debug_capture_p_row.argtypes = [I, I, I, P, P]
+    lib.qattn_debug_capture_p_row.restype = I
     lib.qattn_debug_attention_plan.argtypes = [I, I, I, I, I, ctypes.POINTER(I),
                                               ctypes.POINTER(S)]
     lib.qattn_debug_attention_plan.restype = I
@@ -319,6 +321,18 @@ def debug_set_wait_timeout_ns(ns: int):
 
 def debug_inject_missing_q(enable: bool):
     load().qattn_debug_inject_missing_q(1 if enable else 0)
+
+
+def debug_capture_p_row(enable: bool, slab: int = 0, row: int = 0, codes: torch.Tensor = None,
+                        maxima: torch.Tensor = None):
+    """Test hook: the next D = 128 attention launches copy row `row` of slab `slab`'s P codes
+    (uint8 [steps * 128]) and tile maxima (int32 [steps]) into the given device tensors."""
+    if not enable:
+        _check(load().qattn_debug_capture_p_row(0, 0, 0, None, None), "qattn_debug_capture_p_row")
+        return
+    assert codes.is_cuda and codes.dtype == torch.uint8 and maxima.is_cuda and maxima.dtype == torch.int32
+    _check(load().qattn_debug_capture_p_row(1, slab, row, codes.data_ptr(), maxima.data_ptr()),
+           "qattn_debug_capture_p_row")
 
 
 def debug_attention_plan(B: int, H: int, L: int, D: int, num_sms: int) -> dict:

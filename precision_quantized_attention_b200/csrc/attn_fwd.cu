@@ -54,6 +54,7 @@
 #include <cuda_bf16.h>
 #include <cstdint>
 
+#include "device_once.h"
 #include "launch.h"
 #include "sm100_ptx.cuh"
 #include "softmax_sm100.cuh"
@@ -636,15 +637,14 @@ using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t
                                    CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
 static EncodeTiledFn get_encode_fn() {
-  static EncodeTiledFn fn = nullptr;
-  if (!fn) {
+  static const EncodeTiledFn fn = [] {          // initialised once, thread-safe
     void* p = nullptr;
     cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
-            cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(p);
-  }
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return static_cast<EncodeTiledFn>(nullptr);
+    return reinterpret_cast<EncodeTiledFn>(p);
+  }();
   return fn;
 }
 
@@ -673,15 +673,13 @@ static cudaError_t launch_attn_d(const void* q8, const void* k8, const void* v8,
   if (!make_map(&mq, q8, D, rows_per_slab, slabs) || !make_map(&mk, k8, D, rows_per_slab, slabs) ||
       !make_map(&mv, v8, D, rows_per_slab, slabs))
     return cudaErrorInvalidValue;
-  static int configured_dev_mask = 0;   // bit per device id < 31
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev < 31 && !(configured_dev_mask & (1 << dev))) {
-    cudaError_t e = cudaFuncSetAttribute(k_attn_fp8_fwd<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         Smem<D>::ALLOC);
-    if (e != cudaSuccess) return e;
-    configured_dev_mask |= 1 << dev;
-  }
+  static DeviceOnce smem_attr;                  // per device and per D, set once
+  const cudaError_t ea = static_cast<cudaError_t>(smem_attr.get([] {
+    return static_cast<int>(cudaFuncSetAttribute(k_attn_fp8_fwd<D>,
+                                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                 Smem<D>::ALLOC));
+  }));
+  if (ea != cudaSuccess) return ea;
   k_attn_fp8_fwd<D><<<grid, ATTN_THREADS, Smem<D>::ALLOC, stream>>>(mq, mk, mv, a);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess || combine_ctas == 0) return e;
@@ -733,7 +731,7 @@ cudaError_t launch_attention(const uint8_t* q8, const uint8_t* k8, const uint8_t
                              int B, int H, int L, int D, const int* cu_seqlens, int nseq,
                              int max_seqlen, int total_tokens, const float* s_q, const float* s_k,
                              const float* s_v, float sm_scale, int* err, uint64_t timeout_ns,
-                             int inject_missing_q, void* workspace, size_t workspace_bytes,
+                             const DebugHooks& dbg, void* workspace, size_t workspace_bytes,
                              int num_sms, cudaStream_t stream) {
   AttnArgs a;
   const bool varlen = cu_seqlens != nullptr;
@@ -748,7 +746,7 @@ cudaError_t launch_attention(const uint8_t* q8, const uint8_t* k8, const uint8_t
   a.out = static_cast<__nv_bfloat16*>(out);
   a.err = err;
   a.timeout_ns = timeout_ns;
-  a.inject_missing_q = inject_missing_q;
+  a.inject_missing_q = dbg.inject_missing_q;
   a.part_o = nullptr;
   a.part_ml = nullptr;
   a.pairs_per_head = 0;
@@ -787,7 +785,7 @@ cudaError_t launch_attention(const uint8_t* q8, const uint8_t* k8, const uint8_t
     // pairs of SMs: the two Q tiles of a pair on the two CTAs of a cluster (attn_pair.cu)
     cudaError_t e = launch_attention_pair(q8, k8, v8, out, H, L, cu_seqlens, nseq, max_seqlen,
                                           a.rows_per_slab, slabs, s_q, s_k, s_v, sm_scale, err,
-                                          timeout_ns, inject_missing_q, varlen ? nullptr : &p,
+                                          timeout_ns, dbg, varlen ? nullptr : &p,
                                           a.part_o, stream);
     if (e != cudaSuccess || combine_ctas == 0) return e;
     k_attn_combine<128><<<combine_ctas, COMBINE_WARPS * 32, 0, stream>>>(a);

@@ -58,6 +58,7 @@
 #include <cuda_bf16.h>
 #include <cstdint>
 
+#include "device_once.h"
 #include "launch.h"
 #include "sm100_ptx.cuh"
 #include "softmax_sm100.cuh"
@@ -122,6 +123,9 @@ struct PairArgs {
   int* err;
   uint64_t timeout_ns;
   int inject_missing_q;     // fault injection for tests: the producers never load anything
+  uint8_t* dbg_p;           // test hook (see DebugHooks): P codes of one row, or nullptr
+  int* dbg_m;
+  int dbg_slab, dbg_row;
   // persistent schedule over pairs (dense), one entry per cluster: see k_attn_fp8_fwd's AttnArgs
   int pairs_per_head;
   int nkv;
@@ -212,6 +216,16 @@ struct StepCursor {
 };
 
 }  // namespace
+
+// Test hook: one row's P codes of key step `step` (word w: keys 4w..4w+3) and the step's tile
+// maximum, to the caller's buffers.
+__device__ __forceinline__ void capture_p_row(const PairArgs& args, int step, const uint32_t (&pk)[32],
+                                           float mx) {
+  uint4* dst = reinterpret_cast<uint4*>(args.dbg_p + static_cast<size_t>(step) * pairk::BLOCK_N);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+  args.dbg_m[step] = static_cast<int>(mx);
+}
 
 // Multiplies this thread's row of O (128 FP32 columns of its TMEM lane) by f, 8 columns at a
 // time.  Out of line: only a rise of the row maximum past 2^64 over M_ref takes it.
@@ -530,6 +544,9 @@ __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(168)
           for (int q = 0; q < 4; ++q)
             pk[i / 4 + q] = cvt_e4m3x2(p[4 * q], p[4 * q + 1]) | (cvt_e4m3x2(p[4 * q + 2], p[4 * q + 3]) << 16);
         }
+        if (args.dbg_p != nullptr && sg.slab == args.dbg_slab &&
+            sg.seq_start + sg.q_row0 + static_cast<int>(rank) * BLOCK_M + r == args.dbg_row)
+          capture_p_row(args, sg.kv0 + j, pk, mx);   // test hook: off unless a row is chosen
         // P(s) over the first 32 columns of the buffer (column c: keys 4c..4c+3)
         tmem_st32(tS, pk);
         // M_ref after step s - 1, published by the other warpgroup (waited on at every step so
@@ -657,25 +674,31 @@ static bool pair_map(CUtensorMap* map, const void* ptr, int rows, int slabs, int
 }
 
 // Pair clusters resident at once on the current device (one CTA per SM): the persistent grid.
+// Sets the pair kernel's dynamic-shared-memory size on the current device (once per device).
+static cudaError_t pair_smem_attribute() {
+  static DeviceOnce attr;
+  return static_cast<cudaError_t>(attr.get([] {
+    return static_cast<int>(cudaFuncSetAttribute(k_attn_fp8_pair,
+                                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                 pairk::ALLOC));
+  }));
+}
+
 int attention_pair_units(int num_sms) {
-  static int cached[64] = {0};
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return num_sms / 2;
-  if (dev >= 0 && dev < 64 && cached[dev] > 0) return cached[dev];
-  int n = 0;
-  if (cudaFuncSetAttribute(k_attn_fp8_pair, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           pairk::ALLOC) == cudaSuccess) {
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(static_cast<unsigned>(num_sms & ~1));
-    cfg.blockDim = dim3(pairk::THREADS);
-    cfg.dynamicSmemBytes = pairk::ALLOC;
-    if (cudaOccupancyMaxActiveClusters(&n, k_attn_fp8_pair, &cfg) != cudaSuccess) n = 0;
-  }
-  cudaGetLastError();
-  if (n <= 0 || n > num_sms / 2) n = num_sms / 2;
-  if (n < 1) n = 1;
-  if (dev >= 0 && dev < 64) cached[dev] = n;   // racing first calls store the same value
-  return n;
+  static DeviceOnce units;
+  return units.get([num_sms] {
+    int n = 0;
+    if (pair_smem_attribute() == cudaSuccess) {
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3(static_cast<unsigned>(num_sms & ~1));
+      cfg.blockDim = dim3(pairk::THREADS);
+      cfg.dynamicSmemBytes = pairk::ALLOC;
+      if (cudaOccupancyMaxActiveClusters(&n, k_attn_fp8_pair, &cfg) != cudaSuccess) n = 0;
+    }
+    cudaGetLastError();
+    if (n <= 0 || n > num_sms / 2) n = num_sms / 2;
+    return n < 1 ? 1 : n;
+  });
 }
 
 // Launch of the pair kernel (D = 128).  Dense: the schedule `plan` (planned for
@@ -684,7 +707,7 @@ cudaError_t launch_attention_pair(const uint8_t* q8, const uint8_t* k8, const ui
                                   int H, int L, const int* cu_seqlens, int nseq, int max_seqlen,
                                   int rows_per_slab, int slabs, const float* s_q, const float* s_k,
                                   const float* s_v, float sm_scale, int* err, uint64_t timeout_ns,
-                                  int inject_missing_q, const AttnSplitPlan* plan, void* workspace,
+                                  const DebugHooks& dbg, const AttnSplitPlan* plan, void* workspace,
                                   cudaStream_t stream) {
   using namespace pairk;
   CUtensorMap mq, mk, mv;
@@ -692,8 +715,7 @@ cudaError_t launch_attention_pair(const uint8_t* q8, const uint8_t* k8, const ui
       !pair_map(&mk, k8, rows_per_slab, slabs, D, BLOCK_N / 2) ||
       !pair_map(&mv, v8, rows_per_slab, slabs, D / 2, BLOCK_N))
     return cudaErrorInvalidValue;
-  cudaError_t e = cudaFuncSetAttribute(k_attn_fp8_pair, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       ALLOC);
+  const cudaError_t e = pair_smem_attribute();
   if (e != cudaSuccess) return e;
   PairArgs a;
   a.rows_per_slab = rows_per_slab;
@@ -707,7 +729,11 @@ cudaError_t launch_attention_pair(const uint8_t* q8, const uint8_t* k8, const ui
   a.out = static_cast<__nv_bfloat16*>(out);
   a.err = err;
   a.timeout_ns = timeout_ns;
-  a.inject_missing_q = inject_missing_q;
+  a.inject_missing_q = dbg.inject_missing_q;
+  a.dbg_p = dbg.p_codes;
+  a.dbg_m = dbg.p_maxima;
+  a.dbg_slab = dbg.p_slab;
+  a.dbg_row = dbg.p_row;
   a.pairs_per_head = plan ? plan->pairs_per_head : 0;
   a.nkv = plan ? plan->nkv : 0;
   a.ctas = plan ? plan->ctas : 0;

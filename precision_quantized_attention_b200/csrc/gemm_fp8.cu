@@ -26,6 +26,7 @@
 #include <cuda_runtime.h>
 #include <cstdint>
 
+#include "device_once.h"
 #include "launch.h"
 #include "sm100_ptx.cuh"
 
@@ -416,15 +417,14 @@ using GemmEncodeFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
 static GemmEncodeFn gemm_encode_fn() {
-  static GemmEncodeFn fn = nullptr;
-  if (!fn) {
+  static const GemmEncodeFn fn = [] {           // initialised once, thread-safe
     void* p = nullptr;
     cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
-            cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<GemmEncodeFn>(p);
-  }
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return static_cast<GemmEncodeFn>(nullptr);
+    return reinterpret_cast<GemmEncodeFn>(p);
+  }();
   return fn;
 }
 
@@ -442,33 +442,28 @@ static bool make_map_2d(CUtensorMap* map, const void* ptr, int rows, int K, int 
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// Largest number of pair clusters resident at once (one CTA per SM), per device.
-static int pair_clusters_resident(int num_sms) {
-  static int cached[32] = {0};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev < 32 && cached[dev] > 0) return cached[dev];
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(num_sms & ~1));
-  cfg.blockDim = dim3(gemm2::THREADS);
-  cfg.dynamicSmemBytes = gemm2::ALLOC;
-  int n = 0;
-  if (cudaOccupancyMaxActiveClusters(&n, k_gemm_fp8_pair, &cfg) != cudaSuccess || n <= 0) {
-    cudaGetLastError();
-    n = num_sms / 2;
-  }
-  if (dev < 32) cached[dev] = n;
-  return n;
+// Sets a kernel's dynamic-shared-memory size once per device (per call site's DeviceOnce).
+static bool set_smem_once(DeviceOnce& once, const void* fn, int bytes) {
+  return once.get([fn, bytes] {
+    return static_cast<int>(cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes));
+  }) == static_cast<int>(cudaSuccess);
 }
 
-static bool set_smem_once(const void* fn, int bytes, int* mask) {
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev < 31 && (*mask & (1 << dev))) return true;
-  if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess)
-    return false;
-  if (dev < 31) *mask |= 1 << dev;
-  return true;
+// Largest number of pair clusters resident at once (one CTA per SM), per device.
+static int pair_clusters_resident(int num_sms) {
+  static DeviceOnce resident;
+  return resident.get([num_sms] {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(num_sms & ~1));
+    cfg.blockDim = dim3(gemm2::THREADS);
+    cfg.dynamicSmemBytes = gemm2::ALLOC;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, k_gemm_fp8_pair, &cfg) != cudaSuccess || n <= 0) {
+      cudaGetLastError();
+      n = num_sms / 2;
+    }
+    return n;
+  });
 }
 
 // M <= 128 (one row tile) keeps the one-SM kernel: a 256-row pair tile would be half empty.
@@ -486,22 +481,22 @@ cudaError_t launch_gemm_fp8(const uint8_t* a8, const uint8_t* b8, void* y, int M
   a.timeout_ns = timeout_ns;
   CUtensorMap ma, mb;
   if (M > gemm::BM && num_sms >= 2) {
-    static int configured = 0;
+    static DeviceOnce configured;
     if (!make_map_2d(&ma, a8, M, K, gemm2::BM / 2) || !make_map_2d(&mb, b8, N, K, gemm2::BN / 2))
       return cudaErrorInvalidValue;
-    if (!set_smem_once(reinterpret_cast<const void*>(k_gemm_fp8_pair), gemm2::ALLOC, &configured))
-      return cudaGetLastError();
+    if (!set_smem_once(configured, reinterpret_cast<const void*>(k_gemm_fp8_pair), gemm2::ALLOC))
+      return cudaErrorInvalidValue;
     const int tiles = ((M + gemm2::BM - 1) / gemm2::BM) * ((N + gemm2::BN - 1) / gemm2::BN);
     const int resident = pair_clusters_resident(num_sms);
     const int pairs = tiles < resident ? tiles : resident;
     k_gemm_fp8_pair<<<2 * pairs, gemm2::THREADS, gemm2::ALLOC, stream>>>(ma, mb, a);
     return cudaGetLastError();
   }
-  static int configured = 0;
+  static DeviceOnce configured;
   if (!make_map_2d(&ma, a8, M, K, gemm::BM) || !make_map_2d(&mb, b8, N, K, gemm::BN))
     return cudaErrorInvalidValue;
-  if (!set_smem_once(reinterpret_cast<const void*>(k_gemm_fp8), gemm::ALLOC, &configured))
-    return cudaGetLastError();
+  if (!set_smem_once(configured, reinterpret_cast<const void*>(k_gemm_fp8), gemm::ALLOC))
+    return cudaErrorInvalidValue;
   const int tiles = ((M + gemm::BM - 1) / gemm::BM) * ((N + gemm::BN - 1) / gemm::BN);
   const int grid = tiles < num_sms ? tiles : num_sms;
   k_gemm_fp8<<<grid, gemm::THREADS, gemm::ALLOC, stream>>>(ma, mb, a);

@@ -39,6 +39,19 @@ cudaError_t launch_gemm_fp8(const uint8_t* a8, const uint8_t* b8, void* y, int M
                             const float* s_a, const float* s_b, int* err, uint64_t timeout_ns,
                             int num_sms, cudaStream_t stream);
 
+// Test hooks of the attention launches (all off by default): inject_missing_q makes the producer
+// never load anything (every wait then runs into its limit); p_codes != null makes the D = 128
+// kernel copy, for the query row p_row of slab p_slab (row index within the slab's rows), the
+// 128 E4M3 codes of P of every key step into p_codes[step * 128 + key] and the step's integer
+// tile maximum into p_maxima[step].
+struct DebugHooks {
+  int inject_missing_q = 0;
+  uint8_t* p_codes = nullptr;
+  int* p_maxima = nullptr;
+  int p_slab = -1;
+  int p_row = -1;
+};
+
 // Persistent schedule of a dense attention launch (see plan_attention_split in attn_fwd.cu):
 // ctas CTAs, `whole` whole pairs each, then tail ranges of tail_w key steps; bytes = workspace
 // the cut tail pairs need (0: no pair is cut).
@@ -59,7 +72,7 @@ cudaError_t launch_attention_pair(const uint8_t* q8, const uint8_t* k8, const ui
                                   int H, int L, const int* cu_seqlens, int nseq, int max_seqlen,
                                   int rows_per_slab, int slabs, const float* s_q, const float* s_k,
                                   const float* s_v, float sm_scale, int* err, uint64_t timeout_ns,
-                                  int inject_missing_q, const AttnSplitPlan* plan, void* workspace,
+                                  const DebugHooks& dbg, const AttnSplitPlan* plan, void* workspace,
                                   cudaStream_t stream);
 
 // workspace may be null (no split); it is used only when workspace_bytes covers the plan.
@@ -67,7 +80,7 @@ cudaError_t launch_attention(const uint8_t* q8, const uint8_t* k8, const uint8_t
                              int B, int H, int L, int D, const int* cu_seqlens, int nseq,
                              int max_seqlen, int total_tokens, const float* s_q, const float* s_k,
                              const float* s_v, float sm_scale, int* err, uint64_t timeout_ns,
-                             int inject_missing_q, void* workspace, size_t workspace_bytes,
+                             const DebugHooks& dbg, void* workspace, size_t workspace_bytes,
                              int num_sms, cudaStream_t stream);
 
 }  // namespace qattn

@@ -1,6 +1,7 @@
 // qattn_api.cu -- the C ABI (include/qattn.h): argument checks, device checks, launches.
 #include <cuda_runtime.h>
 #include <cstdint>
+#include <mutex>
 
 #include "launch.h"
 #include "qattn.h"
@@ -16,14 +17,15 @@ constexpr int kMaxDevices = 64;
 constexpr uint64_t kDefaultTimeoutNs = 2000000000ull;
 
 struct DeviceInfo {
-  bool ready = false;
+  cudaError_t setup = cudaSuccess;   // error of the set-up below, if any
   bool supported = false;
   int num_sms = 0;
   int* err = nullptr;
 };
 DeviceInfo g_dev[kMaxDevices];
+std::once_flag g_dev_once[kMaxDevices];
 uint64_t g_timeout_ns = kDefaultTimeoutNs;
-int g_inject_missing_q = 0;
+qattn::DebugHooks g_dbg;          // test hooks (qattn_debug_*)
 
 thread_local int t_last_cuda_error = 0;   // qattn_last_cuda_error: per calling host thread
 
@@ -33,28 +35,29 @@ qattn_status from_cuda(cudaError_t e) {
   return QATTN_ERR_CUDA;
 }
 
-// Per-device setup on first use: capability check, SM count, address of the error word.
+// Per-device set-up on first use, once per device and thread-safe (std::call_once): capability
+// check, SM count, device address of the error word.  Callers on other threads wait for it.
 qattn_status device_info(DeviceInfo** out) {
   int dev = 0;
   const cudaError_t ge = cudaGetDevice(&dev);
   if (ge != cudaSuccess) return from_cuda(ge);
   if (dev < 0 || dev >= kMaxDevices) return QATTN_ERR_CUDA;
   DeviceInfo& d = g_dev[dev];
-  if (!d.ready) {
+  std::call_once(g_dev_once[dev], [&d, dev] {
     int major = 0, minor = 0, sms = 0;
-    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
-        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
-        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-      return QATTN_ERR_CUDA;
-    d.supported = (major == 10 && minor == 0);
+    cudaError_t e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    d.supported = e == cudaSuccess && major == 10 && minor == 0;
     d.num_sms = sms;
-    if (d.supported) {
+    if (e == cudaSuccess && d.supported) {
       void* p = nullptr;
-      if (cudaGetSymbolAddress(&p, g_qattn_error) != cudaSuccess) return QATTN_ERR_CUDA;
+      e = cudaGetSymbolAddress(&p, g_qattn_error);
       d.err = static_cast<int*>(p);
     }
-    d.ready = true;
-  }
+    d.setup = e;
+  });
+  if (d.setup != cudaSuccess) return from_cuda(d.setup);
   if (!d.supported) return QATTN_ERR_UNSUPPORTED;
   *out = &d;
   return QATTN_OK;
@@ -271,7 +274,7 @@ qattn_status qattn_forward_ws(const uint8_t* q8, const uint8_t* k8, const uint8_
     return QATTN_ERR_INVALID_ARG;
   return from_cuda(qattn::launch_attention(q8, k8, v8, out_bf16, B, H, L, D, nullptr, 0, L, L,
                                            scales->s_q, scales->s_k, scales->s_v, sm_scale,
-                                           d->err, g_timeout_ns, g_inject_missing_q,
+                                           d->err, g_timeout_ns, g_dbg,
                                            workspace_dev, workspace_bytes, d->num_sms,
                                            reinterpret_cast<cudaStream_t>(stream)));
 }
@@ -308,7 +311,7 @@ qattn_status qattn_forward_varlen(const uint8_t* q8, const uint8_t* k8, const ui
   return from_cuda(qattn::launch_attention(q8, k8, v8, out_bf16, 1, H, 0, D, cu_seqlens_dev,
                                            nseq, max_seqlen, total_tokens, scales->s_q,
                                            scales->s_k, scales->s_v, sm_scale, d->err,
-                                           g_timeout_ns, g_inject_missing_q, nullptr, 0,
+                                           g_timeout_ns, g_dbg, nullptr, 0,
                                            d->num_sms, reinterpret_cast<cudaStream_t>(stream)));
 }
 
@@ -351,7 +354,25 @@ void qattn_debug_set_wait_timeout_ns(uint64_t ns) {
   g_timeout_ns = ns ? ns : kDefaultTimeoutNs;
 }
 
-void qattn_debug_inject_missing_q(int enable) { g_inject_missing_q = enable ? 1 : 0; }
+void qattn_debug_inject_missing_q(int enable) { g_dbg.inject_missing_q = enable ? 1 : 0; }
+
+qattn_status qattn_debug_capture_p_row(int enable, int slab, int row, uint8_t* codes_dev,
+                                       int* maxima_dev) {
+  if (!enable) {
+    g_dbg.p_codes = nullptr;
+    g_dbg.p_maxima = nullptr;
+    g_dbg.p_slab = g_dbg.p_row = -1;
+    return QATTN_OK;
+  }
+  if (!codes_dev || !maxima_dev || !aligned(codes_dev, 16) || !aligned(maxima_dev, 4) || slab < 0 ||
+      row < 0)
+    return QATTN_ERR_INVALID_ARG;
+  g_dbg.p_codes = codes_dev;
+  g_dbg.p_maxima = maxima_dev;
+  g_dbg.p_slab = slab;
+  g_dbg.p_row = row;
+  return QATTN_OK;
+}
 
 qattn_status qattn_debug_attention_plan(int B, int H, int L, int D, int num_sms, int* plan,
                                         size_t* workspace_bytes) {

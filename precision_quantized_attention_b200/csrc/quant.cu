@@ -14,6 +14,7 @@
 #include <type_traits>
 #include <cstdint>
 
+#include "device_once.h"
 #include "launch.h"
 #include "sm100_ptx.cuh"
 
@@ -880,16 +881,24 @@ cudaError_t launch_quant_fp4_block(const void* x, size_t n, const float* amax, u
   return cudaGetLastError();
 }
 
+// Co-resident CTAs per SM of a cooperative kernel with FUSED_THREADS threads (0 on error).
+template <class K>
+static int blocks_per_sm_of(K fn) {
+  int n = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, reinterpret_cast<const void*>(fn), FUSED_THREADS,
+                                                    0) != cudaSuccess) {
+    cudaGetLastError();
+    return 0;
+  }
+  return n;
+}
+
 cudaError_t launch_calib_quant_fp8(const void* x, size_t n, float* amax, uint8_t* out,
                                    float* scale, void* workspace, uint64_t limit_ns, int* err,
                                    int num_sms, cudaStream_t stream) {
-  static int blocks_per_sm = 0;
-  if (blocks_per_sm == 0) {
-    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&blocks_per_sm,
-                                                                  k_calib_quant_fp8,
-                                                                  FUSED_THREADS, 0);
-    if (e != cudaSuccess || blocks_per_sm < 1) return e != cudaSuccess ? e : cudaErrorInvalidValue;
-  }
+  static DeviceOnce occ;
+  const int blocks_per_sm = occ.get([] { return blocks_per_sm_of(k_calib_quant_fp8); });
+  if (blocks_per_sm < 1) return cudaErrorInvalidValue;
   const size_t nvec = n / 8;
   const int ntail = static_cast<int>(n - nvec * 8);
   size_t want = (nvec + FUSED_THREADS * 4 - 1) / (FUSED_THREADS * 4);   // >= 4 vectors/thread
@@ -914,12 +923,10 @@ cudaError_t launch_calib_quant_qkv(const void* const* x, uint8_t* const* codes8,
                                    uint8_t* const* bscale, float* const* gscale, size_t n, int mode,
                                    void* workspace, uint64_t limit_ns, int* err, int num_sms,
                                    cudaStream_t stream) {
-  static int bps[2] = {0, 0};
+  static DeviceOnce occ[2];
   const void* fn = mode == 0 ? (const void*)k_calib_quant_qkv<0> : (const void*)k_calib_quant_qkv<1>;
-  if (bps[mode] == 0) {
-    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&bps[mode], fn, FUSED_THREADS, 0);
-    if (e != cudaSuccess || bps[mode] < 1) return e != cudaSuccess ? e : cudaErrorInvalidValue;
-  }
+  const int bps_mode = occ[mode].get([fn] { return blocks_per_sm_of(fn); });
+  if (bps_mode < 1) return cudaErrorInvalidValue;
   QkvArgs a;
   for (int i = 0; i < QKV; ++i) {
     a.t[i].x = static_cast<const uint4*>(x[i]);
@@ -936,7 +943,7 @@ cudaError_t launch_calib_quant_qkv(const void* const* x, uint8_t* const* codes8,
   a.ws = static_cast<QkvWorkspace*>(workspace);
   const size_t units = mode == 0 ? n / 8 : n / 16;
   const size_t want = (units + FUSED_THREADS * 4 - 1) / (FUSED_THREADS * 4);
-  const size_t cap = static_cast<size_t>(num_sms) * bps[mode];
+  const size_t cap = static_cast<size_t>(num_sms) * bps_mode;
   const unsigned grid = static_cast<unsigned>(want < 1 ? 1 : (want < cap ? want : cap));
   void* args[] = {(void*)&a};
   return cudaLaunchCooperativeKernel(fn, dim3(grid), dim3(FUSED_THREADS), args, 0, stream);
@@ -980,12 +987,9 @@ cudaError_t launch_calib_quant_fp4_block(const void* x, size_t n, float* amax, u
                                          uint8_t* bscale, float* gscale, uint8_t* codes8,
                                          float* scale8, void* workspace, uint64_t limit_ns,
                                          int* err, int num_sms, cudaStream_t stream) {
-  static int blocks_per_sm = 0;
-  if (blocks_per_sm == 0) {
-    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(
-        &blocks_per_sm, k_calib_quant_fp4_block, FUSED_THREADS, 0);
-    if (e != cudaSuccess || blocks_per_sm < 1) return e != cudaSuccess ? e : cudaErrorInvalidValue;
-  }
+  static DeviceOnce occ;
+  const int blocks_per_sm = occ.get([] { return blocks_per_sm_of(k_calib_quant_fp4_block); });
+  if (blocks_per_sm < 1) return cudaErrorInvalidValue;
   const size_t nblocks = n / 16;
   size_t want = (nblocks + FUSED_THREADS * 2 - 1) / (FUSED_THREADS * 2);
   size_t cap = static_cast<size_t>(num_sms) * blocks_per_sm;

@@ -1,0 +1,85 @@
+"""The P codes of the CUDA path, key by key, against the method's admissible codes.
+
+The blog ("Optimizing FLUX.1 Kontext for Image Editing with Low-Precision Quantization",
+"Workflow and quantization", second SDPA bullet) fixes BMM1's accumulation only as "higher
+precision": an FP32 accumulator may sum in another order than the oracle's exact sum, which moves
+each base-2 score S' by up to the oracle's radius delta, and where 2^(S' - M +- delta) * 448
+straddles an E4M3 rounding boundary both codes are results of the method.  On the L=8704 editing
+workload with outlier channels, rows are nearly one-hot and one such code can move an output by a
+few percent.  This test takes the sampled row whose output is farthest from the oracle (and a few
+ordinary rows), captures every P code the kernel computes for it (qattn_debug_capture_p_row), and
+checks each against the oracle's code for that key:
+  * equal after the exact rescaling 2^(tile max - M) (the kernel quantizes P relative to its tile's
+    integer maximum, the oracle relative to the row's; E4M3 rounding commutes with powers of two
+    in the normal range), or
+  * inside the oracle's admissible range [lo, hi] of that key (an accumulation-order tie), or
+  * for an oracle code in E4M3's subnormal range (below 2^-6), within one subnormal step 2^-9
+    (the kernel's finer scale rounds such values on a finer grid).
+Anything else would be a kernel error."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import precision_quantized_attention_b200 as qa
+import workloads
+from parity import gpu_path, oracle_path
+
+pytestmark = pytest.mark.gpu
+
+
+def _captured_row(path, slab, t, nsteps):
+    codes = torch.zeros(nsteps * 128, dtype=torch.uint8, device="cuda")
+    maxima = torch.zeros(nsteps, dtype=torch.int32, device="cuda")
+    qa._lib.debug_capture_p_row(True, slab, t, codes, maxima)
+    try:
+        path.attend()
+        assert qa.get_error() == 0
+    finally:
+        qa._lib.debug_capture_p_row(False)
+    return codes.cpu().numpy(), maxima.cpu().numpy()
+
+
+def _classify(w, path, q8, k8, row, tbl):
+    B, H, T, D = w.shape
+    slab, t = divmod(row, T)
+    nsteps = (T + 127) // 128
+    gcode, gmax = _captured_row(path, slab, t, nsteps)
+    gcode = gcode[:T]
+    code, x, delta, lo, hi, M, l = oracle.p_row_detail(q8, k8, w.shape, path.scale[0].item(),
+                                                       path.scale[1].item(), row, w.sm_scale)
+    step = np.arange(T) // 128
+    assert np.all(gmax[step] <= M)                          # every tile maximum <= the row's
+    v_gpu = tbl[gcode] * np.exp2(gmax[step].astype(np.float64) - M)   # at the oracle's scale
+    v_or = tbl[code]
+    same = v_gpu == v_or
+    tie = ~same & (v_gpu >= tbl[lo]) & (v_gpu <= tbl[hi])
+    sub = ~same & ~tie & (v_or < 2.0 ** -6) & (np.abs(v_gpu - v_or) <= 2.0 ** -9)
+    bad = ~(same | tie | sub)
+    return {"row": row, "differ": int(np.sum(~same)), "ties": int(np.sum(tie)),
+            "subnormal": int(np.sum(sub)), "bad": np.flatnonzero(bad), "M": M}
+
+
+def test_edit_fp8_p_codes_differ_only_by_admissible_ties():
+    w = workloads.WORKLOADS["edit_fp8"]
+    q, k, v = workloads.make_qkv(w)
+    path = gpu_path(w, q, k, v)
+    rows = workloads.sample_rows(w, per_head=48).numpy()
+    want = oracle_path(w, q, k, v, rows=rows)
+    got = path.out.float().reshape(-1, w.D)[torch.as_tensor(rows, device="cuda")].cpu().numpy()
+    err = np.abs(got.reshape(want.shape) - want).max(axis=-1)
+    order = np.argsort(err)
+    chosen = [int(rows[order[-1]])] + [int(rows[order[i]]) for i in (len(order) // 2, len(order) // 3)]
+    q8, k8 = path.codes[0].cpu().numpy(), path.codes[1].cpu().numpy()
+    tbl = oracle.e4m3_table().astype(np.float64)
+    report = []
+    for row in chosen:
+        r = _classify(w, path, q8, k8, row, tbl)
+        report.append(r)
+        assert r["bad"].size == 0, f"row {row}: codes outside the admissible range at keys {r['bad'][:16]}"
+    worst = report[0]
+    print(f"worst sampled row {worst['row']} (max-abs {err[order[-1]]:.3e}): {worst['differ']} of "
+          f"{w.L} codes differ ({worst['ties']} accumulation-order ties, {worst['subnormal']} "
+          f"subnormal); ordinary rows: {[(r['row'], r['differ']) for r in report[1:]]}")
+    for r in report[1:]:
+        assert r["differ"] - r["subnormal"] <= 16      # ordinary rows: at most a handful of ties

@@ -234,3 +234,35 @@ def test_ambiguity_is_zero_without_p_quantization_and_small_otherwise():
     _, amb0 = oracle.attention_e4m3(q8, q8, q8, w.shape, sq, sq, sq, flags=oracle.FP32,
                                     with_ambiguity=True)
     assert np.all(amb0 == 0)
+
+
+def test_p_row_detail_rebuilds_the_row_and_its_ambiguity():
+    """oracle.p_row_detail gives one row's P codes, x = S' - M, the radius delta and the code
+    range [lo, hi]; from them the row's output (sum_j val(code_j) v_j * s_v / 448 / l) and its
+    ambiguity bound (sum_j max|val(lo or hi) - val(code)| |v_j| * s_v / 448 / l) are rebuilt
+    and must equal attention_e4m3's, on peaked rows (outlier channels) and plain ones."""
+    tbl = oracle.e4m3_table().astype(np.float64)
+    for outliers, seed in ((4, 33), (0, 34)):
+        w = workloads.custom("detail", "fp8", 1, 2, 300, 64, seed=seed, outliers=outliers)
+        q, k, v = workloads.make_qkv(w)
+        q8, sq, _ = oracle.quantize_tensor(q, "fp8")
+        k8, sk, _ = oracle.quantize_tensor(k, "fp8")
+        v8, sv, _ = oracle.quantize_tensor(v, "fp8")
+        B, H, T, D = w.shape
+        rows = [0, 17, 299, T + 5, 2 * T - 1]
+        want, amb = oracle.attention_e4m3(q8, k8, v8, w.shape, sq, sk, sv, w.sm_scale, rows=rows,
+                                          with_ambiguity=True)
+        V = tbl[v8.reshape(B * H, T, D)]
+        for i, row in enumerate(rows):
+            code, x, delta, lo, hi, M, l = oracle.p_row_detail(q8, k8, w.shape, sq, sk, row, w.sm_scale)
+            assert code.shape == (T,) and M == np.ceil(M) and np.all(x <= 0) and np.all(delta > 0)
+            # the code is e4m3 of fl32(2^fl32(x)) * 448, within its own range
+            p = np.exp2(x.astype(np.float32)).astype(np.float32)
+            assert np.array_equal(code, np.array([oracle.e4m3_from_float(float(np.float32(pi * 448.0)))
+                                                  for pi in p], dtype=np.uint8))
+            assert np.all(tbl[lo] <= tbl[code]) and np.all(tbl[code] <= tbl[hi])
+            post = np.float64(sv) / 448.0 / l
+            vv = V[row // T]
+            np.testing.assert_allclose((tbl[code] @ vv) * post, want[i], rtol=1e-12, atol=1e-15)
+            a = np.maximum(np.abs(tbl[lo] - tbl[code]), np.abs(tbl[hi] - tbl[code]))
+            np.testing.assert_allclose((a @ np.abs(vv)) * post, amb[i], rtol=1e-12, atol=1e-15)
