@@ -311,9 +311,54 @@ def run_mode_extra(w, flush, steps, warmup):
     attn = sum(e[1].elapsed_time(e[2]) for e in ev) / steps
     quant = sum(e[0].elapsed_time(e[1]) for e in ev) / steps
     quant_static = time_quantize(w, qd, kd, vd, path.amax.tolist(), flush, steps)
-    return {"workload": w.name, "steps": steps, "step_ms": step, "attn_ms": attn,
-            "quant_ms": quant, "quant_static_ms": quant_static, "flops": w.flops,
-            "numel": q.numel(), "w": w}
+    out = {"workload": w.name, "steps": steps, "step_ms": step, "attn_ms": attn,
+           "quant_ms": quant, "quant_static_ms": quant_static, "flops": w.flops,
+           "numel": q.numel(), "w": w}
+    if w.mode == "fp4":
+        out["fp4_direct"] = fp4_direct_estimate(qd, kd, vd, path.amax, flush, steps)
+    return out
+
+
+def fp4_direct_estimate(qd, kd, vd, amax, flush, steps):
+    """What attention reading the packed E2M1 codes directly (instead of the FP8 requant codes)
+    would save: the requant output's write in the quantize pass; the attention kernel itself is
+    bound by its softmax, not by its 80 MB of code reads.  Times the per-tensor static FP4
+    quantize of Q, K, V with and without the FP8 requant output."""
+    import precision_quantized_attention_b200 as qa
+    n = qd.numel()
+    u8 = dict(dtype=torch.uint8, device="cuda")
+    e2m1 = [torch.empty(n // 2, **u8) for _ in range(3)]
+    bs = [torch.empty(n // 16, **u8) for _ in range(3)]
+    c8 = [torch.empty(n, **u8) for _ in range(3)]
+    gs = [torch.zeros(1, device="cuda") for _ in range(3)]
+    s8 = [torch.zeros(1, device="cuda") for _ in range(3)]
+    am = [amax[i:i + 1] for i in range(3)]
+
+    def run(requant):
+        for i, x in enumerate((qd, kd, vd)):
+            qa.quantize_fp4_block(x, am[i], e2m1[i], bs[i], gs[i], c8[i] if requant else None,
+                                  s8[i] if requant else None)
+
+    times = {}
+    for requant in (True, False):
+        for _ in range(3):
+            run(requant)
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(steps)]
+        for e0, e1 in ev:
+            flush()
+            e0.record()
+            run(requant)
+            e1.record()
+        torch.cuda.synchronize()
+        times[requant] = sum(e0.elapsed_time(e1) for e0, e1 in ev) / steps
+    if qa.get_error() != 0:
+        raise RuntimeError("device error in the FP4-direct estimate")
+    return {"quant_with_fp8_requant_ms": times[True], "quant_without_ms": times[False],
+            "saving_ms": times[True] - times[False],
+            "how": "per-tensor static FP4 quantize of Q, K, V with and without the FP8 requant "
+                   "output (qattn_quantize_fp4_block); the attention kernel would read E2M1 + "
+                   "block scales instead of E4M3 codes"}
 
 
 def measured_fp8_rates(flush, reps=5):
@@ -490,7 +535,8 @@ def report(args, w, qkv, rank, world, ms, attn, quant, e2e_ms, clocks, launches,
                "quantize": {"ms": x["quant_ms"], "algorithmic_bytes": qb4,
                             "frac_hbm": qb4 / (x["quant_ms"] * 1e-3) / 1e9 / hbm_gbs,
                             "static": {"ms": x["quant_static_ms"],
-                                       "frac_hbm": qb4 / (x["quant_static_ms"] * 1e-3) / 1e9 / hbm_gbs}}}
+                                       "frac_hbm": qb4 / (x["quant_static_ms"] * 1e-3) / 1e9 / hbm_gbs}},
+               "fp4_direct_estimate": x.get("fp4_direct")}
     result = {
         "metric": "quantized attention TFLOP/s @L=8704,H=24,D=128 and % of B200 FP8 peak",
         "value": world * flops / (ms * 1e-3) / 1e12,
@@ -589,9 +635,9 @@ def run_reference(args):
 
 
 # The transformer block's FP8 linear layers on the joint sequence (M = 512 + 4096 + 4096 tokens,
-# hidden 3072): the QKV projection and the two MLP GEMMs.
-GEMM_SHAPES = {"qkv_proj": (8704, 9216, 3072), "mlp_up": (8704, 12288, 3072),
-               "mlp_down": (8704, 3072, 12288)}
+# hidden 3072): the QKV and output projections and the two MLP GEMMs.
+GEMM_SHAPES = {"qkv_proj": (8704, 9216, 3072), "out_proj": (8704, 3072, 3072),
+               "mlp_up": (8704, 12288, 3072), "mlp_down": (8704, 3072, 12288)}
 
 
 def run_gemm(args):
@@ -646,6 +692,7 @@ def run_gemm(args):
                        "cores": os.cpu_count(), "kind": "oracle", "seconds": dt,
                        "sample": f"16 of {M} rows of {name} (numpy FP64 matmul)"}
     value = total_flops / (total_ms * 1e-3) / 1e12
+    fused = v_projection_fused(flush, args.steps)
     # the burst GEMM figure, unless the power cap held the clock down during the timed launches:
     # then the figure measured over a seconds-long loop under the cap (when the peaks file has it)
     clk = clocks.summary()
@@ -661,22 +708,71 @@ def run_gemm(args):
         rec["frac"] = rec["tflops"] / fp8_peak
     print(json.dumps({
         "metric": "FP8 GEMM TFLOP/s on the FLUX.1 Kontext block's linear layers "
-                  "(QKV projection and MLP, 8704 tokens, hidden 3072)",
+                  "(QKV and output projections, MLP; 8704 tokens, hidden 3072)",
         "value": value, "unit": "TFLOP/s", "n_gpus": 1, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": total_ms, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "e4m3",
         "data": "synthetic: seeded random E4M3 codes, per-tensor multipliers 0.01 and 0.002",
-        "config": {"workload": "qkv_proj 8704x9216x3072, mlp_up 8704x12288x3072, "
-                               "mlp_down 8704x3072x12288 (M x N x K)",
+        "config": {"workload": "qkv_proj 8704x9216x3072, out_proj 8704x3072x3072, "
+                               "mlp_up 8704x12288x3072, mlp_down 8704x3072x12288 (M x N x K)",
                    "l2": "flushed before every launch, outside the timed events"},
         "roofline": {"bound": "tensor", "achieved": value, "peak": fp8_peak, "unit": "TFLOP/s",
                      "frac": value / fp8_peak, "traffic": None, "kernel": "k_gemm_fp8_pair",
                      "peak_source": f"{peak_kind} bf16 {bf16_tf} TFLOP/s x {FP8_PER_BF16} "
                                     "(nominal FP8/BF16 ratio)", "per_shape": per_shape},
-        "gpu_launches": 3 * args.steps,
+        "v_projection_fused_quantize": fused,
+        "gpu_launches": len(GEMM_SHAPES) * args.steps,
         "clocks": clk,
         "cpu_baseline": cpu,
     }), flush=True)
+
+
+def v_projection_fused(flush, steps):
+    """The value projection (8704 tokens, 3072 -> 3072) feeding the attention's V codes, with
+    static scales: the GEMM's bf16 output then a separate quantize launch, against the GEMM with
+    the quantize fused into its epilogue (qattn_gemm_fp8_e4m3, codes only)."""
+    import precision_quantized_attention_b200 as qa
+    M, N, K = GEMM_SHAPES["out_proj"]               # same shape as the value projection
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(11)
+    a8 = torch.randint(0, 256, (M, K), dtype=torch.uint8, device="cuda", generator=gen)
+    b8 = torch.randint(0, 256, (N, K), dtype=torch.uint8, device="cuda", generator=gen)
+    a8 = torch.where((a8 & 0x7F) == 0x7F, a8 ^ 1, a8)
+    b8 = torch.where((b8 & 0x7F) == 0x7F, b8 ^ 1, b8)
+    sa, sb = torch.tensor([0.01], device="cuda"), torch.tensor([0.002], device="cuda")
+    y = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
+    codes = torch.empty(M, N, dtype=torch.uint8, device="cuda")
+    scale = torch.zeros(1, device="cuda")
+    qa.gemm_fp8(a8, b8, y, sa, sb)
+    amax = y.float().abs().max().reshape(1)          # the static calibration
+
+    def separate():
+        qa.gemm_fp8(a8, b8, y, sa, sb)
+        qa.quantize_fp8(y.reshape(-1), amax, codes.reshape(-1), scale)
+
+    def fused_call():
+        qa.gemm_fp8_e4m3(a8, b8, codes, sa, sb, amax, scale)
+
+    def ms(fn):
+        for _ in range(3):
+            fn()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(steps)]
+        for e0, e1 in ev:
+            flush()
+            e0.record()
+            fn()
+            e1.record()
+        torch.cuda.synchronize()
+        return sum(e0.elapsed_time(e1) for e0, e1 in ev) / steps
+
+    t_sep, t_fused = ms(separate), ms(fused_call)
+    if qa.get_error() != 0:
+        raise RuntimeError("device error in the fused value-projection timing")
+    return {"shape": f"{M}x{N}x{K}", "gemm_then_quantize_ms": t_sep, "fused_ms": t_fused,
+            "saved_ms": t_sep - t_fused,
+            "how": "static amax; separate = qattn_gemm_fp8 (bf16 out) + qattn_quantize_fp8; fused = "
+                   "qattn_gemm_fp8_e4m3 (codes only)"}
 
 
 def main():

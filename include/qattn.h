@@ -179,6 +179,23 @@ QATTN_API qattn_status qattn_gemm_fp8(const uint8_t* a8, const uint8_t* b8, void
                                       int N, int K, const float* s_a_dev, const float* s_b_dev,
                                       qattn_stream_t stream);
 
+/* The same GEMM with the per-tensor FP8 FakeQuantize of its output fused into the epilogue, for
+ * a projection whose output goes straight to the quantized attention (the value projection: no
+ * RoPE or normalization lies between it and SDPA).  The scale is static, from a given amax (the
+ * blog's post-training calibration, "Workflow and quantization", flow steps 3-4):
+ *   s = fl32(amax / 448) (amax == 0: s = 1), written to *scale_out_dev;
+ *   codes_out[m, n] = e4m3(fl32(y[m, n] / s)), y[m, n] the bf16 value qattn_gemm_fp8 computes,
+ * i.e. exactly what qattn_quantize_fp8(y, amax) would write from that bf16 output (round to
+ * nearest even, saturating; values above the amax saturate).  y_bf16 may be null (codes only)
+ * or receive the bf16 output as well.  codes_out: [M, N] bytes, 16-byte aligned; amax_dev,
+ * scale_out_dev: device floats.  A non-finite amax writes no code and records
+ * QATTN_ERR_NONFINITE (qattn_get_error).  Other requirements as qattn_gemm_fp8. */
+QATTN_API qattn_status qattn_gemm_fp8_e4m3(const uint8_t* a8, const uint8_t* b8, void* y_bf16,
+                                           uint8_t* codes_out, int M, int N, int K,
+                                           const float* s_a_dev, const float* s_b_dev,
+                                           const float* amax_dev, float* scale_out_dev,
+                                           qattn_stream_t stream);
+
 /* qattn_calibrate_quantize_fp8 without a caller workspace (the blog has no counterpart: this is
  * a calling convention, not part of the method).  For callers that cannot supply a scratch
  * buffer -- C code with no device allocator at the call site, or a runtime whose device memory

@@ -23,12 +23,13 @@ EXPORTS = (
     "qattn_forward_varlen", "qattn_get_error", "qattn_calibrate_quantize_fp8",
     "qattn_calibrate_quantize_fp4_block", "qattn_calibrate_quantize_fp8_noalloc",
     "qattn_calibrate_quantize_qkv", "qattn_quantize_qkv", "qattn_forward_ws", "qattn_gemm_fp8",
+    "qattn_gemm_fp8_e4m3",
     "qattn_status_str", "qattn_last_cuda_error",
     "qattn_forward_workspace_bytes",
     "qattn_debug_set_wait_timeout_ns", "qattn_debug_inject_missing_q", "qattn_debug_capture_p_row",
     "qattn_debug_attention_plan",
 )
-_RETURNS_STATUS = EXPORTS[:13]
+_RETURNS_STATUS = EXPORTS[:14]
 FUSED_WORKSPACE_BYTES = 256     # QATTN_FUSED_WORKSPACE_BYTES
 
 
@@ -75,6 +76,7 @@ def load() -> ctypes.CDLL:
     lib.qattn_calibrate_quantize_qkv.argtypes = [ctypes.POINTER(QuantIO), S, I, P, S, P]
     lib.qattn_quantize_qkv.argtypes = [ctypes.POINTER(QuantIO), S, I, P]
     lib.qattn_gemm_fp8.argtypes = [P, P, P, I, I, I, P, P, P]
+    lib.qattn_gemm_fp8_e4m3.argtypes = [P, P, P, P, I, I, I, P, P, P, P, P]
     lib.qattn_forward.argtypes = [P, P, P, P, I, I, I, I, ctypes.POINTER(_Scales), F, I, P]
     lib.qattn_forward_varlen.argtypes = [P, P, P, P, P, I, I, I, I, I, ctypes.POINTER(_Scales),
                                          F, I, P]
@@ -265,6 +267,25 @@ def gemm_fp8(a8, b8, y, s_a, s_b, stream=None):
                                  _dev(y, torch.bfloat16, "y"), M, N, K,
                                  _dev(s_a, torch.float32, "s_a"), _dev(s_b, torch.float32, "s_b"),
                                  _stream(stream)), "qattn_gemm_fp8")
+
+
+def gemm_fp8_e4m3(a8, b8, codes, s_a, s_b, amax, scale_out, y=None, stream=None):
+    """The FP8 GEMM with its bf16 output quantized to E4M3 in the epilogue under a static amax:
+    codes [M, N] uint8 = e4m3(y / s), s = amax / 448 written to scale_out (one-element float32
+    device tensors); y [M, N] bf16 optional.  K % 128 == 0, N % 32 == 0."""
+    if a8.dim() != 2 or b8.dim() != 2 or a8.shape[1] != b8.shape[1]:
+        raise ValueError("a8 [M, K] and b8 [N, K] with the same K")
+    M, K = a8.shape
+    N = b8.shape[0]
+    if tuple(codes.shape) != (M, N) or (y is not None and tuple(y.shape) != (M, N)):
+        raise ValueError("codes (and y) must be [M, N]")
+    _check(load().qattn_gemm_fp8_e4m3(_dev(a8, torch.uint8, "a8"), _dev(b8, torch.uint8, "b8"),
+                                      None if y is None else _dev(y, torch.bfloat16, "y"),
+                                      _dev(codes, torch.uint8, "codes"), M, N, K,
+                                      _dev(s_a, torch.float32, "s_a"), _dev(s_b, torch.float32, "s_b"),
+                                      _dev(amax, torch.float32, "amax"),
+                                      _dev(scale_out, torch.float32, "scale_out"), _stream(stream)),
+           "qattn_gemm_fp8_e4m3")
 
 
 def _scales(s_q, s_k, s_v):

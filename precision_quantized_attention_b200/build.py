@@ -13,7 +13,7 @@ CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(os.path.dirname(HERE), "include")
 LIB = os.path.join(HERE, "libqattn.so")
 SOURCES = ["qattn_api.cu", "quant.cu", "attn_fwd.cu", "attn_pair.cu", "noalloc.cu", "gemm_fp8.cu"]
-HEADERS = ["sm100_ptx.cuh", "softmax_sm100.cuh", "launch.h", "device_once.h"]
+HEADERS = ["sm100_ptx.cuh", "softmax_sm100.cuh", "launch.h", "device_once.h", "quant_math.cuh"]
 
 
 def nvcc() -> str:

@@ -694,13 +694,16 @@ static cudaError_t launch_attn_d(const void* q8, const void* k8, const void* v8,
 // has a handful of parts at most) and at most one pair; when the even share would be 0.8 of a
 // pair or more, or would save fewer than 4 key steps, the tail pairs stay whole (one per CTA).
 // bytes = the workspace the cut pairs' partial results need (0: no pair is cut).
+#ifndef QATTN_TAIL_MIN_DIV
+#define QATTN_TAIL_MIN_DIV 4        // a tail range is at least 1/QATTN_TAIL_MIN_DIV of a pair
+#endif
 AttnSplitPlan plan_attention_split(int B, int H, int L, int D, int num_sms) {
   AttnSplitPlan p;
   p.pairs_per_head = (L + NQ * BLOCK_M - 1) / (NQ * BLOCK_M);
   const long long pairs = static_cast<long long>(p.pairs_per_head) * H * B;
   p.nkv = (L + BLOCK_N - 1) / BLOCK_N;
   const long long steps = pairs * p.nkv;
-  const int wmin = (p.nkv + 3) / 4;
+  const int wmin = (p.nkv + QATTN_TAIL_MIN_DIV - 1) / QATTN_TAIL_MIN_DIV;
   const long long want = (steps + wmin - 1) / wmin;
   p.ctas = static_cast<int>(want < num_sms ? want : num_sms);
   if (p.ctas < 1) p.ctas = 1;

@@ -495,6 +495,8 @@ __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(168)
       float m_w = 0.0f;                            // to m_w, the largest tile maximum it has seen
       bool mine_before = false;
       float m_ref = 0.0f;
+      const bool capture = args.dbg_p != nullptr && sg.slab == args.dbg_slab &&
+                           sg.seq_start + sg.q_row0 + static_cast<int>(rank) * BLOCK_M + r == args.dbg_row;
       for (int j = (s0 & 1) == wg ? 0 : 1; j < n; j += 2) {
         const int s = s0 + j;
         const int b = s % NSBUF;
@@ -544,9 +546,9 @@ __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(168)
           for (int q = 0; q < 4; ++q)
             pk[i / 4 + q] = cvt_e4m3x2(p[4 * q], p[4 * q + 1]) | (cvt_e4m3x2(p[4 * q + 2], p[4 * q + 3]) << 16);
         }
-        if (args.dbg_p != nullptr && sg.slab == args.dbg_slab &&
-            sg.seq_start + sg.q_row0 + static_cast<int>(rank) * BLOCK_M + r == args.dbg_row)
-          capture_p_row(args, sg.kv0 + j, pk, mx);   // test hook: off unless a row is chosen
+#ifndef QATTN_NO_CAPTURE_HOOK
+        if (capture) capture_p_row(args, sg.kv0 + j, pk, mx);   // test hook: off unless a row is chosen
+#endif
         // P(s) over the first 32 columns of the buffer (column c: keys 4c..4c+3)
         tmem_st32(tS, pk);
         // M_ref after step s - 1, published by the other warpgroup (waited on at every step so

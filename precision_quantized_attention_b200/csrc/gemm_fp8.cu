@@ -27,6 +27,7 @@
 #include <cstdint>
 
 #include "device_once.h"
+#include "quant_math.cuh"
 #include "launch.h"
 #include "sm100_ptx.cuh"
 
@@ -59,10 +60,69 @@ struct GemmArgs {
   int M, N, K;
   const float* s_a;
   const float* s_b;
-  __nv_bfloat16* y;
+  __nv_bfloat16* y;         // bf16 output, or nullptr (codes only)
   int* err;
   uint64_t timeout_ns;
+  // optional per-tensor FP8 quantization of the bf16 output with a given (static) amax: codes
+  // [M, N] = e4m3(fl32(y / s)), s = fl32(amax / 448) (amax == 0: s = 1) written to *scale_out
+  uint8_t* codes;
+  const float* amax;
+  float* scale_out;
 };
+
+// Per-tensor scale of the epilogue's E4M3 codes from the given amax: (s, RN(1 / s), Markstein
+// usable); ok = false (and a non-finite error recorded once) when the amax is not finite.
+struct CodeScale {
+  float s, r;
+  bool fast, ok;
+};
+__device__ __forceinline__ CodeScale code_scale(const GemmArgs& a) {
+  CodeScale cs{1.0f, 1.0f, true, false};
+  if (!a.codes) return cs;
+  const float amax = __ldg(a.amax);
+  if (!(amax <= 3.402823466e38f)) {              // inf or NaN: no code is written
+    if (blockIdx.x == 0 && threadIdx.x == 64) atomicExch(a.err, DEV_ERR_NONFINITE);
+    return cs;
+  }
+  cs.s = amax == 0.0f ? 1.0f : __fdiv_rn(amax, 448.0f);
+  cs.r = __frcp_rn(cs.s);
+  cs.fast = markstein_ok(cs.s);
+  cs.ok = true;
+  if (blockIdx.x == 0 && threadIdx.x == 64) *a.scale_out = cs.s;
+  return cs;
+}
+
+// Epilogue of 32 columns of one row: bf16 of acc * scale to y (if any) and, when the codes are
+// requested, their E4M3 codes (the bf16 values quantized exactly as qattn_quantize_fp8 would).
+__device__ __forceinline__ void epilogue32(const GemmArgs& a, const CodeScale& cs, const uint32_t (&v)[32],
+                                           float scale, size_t off) {
+  uint32_t packed[16];
+#pragma unroll
+  for (int e = 0; e < 16; ++e) {
+    const __nv_bfloat162 b2 = __floats2bfloat162_rn(__uint_as_float(v[2 * e]) * scale,
+                                                    __uint_as_float(v[2 * e + 1]) * scale);
+    packed[e] = *reinterpret_cast<const uint32_t*>(&b2);
+  }
+  if (a.y) {
+    uint4* dst = reinterpret_cast<uint4*>(a.y + off);
+#pragma unroll
+    for (int e = 0; e < 4; ++e)
+      dst[e] = make_uint4(packed[4 * e], packed[4 * e + 1], packed[4 * e + 2], packed[4 * e + 3]);
+  }
+  if (cs.ok) {
+    uint32_t c[8];
+    if (cs.fast) {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) c[e] = quant4_e4m3<true>(packed[2 * e], packed[2 * e + 1], cs.s, cs.r);
+    } else {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) c[e] = quant4_e4m3<false>(packed[2 * e], packed[2 * e + 1], cs.s, cs.r);
+    }
+    uint4* dst = reinterpret_cast<uint4*>(a.codes + off);
+    dst[0] = make_uint4(c[0], c[1], c[2], c[3]);
+    dst[1] = make_uint4(c[4], c[5], c[6], c[7]);
+  }
+}
 
 __global__ void __launch_bounds__(gemm::THREADS, 1)
     k_gemm_fp8(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
@@ -169,6 +229,7 @@ __global__ void __launch_bounds__(gemm::THREADS, 1)
     const int r = quarter * 32 + lane;             // row within the tile
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
     const float scale = __ldg(args.s_a) * __ldg(args.s_b);
+    const CodeScale cs = code_scale(args);
     int i = 0;
     for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++i) {
       const int ab = i & 1;
@@ -176,26 +237,15 @@ __global__ void __launch_bounds__(gemm::THREADS, 1)
       if (!__all_sync(0xFFFFFFFFu, ok)) break;
       tc_fence_after();
       const int m = (t % tiles_m) * BM + r, n0 = (t / tiles_m) * BN;
-      __nv_bfloat16* yrow = args.y + static_cast<size_t>(m) * args.N + n0;
+      const size_t row_off = static_cast<size_t>(m) * args.N + n0;
       const uint32_t acc = tmem + lane_off + static_cast<uint32_t>(ab * BN);
 #pragma unroll 1
       for (int c = 0; c < BN / 32; ++c) {
         uint32_t v[32];
         tmem_ld32(acc + c * 32, v);
         tmem_wait_ld();
-        if (m < args.M && n0 + c * 32 < args.N) {   // N % 32 == 0: a chunk is all in or out
-          uint32_t packed[16];
-#pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const __nv_bfloat162 b2 = __floats2bfloat162_rn(__uint_as_float(v[2 * e]) * scale,
-                                                            __uint_as_float(v[2 * e + 1]) * scale);
-            packed[e] = *reinterpret_cast<const uint32_t*>(&b2);
-          }
-          uint4* dst = reinterpret_cast<uint4*>(yrow + c * 32);
-#pragma unroll
-          for (int e = 0; e < 4; ++e)
-            dst[e] = make_uint4(packed[4 * e], packed[4 * e + 1], packed[4 * e + 2], packed[4 * e + 3]);
-        }
+        if (m < args.M && n0 + c * 32 < args.N)     // N % 32 == 0: a chunk is all in or out
+          epilogue32(args, cs, v, scale, row_off + c * 32);
       }
       tc_fence_before();
       mbar_arrive(BAR(B_ACCE + ab));               // accumulator read out
@@ -365,6 +415,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(gemm2::THREADS, 1)
     const int r = quarter * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
     const float scale = __ldg(args.s_a) * __ldg(args.s_b);
+    const CodeScale cs = code_scale(args);
     int i = 0;
     for (int t = pair; t < tiles; t += npairs, ++i) {
       const int ab = i & 1;
@@ -373,26 +424,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(gemm2::THREADS, 1)
       tc_fence_after();
       const int m = (t % tiles_m) * BM + static_cast<int>(rank) * (BM / 2) + r;
       const int n0 = (t / tiles_m) * BN;
-      __nv_bfloat16* yrow = args.y + static_cast<size_t>(m) * args.N + n0;
+      const size_t row_off = static_cast<size_t>(m) * args.N + n0;
       const uint32_t acc = tmem + lane_off + static_cast<uint32_t>(ab * BN);
 #pragma unroll 1
       for (int c = 0; c < BN / 32; ++c) {
         uint32_t v[32];
         tmem_ld32(acc + c * 32, v);
         tmem_wait_ld();
-        if (m < args.M && n0 + c * 32 < args.N) {
-          uint32_t packed[16];
-#pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const __nv_bfloat162 b2 = __floats2bfloat162_rn(__uint_as_float(v[2 * e]) * scale,
-                                                            __uint_as_float(v[2 * e + 1]) * scale);
-            packed[e] = *reinterpret_cast<const uint32_t*>(&b2);
-          }
-          uint4* dst = reinterpret_cast<uint4*>(yrow + c * 32);
-#pragma unroll
-          for (int e = 0; e < 4; ++e)
-            dst[e] = make_uint4(packed[4 * e], packed[4 * e + 1], packed[4 * e + 2], packed[4 * e + 3]);
-        }
+        if (m < args.M && n0 + c * 32 < args.N) epilogue32(args, cs, v, scale, row_off + c * 32);
       }
       tc_fence_before();
       __syncwarp();
@@ -469,8 +508,12 @@ static int pair_clusters_resident(int num_sms) {
 // M <= 128 (one row tile) keeps the one-SM kernel: a 256-row pair tile would be half empty.
 cudaError_t launch_gemm_fp8(const uint8_t* a8, const uint8_t* b8, void* y, int M, int N, int K,
                             const float* s_a, const float* s_b, int* err, uint64_t timeout_ns,
-                            int num_sms, cudaStream_t stream) {
+                            int num_sms, cudaStream_t stream, uint8_t* codes, const float* amax,
+                            float* scale_out) {
   GemmArgs a;
+  a.codes = codes;
+  a.amax = amax;
+  a.scale_out = scale_out;
   a.M = M;
   a.N = N;
   a.K = K;

@@ -34,10 +34,13 @@ cudaError_t launch_quant_qkv(const void* const* x, uint8_t* const* codes8, float
                              float* const* gscale, size_t n, int mode, int* err, int num_sms,
                              cudaStream_t stream);
 
-// Y[M, N] (bf16) = (A8[M, K] B8[N, K]^T) * s_a * s_b; K % 128 == 0, N % 32 == 0.
+// Y[M, N] (bf16) = (A8[M, K] B8[N, K]^T) * s_a * s_b; K % 128 == 0, N % 32 == 0.  y may be null
+// when codes are requested; codes (optional): the E4M3 codes of the bf16 Y under the given amax
+// (scale s = amax / 448 written to *scale_out).
 cudaError_t launch_gemm_fp8(const uint8_t* a8, const uint8_t* b8, void* y, int M, int N, int K,
                             const float* s_a, const float* s_b, int* err, uint64_t timeout_ns,
-                            int num_sms, cudaStream_t stream);
+                            int num_sms, cudaStream_t stream, uint8_t* codes = nullptr,
+                            const float* amax = nullptr, float* scale_out = nullptr);
 
 // Test hooks of the attention launches (all off by default): inject_missing_q makes the producer
 // never load anything (every wait then runs into its limit); p_codes != null makes the D = 128

@@ -256,6 +256,26 @@ qattn_status qattn_gemm_fp8(const uint8_t* a8, const uint8_t* b8, void* y_bf16, 
                                           reinterpret_cast<cudaStream_t>(stream)));
 }
 
+qattn_status qattn_gemm_fp8_e4m3(const uint8_t* a8, const uint8_t* b8, void* y_bf16,
+                                 uint8_t* codes_out, int M, int N, int K, const float* s_a_dev,
+                                 const float* s_b_dev, const float* amax_dev, float* scale_out_dev,
+                                 qattn_stream_t stream) {
+  if (!a8 || !b8 || !codes_out || !s_a_dev || !s_b_dev || !amax_dev || !scale_out_dev)
+    return QATTN_ERR_INVALID_ARG;
+  if (M < 1 || N < 32 || K < 128 || N % 32 != 0 || K % 128 != 0) return QATTN_ERR_INVALID_ARG;
+  if (!aligned(a8, 16) || !aligned(b8, 16) || (y_bf16 && !aligned(y_bf16, 16)) ||
+      !aligned(codes_out, 16) || !aligned(s_a_dev, 4) || !aligned(s_b_dev, 4) ||
+      !aligned(amax_dev, 4) || !aligned(scale_out_dev, 4))
+    return QATTN_ERR_INVALID_ARG;
+  DeviceInfo* d = nullptr;
+  qattn_status st = device_info(&d);
+  if (st != QATTN_OK) return st;
+  return from_cuda(qattn::launch_gemm_fp8(a8, b8, y_bf16, M, N, K, s_a_dev, s_b_dev, d->err,
+                                          g_timeout_ns, d->num_sms,
+                                          reinterpret_cast<cudaStream_t>(stream), codes_out,
+                                          amax_dev, scale_out_dev));
+}
+
 qattn_status qattn_forward_ws(const uint8_t* q8, const uint8_t* k8, const uint8_t* v8,
                               void* out_bf16, int B, int H, int L, int D,
                               const qattn_scales* scales, float sm_scale, qattn_mode mode,

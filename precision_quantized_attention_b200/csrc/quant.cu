@@ -15,6 +15,7 @@
 #include <cstdint>
 
 #include "device_once.h"
+#include "quant_math.cuh"
 #include "launch.h"
 #include "sm100_ptx.cuh"
 
@@ -69,45 +70,6 @@ __global__ void __launch_bounds__(256) k_amax_bf16(const uint4* __restrict__ xv,
       atomicMax(amax_bits, m << 16);
     }
   }
-}
-
-// -------------------------------------------------------------------------------------------
-// Correctly rounded x / s for a divisor shared by many elements (Markstein's theorem: with
-// r = RN(1/s) and q0 = RN(x * r), which is within one ulp of x / s, the residual
-// x - q0 * s is exact in one FMA and RN(q0 + residual * r) = RN(x / s)).  Three FMA-pipe
-// instructions instead of a division; valid while s, r and the residual stay normal, which
-// `markstein_ok` checks once per divisor (callers use __fdiv_rn otherwise).  Quotients so small
-// that they leave the normal range map to a signed zero E4M3/E2M1 code either way.
-// -------------------------------------------------------------------------------------------
-__device__ __forceinline__ bool markstein_ok(float s) {
-  const float a = fabsf(s);
-  return a >= 0x1p-100f && a <= 0x1p+100f;
-}
-
-// s > 0, so RN(x / s) has the sign of x; copysign restores it where the correction step's
-// sum of zeros would not (x = -0, or a quotient that underflows).
-__device__ __forceinline__ float div_rn_by(float x, float s, float r) {
-  const float q0 = __fmul_rn(x, r);
-  const float e = __fmaf_rn(-q0, s, x);
-  return copysignf(__fmaf_rn(e, r, q0), x);
-}
-
-// -------------------------------------------------------------------------------------------
-// Per-tensor FP8: s = fl32(amax / 448), code = e4m3(fl32(x / s)); amax == 0 gives s = 1.
-// -------------------------------------------------------------------------------------------
-__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
-__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
-
-template <bool FAST>
-__device__ __forceinline__ float div_s(float x, float s, float r) {
-  return FAST ? div_rn_by(x, s, r) : __fdiv_rn(x, s);
-}
-
-template <bool FAST>
-__device__ __forceinline__ uint32_t quant4_e4m3(uint32_t w0, uint32_t w1, float s, float r) {
-  const uint32_t lo = cvt_e4m3x2(div_s<FAST>(bf16_lo(w0), s, r), div_s<FAST>(bf16_hi(w0), s, r));
-  const uint32_t hi = cvt_e4m3x2(div_s<FAST>(bf16_lo(w1), s, r), div_s<FAST>(bf16_hi(w1), s, r));
-  return lo | (hi << 16);
 }
 
 __global__ void __launch_bounds__(256) k_quant_fp8(const uint4* __restrict__ xv, size_t nvec,
@@ -765,6 +727,10 @@ __global__ void __launch_bounds__(FUSED_THREADS) k_calib_quant_qkv(const QkvArgs
 // -------------------------------------------------------------------------------------------
 constexpr int STATIC_THREADS = 256;
 constexpr int STATIC_UNROLL = 4;           // 16-byte loads in flight per thread (FP8)
+#ifndef QATTN_STATIC_FP4_UNROLL
+#define QATTN_STATIC_FP4_UNROLL 2
+#endif
+constexpr int STATIC_FP4_UNROLL = QATTN_STATIC_FP4_UNROLL;   // 16-element blocks in flight (FP4)
 
 template <int MODE>
 __global__ void __launch_bounds__(STATIC_THREADS) k_quant_qkv(const __grid_constant__ QkvArgs a) {
@@ -825,11 +791,16 @@ __global__ void __launch_bounds__(STATIC_THREADS) k_quant_qkv(const __grid_const
     const uint4* xv = tp.x;
     uint4* c8 = reinterpret_cast<uint4*>(tp.codes8);
     size_t b = i0;
-    for (; b + T < nblocks; b += 2 * T) {         // two blocks' loads in flight
-      const uint4 a0 = __ldcs(xv + 2 * b), a1 = __ldcs(xv + 2 * b + 1);
-      const uint4 d0 = __ldcs(xv + 2 * (b + T)), d1 = __ldcs(xv + 2 * (b + T) + 1);
-      fp4_block(a0, a1, b, six_sg, &tab, tp.e2m1, tp.bscale, c8);
-      fp4_block(d0, d1, b + T, six_sg, &tab, tp.e2m1, tp.bscale, c8);
+    constexpr size_t UB = STATIC_FP4_UNROLL;
+    for (; b + (UB - 1) * T < nblocks; b += UB * T) {   // UB blocks' loads in flight
+      uint4 x0[UB], x1[UB];
+#pragma unroll
+      for (size_t u = 0; u < UB; ++u) {
+        x0[u] = __ldcs(xv + 2 * (b + u * T));
+        x1[u] = __ldcs(xv + 2 * (b + u * T) + 1);
+      }
+#pragma unroll
+      for (size_t u = 0; u < UB; ++u) fp4_block(x0[u], x1[u], b + u * T, six_sg, &tab, tp.e2m1, tp.bscale, c8);
     }
     for (; b < nblocks; b += T)
       fp4_block(__ldcs(xv + 2 * b), __ldcs(xv + 2 * b + 1), b, six_sg, &tab, tp.e2m1, tp.bscale, c8);
@@ -971,7 +942,7 @@ cudaError_t launch_quant_qkv(const void* const* x, uint8_t* const* codes8, float
   // per tensor: enough CTAs for four 16-byte vectors (FP8) or two blocks (FP4) per thread, at
   // most 4 CTAs of 256 threads per SM (3 tensors: 12 per SM)
   const size_t per_cta = mode == 0 ? static_cast<size_t>(STATIC_THREADS) * STATIC_UNROLL * 8
-                                   : static_cast<size_t>(STATIC_THREADS) * 2 * 16;
+                                   : static_cast<size_t>(STATIC_THREADS) * STATIC_FP4_UNROLL * 16;
   size_t want = (n + per_cta - 1) / per_cta;
   const size_t cap = static_cast<size_t>(num_sms) * 4;
   if (want < 1) want = 1;

@@ -136,3 +136,26 @@ def test_gemm_argument_errors():
                {"s_a": ctypes.c_void_p(0x10002)}, {"M": 0}, {"N": 16}, {"N": 48}, {"K": 64},
                {"K": 200}):
         assert call(**kw) == _lib.ERR_INVALID_ARG, kw
+
+
+def test_gemm_e4m3_argument_errors():
+    """qattn_gemm_fp8_e4m3 refuses on the host, before any launch: null codes, amax or scale
+    output, misaligned buffers (a null y is allowed: codes only), and the shapes qattn_gemm_fp8
+    refuses."""
+    lib = _lib.load()
+    g = lib.qattn_gemm_fp8_e4m3
+    s0 = ctypes.c_void_p(0)
+    names = ("a8", "b8", "y", "codes", "M", "N", "K", "s_a", "s_b", "amax", "scale")
+    ok = (FAKE, FAKE, FAKE, FAKE, 256, 256, 256, FAKE, FAKE, FAKE, FAKE, s0)
+
+    def call(**kw):
+        a = list(ok)
+        for i, name in enumerate(names):
+            if name in kw:
+                a[i] = kw[name]
+        return g(*a)
+
+    for kw in ({"a8": None}, {"b8": None}, {"codes": None}, {"s_a": None}, {"s_b": None},
+               {"amax": None}, {"scale": None}, {"codes": MISALIGNED}, {"y": MISALIGNED},
+               {"amax": ctypes.c_void_p(0x10002)}, {"M": 0}, {"N": 48}, {"K": 200}):
+        assert call(**kw) == _lib.ERR_INVALID_ARG, kw

@@ -50,7 +50,8 @@ def test_small_shapes_all_elements(M, N, K):
     _check(y.float().cpu().numpy(), want, bound, K)
 
 
-@pytest.mark.parametrize("M,N,K", [(8704, 9216, 3072), (8704, 12288, 3072), (8704, 3072, 12288)])
+@pytest.mark.parametrize("M,N,K", [(8704, 9216, 3072), (8704, 3072, 3072), (8704, 12288, 3072),
+                                   (8704, 3072, 12288)])
 def test_kontext_block_shapes_sampled_rows(M, N, K):
     """The joint sequence (512 text + 4096 target + 4096 context tokens) through the block's QKV
     projection (3072 -> 3 x 3072) and the MLP (3072 -> 12288 -> 3072): every column of 64
@@ -69,3 +70,65 @@ def test_repeatable_and_scales_applied():
                 torch.tensor([sa * 2], device="cuda"), torch.tensor([sb], device="cuda"))
     assert qa.get_error() == 0
     assert torch.equal(y2.float(), (y.float() * 2))   # a power of two: exact in bf16
+
+
+def _fused(M, N, K, seed, amax_factor=1.0, with_y=True):
+    """gemm_fp8_e4m3 on seeded codes; amax = amax_factor * max |bf16 y| of the plain GEMM (a
+    static calibration).  Returns (a8, b8, s_a, s_b, y of the plain GEMM, y of the fused call or
+    None, codes, scale, amax)."""
+    a8, b8, sa, sb, y = _run(M, N, K, seed)
+    amax = float(y.float().abs().max().item()) * amax_factor
+    codes = torch.full((M, N), 0x55, dtype=torch.uint8, device="cuda")
+    scale = torch.zeros(1, device="cuda")
+    y2 = torch.full((M, N), float("nan"), dtype=torch.bfloat16, device="cuda") if with_y else None
+    qa.gemm_fp8_e4m3(torch.from_numpy(a8).cuda(), torch.from_numpy(b8).cuda(), codes,
+                     torch.tensor([sa], device="cuda"), torch.tensor([sb], device="cuda"),
+                     torch.tensor([amax], dtype=torch.float32, device="cuda"), scale, y=y2)
+    assert qa.get_error() == 0
+    return a8, b8, sa, sb, y, y2, codes, scale, np.float32(amax)
+
+
+@pytest.mark.parametrize("M,N,K,amax_factor", [(100, 288, 256, 1.0),       # one-SM kernel
+                                               (130, 288, 256, 1.0), (300, 512, 384, 0.5),
+                                               (2560, 2080, 256, 2.0)])    # SM pairs
+def test_fused_e4m3_codes_are_the_quantized_bf16_output(M, N, K, amax_factor):
+    """The codes of gemm_fp8_e4m3 are exactly oracle.quantize_fp8 of the GEMM's own bf16 output
+    under the given amax (also when the amax is below the output's maximum: saturation), the
+    written scale is the oracle's, the bf16 output of the fused call equals the plain GEMM's,
+    and that bf16 output meets the oracle's GEMM bound."""
+    a8, b8, sa, sb, y, y2, codes, scale, amax = _fused(M, N, K, seed=M * 7 + N, amax_factor=amax_factor)
+    assert torch.equal(y2, y)
+    want_codes, want_scale = oracle.quantize_fp8(y.cpu().reshape(-1), float(amax))
+    assert np.array_equal(codes.cpu().numpy().reshape(-1), want_codes)
+    assert np.float32(scale.item()) == want_scale
+    want, bound = oracle.gemm_e4m3(a8, b8, sa, sb)
+    _check(y.float().cpu().numpy(), want, bound, K)
+    # codes only (no bf16 output): the same codes
+    _, _, _, _, _, _, codes2, _, _ = _fused(M, N, K, seed=M * 7 + N, amax_factor=amax_factor, with_y=False)
+    assert torch.equal(codes2, codes)
+
+
+def test_fused_e4m3_value_projection_against_the_oracle_bf16_path():
+    """The value projection of the joint sequence (8704 tokens, 3072 -> 3072): the fused codes
+    equal the quantized GPU bf16 output everywhere, and differ from the quantized oracle bf16
+    output only where the FP32 accumulation order tipped a bf16 rounding (a few in a million)."""
+    M, N, K = 8704, 3072, 3072
+    a8, b8, sa, sb, y, _, codes, scale, amax = _fused(M, N, K, seed=21, with_y=False)
+    want_codes, _ = oracle.quantize_fp8(y.cpu().reshape(-1), float(amax))
+    assert np.array_equal(codes.cpu().numpy().reshape(-1), want_codes)
+    rows = np.unique(np.concatenate([[0, M - 1], np.random.default_rng(2).integers(0, M, 62)]))
+    want, _ = oracle.gemm_e4m3(a8, b8, sa, sb, rows=rows)
+    want_bf16 = torch.from_numpy(want.astype(np.float32)).to(torch.bfloat16)
+    orc_codes, _ = oracle.quantize_fp8(want_bf16.reshape(-1), float(amax))
+    got = codes.cpu().numpy()[rows].reshape(-1)
+    assert np.mean(got != orc_codes) < 1e-4
+
+
+def test_fused_e4m3_nonfinite_amax_writes_no_code():
+    a8, b8, sa, sb, y = _run(130, 288, 256, seed=5)
+    codes = torch.full((130, 288), 0x55, dtype=torch.uint8, device="cuda")
+    qa.gemm_fp8_e4m3(torch.from_numpy(a8).cuda(), torch.from_numpy(b8).cuda(), codes,
+                     torch.tensor([sa], device="cuda"), torch.tensor([sb], device="cuda"),
+                     torch.tensor([float("inf")], device="cuda"), torch.zeros(1, device="cuda"))
+    assert qa.get_error() == qa._lib.ERR_NONFINITE
+    assert bool((codes == 0x55).all())
