@@ -34,13 +34,20 @@ BF16_FALLBACK_TFLOPS = 1590.0
 FP8_PER_BF16 = 2.0          # nominal dense FP8 / BF16 tensor throughput ratio on B200
 L2_FLUSH_BYTES = 256 << 20
 # DRAM bytes (read + write) of one launch of the attention kernel at L=8704 (B=1, H=24, D=128),
-# from ncu on the current kernel:
-#   ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum --clock-control none \
-#       -k regex:k_attn_fp8 -s 3 -c 1 python bench.py --steps 1 --warmup 3 --no-cpu-baseline --no-e2e
-# None until captured for this kernel (re-capture whenever the kernel changes).  Other shapes of
-# the same kernel: scaled by their algorithmic bytes (Q8 + K8 + V8 + bf16 output), and so marked.
-ATTN_TRAFFIC_L8704 = None
+# from ncu on the current kernel (80.30 MB read + 22.40 MB written):
+#   ncu --set full --clock-control none -k regex:k_attn_fp8_pair -s 3 -c 1 -o attn_pair \
+#       python bench.py --steps 1 --warmup 3 --no-cpu-baseline --no-e2e --no-extras
+# Set to None whenever the kernel changes, until captured again.  Other shapes of the same
+# kernel: scaled by their algorithmic bytes (Q8 + K8 + V8 + bf16 output), and so marked.
+ATTN_TRAFFIC_L8704 = 102706432
 ATTN_TRAFFIC_SOURCE = "ncu dram__bytes_read.sum + dram__bytes_write.sum, one launch, L=8704"
+# DRAM bytes (read + write) of one Q, K, V quantize launch at L=8704 (B=1, H=24, D=128), from
+#   ncu --metrics gpu__time_duration.sum,dram__bytes_read.sum,dram__bytes_write.sum,lts__t_sector_hit_rate.pct \
+#       --clock-control none -k regex:"k_quant_qkv|k_calib_quant_qkv" -s 3 -c 1 --csv --log-file q.csv \
+#       python bench.py --steps 1 --warmup 3 --no-cpu-baseline --no-e2e --no-extras [--mode fp4] [--static-scales]
+# keyed by (mode, static scales); None again whenever those kernels change.
+QUANT_TRAFFIC_L8704 = {("fp8", False): 207469312, ("fp8", True): 202917120,
+                       ("fp4", False): 262223104, ("fp4", True): 235917824}
 ATTN_KERNEL = {128: "k_attn_fp8_pair (cluster of two CTAs per pair of Q tiles)", 64: "k_attn_fp8_fwd<64>"}
 
 
@@ -55,6 +62,13 @@ def attn_traffic(w):
         return ATTN_TRAFFIC_L8704, ATTN_TRAFFIC_SOURCE
     return ATTN_TRAFFIC_L8704 * algo / algo_ref, (ATTN_TRAFFIC_SOURCE +
                                                   ", scaled by this workload's algorithmic bytes")
+
+
+def quant_traffic(w, static):
+    """DRAM bytes of the quantize launch per the ncu capture, for the L=8704 shape only."""
+    if w.varlen or (w.L, w.H, w.B, w.D) != (8704, 24, 1, 128):
+        return None
+    return QUANT_TRAFFIC_L8704.get((w.mode, bool(static)))
 
 
 def load_peaks():
@@ -510,6 +524,7 @@ def report(args, w, qkv, rank, world, ms, attn, quant, e2e_ms, clocks, launches,
                 "gbs": quant_bytes / (quant * 1e-3) / 1e9,
                 "frac_hbm": quant_bytes / (quant * 1e-3) / 1e9 / hbm_gbs,
                 "hbm_peak_gbs": hbm_gbs, "launches": 1,
+                "traffic": quant_traffic(w, args.static_scales),
                 "path": ("static scales (qattn_quantize_qkv, one pass)" if args.static_scales
                          else "calibrated every step (qattn_calibrate_quantize_qkv: amax, grid "
                               "barrier, quantize)")}
@@ -517,6 +532,7 @@ def report(args, w, qkv, rank, world, ms, attn, quant, e2e_ms, clocks, launches,
         qs = extra["quant_static_ms"]
         quantize["static"] = {"ms": qs, "gbs": quant_bytes / (qs * 1e-3) / 1e9,
                               "frac_hbm": quant_bytes / (qs * 1e-3) / 1e9 / hbm_gbs,
+                              "traffic": quant_traffic(w, True),
                               "path": "static scales (qattn_quantize_qkv, one pass), the amax "
                                       "calibrated in the timed steps"}
     fp4 = None
@@ -534,8 +550,10 @@ def report(args, w, qkv, rank, world, ms, attn, quant, e2e_ms, clocks, launches,
                             "kernel": ATTN_KERNEL[w4.D]},
                "quantize": {"ms": x["quant_ms"], "algorithmic_bytes": qb4,
                             "frac_hbm": qb4 / (x["quant_ms"] * 1e-3) / 1e9 / hbm_gbs,
+                            "traffic": quant_traffic(w4, False),
                             "static": {"ms": x["quant_static_ms"],
-                                       "frac_hbm": qb4 / (x["quant_static_ms"] * 1e-3) / 1e9 / hbm_gbs}},
+                                       "frac_hbm": qb4 / (x["quant_static_ms"] * 1e-3) / 1e9 / hbm_gbs,
+                                       "traffic": quant_traffic(w4, True)}},
                "fp4_direct_estimate": x.get("fp4_direct")}
     result = {
         "metric": "quantized attention TFLOP/s @L=8704,H=24,D=128 and % of B200 FP8 peak",
