@@ -52,10 +52,23 @@ typedef enum {
   QATTN_ERR_UNSUPPORTED = 2,
   QATTN_ERR_CUDA = 3,
   QATTN_ERR_NONFINITE = 4,
-  QATTN_ERR_TIMEOUT = 5
+  QATTN_ERR_TIMEOUT = 5,
+  /* checked build only (libqattn_checked.so): a kernel found an index outside its buffer and
+   * skipped that access; the results are then incomplete */
+  QATTN_ERR_BOUNDS = 6
 } qattn_status;
 
-typedef enum { QATTN_MODE_FP8 = 0, QATTN_MODE_FP4 = 1 } qattn_mode;
+typedef enum {
+  QATTN_MODE_FP8 = 0,
+  QATTN_MODE_FP4 = 1,
+  /* Debug switch of the attention calls (qattn_forward, _ws, _varlen), OR'ed into the mode: P is
+   * not quantized.  The same codes, scales and FP32 softmax with the integer row maximum M, but
+   * BMM2 takes P in FP32: O = (sum_j p_j val(v_j)) * s_v / l with p_j = 2^fl32(S'_j - M) (the
+   * blog's steps without the fourth SDPA bullet's P quantization), from a plain CUDA-core
+   * kernel, not the tensor-core path: for isolating the error the P codes add.  The workspace
+   * of qattn_forward_ws is not used. */
+  QATTN_FLAG_P_UNQUANTIZED = 0x100
+} qattn_mode;
 
 /* Per-tensor dequantization multipliers of the E4M3 inputs of qattn_forward: value of an
  * element = val(code) * (*s).  All three are device pointers to one float each, as written by
@@ -260,7 +273,8 @@ QATTN_API qattn_status qattn_forward_varlen(const uint8_t* q8, const uint8_t* k8
                                   qattn_stream_t stream);
 
 /* Synchronizes `stream`, then returns and clears the current device's error word: QATTN_OK,
- * QATTN_ERR_NONFINITE or QATTN_ERR_TIMEOUT (or QATTN_ERR_CUDA if the synchronization failed). */
+ * QATTN_ERR_NONFINITE, QATTN_ERR_TIMEOUT or (checked build) QATTN_ERR_BOUNDS (or QATTN_ERR_CUDA
+ * if the synchronization failed). */
 QATTN_API qattn_status qattn_get_error(qattn_stream_t stream);
 
 /* Human-readable name of a status code (static storage). */
@@ -270,6 +284,20 @@ QATTN_API const char* qattn_status_str(qattn_status status);
  * this library returned on the calling host thread, or 0 if none has.  Argument checks and
  * device error words do not change it.  Lets a caller report which CUDA call failed. */
 QATTN_API int qattn_last_cuda_error(void);
+
+/* How this library was built: bit 0 set for the checked build (libqattn_checked.so, compiled
+ * with QATTN_CHECKED), in which every kernel tests the global-memory indices it computes (output
+ * rows, workspace slots, tile and TMA coordinates, element and block indices) against the
+ * extents of its buffers, records QATTN_ERR_BOUNDS in the error word on a miss and skips that
+ * access instead of trapping.  No device needed. */
+QATTN_API int qattn_build_info(void);
+
+/* Test hook of the checked build, not part of the method: with enable != 0 the next
+ * qattn_quantize_fp8 launches run their element loop one 8-element vector past n (as an index
+ * bug would), so the bounds checks must catch the extra vector, record QATTN_ERR_BOUNDS and skip
+ * it; the first n codes are still written.  The normal build has no such switch: there it
+ * returns QATTN_ERR_UNSUPPORTED and changes nothing. */
+QATTN_API qattn_status qattn_debug_inject_oob(int enable);
 
 /* Test hooks, not part of the method.  qattn_debug_set_wait_timeout_ns sets the limit after
  * which a wait inside the attention kernel gives up (default 2 s; 0 restores the default).

@@ -12,10 +12,13 @@ import os
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libqattn.so")
+# QATTN_DEBUG=1 selects the checked build (device bounds checks that record QATTN_ERR_BOUNDS)
+CHECKED = os.environ.get("QATTN_DEBUG") == "1"
+LIB_PATH = os.path.join(_HERE, "libqattn_checked.so" if CHECKED else "libqattn.so")
 
-OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_NONFINITE, ERR_TIMEOUT = range(6)
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_NONFINITE, ERR_TIMEOUT, ERR_BOUNDS = range(7)
 MODE_FP8, MODE_FP4 = 0, 1
+FLAG_P_UNQUANTIZED = 0x100   # OR into the mode of forward(): P stays FP32 (debug path)
 
 # every symbol the header declares
 EXPORTS = (
@@ -27,7 +30,7 @@ EXPORTS = (
     "qattn_status_str", "qattn_last_cuda_error",
     "qattn_forward_workspace_bytes",
     "qattn_debug_set_wait_timeout_ns", "qattn_debug_inject_missing_q", "qattn_debug_capture_p_row",
-    "qattn_debug_attention_plan",
+    "qattn_debug_attention_plan", "qattn_build_info", "qattn_debug_inject_oob",
 )
 _RETURNS_STATUS = EXPORTS[:14]
 FUSED_WORKSPACE_BYTES = 256     # QATTN_FUSED_WORKSPACE_BYTES
@@ -64,7 +67,8 @@ def load() -> ctypes.CDLL:
         return _lib
     if not os.path.exists(LIB_PATH):
         raise ImportError(f"{LIB_PATH} is missing: build it with "
-                          "`python -m precision_quantized_attention_b200.build`")
+                          "`python -m precision_quantized_attention_b200.build"
+                          + (" --checked`" if CHECKED else "`"))
     lib = ctypes.CDLL(LIB_PATH)
     P, S, I, F = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int, ctypes.c_float
     lib.qattn_calibrate_amax.argtypes = [P, S, P, P]
@@ -92,6 +96,10 @@ def load() -> ctypes.CDLL:
     lib.qattn_debug_set_wait_timeout_ns.restype = None
     lib.qattn_debug_inject_missing_q.argtypes = [I]
     lib.qattn_debug_inject_missing_q.restype = None
+    lib.qattn_build_info.argtypes = []
+    lib.qattn_build_info.restype = I
+    lib.qattn_debug_inject_oob.argtypes = [I]
+    lib.qattn_debug_inject_oob.restype = I
     lib.qattn_debug_capture_p_row.argtypes = [I, I, I, P, P]
     lib.qattn_debug_capture_p_row.restype = I
     lib.qattn_debug_attention_plan.argtypes = [I, I, I, I, I, ctypes.POINTER(I),
@@ -342,6 +350,17 @@ def debug_set_wait_timeout_ns(ns: int):
 
 def debug_inject_missing_q(enable: bool):
     load().qattn_debug_inject_missing_q(1 if enable else 0)
+
+
+def build_info() -> int:
+    """Bit 0: the loaded library is the checked build (QATTN_DEBUG=1)."""
+    return int(load().qattn_build_info())
+
+
+def debug_inject_oob(enable: bool):
+    """Checked build only: the next quantize_fp8 launches loop one 8-element vector past n, which
+    the device bounds checks must stop (QATTN_ERR_BOUNDS).  Raises QattnError in the normal build."""
+    _check(load().qattn_debug_inject_oob(1 if enable else 0), "qattn_debug_inject_oob")
 
 
 def debug_capture_p_row(enable: bool, slab: int = 0, row: int = 0, codes: torch.Tensor = None,

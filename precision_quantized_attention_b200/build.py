@@ -1,6 +1,10 @@
-"""Builds libqattn.so in-tree with nvcc for sm_100a (no GPU needed to compile).
+"""Builds libqattn.so in-tree with nvcc for sm_100a (no GPU needed to compile), and with
+``--checked`` (or QATTN_DEBUG=1 in the environment) also the checked build libqattn_checked.so:
+the same sources compiled with QATTN_CHECKED, whose kernels test the global-memory indices they
+compute against their buffers' extents and record QATTN_ERR_BOUNDS instead of trapping.  The
+binding loads the checked library when QATTN_DEBUG=1 is set.
 
-    python -m precision_quantized_attention_b200.build
+    python -m precision_quantized_attention_b200.build [--checked] [-v]
 """
 from __future__ import annotations
 
@@ -12,7 +16,9 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(os.path.dirname(HERE), "include")
 LIB = os.path.join(HERE, "libqattn.so")
-SOURCES = ["qattn_api.cu", "quant.cu", "attn_fwd.cu", "attn_pair.cu", "noalloc.cu", "gemm_fp8.cu"]
+LIB_CHECKED = os.path.join(HERE, "libqattn_checked.so")
+SOURCES = ["qattn_api.cu", "quant.cu", "attn_fwd.cu", "attn_pair.cu", "attn_debug.cu", "noalloc.cu",
+           "gemm_fp8.cu"]
 HEADERS = ["sm100_ptx.cuh", "softmax_sm100.cuh", "launch.h", "device_once.h", "quant_math.cuh"]
 
 
@@ -30,24 +36,29 @@ def flags(verbose_ptxas: bool = False) -> list[str]:
     return f
 
 
-def _stale() -> bool:
-    if not os.path.exists(LIB):
+def _stale(lib: str) -> bool:
+    if not os.path.exists(lib):
         return True
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     deps = [os.path.join(CSRC, s) for s in SOURCES + HEADERS] + [os.path.join(INCLUDE, "qattn.h")]
     return any(os.path.getmtime(p) > t for p in deps)
 
 
-def build(force: bool = False, verbose_ptxas: bool = False) -> str:
-    if not force and not _stale():
-        return LIB
-    tmp = LIB + f".tmp{os.getpid()}"
-    cmd = [nvcc(), *flags(verbose_ptxas), "-shared", "-o", tmp,
-           *[os.path.join(CSRC, s) for s in SOURCES]]
+def build(force: bool = False, verbose_ptxas: bool = False, checked: bool = False) -> str:
+    """Builds libqattn.so (checked=False) or libqattn_checked.so (checked=True) if stale."""
+    lib = LIB_CHECKED if checked else LIB
+    if not force and not _stale(lib):
+        return lib
+    tmp = lib + f".tmp{os.getpid()}"
+    cmd = [nvcc(), *flags(verbose_ptxas), *(["-DQATTN_CHECKED"] if checked else []), "-shared",
+           "-o", tmp, *[os.path.join(CSRC, s) for s in SOURCES]]
     subprocess.check_call(cmd)
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, lib)
+    return lib
 
 
 if __name__ == "__main__":
-    print(build(force=True, verbose_ptxas="-v" in sys.argv))
+    v = "-v" in sys.argv
+    print(build(force=True, verbose_ptxas=v))
+    if "--checked" in sys.argv or os.environ.get("QATTN_DEBUG") == "1":
+        print(build(force=True, verbose_ptxas=v, checked=True))

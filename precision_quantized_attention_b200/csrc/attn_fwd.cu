@@ -100,6 +100,10 @@ struct AttnArgs {
   int tail_w;               // tail key steps per CTA, 1..nkv (nkv: no pair is cut)
   float* part_o;
   float2* part_ml;
+  // extents for the checked build's index tests: slabs of the tensors (the output has
+  // slabs * rows_per_slab rows) and rows of partial results the workspace holds
+  int slabs;
+  long long part_rows;
 };
 
 // One unit of a CTA's work: key steps [kv0, kv1) of one pair of Q tiles.
@@ -253,6 +257,9 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
         if (nk >= KSTAGES &&
             !mbar_wait(BAR(B_KEMPTY + s), ((nk / KSTAGES) - 1) & 1, tlim, abort_flag, args.err))
           return false;
+        // a tile starting past the sequence would load zeros: an index error (recorded; the
+        // load itself stays in the tensor map's bounds checking)
+        (void)QATTN_IN_BOUNDS(args.err, kv * BLOCK_N < sg.seq_len);
         mbar_arrive_expect_tx(BAR(B_KFULL + s), SL::TILE_KV);
         tma_load_3d(base_u32 + SL::OFF_K + s * SL::TILE_KV, &tm_k, BAR(B_KFULL + s), 0,
                     sg.seq_start + kv * BLOCK_N, sg.slab);
@@ -264,6 +271,7 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
         if (nv >= VSTAGES &&
             !mbar_wait(BAR(B_VEMPTY + s), ((nv / VSTAGES) - 1) & 1, tlim, abort_flag, args.err))
           return false;
+        (void)QATTN_IN_BOUNDS(args.err, kv * BLOCK_N < sg.seq_len);
         mbar_arrive_expect_tx(BAR(B_VFULL + s), SL::TILE_KV);
         tma_load_3d(base_u32 + SL::OFF_V + s * SL::TILE_KV, &tm_v, BAR(B_VFULL + s), 0,
                     sg.seq_start + kv * BLOCK_N, sg.slab);
@@ -276,6 +284,8 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
         const int b = i & 1;
         if (i >= 2 && !mbar_wait(BAR(B_QEMPTY + b), ((i >> 1) - 1) & 1, tlim, abort_flag, args.err))
           break;
+        (void)QATTN_IN_BOUNDS(args.err, sg.q_row0 < sg.seq_len && sg.slab < args.slabs &&
+                                            sg.seq_start + sg.seq_len <= args.rows_per_slab);
         mbar_arrive_expect_tx(BAR(B_QFULL + b), NQ * SL::TILE_Q);
         for (int t = 0; t < NQ; ++t)
           tma_load_3d(base_u32 + SL::OFF_Q + (b * NQ + t) * SL::TILE_Q, &tm_q, BAR(B_QFULL + b), 0,
@@ -504,7 +514,8 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
         const int row = sg.q_row0 + t * BLOCK_M + r;
         const bool valid = row < sg.seq_len;
         const float f_ref = exp2_int(static_cast<int>(m_ref - m_run));   // O relative to m_run
-        if (sg.slot >= 0) {
+        if (sg.slot >= 0 && QATTN_IN_BOUNDS(args.err, (static_cast<long long>(sg.slot) * NQ + t + 1) *
+                                                          BLOCK_M <= args.part_rows)) {
           // partial result of this segment: raw O row, running max and row sum
           const size_t slot = static_cast<size_t>(sg.slot) * NQ + t;
           float4* po = reinterpret_cast<float4*>(args.part_o + (slot * BLOCK_M + r) * D);
@@ -519,7 +530,7 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
                                            __uint_as_float(v[4 * i + 2]) * f_ref, __uint_as_float(v[4 * i + 3]) * f_ref);
           }
           args.part_ml[slot * BLOCK_M + r] = make_float2(m_run, l);
-        } else {
+        } else if (sg.slot < 0) {
         const float scale = __ldg(args.s_v) / l * f_ref;   // O = acc * s_v / 448 / (l / 448)
         __nv_bfloat16* orow =
             args.out + (static_cast<size_t>(sg.slab) * args.rows_per_slab + sg.seq_start + row) * D;
@@ -535,7 +546,8 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
                                                             __uint_as_float(v[2 * i + 1]) * scale);
             packed[i] = *reinterpret_cast<const uint32_t*>(&b2);
           }
-          if (valid) {
+          if (valid && QATTN_IN_BOUNDS(args.err, static_cast<long long>(sg.slab) * args.rows_per_slab +
+                                                     sg.seq_start + row < static_cast<long long>(args.slabs) * args.rows_per_slab)) {
             uint4* dst = reinterpret_cast<uint4*>(orow + c4 * 32);
 #pragma unroll
             for (int i = 0; i < 4; ++i)
@@ -593,6 +605,10 @@ __global__ void __launch_bounds__(COMBINE_WARPS * 32) k_attn_combine(const AttnA
   auto slot = [&](int c) {
     return static_cast<size_t>(2 * c + (c * W < g0 ? 1 : 0)) * NQ + t;
   };
+  if (!QATTN_IN_BOUNDS(args.err, c_first >= 0 && c_last < args.ctas &&
+                                     static_cast<long long>(slot(c_last) + 1) * BLOCK_M <= args.part_rows &&
+                                     static_cast<long long>(bz * args.H + h) < args.slabs))
+    return;
   float M = -INFINITY;
   for (int c = c_first; c <= c_last; ++c) M = fmaxf(M, args.part_ml[slot(c) * BLOCK_M + r].x);
   float l = 0.0f;
@@ -752,6 +768,7 @@ cudaError_t launch_attention(const uint8_t* q8, const uint8_t* k8, const uint8_t
   a.inject_missing_q = dbg.inject_missing_q;
   a.part_o = nullptr;
   a.part_ml = nullptr;
+  a.part_rows = 0;
   a.pairs_per_head = 0;
   a.nkv = 0;
   a.ctas = 0;
@@ -759,6 +776,7 @@ cudaError_t launch_attention(const uint8_t* q8, const uint8_t* k8, const uint8_t
   a.tail_pairs = 0;
   a.tail_w = 1;
   const int slabs = varlen ? H : B * H;
+  a.slabs = slabs;
   dim3 grid;
   int combine_ctas = 0;
   AttnSplitPlan p{};
@@ -780,6 +798,7 @@ cudaError_t launch_attention(const uint8_t* q8, const uint8_t* k8, const uint8_t
       const size_t o_elems = static_cast<size_t>(2) * p.ctas * NQ * BLOCK_M * D;
       a.part_o = static_cast<float*>(workspace);
       a.part_ml = reinterpret_cast<float2*>(a.part_o + o_elems);
+      a.part_rows = static_cast<long long>(2) * p.ctas * NQ * BLOCK_M;
       combine_ctas = p.tail_pairs * NQ * BLOCK_M / COMBINE_WARPS;
     }
     grid = dim3(p.ctas, 1, 1);

@@ -135,6 +135,11 @@ struct PairArgs {
   int tail_w;
   float* part_o;
   float2* part_ml;
+  // extents for the checked build's index tests: slabs of the tensors, rows of partial results
+  // the workspace holds, key steps the P-capture buffers hold
+  int slabs;
+  long long part_rows;
+  int dbg_steps;
 };
 
 namespace {
@@ -221,6 +226,7 @@ struct StepCursor {
 // maximum, to the caller's buffers.
 __device__ __forceinline__ void capture_p_row(const PairArgs& args, int step, const uint32_t (&pk)[32],
                                            float mx) {
+  if (!QATTN_IN_BOUNDS(args.err, step < args.dbg_steps)) return;
   uint4* dst = reinterpret_cast<uint4*>(args.dbg_p + static_cast<size_t>(step) * pairk::BLOCK_N);
 #pragma unroll
   for (int i = 0; i < 8; ++i) dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
@@ -252,6 +258,9 @@ __device__ __noinline__ void pair_epilogue(const PairArgs& args, const PSeg& sg,
   constexpr int D = pairk::D;
   const int row = sg.q_row0 + rank * pairk::BLOCK_M + r;
   if (sg.slot >= 0) {
+    if (!QATTN_IN_BOUNDS(args.err, (static_cast<long long>(sg.slot) * 2 + rank + 1) * pairk::BLOCK_M <=
+                                       args.part_rows))
+      return;
     const size_t slot = static_cast<size_t>(sg.slot) * 2 + rank;
     float4* po = reinterpret_cast<float4*>(args.part_o + (slot * pairk::BLOCK_M + r) * D);
 #pragma unroll 1
@@ -267,7 +276,10 @@ __device__ __noinline__ void pair_epilogue(const PairArgs& args, const PSeg& sg,
     args.part_ml[slot * pairk::BLOCK_M + r] = make_float2(m_fin, l_tot);
     return;
   }
-  const bool valid = row < sg.seq_len;
+  const bool valid = row < sg.seq_len &&
+                     QATTN_IN_BOUNDS(args.err, static_cast<long long>(sg.slab) * args.rows_per_slab +
+                                                   sg.seq_start + row <
+                                               static_cast<long long>(args.slabs) * args.rows_per_slab);
   const float scale = __ldg(args.s_v) / l_tot * f_ref;   // O = acc * s_v / 448 / (l / 448)
   __nv_bfloat16* orow =
       args.out + (static_cast<size_t>(sg.slab) * args.rows_per_slab + sg.seq_start + row) * D;
@@ -358,7 +370,12 @@ __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(168)
       StepCursor lc;
       lc.start(args);
       while (ok && lc.valid) {
+        // tiles starting past the sequence would load zeros: index errors (recorded; the loads
+        // themselves stay in the tensor maps' bounds checking)
+        (void)QATTN_IN_BOUNDS(args.err, (lc.sg.kv0 + lc.j) * BLOCK_N < lc.sg.seq_len);
         if (lc.j == 0) {
+          (void)QATTN_IN_BOUNDS(args.err, lc.sg.q_row0 < lc.sg.seq_len && lc.sg.slab < args.slabs &&
+                                              lc.sg.seq_start + lc.sg.seq_len <= args.rows_per_slab);
           const int i = lc.seg, b = i & 1;
           if (i >= 2 && !mbar_wait(BAR(B_QEMPTY + b), ((i >> 1) - 1) & 1, tlim, abort_flag, args.err)) {
             ok = false;
@@ -744,6 +761,9 @@ cudaError_t launch_attention_pair(const uint8_t* q8, const uint8_t* k8, const ui
   a.tail_w = plan ? plan->tail_w : 1;
   a.part_o = nullptr;
   a.part_ml = nullptr;
+  a.slabs = slabs;
+  a.part_rows = 0;
+  a.dbg_steps = ((cu_seqlens ? max_seqlen : L) + BLOCK_N - 1) / BLOCK_N;
   dim3 grid;
   if (cu_seqlens) {
     grid = dim3(2 * ((max_seqlen + 2 * BLOCK_M - 1) / (2 * BLOCK_M)), H, nseq);
@@ -752,6 +772,7 @@ cudaError_t launch_attention_pair(const uint8_t* q8, const uint8_t* k8, const ui
       const size_t o_elems = static_cast<size_t>(2) * plan->ctas * 2 * BLOCK_M * D;
       a.part_o = static_cast<float*>(workspace);
       a.part_ml = reinterpret_cast<float2*>(a.part_o + o_elems);
+      a.part_rows = static_cast<long long>(2) * plan->ctas * 2 * BLOCK_M;
     }
     grid = dim3(2 * plan->ctas, 1, 1);
   }

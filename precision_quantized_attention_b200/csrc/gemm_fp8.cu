@@ -96,6 +96,7 @@ __device__ __forceinline__ CodeScale code_scale(const GemmArgs& a) {
 // requested, their E4M3 codes (the bf16 values quantized exactly as qattn_quantize_fp8 would).
 __device__ __forceinline__ void epilogue32(const GemmArgs& a, const CodeScale& cs, const uint32_t (&v)[32],
                                            float scale, size_t off) {
+  if (!QATTN_IN_BOUNDS(a.err, off + 32 <= static_cast<size_t>(a.M) * a.N)) return;
   uint32_t packed[16];
 #pragma unroll
   for (int e = 0; e < 16; ++e) {
@@ -172,6 +173,8 @@ __global__ void __launch_bounds__(gemm::THREADS, 1)
       bool ok = true;
       for (int t = blockIdx.x; ok && t < tiles; t += gridDim.x) {
         const int m0 = (t % tiles_m) * BM, n0 = (t / tiles_m) * BN;
+        // a tile starting past the output would be computed from zero fill: an index error
+        (void)QATTN_IN_BOUNDS(args.err, m0 < args.M && n0 < args.N);
         for (int kb = 0; kb < kblocks; ++kb, ++u) {
           const int s = u % STAGES;
           if (u >= STAGES &&
@@ -352,6 +355,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(gemm2::THREADS, 1)
       for (int t = pair; ok && t < tiles; t += npairs) {
         const int m0 = (t % tiles_m) * BM + static_cast<int>(rank) * (BM / 2);
         const int n0 = (t / tiles_m) * BN + static_cast<int>(rank) * (BN / 2);
+        // the pair's tile must start inside the output (a CTA's half may lie past it: zero fill)
+        (void)QATTN_IN_BOUNDS(args.err, (t % tiles_m) * BM < args.M && (t / tiles_m) * BN < args.N);
         for (int kb = 0; kb < kblocks; ++kb, ++u) {
           const int s = u % STAGES;
           if (u >= STAGES &&

@@ -12,7 +12,8 @@ namespace qattn {
 cudaError_t launch_amax(const void* x, size_t n, float* amax, int* err, int num_sms,
                         cudaStream_t stream);
 cudaError_t launch_quant_fp8(const void* x, size_t n, const float* amax, uint8_t* out,
-                             float* scale, int* err, int num_sms, cudaStream_t stream);
+                             float* scale, int* err, int num_sms, cudaStream_t stream,
+                             int inject_oob = 0);
 cudaError_t launch_quant_fp4_block(const void* x, size_t n, const float* amax, uint8_t* packed,
                                    uint8_t* bscale, float* gscale, uint8_t* codes8, float* scale8,
                                    int* err, int num_sms, cudaStream_t stream);
@@ -49,11 +50,20 @@ cudaError_t launch_gemm_fp8(const uint8_t* a8, const uint8_t* b8, void* y, int M
 // tile maximum into p_maxima[step].
 struct DebugHooks {
   int inject_missing_q = 0;
+  int inject_oob = 0;              // checked build only: qattn_quantize_fp8 loops one vector past n
   uint8_t* p_codes = nullptr;
   int* p_maxima = nullptr;
   int p_slab = -1;
   int p_row = -1;
 };
+
+// The attention with P left unquantized (QATTN_FLAG_P_UNQUANTIZED, a debug path; attn_debug.cu):
+// dense (cu_seqlens == nullptr: B, H, L) or varlen (cu_seqlens, nseq, max_seqlen, total_tokens, H).
+cudaError_t launch_attention_p_unquantized(const uint8_t* q8, const uint8_t* k8, const uint8_t* v8,
+                                           void* out, int B, int H, int L, int D,
+                                           const int* cu_seqlens, int nseq, int max_seqlen,
+                                           int total_tokens, const float* s_q, const float* s_k,
+                                           const float* s_v, float sm_scale, cudaStream_t stream);
 
 // Persistent schedule of a dense attention launch (see plan_attention_split in attn_fwd.cu):
 // ctas CTAs, `whole` whole pairs each, then tail ranges of tail_w key steps; bytes = workspace

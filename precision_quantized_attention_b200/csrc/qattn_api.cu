@@ -75,8 +75,13 @@ qattn_status check_attention_common(const uint8_t* q8, const uint8_t* k8, const 
     return QATTN_ERR_INVALID_ARG;
   if (H < 1 || !(sm_scale > 0.0f) || !(sm_scale < 3.0e38f)) return QATTN_ERR_INVALID_ARG;
   if (D != 64 && D != 128) return QATTN_ERR_UNSUPPORTED;
-  if (mode != QATTN_MODE_FP8 && mode != QATTN_MODE_FP4) return QATTN_ERR_INVALID_ARG;
+  const int base = static_cast<int>(mode) & ~static_cast<int>(QATTN_FLAG_P_UNQUANTIZED);
+  if (base != QATTN_MODE_FP8 && base != QATTN_MODE_FP4) return QATTN_ERR_INVALID_ARG;
   return QATTN_OK;
+}
+
+bool p_unquantized(qattn_mode mode) {
+  return (static_cast<int>(mode) & static_cast<int>(QATTN_FLAG_P_UNQUANTIZED)) != 0;
 }
 
 }  // namespace
@@ -104,7 +109,8 @@ qattn_status qattn_quantize_fp8(const void* x_bf16, size_t n, const float* amax_
   qattn_status st = device_info(&d);
   if (st != QATTN_OK) return st;
   return from_cuda(qattn::launch_quant_fp8(x_bf16, n, amax_dev, out_e4m3, scale_dev, d->err,
-                                           d->num_sms, reinterpret_cast<cudaStream_t>(stream)));
+                                           d->num_sms, reinterpret_cast<cudaStream_t>(stream),
+                                           g_dbg.inject_oob));
 }
 
 qattn_status qattn_quantize_fp4_block(const void* x_bf16, size_t n, const float* amax_dev,
@@ -292,6 +298,12 @@ qattn_status qattn_forward_ws(const uint8_t* q8, const uint8_t* k8, const uint8_
   if (workspace_dev != nullptr &&
       workspace_bytes < qattn::attention_plan(B, H, L, D, d->num_sms).bytes)
     return QATTN_ERR_INVALID_ARG;
+  if (p_unquantized(mode)) {
+    if (static_cast<int64_t>(B) * H > 65535) return QATTN_ERR_UNSUPPORTED;
+    return from_cuda(qattn::launch_attention_p_unquantized(
+        q8, k8, v8, out_bf16, B, H, L, D, nullptr, 0, L, L, scales->s_q, scales->s_k, scales->s_v,
+        sm_scale, reinterpret_cast<cudaStream_t>(stream)));
+  }
   return from_cuda(qattn::launch_attention(q8, k8, v8, out_bf16, B, H, L, D, nullptr, 0, L, L,
                                            scales->s_q, scales->s_k, scales->s_v, sm_scale,
                                            d->err, g_timeout_ns, g_dbg,
@@ -328,6 +340,10 @@ qattn_status qattn_forward_varlen(const uint8_t* q8, const uint8_t* k8, const ui
   DeviceInfo* d = nullptr;
   st = device_info(&d);
   if (st != QATTN_OK) return st;
+  if (p_unquantized(mode))
+    return from_cuda(qattn::launch_attention_p_unquantized(
+        q8, k8, v8, out_bf16, 1, H, 0, D, cu_seqlens_dev, nseq, max_seqlen, total_tokens,
+        scales->s_q, scales->s_k, scales->s_v, sm_scale, reinterpret_cast<cudaStream_t>(stream)));
   return from_cuda(qattn::launch_attention(q8, k8, v8, out_bf16, 1, H, 0, D, cu_seqlens_dev,
                                            nseq, max_seqlen, total_tokens, scales->s_q,
                                            scales->s_k, scales->s_v, sm_scale, d->err,
@@ -352,6 +368,7 @@ qattn_status qattn_get_error(qattn_stream_t stream) {
     case 0: return QATTN_OK;
     case qattn::DEV_ERR_NONFINITE: return QATTN_ERR_NONFINITE;
     case qattn::DEV_ERR_TIMEOUT: return QATTN_ERR_TIMEOUT;
+    case qattn::DEV_ERR_BOUNDS: return QATTN_ERR_BOUNDS;
     default: return QATTN_ERR_CUDA;
   }
 }
@@ -366,6 +383,7 @@ const char* qattn_status_str(qattn_status status) {
     case QATTN_ERR_CUDA: return "QATTN_ERR_CUDA";
     case QATTN_ERR_NONFINITE: return "QATTN_ERR_NONFINITE";
     case QATTN_ERR_TIMEOUT: return "QATTN_ERR_TIMEOUT";
+    case QATTN_ERR_BOUNDS: return "QATTN_ERR_BOUNDS";
   }
   return "QATTN_ERR_UNKNOWN";
 }
@@ -375,6 +393,24 @@ void qattn_debug_set_wait_timeout_ns(uint64_t ns) {
 }
 
 void qattn_debug_inject_missing_q(int enable) { g_dbg.inject_missing_q = enable ? 1 : 0; }
+
+int qattn_build_info(void) {
+#ifdef QATTN_CHECKED
+  return 1;
+#else
+  return 0;
+#endif
+}
+
+qattn_status qattn_debug_inject_oob(int enable) {
+#ifdef QATTN_CHECKED
+  g_dbg.inject_oob = enable ? 1 : 0;
+  return QATTN_OK;
+#else
+  (void)enable;
+  return QATTN_ERR_UNSUPPORTED;
+#endif
+}
 
 qattn_status qattn_debug_capture_p_row(int enable, int slab, int row, uint8_t* codes_dev,
                                        int* maxima_dev) {

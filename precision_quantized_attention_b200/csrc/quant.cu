@@ -72,7 +72,10 @@ __global__ void __launch_bounds__(256) k_amax_bf16(const uint4* __restrict__ xv,
   }
 }
 
+// nloop: the element loop's bound in 8-element vectors, nvec except under the checked build's
+// injection test (nvec + 1), where the bounds checks must stop the extra vector.
 __global__ void __launch_bounds__(256) k_quant_fp8(const uint4* __restrict__ xv, size_t nvec,
+                                                   size_t nloop,
                                                    const uint16_t* __restrict__ xtail, int ntail,
                                                    const float* __restrict__ amax_p,
                                                    uint2* __restrict__ outv,
@@ -90,12 +93,14 @@ __global__ void __launch_bounds__(256) k_quant_fp8(const uint4* __restrict__ xv,
   const size_t stride = static_cast<size_t>(gridDim.x) * blockDim.x;
   const size_t i0 = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (markstein_ok(s)) {
-    for (size_t i = i0; i < nvec; i += stride) {
+    for (size_t i = i0; i < nloop; i += stride) {
+      if (!QATTN_IN_BOUNDS(err, i < nvec)) continue;
       const uint4 a = __ldcs(xv + i);
       __stcs(outv + i, make_uint2(quant4_e4m3<true>(a.x, a.y, s, r), quant4_e4m3<true>(a.z, a.w, s, r)));
     }
   } else {
-    for (size_t i = i0; i < nvec; i += stride) {
+    for (size_t i = i0; i < nloop; i += stride) {
+      if (!QATTN_IN_BOUNDS(err, i < nvec)) continue;
       const uint4 a = __ldcs(xv + i);
       __stcs(outv + i, make_uint2(quant4_e4m3<false>(a.x, a.y, s, r), quant4_e4m3<false>(a.z, a.w, s, r)));
     }
@@ -188,8 +193,13 @@ __device__ __forceinline__ void fp4_block(uint4 a0, uint4 a1, size_t b, float si
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
       const float x0 = bf16_lo(w[i]), x1 = bf16_hi(w[i]);
-      const float q0 = fast_eff ? div_rn_by(x0, eff, r_eff) : __fdiv_rn(x0, eff);
-      const float q1 = fast_eff ? div_rn_by(x1, eff, r_eff) : __fdiv_rn(x1, eff);
+      float q0, q1;
+      if (fast_eff) {
+        div2_rn_by(x0, x1, eff, r_eff, q0, q1);
+      } else {
+        q0 = __fdiv_rn(x0, eff);
+        q1 = __fdiv_rn(x1, eff);
+      }
       const uint32_t byte = cvt_e2m1x2(q0, q1);
       if (i < 4) pk0 |= byte << (8 * i);
       else pk1 |= byte << (8 * (i - 4));
@@ -832,12 +842,16 @@ cudaError_t launch_amax(const void* x, size_t n, float* amax, int* err, int num_
 }
 
 cudaError_t launch_quant_fp8(const void* x, size_t n, const float* amax, uint8_t* out,
-                             float* scale, int* err, int num_sms, cudaStream_t stream) {
+                             float* scale, int* err, int num_sms, cudaStream_t stream,
+                             int inject_oob) {
   const size_t nvec = n / 8;
   const int ntail = static_cast<int>(n - nvec * 8);
   const uint16_t* xs = static_cast<const uint16_t*>(x);
+#ifndef QATTN_CHECKED
+  inject_oob = 0;                  // only the checked build can stop the extra vector
+#endif
   k_quant_fp8<<<grid_for(nvec, num_sms), 256, 0, stream>>>(
-      static_cast<const uint4*>(x), nvec, xs + nvec * 8, ntail, amax,
+      static_cast<const uint4*>(x), nvec, nvec + (inject_oob ? 1 : 0), xs + nvec * 8, ntail, amax,
       reinterpret_cast<uint2*>(out), out + nvec * 8, scale, err);
   return cudaGetLastError();
 }

@@ -31,6 +31,26 @@ __device__ __forceinline__ float div_rn_by(float x, float s, float r) {
   return copysignf(__fmaf_rn(e, r, q0), x);
 }
 
+// Two quotients at once with packed f32x2 arithmetic: lane by lane the operations and roundings
+// of div_rn_by (q0 = RN(x r), e = RN(x - q0 s) exact, RN(q0 + e r)), so the results are
+// identical, in three instructions for two elements.  Used by the FP4 block quantize, whose
+// per-element quotients dominate its instruction count.
+__device__ __forceinline__ void div2_rn_by(float x0, float x1, float s, float r, float& q0, float& q1) {
+  float a, b;
+  asm("{\n\t.reg .b64 x, q, e, rr, ns;\n\t"
+      "mov.b64 x, {%2, %3};\n\t"
+      "mov.b64 rr, {%4, %4};\n\t"
+      "mov.b64 ns, {%5, %5};\n\t"
+      "mul.rn.f32x2 q, x, rr;\n\t"
+      "fma.rn.f32x2 e, q, ns, x;\n\t"
+      "fma.rn.f32x2 q, e, rr, q;\n\t"
+      "mov.b64 {%0, %1}, q;\n\t}"
+      : "=f"(a), "=f"(b)
+      : "f"(x0), "f"(x1), "f"(r), "f"(-s));
+  q0 = copysignf(a, x0);
+  q1 = copysignf(b, x1);
+}
+
 // -------------------------------------------------------------------------------------------
 // Per-tensor FP8: s = fl32(amax / 448), code = e4m3(fl32(x / s)); amax == 0 gives s = 1.
 // -------------------------------------------------------------------------------------------

@@ -11,7 +11,22 @@ namespace qattn {
 // ----------------------------------------------------------------------------------------------
 // Error word shared by every kernel of the library (one per device, cleared by the host).
 // ----------------------------------------------------------------------------------------------
-enum : int { DEV_OK = 0, DEV_ERR_NONFINITE = 4, DEV_ERR_TIMEOUT = 5 };
+enum : int { DEV_OK = 0, DEV_ERR_NONFINITE = 4, DEV_ERR_TIMEOUT = 5, DEV_ERR_BOUNDS = 6 };
+
+// Checked build (compiled with QATTN_CHECKED: libqattn_checked.so, loaded under QATTN_DEBUG=1):
+// QATTN_IN_BOUNDS(err, cond) tests that an index a kernel is about to use lies inside its
+// buffer; if not, it records DEV_ERR_BOUNDS in the error word and yields false, and the caller
+// skips the access (no trap, the context stays usable).  In the normal build it is `true`, the
+// condition is not evaluated, and nothing is compiled in.
+#ifdef QATTN_CHECKED
+__device__ __forceinline__ bool qattn_bounds_failed(int* err) {
+  atomicExch(err, DEV_ERR_BOUNDS);
+  return false;
+}
+#define QATTN_IN_BOUNDS(err, cond) ((cond) ? true : ::qattn::qattn_bounds_failed(err))
+#else
+#define QATTN_IN_BOUNDS(err, cond) true
+#endif
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));

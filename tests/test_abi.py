@@ -159,3 +159,44 @@ def test_gemm_e4m3_argument_errors():
                {"amax": None}, {"scale": None}, {"codes": MISALIGNED}, {"y": MISALIGNED},
                {"amax": ctypes.c_void_p(0x10002)}, {"M": 0}, {"N": 48}, {"K": 200}):
         assert call(**kw) == _lib.ERR_INVALID_ARG, kw
+
+
+def test_checked_build_exports_the_same_symbols_and_says_so():
+    """libqattn_checked.so (QATTN_DEBUG=1) is the same C ABI compiled with device bounds checks:
+    it exports every declared symbol, reports bit 0 in qattn_build_info, accepts the overrun
+    injection and names QATTN_ERR_BOUNDS; the normal build reports 0 and refuses the injection."""
+    from precision_quantized_attention_b200 import build
+    path = build.build(checked=True)             # a no-op when it is up to date
+    checked = ctypes.CDLL(path)
+    for name in _declared():
+        assert hasattr(checked, name), name
+    checked.qattn_status_str.restype = ctypes.c_char_p
+    assert checked.qattn_build_info() == 1
+    assert checked.qattn_debug_inject_oob(0) == _lib.OK
+    assert checked.qattn_status_str(_lib.ERR_BOUNDS) == b"QATTN_ERR_BOUNDS"
+    normal = _lib.load()
+    if not _lib.CHECKED:
+        assert normal.qattn_build_info() == 0
+        assert normal.qattn_debug_inject_oob(1) == _lib.ERR_UNSUPPORTED
+
+
+def test_p_unquantized_flag_is_validated_on_the_host():
+    """QATTN_FLAG_P_UNQUANTIZED combines with either mode; other high bits are refused, and the
+    flag's own limit (B * H grid rows <= 65535) is checked on the host."""
+    lib = _lib.load()
+    s0 = ctypes.c_void_p(0)
+    sc = _lib._Scales(0x10000, 0x10000, 0x10000)
+    fwd = lib.qattn_forward
+    flag = _lib.FLAG_P_UNQUANTIZED
+    assert fwd(FAKE, FAKE, FAKE, FAKE, 1, 1, 16, 64, ctypes.byref(sc), 0.1, 0x200, s0) == _lib.ERR_INVALID_ARG
+    assert fwd(FAKE, FAKE, FAKE, FAKE, 1, 1, 16, 64, ctypes.byref(sc), 0.1, flag | 2, s0) == _lib.ERR_INVALID_ARG
+    assert fwd(FAKE, FAKE, FAKE, FAKE, 1, 1, 0, 64, ctypes.byref(sc), 0.1, flag, s0) == _lib.ERR_INVALID_ARG
+    assert fwd(FAKE, FAKE, FAKE, FAKE, 1, 1, 16, 96, ctypes.byref(sc), 0.1, flag | 1, s0) == _lib.ERR_UNSUPPORTED
+    if not _gpu():
+        return
+    assert fwd(FAKE, FAKE, FAKE, FAKE, 300, 300, 16, 64, ctypes.byref(sc), 0.1, flag, s0) == _lib.ERR_UNSUPPORTED
+
+
+def _gpu():
+    import torch
+    return torch.cuda.is_available()

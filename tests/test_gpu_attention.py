@@ -242,3 +242,43 @@ def test_large_and_staggered_rises_of_the_row_max():
     got = path.out.float().cpu().numpy()
     rel, mx = assert_close(got, oracle_path(w, q, k, v), "staggered rises")
     print(f"staggered rises: rel-L2 {rel:.2e} max-abs {mx:.2e}")
+
+
+def _p_unquantized(path, w):
+    """The debug switch: the same codes and scales through the attention with P left FP32."""
+    out = torch.empty_like(path.out)
+    s = path.scale
+    mode = (qa.MODE_FP8 if w.mode == "fp8" else qa.MODE_FP4) | qa._lib.FLAG_P_UNQUANTIZED
+    if w.varlen:
+        qa.forward_varlen(path.codes[0], path.codes[1], path.codes[2], out, path.cu,
+                          path.max_seqlen, s[0:1], s[1:2], s[2:3], w.sm_scale, mode)
+    else:
+        qa.forward(path.codes[0], path.codes[1], path.codes[2], out, s[0:1], s[1:2], s[2:3],
+                   w.sm_scale, mode)
+    assert qa.get_error() == 0
+    return out.float().cpu().numpy().reshape(-1, w.D)
+
+
+@pytest.mark.parametrize("name,mode,B,H,L,D,lens", [
+    ("dense300", "fp8", 2, 3, 300, 128, None), ("dense129_d64", "fp8", 1, 2, 129, 64, None),
+    ("dense1000_fp4", "fp4", 1, 2, 1000, 128, None), ("varlen", "fp8", None, 3, None, 128, [1, 200, 129])])
+def test_p_unquantized_switch_matches_the_oracle_without_p_quantization(name, mode, B, H, L, D, lens):
+    """QATTN_FLAG_P_UNQUANTIZED runs the method with P left in FP32; it must equal the oracle's
+    FP32-softmax attention without P quantization (flag FP32 only) on the same codes and scales,
+    within the bf16 rounding of the output (2^-8 relative) plus FP32 accumulation noise; and the
+    quantized-P output must differ from it by the (small) error of the P codes alone."""
+    w = workloads.custom(name, mode, B, H, L, D, seed=41, varlen_lens=lens)
+    q, k, v = workloads.make_qkv(w)
+    path = gpu_path(w, q, k, v)
+    got = _p_unquantized(path, w)
+    sc = [float(x) for x in path.scale.cpu()]
+    want = oracle.attention_e4m3(path.codes[0].cpu().numpy(), path.codes[1].cpu().numpy(),
+                                 path.codes[2].cpu().numpy(), w.shape, *sc, sm_scale=w.sm_scale,
+                                 flags=oracle.FP32, cu_seqlens=w.cu_seqlens).reshape(-1, w.D)
+    bound = 2.0 ** -8 * np.abs(want) + 1e-5 * np.abs(want).max()
+    excess = np.abs(got - want) - bound
+    assert excess.max() <= 0.0, f"{name}: worst excess {excess.max():.3e}"
+    quantized = path.out.float().cpu().numpy().reshape(-1, w.D)
+    rel_p, _ = compare(quantized, want)
+    print(f"{name}: error of the P codes alone (rel-L2) {rel_p:.2e}")
+    assert 0.0 < rel_p < 3e-2
