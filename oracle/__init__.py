@@ -304,6 +304,41 @@ def method_forward(q, k, v, mode="fp8", sm_scale=None, cu_seqlens=None, rows=Non
                           with_ambiguity)
 
 
+def e2m1_table() -> np.ndarray:
+    """Values of the 16 E2M1 codes."""
+    return np.array([e2m1_to_float(c) for c in range(16)], dtype=np.float64)
+
+
+def unpack_e2m1(packed, k: int) -> np.ndarray:
+    """E2M1 codes [rows, k] from their packed form [rows, k / 2]: element 2i in the low nibble of
+    byte i, element 2i + 1 in the high nibble (the layout quantize_fp4_block writes)."""
+    p = np.asarray(packed, dtype=np.uint8).reshape(-1, k // 2)
+    codes = np.empty((p.shape[0], k), dtype=np.uint8)
+    codes[:, 0::2] = p & 0x0F
+    codes[:, 1::2] = p >> 4
+    return codes
+
+
+def gemm_fp4_block(a_packed, a_bscale, sg_a, b_packed, b_bscale, sg_b, k: int, rows=None):
+    """The per-block FP4 linear layer, Y = X W^T, as its plain definition in FP64.  X [M, k] and
+    W [N, k] are in the per-block FP4 format of quantize_fp4_block: packed E2M1 codes [rows, k/2],
+    E4M3 block scales [rows, k/16] (block b covers columns 16 b .. 16 b + 15) and a per-tensor
+    FP32 scale s_g;
+        Y[m, n] = (sum_k val(a[m, k]) val(sa[m, k/16]) val(b[n, k]) val(sb[n, k/16])) sg_a sg_b,
+    the per-tensor scales applied once to the block-scaled dot product (as a block-scaled tensor
+    core GEMM does), not through the FP32-rounded per-element dequantization of
+    dequant_fp4_block.  numpy matmul as the library primitive; the block-scaled values are exact
+    in FP64.  rows: optional row indices of Y.  Returns (Y, bound), bound[m, n] = sum_k |terms|,
+    the scale an FP32 accumulation error is relative to."""
+    t2, t8 = e2m1_table(), e4m3_table()
+    a = t2[unpack_e2m1(a_packed, k)] * np.repeat(t8[np.asarray(a_bscale, np.uint8).reshape(-1, k // 16)], 16, axis=1)
+    b = t2[unpack_e2m1(b_packed, k)] * np.repeat(t8[np.asarray(b_bscale, np.uint8).reshape(-1, k // 16)], 16, axis=1)
+    if rows is not None:
+        a = a[np.asarray(rows)]
+    g = float(np.float32(sg_a)) * float(np.float32(sg_b))
+    return (a @ b.T) * g, (np.abs(a) @ np.abs(b).T) * abs(g)
+
+
 def gemm_e4m3(a8, b8, s_a, s_b, rows=None):
     """The FP8 linear layer, Y = X W^T, as its plain definition in FP64: a8 [M, K] and b8 [N, K]
     E4M3 codes (uint8), s_a, s_b their per-tensor dequantization multipliers;
