@@ -32,6 +32,7 @@ import workloads  # noqa: E402
 HBM_FALLBACK_GBS = 6650.0
 BF16_FALLBACK_TFLOPS = 1590.0
 FP8_PER_BF16 = 2.0          # nominal dense FP8 / BF16 tensor throughput ratio on B200
+FP4_PER_BF16 = 4.0          # nominal dense FP4 / BF16 ratio (9 vs 2.25 PFLOP/s)
 L2_FLUSH_BYTES = 256 << 20
 # DRAM bytes (read + write) of one launch of the attention kernel at L=8704 (B=1, H=24, D=128),
 # from ncu on the current kernel (80.30 MB read + 22.40 MB written):
@@ -711,6 +712,7 @@ def run_gemm(args):
                        "sample": f"16 of {M} rows of {name} (numpy FP64 matmul)"}
     value = total_flops / (total_ms * 1e-3) / 1e12
     fused = v_projection_fused(flush, args.steps)
+    fp4 = fp4_gemm_rates(flush, args.steps, args.warmup)
     # the burst GEMM figure, unless the power cap held the clock down during the timed launches:
     # then the figure measured over a seconds-long loop under the cap (when the peaks file has it)
     clk = clocks.summary()
@@ -724,6 +726,12 @@ def run_gemm(args):
     fp8_peak = bf16_tf * FP8_PER_BF16
     for rec in per_shape.values():
         rec["frac"] = rec["tflops"] / fp8_peak
+    fp4_peak = bf16_tf * FP4_PER_BF16
+    for rec in fp4["per_shape"].values():
+        rec["frac"] = rec["tflops"] / fp4_peak
+    fp4["peak"] = fp4_peak
+    fp4["peak_source"] = f"{peak_kind} bf16 {bf16_tf} TFLOP/s x {FP4_PER_BF16} (nominal FP4/BF16 ratio)"
+    fp4["frac"] = fp4["value"] / fp4_peak
     print(json.dumps({
         "metric": "FP8 GEMM TFLOP/s on the FLUX.1 Kontext block's linear layers "
                   "(QKV and output projections, MLP; 8704 tokens, hidden 3072)",
@@ -739,10 +747,48 @@ def run_gemm(args):
                      "peak_source": f"{peak_kind} bf16 {bf16_tf} TFLOP/s x {FP8_PER_BF16} "
                                     "(nominal FP8/BF16 ratio)", "per_shape": per_shape},
         "v_projection_fused_quantize": fused,
+        "fp4": fp4,
         "gpu_launches": len(GEMM_SHAPES) * args.steps,
         "clocks": clk,
         "cpu_baseline": cpu,
     }), flush=True)
+
+
+def fp4_gemm_rates(flush, steps, warmup):
+    """The per-block FP4 GEMM (qattn_gemm_fp4) on the same shapes: seeded random packed E2M1
+    codes and E4M3 block scales, timed like the FP8 launches."""
+    import precision_quantized_attention_b200 as qa
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(9)
+    per_shape, flops_sum, ms_sum = {}, 0.0, 0.0
+    for name, (M, N, K) in GEMM_SHAPES.items():
+        xp = torch.randint(0, 256, (M, K // 2), dtype=torch.uint8, device="cuda", generator=gen)
+        wp = torch.randint(0, 256, (N, K // 2), dtype=torch.uint8, device="cuda", generator=gen)
+        xb = torch.randint(0, 0x7F, (M, K // 16), dtype=torch.uint8, device="cuda", generator=gen)
+        wb = torch.randint(0, 0x7F, (N, K // 16), dtype=torch.uint8, device="cuda", generator=gen)
+        sx, sw = torch.tensor([0.01], device="cuda"), torch.tensor([0.002], device="cuda")
+        y = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
+        for _ in range(warmup):
+            qa.gemm_fp4(xp, xb, sx, wp, wb, sw, y)
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(steps)]
+        torch.cuda.synchronize()
+        for e0, e1 in ev:
+            flush()
+            e0.record()
+            qa.gemm_fp4(xp, xb, sx, wp, wb, sw, y)
+            e1.record()
+        torch.cuda.synchronize()
+        if qa.get_error() != 0:
+            raise RuntimeError("device error during the FP4 GEMM timing")
+        ms = sum(e0.elapsed_time(e1) for e0, e1 in ev) / len(ev)
+        flops = 2.0 * M * N * K
+        per_shape[name] = {"M": M, "N": N, "K": K, "ms": ms, "tflops": flops / (ms * 1e-3) / 1e12}
+        flops_sum += flops
+        ms_sum += ms
+    return {"kernel": "k_gemm_fp4 (kind::mxf4nvf4, 128 x 128 tiles, one SM each)",
+            "value": flops_sum / (ms_sum * 1e-3) / 1e12, "unit": "TFLOP/s", "ms": ms_sum,
+            "per_shape": per_shape, "gpu_launches": len(GEMM_SHAPES) * steps}
 
 
 def v_projection_fused(flush, steps):

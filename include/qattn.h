@@ -209,6 +209,22 @@ QATTN_API qattn_status qattn_gemm_fp8_e4m3(const uint8_t* a8, const uint8_t* b8,
                                            const float* amax_dev, float* scale_out_dev,
                                            qattn_stream_t stream);
 
+/* The block's linear layers in the per-block FP4 format (the blog's per-block FP4 quant config,
+ * "Workflow and quantization"; Fig. 3): Y = X W^T with
+ *   Y[m, n] = bf16((sum_k val(x[m,k]) val(sx[m,k/16]) val(w[n,k]) val(sw[n,k/16])) * sg_x * sg_w)
+ * on block-scaled FP4 tensor cores (FP32 accumulation).  X [M, K] and W [N, K] as
+ * qattn_quantize_fp4_block writes them: x_e2m1 / w_e2m1 packed E2M1 codes, rows of K / 2 bytes
+ * (element 2i in the low nibble of byte i); x_bscale / w_bscale E4M3 block scales, [rows, K / 16]
+ * row-major (block b covers K elements 16 b .. 16 b + 15, codes 0x00..0x7E); sg_x_dev /
+ * sg_w_dev one-element device FP32 per-tensor scales; y_bf16 [M, N] row-major.  All device,
+ * caller-owned, 16-byte aligned (the scales 4-byte); M >= 1, N >= 32 with N % 32 == 0,
+ * K >= 256 with K % 256 == 0, else QATTN_ERR_INVALID_ARG.  Timeouts of the kernel's bounded
+ * waits are reported by qattn_get_error. */
+QATTN_API qattn_status qattn_gemm_fp4(const uint8_t* x_e2m1, const uint8_t* x_bscale,
+                                      const float* sg_x_dev, const uint8_t* w_e2m1,
+                                      const uint8_t* w_bscale, const float* sg_w_dev, void* y_bf16,
+                                      int M, int N, int K, qattn_stream_t stream);
+
 /* qattn_calibrate_quantize_fp8 without a caller workspace (the blog has no counterpart: this is
  * a calling convention, not part of the method).  For callers that cannot supply a scratch
  * buffer -- C code with no device allocator at the call site, or a runtime whose device memory

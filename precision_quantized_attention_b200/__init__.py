@@ -18,11 +18,11 @@ from . import _lib
 from ._lib import (MODE_FP4, MODE_FP8, QattnError, calibrate_amax, calibrate_quantize_fp4_block,
                    calibrate_quantize_fp8, calibrate_quantize_qkv, forward, forward_varlen,
                    forward_workspace_bytes, get_error, new_workspace, quantize_fp4_block,
-                   quantize_fp8, quantize_qkv, gemm_fp8, gemm_fp8_e4m3)
+                   quantize_fp8, quantize_qkv, gemm_fp4, gemm_fp8, gemm_fp8_e4m3)
 
 __all__ = ["QuantizedAttention", "calibrate_amax", "quantize_fp8", "quantize_fp4_block",
            "calibrate_quantize_fp8", "calibrate_quantize_fp4_block", "calibrate_quantize_qkv",
-           "quantize_qkv", "gemm_fp8", "gemm_fp8_e4m3",
+           "quantize_qkv", "gemm_fp8", "gemm_fp8_e4m3", "gemm_fp4",
            "new_workspace", "forward", "forward_workspace_bytes",
            "forward_varlen", "get_error", "QattnError", "MODE_FP8", "MODE_FP4"]
 

@@ -26,13 +26,13 @@ EXPORTS = (
     "qattn_forward_varlen", "qattn_get_error", "qattn_calibrate_quantize_fp8",
     "qattn_calibrate_quantize_fp4_block", "qattn_calibrate_quantize_fp8_noalloc",
     "qattn_calibrate_quantize_qkv", "qattn_quantize_qkv", "qattn_forward_ws", "qattn_gemm_fp8",
-    "qattn_gemm_fp8_e4m3",
+    "qattn_gemm_fp8_e4m3", "qattn_gemm_fp4",
     "qattn_status_str", "qattn_last_cuda_error",
     "qattn_forward_workspace_bytes",
     "qattn_debug_set_wait_timeout_ns", "qattn_debug_inject_missing_q", "qattn_debug_capture_p_row",
     "qattn_debug_attention_plan", "qattn_build_info", "qattn_debug_inject_oob",
 )
-_RETURNS_STATUS = EXPORTS[:14]
+_RETURNS_STATUS = EXPORTS[:15]
 FUSED_WORKSPACE_BYTES = 256     # QATTN_FUSED_WORKSPACE_BYTES
 
 
@@ -81,6 +81,7 @@ def load() -> ctypes.CDLL:
     lib.qattn_quantize_qkv.argtypes = [ctypes.POINTER(QuantIO), S, I, P]
     lib.qattn_gemm_fp8.argtypes = [P, P, P, I, I, I, P, P, P]
     lib.qattn_gemm_fp8_e4m3.argtypes = [P, P, P, P, I, I, I, P, P, P, P, P]
+    lib.qattn_gemm_fp4.argtypes = [P, P, P, P, P, P, P, I, I, I, P]
     lib.qattn_forward.argtypes = [P, P, P, P, I, I, I, I, ctypes.POINTER(_Scales), F, I, P]
     lib.qattn_forward_varlen.argtypes = [P, P, P, P, P, I, I, I, I, I, ctypes.POINTER(_Scales),
                                          F, I, P]
@@ -294,6 +295,21 @@ def gemm_fp8_e4m3(a8, b8, codes, s_a, s_b, amax, scale_out, y=None, stream=None)
                                       _dev(amax, torch.float32, "amax"),
                                       _dev(scale_out, torch.float32, "scale_out"), _stream(stream)),
            "qattn_gemm_fp8_e4m3")
+
+
+def gemm_fp4(x_e2m1, x_bscale, sg_x, w_e2m1, w_bscale, sg_w, y, stream=None):
+    """Per-block FP4 GEMM, Y = X W^T: x_e2m1 uint8 [M, K/2] packed E2M1, x_bscale uint8 [M, K/16]
+    E4M3 block scales, sg_x float32 [1] per-tensor scale (W likewise with N rows); y bf16 [M, N].
+    K % 256 == 0, N % 32 == 0."""
+    M, N = y.shape
+    K = 2 * x_e2m1.shape[-1]
+    if (tuple(x_e2m1.shape) != (M, K // 2) or tuple(w_e2m1.shape) != (N, K // 2) or
+            tuple(x_bscale.shape) != (M, K // 16) or tuple(w_bscale.shape) != (N, K // 16)):
+        raise ValueError("x_e2m1 [M, K/2], x_bscale [M, K/16], w_e2m1 [N, K/2], w_bscale [N, K/16]")
+    _check(load().qattn_gemm_fp4(_dev(x_e2m1, torch.uint8, "x_e2m1"), _dev(x_bscale, torch.uint8, "x_bscale"),
+                                 _dev(sg_x, torch.float32, "sg_x"), _dev(w_e2m1, torch.uint8, "w_e2m1"),
+                                 _dev(w_bscale, torch.uint8, "w_bscale"), _dev(sg_w, torch.float32, "sg_w"),
+                                 _dev(y, torch.bfloat16, "y"), M, N, K, _stream(stream)), "qattn_gemm_fp4")
 
 
 def _scales(s_q, s_k, s_v):

@@ -1,0 +1,332 @@
+// gemm_fp4.cu -- per-block FP4 GEMM (E2M1 values, an E4M3 scale per 16 elements, a per-tensor
+// FP32 scale) for sm_100a: TMA + block-scaled tcgen05.mma (kind::mxf4nvf4) + TMEM.
+//
+// The linear layers of the transformer block in the blog's per-block FP4 post-training
+// quantization (NVIDIA developer blog "Optimizing FLUX.1 Kontext for Image Editing with
+// Low-Precision Quantization", "Workflow and quantization": the quant config takes per-tensor
+// FP8 or per-block FP4; Fig. 3 puts the GEMMs and the SDPA at about 75 % of the block's time).
+// Operands are in the format qattn_quantize_fp4_block writes: X [M, K] and W [N, K] as packed
+// E2M1 codes (element 2i in the low nibble of byte i, rows K / 2 bytes long), E4M3 block scales
+// [rows, K / 16] row-major (block b covers K elements 16 b .. 16 b + 15), and a per-tensor scale
+// s_g.  Computed here:
+//   Y[m, n] = bf16( (sum_k val(x[m,k]) val(sx[m,k/16]) val(w[n,k]) val(sw[n,k/16])) * fl32(sg_x sg_w) )
+// with the block-scaled products accumulated in FP32 by the tensor cores.
+//
+// One persistent kernel, 320 threads, one SM per 128 x 128 output tile (m-fastest order):
+//   warp 0      TMA producer: per 256-element (128-byte) K block the X tile (128 rows) and the W
+//               tile (128 rows), 128-byte swizzle, into a 4-stage ring.
+//   warp 1      MMA issuer (one thread) and TMEM owner: four K = 64 block-scaled MMAs per K
+//               block into one of two 128-column FP32 accumulators.
+//   warps 2-5   epilogue: thread = output row = TMEM lane; 32 columns at a time, scaled by
+//               sg_x sg_w, rounded to bf16, stored.
+//   warps 6-9   scale factors: per K block, each of the tile's rows' 16 block scales is one
+//               16-byte load from the row-major scale arrays; every warp writes them into its own
+//               lane quarter of a 4-stage TMEM ring (32 columns a stage: X's, then W's), as the
+//               block-scaled MMA reads them: row r's four factors of a K = 64 step form the word at
+//               lane r % 32, column (step * 4 + r / 32), replicated in every lane quarter.
+// The MMA commit of a K block frees both its shared-memory stage and its scale-factor stage.
+// All waits are bounded (a global-timer limit).
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <cstdint>
+
+#include "device_once.h"
+#include "launch.h"
+#include "sm100_ptx.cuh"
+
+namespace qattn {
+
+namespace gemm4 {
+constexpr int BM = 128;                  // output rows per tile (= TMEM lanes)
+constexpr int BN = 128;                  // output columns per tile (MMA N)
+constexpr int BK = 256;                  // K elements per stage (128 bytes of E2M1 per row)
+constexpr int BKB = BK / 2;              // bytes per row per stage
+constexpr int STAGES = 4;
+constexpr int THREADS = 320;
+constexpr int WARP_LOAD = 0, WARP_MMA = 1, WARP_SF0 = 6;   // warps 2-5: epilogue
+constexpr int TILE_A = BM * BKB;         // 16 KB
+constexpr int TILE_B = BN * BKB;         // 16 KB
+constexpr int OFF_A = 0;
+constexpr int OFF_B = OFF_A + STAGES * TILE_A;
+constexpr int OFF_BAR = OFF_B + STAGES * TILE_B;
+// barriers: full[STAGES] (TMA), sf_full[STAGES], empty[STAGES], acc_full[2], acc_empty[2], drain
+constexpr int B_FULL = 0, B_SFFULL = STAGES, B_EMPTY = 2 * STAGES, B_ACCF = 3 * STAGES;
+constexpr int B_ACCE = B_ACCF + 2, B_DRAIN = B_ACCE + 2, NBARS = B_DRAIN + 1;
+constexpr int OFF_TMEM = OFF_BAR + 8 * NBARS;
+constexpr int OFF_ABORT = OFF_TMEM + 4;
+constexpr int BYTES = OFF_ABORT + 4;
+constexpr int ALLOC = BYTES + 1024;      // slack for 1024-byte alignment
+static_assert(TILE_A % 1024 == 0 && TILE_B % 1024 == 0, "alignment");
+static_assert(ALLOC <= 227 * 1024, "shared memory per CTA");
+// TMEM: accumulators at columns 0 and BN; scale-factor stage s at SF0 + 32 s (16 columns of X's
+// factors, 16 of W's: K = 64 step kk, row group c = r / 32 in column kk * 4 + c)
+constexpr uint32_t SF0 = 2 * BN;
+constexpr uint32_t SF_COLS = 32;
+constexpr uint32_t TMEM_COLS = 512;
+static_assert(SF0 + STAGES * SF_COLS <= TMEM_COLS, "TMEM budget");
+constexpr uint32_t IDESC = idesc_mxf4_e2m1(BM, BN);
+}  // namespace gemm4
+
+struct Gemm4Args {
+  int M, N, K;
+  const uint8_t* sx;        // X's block scales [M, K / 16]
+  const uint8_t* sw;        // W's block scales [N, K / 16]
+  const float* sg_x;
+  const float* sg_w;
+  __nv_bfloat16* y;
+  int* err;
+  uint64_t timeout_ns;
+};
+
+__global__ void __launch_bounds__(gemm4::THREADS, 1)
+    k_gemm_fp4(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
+               const __grid_constant__ Gemm4Args args) {
+  using namespace gemm4;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_u32 = smem_u32(smem_raw);
+  const uint32_t base_u32 = (raw_u32 + 1023u) & ~1023u;
+  uint8_t* base = smem_raw + (base_u32 - raw_u32);
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  const int tiles_m = (args.M + BM - 1) / BM;
+  const int tiles = tiles_m * ((args.N + BN - 1) / BN);
+  const int kblocks = args.K / BK;
+  if (static_cast<int>(blockIdx.x) >= tiles) return;   // uniform over the CTA
+
+  const uint32_t bar0 = base_u32 + OFF_BAR;
+  auto BAR = [&](int i) { return bar0 + 8u * static_cast<uint32_t>(i); };
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(base + OFF_ABORT);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base + OFF_TMEM);
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < STAGES; ++i) {
+      mbar_init(BAR(B_FULL + i), 1);
+      mbar_init(BAR(B_SFFULL + i), 4);           // one arrival per scale-factor warp
+      mbar_init(BAR(B_EMPTY + i), 1);
+    }
+    for (int b = 0; b < 2; ++b) { mbar_init(BAR(B_ACCF + b), 1); mbar_init(BAR(B_ACCE + b), 128); }
+    mbar_init(BAR(B_DRAIN), 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == WARP_MMA) {
+    tmem_alloc(base_u32 + OFF_TMEM, TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint64_t tlim = args.timeout_ns;
+
+  if (warp == WARP_LOAD) {
+    // ======================= TMA producer =======================
+    if (lane == 0) {
+      tma_prefetch_desc(&tm_a);
+      tma_prefetch_desc(&tm_b);
+      int u = 0;                                   // K blocks issued (ring position)
+      bool ok = true;
+      for (int t = blockIdx.x; ok && t < tiles; t += gridDim.x) {
+        const int m0 = (t % tiles_m) * BM, n0 = (t / tiles_m) * BN;
+        (void)QATTN_IN_BOUNDS(args.err, m0 < args.M && n0 < args.N);
+        for (int kb = 0; kb < kblocks; ++kb, ++u) {
+          const int s = u % STAGES;
+          if (u >= STAGES &&
+              !mbar_wait(BAR(B_EMPTY + s), ((u / STAGES) - 1) & 1, tlim, abort_flag, args.err)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(BAR(B_FULL + s), TILE_A + TILE_B);
+          tma_load_2d(base_u32 + OFF_A + s * TILE_A, &tm_a, BAR(B_FULL + s), kb * BKB, m0);
+          tma_load_2d(base_u32 + OFF_B + s * TILE_B, &tm_b, BAR(B_FULL + s), kb * BKB, n0);
+        }
+      }
+      // drain: every issued load has landed before the CTA may exit (instant when healthy)
+      for (int j = u - 1; j >= 0 && j >= u - STAGES; --j)
+        mbar_drain(BAR(B_FULL + j % STAGES), (j / STAGES) & 1, tlim);
+    }
+  } else if (warp >= WARP_SF0) {
+    // ======================= scale factors into TMEM =======================
+    const int quarter = warp & 3;                  // this warp's TMEM lane quarter
+    const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+    const size_t row_bytes = static_cast<size_t>(args.K / 16);
+    int u = 0;
+    bool ok = true;
+    for (int t = blockIdx.x; ok && t < tiles; t += gridDim.x) {
+      const int m0 = (t % tiles_m) * BM, n0 = (t / tiles_m) * BN;
+      for (int kb = 0; kb < kblocks; ++kb, ++u) {
+        const int s = u % STAGES;
+        if (u >= STAGES) {
+          ok = mbar_wait(BAR(B_EMPTY + s), ((u / STAGES) - 1) & 1, tlim, abort_flag, args.err);
+          if (!__all_sync(0xFFFFFFFFu, ok)) { ok = false; break; }
+        }
+        // row group c of the tile: rows 32 c + lane; 16 factors (16 bytes) of the K block each
+        uint32_t v[32];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const int rx = m0 + 32 * c + lane, rw = n0 + 32 * c + lane;
+          uint4 fx = make_uint4(0u, 0u, 0u, 0u), fw = make_uint4(0u, 0u, 0u, 0u);
+          if (rx < args.M)
+            fx = __ldg(reinterpret_cast<const uint4*>(args.sx + static_cast<size_t>(rx) * row_bytes) + kb);
+          if (rw < args.N)
+            fw = __ldg(reinterpret_cast<const uint4*>(args.sw + static_cast<size_t>(rw) * row_bytes) + kb);
+          v[c] = fx.x; v[4 + c] = fx.y; v[8 + c] = fx.z; v[12 + c] = fx.w;
+          v[16 + c] = fw.x; v[20 + c] = fw.y; v[24 + c] = fw.z; v[28 + c] = fw.w;
+        }
+        tmem_st32(tmem + lane_off + SF0 + static_cast<uint32_t>(s) * SF_COLS, v);
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(BAR(B_SFFULL + s));
+      }
+    }
+  } else if (warp == WARP_MMA) {
+    // ======================= MMA issuer =======================
+    if (lane == 0) {
+      int u = 0, i = 0;                            // K blocks consumed; tiles of this CTA
+      bool ok = true;
+      for (int t = blockIdx.x; ok && t < tiles; t += gridDim.x, ++i) {
+        const int ab = i & 1;                      // accumulator of this tile
+        if (i >= 2)
+          ok = mbar_wait(BAR(B_ACCE + ab), ((i >> 1) - 1) & 1, tlim, abort_flag, args.err);
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t acc = tmem + static_cast<uint32_t>(ab * BN);
+        for (int kb = 0; kb < kblocks; ++kb, ++u) {
+          const int s = u % STAGES;
+          ok = mbar_wait(BAR(B_FULL + s), (u / STAGES) & 1, tlim, abort_flag, args.err) &&
+               mbar_wait(BAR(B_SFFULL + s), (u / STAGES) & 1, tlim, abort_flag, args.err);
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t a_s = base_u32 + OFF_A + s * TILE_A;
+          const uint32_t b_s = base_u32 + OFF_B + s * TILE_B;
+          const uint32_t sf = tmem + SF0 + static_cast<uint32_t>(s) * SF_COLS;
+#pragma unroll
+          for (int kk = 0; kk < BK / 64; ++kk) {
+            // K-major rows of 128 bytes, 128-byte swizzle, 8-row atoms (SBO 1024); a K = 64 step
+            // is 32 bytes of packed E2M1
+            const uint64_t da = smem_desc(a_s + kk * 32, 16, 1024, 2u);
+            const uint64_t db = smem_desc(b_s + kk * 32, 16, 1024, 2u);
+            mma_mxf4_ss(acc, da, db, IDESC, sf + kk * 4, sf + 16 + kk * 4, (kb > 0 || kk > 0) ? 1u : 0u);
+          }
+          mma_commit(BAR(B_EMPTY + s));           // stage and factors free once these complete
+        }
+        if (ok) mma_commit(BAR(B_ACCF + ab));     // accumulator complete
+      }
+      mma_commit(BAR(B_DRAIN));
+      mbar_drain(BAR(B_DRAIN), 0, tlim);
+    }
+  } else {
+    // ======================= epilogue warps =======================
+    const int quarter = warp & 3;
+    const int r = quarter * 32 + lane;             // row within the tile
+    const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+    const float scale = __ldg(args.sg_x) * __ldg(args.sg_w);
+    int i = 0;
+    for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++i) {
+      const int ab = i & 1;
+      const bool ok = mbar_wait(BAR(B_ACCF + ab), (i >> 1) & 1, tlim, abort_flag, args.err);
+      if (!__all_sync(0xFFFFFFFFu, ok)) break;
+      tc_fence_after();
+      const int m = (t % tiles_m) * BM + r, n0 = (t / tiles_m) * BN;
+      const uint32_t acc = tmem + lane_off + static_cast<uint32_t>(ab * BN);
+#pragma unroll 1
+      for (int c = 0; c < BN / 32; ++c) {
+        uint32_t v[32];
+        tmem_ld32(acc + c * 32, v);
+        tmem_wait_ld();
+        const size_t off = static_cast<size_t>(m) * args.N + n0 + c * 32;
+        // N % 32 == 0: a 32-column chunk is all in or all out
+        if (m < args.M && n0 + c * 32 < args.N &&
+            QATTN_IN_BOUNDS(args.err, off + 32 <= static_cast<size_t>(args.M) * args.N)) {
+          uint32_t packed[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const __nv_bfloat162 b2 = __floats2bfloat162_rn(__uint_as_float(v[2 * e]) * scale,
+                                                            __uint_as_float(v[2 * e + 1]) * scale);
+            packed[e] = *reinterpret_cast<const uint32_t*>(&b2);
+          }
+          uint4* dst = reinterpret_cast<uint4*>(args.y + off);
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            dst[e] = make_uint4(packed[4 * e], packed[4 * e + 1], packed[4 * e + 2], packed[4 * e + 3]);
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(BAR(B_ACCE + ab));               // accumulator read out
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == WARP_MMA) {
+    tc_fence_after();
+    tmem_dealloc(tmem, TMEM_COLS);
+  }
+}
+
+// ---------------------------------------------------------------------------------------------
+// Host side
+// ---------------------------------------------------------------------------------------------
+using Gemm4EncodeFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static Gemm4EncodeFn gemm4_encode_fn() {
+  static const Gemm4EncodeFn fn = [] {          // initialised once, thread-safe
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return static_cast<Gemm4EncodeFn>(nullptr);
+    return reinterpret_cast<Gemm4EncodeFn>(p);
+  }();
+  return fn;
+}
+
+// Packed E2M1 [rows, K / 2 bytes]; box of 128 rows x 128 bytes, 128-byte swizzle; reads past the
+// last row return zeros.
+static bool make_map_e2m1(CUtensorMap* map, const void* ptr, int rows, int K) {
+  Gemm4EncodeFn enc = gemm4_encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(K / 2), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(K / 2)};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(gemm4::BKB), static_cast<cuuint32_t>(gemm4::BM)};
+  cuuint32_t estr[2] = {1u, 1u};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(ptr), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+cudaError_t launch_gemm_fp4(const uint8_t* x, const uint8_t* sx, const float* sg_x, const uint8_t* w,
+                            const uint8_t* sw, const float* sg_w, void* y, int M, int N, int K,
+                            int* err, uint64_t timeout_ns, int num_sms, cudaStream_t stream) {
+  static_assert(gemm4::BM == gemm4::BN, "one box shape serves both operands");
+  Gemm4Args a;
+  a.M = M;
+  a.N = N;
+  a.K = K;
+  a.sx = sx;
+  a.sw = sw;
+  a.sg_x = sg_x;
+  a.sg_w = sg_w;
+  a.y = static_cast<__nv_bfloat16*>(y);
+  a.err = err;
+  a.timeout_ns = timeout_ns;
+  CUtensorMap ma, mb;
+  if (!make_map_e2m1(&ma, x, M, K) || !make_map_e2m1(&mb, w, N, K)) return cudaErrorInvalidValue;
+  static DeviceOnce configured;
+  const int set = configured.get([] {
+    return static_cast<int>(cudaFuncSetAttribute(k_gemm_fp4, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                 gemm4::ALLOC));
+  });
+  if (set != static_cast<int>(cudaSuccess)) return static_cast<cudaError_t>(set);
+  const int tiles = ((M + gemm4::BM - 1) / gemm4::BM) * ((N + gemm4::BN - 1) / gemm4::BN);
+  const int grid = tiles < num_sms ? tiles : num_sms;
+  k_gemm_fp4<<<grid, gemm4::THREADS, gemm4::ALLOC, stream>>>(ma, mb, a);
+  return cudaGetLastError();
+}
+
+}  // namespace qattn

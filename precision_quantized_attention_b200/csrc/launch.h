@@ -57,6 +57,12 @@ struct DebugHooks {
   int p_row = -1;
 };
 
+// Per-block FP4 GEMM (gemm_fp4.cu): Y [M, N] bf16 = X W^T from packed E2M1 codes, E4M3 block
+// scales (one per 16 K elements, row-major) and per-tensor scales.  K % 256 == 0, N % 32 == 0.
+cudaError_t launch_gemm_fp4(const uint8_t* x, const uint8_t* sx, const float* sg_x, const uint8_t* w,
+                            const uint8_t* sw, const float* sg_w, void* y, int M, int N, int K,
+                            int* err, uint64_t timeout_ns, int num_sms, cudaStream_t stream);
+
 // The attention with P left unquantized (QATTN_FLAG_P_UNQUANTIZED, a debug path; attn_debug.cu):
 // dense (cu_seqlens == nullptr: B, H, L) or varlen (cu_seqlens, nseq, max_seqlen, total_tokens, H).
 cudaError_t launch_attention_p_unquantized(const uint8_t* q8, const uint8_t* k8, const uint8_t* v8,

@@ -282,6 +282,23 @@ qattn_status qattn_gemm_fp8_e4m3(const uint8_t* a8, const uint8_t* b8, void* y_b
                                           amax_dev, scale_out_dev));
 }
 
+qattn_status qattn_gemm_fp4(const uint8_t* x_e2m1, const uint8_t* x_bscale, const float* sg_x_dev,
+                           const uint8_t* w_e2m1, const uint8_t* w_bscale, const float* sg_w_dev,
+                           void* y_bf16, int M, int N, int K, qattn_stream_t stream) {
+  if (!x_e2m1 || !x_bscale || !sg_x_dev || !w_e2m1 || !w_bscale || !sg_w_dev || !y_bf16)
+    return QATTN_ERR_INVALID_ARG;
+  if (M < 1 || N < 32 || K < 256 || N % 32 != 0 || K % 256 != 0) return QATTN_ERR_INVALID_ARG;
+  if (!aligned(x_e2m1, 16) || !aligned(w_e2m1, 16) || !aligned(x_bscale, 16) ||
+      !aligned(w_bscale, 16) || !aligned(y_bf16, 16) || !aligned(sg_x_dev, 4) || !aligned(sg_w_dev, 4))
+    return QATTN_ERR_INVALID_ARG;
+  DeviceInfo* d = nullptr;
+  qattn_status st = device_info(&d);
+  if (st != QATTN_OK) return st;
+  return from_cuda(qattn::launch_gemm_fp4(x_e2m1, x_bscale, sg_x_dev, w_e2m1, w_bscale, sg_w_dev,
+                                          y_bf16, M, N, K, d->err, g_timeout_ns, d->num_sms,
+                                          reinterpret_cast<cudaStream_t>(stream)));
+}
+
 qattn_status qattn_forward_ws(const uint8_t* q8, const uint8_t* k8, const uint8_t* v8,
                               void* out_bf16, int B, int H, int L, int D,
                               const qattn_scales* scales, float sm_scale, qattn_mode mode,

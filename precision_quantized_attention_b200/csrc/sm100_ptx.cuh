@@ -297,6 +297,22 @@ __device__ __forceinline__ void mma_f8_ss(uint32_t d_tmem, uint64_t a_desc, uint
       : "memory");
 }
 
+// Block-scaled FP4 (kind::mxf4nvf4, packed E2M1 operands from shared memory, E4M3 scale
+// factors, one per 16 K elements), one issuing thread: D[tmem] (+)= (A * SFA) * (B * SFB)^T over
+// K = 64.  sfa_tmem / sfb_tmem address the factors: row r's four factors (its 64 K elements) are
+// the four bytes of the 32-bit word at lane r % 32, column base + r / 32, in every lane quarter.
+__device__ __forceinline__ void mma_mxf4_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                            uint32_t idesc, uint32_t sfa_tmem, uint32_t sfb_tmem,
+                                            uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %6, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%4], [%5], p;\n\t}" ::"r"(
+          d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(sfa_tmem), "r"(sfb_tmem), "r"(accumulate)
+      : "memory");
+}
+
 // Block-scaled, A from tensor memory (kind::mxf8f6f4, E8M0 scale factors, one per 32 K
 // elements; A's row m in lane m, element k in column k/4, byte k%4), one issuing thread:
 // D[tmem] (+)= (A[tmem] * SFA) * (B[smem desc] * SFB).  sfa_tmem / sfb_tmem address 4-column
@@ -425,6 +441,14 @@ __host__ __device__ constexpr uint32_t idesc_mxf8_e4m3(uint32_t M, uint32_t N, b
                                                        uint32_t sf_id) {
   return ((sf_id & 3u) << 4) | ((b_mn_major ? 1u : 0u) << 16) | ((N >> 3) << 17) | (1u << 23) |
          ((M >> 4) << 24) | ((sf_id & 3u) << 29);
+}
+
+// Instruction descriptor of kind::mxf4nvf4 (block-scaled FP4): A and B E2M1 (format 1 in
+// [7,10) and [10,13)), both K-major, N >> 3 in [17,23), scale factors E4M3 (bit 23 clear),
+// M >> 4 in [24,29), scale-factor bytes 0 (the four factors of a K = 64 step fill the word),
+// K = 64 (bit 31 clear).
+__host__ __device__ constexpr uint32_t idesc_mxf4_e2m1(uint32_t M, uint32_t N) {
+  return (1u << 7) | (1u << 10) | ((N >> 3) << 17) | ((M >> 4) << 24);
 }
 
 // ----------------------------------------------------------------------------------------------

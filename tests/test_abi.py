@@ -200,3 +200,16 @@ def test_p_unquantized_flag_is_validated_on_the_host():
 def _gpu():
     import torch
     return torch.cuda.is_available()
+
+
+def test_gemm_fp4_argument_errors():
+    lib = _lib.load()
+    s0 = ctypes.c_void_p(0)
+    g = lib.qattn_gemm_fp4
+    ok = (FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE)
+    assert g(None, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 128, 128, 256, s0) == _lib.ERR_INVALID_ARG
+    assert g(*ok, 128, 128, 128, s0) == _lib.ERR_INVALID_ARG           # K < 256
+    assert g(*ok, 128, 128, 384, s0) == _lib.ERR_INVALID_ARG           # K % 256 != 0
+    assert g(*ok, 128, 48, 256, s0) == _lib.ERR_INVALID_ARG            # N % 32 != 0
+    assert g(*ok, 0, 128, 256, s0) == _lib.ERR_INVALID_ARG
+    assert g(FAKE, MISALIGNED, FAKE, FAKE, FAKE, FAKE, FAKE, 128, 128, 256, s0) == _lib.ERR_INVALID_ARG

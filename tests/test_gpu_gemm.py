@@ -132,3 +132,73 @@ def test_fused_e4m3_nonfinite_amax_writes_no_code():
                      torch.tensor([float("inf")], device="cuda"), torch.zeros(1, device="cuda"))
     assert qa.get_error() == qa._lib.ERR_NONFINITE
     assert bool((codes == 0x55).all())
+
+
+# --- per-block FP4 GEMM (kind::mxf4nvf4) vs oracle.gemm_fp4_block ---------------------------
+def _fp4_operands(rng, rows, K):
+    """Random packed E2M1 codes (all 16 codes) and E4M3 block scales (every finite non-negative
+    code 0x00..0x7E, subnormals included)."""
+    return (rng.integers(0, 256, size=(rows, K // 2), dtype=np.uint8),
+            rng.integers(0, 0x7F, size=(rows, K // 16), dtype=np.uint8))
+
+
+def _run_fp4(M, N, K, seed, sg_x=0.01, sg_w=0.002):
+    rng = np.random.default_rng(seed)
+    (xp, xb), (wp, wb) = _fp4_operands(rng, M, K), _fp4_operands(rng, N, K)
+    y = torch.full((M, N), float("nan"), dtype=torch.bfloat16, device="cuda")
+    dev = lambda a: torch.from_numpy(a).cuda()
+    qa.gemm_fp4(dev(xp), dev(xb), torch.tensor([sg_x], device="cuda"), dev(wp), dev(wb),
+                torch.tensor([sg_w], device="cuda"), y)
+    assert qa.get_error() == 0
+    return (xp, xb, np.float32(sg_x), wp, wb, np.float32(sg_w)), y
+
+
+@pytest.mark.parametrize("M,N,K", [(1, 32, 256), (128, 128, 256), (130, 288, 512), (300, 512, 768),
+                                   (257, 96, 1024), (2560, 2080, 256)])
+def test_fp4_small_shapes_all_elements(M, N, K):
+    """Ragged row and column tiles (N not a multiple of 128), one and several 256-element K
+    blocks, several tiles per SM (2560 x 2080: 340 tiles of 128 x 128); the bar of the FP8 GEMM:
+    FP32 accumulation (K * 2^-24 of the sum of |terms|) plus the bf16 rounding (2^-8)."""
+    ops, y = _run_fp4(M, N, K, seed=M + 3 * N + K)
+    want, bound = oracle.gemm_fp4_block(*ops, K)
+    _check(y.float().cpu().numpy(), want, bound, K)
+
+
+@pytest.mark.parametrize("M,N,K", [(8704, 9216, 3072), (8704, 3072, 3072), (8704, 12288, 3072),
+                                   (8704, 3072, 12288)])
+def test_fp4_kontext_block_shapes_sampled_rows(M, N, K):
+    ops, y = _run_fp4(M, N, K, seed=K + 1)
+    rows = np.unique(np.concatenate([[0, M - 1], np.random.default_rng(3).integers(0, M, 62)]))
+    want, bound = oracle.gemm_fp4_block(*ops, K, rows=rows)
+    _check(y[torch.as_tensor(rows, device="cuda")].float().cpu().numpy(), want, bound, K)
+
+
+def test_fp4_gemm_of_operands_quantized_on_the_gpu():
+    """bf16 X and W through qattn_quantize_fp4_block (bit-exact with the oracle's quantizer),
+    then the FP4 GEMM: within the accumulation bar of the oracle on those codes, and near the
+    bf16 product (the FP4 quantization error of Gaussian data, about 10 % per element)."""
+    g = torch.Generator().manual_seed(2)
+    M, N, K = 300, 256, 512
+    x = torch.randn(M, K, generator=g).to(torch.bfloat16).cuda()
+    w = torch.randn(N, K, generator=g).to(torch.bfloat16).cuda()
+    ops = []
+    for t in (x, w):
+        rows = t.shape[0]
+        amax = torch.zeros(1, device="cuda")
+        qa.calibrate_amax(t.reshape(-1), amax)
+        e2m1 = torch.empty(rows * K // 2, dtype=torch.uint8, device="cuda")
+        bs = torch.empty(rows * K // 16, dtype=torch.uint8, device="cuda")
+        sg = torch.zeros(1, device="cuda")
+        qa.quantize_fp4_block(t.reshape(-1), amax, e2m1, bs, sg)
+        ops.append((e2m1.reshape(rows, K // 2), bs.reshape(rows, K // 16), sg))
+    y = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
+    qa.gemm_fp4(*ops[0], *ops[1], y)
+    assert qa.get_error() == 0
+    host = [a.cpu().numpy() for o in ops for a in o]
+    want, bound = oracle.gemm_fp4_block(host[0], host[1], host[2][0], host[3], host[4], host[5][0], K)
+    got = y.float().cpu().numpy()
+    _check(got, want, bound, K)
+    ref = (x.float() @ w.float().T).cpu().numpy()
+    rel = np.linalg.norm(got - ref) / np.linalg.norm(ref)
+    print(f"FP4 GEMM vs the bf16 product: rel-L2 {rel:.3f}")
+    assert rel < 0.25
