@@ -14,16 +14,17 @@
 //
 // One persistent kernel, 320 threads, one SM per 128 x 128 output tile (m-fastest order):
 //   warp 0      TMA producer: per 256-element (128-byte) K block the X tile (128 rows) and the W
-//               tile (128 rows), 128-byte swizzle, into a 4-stage ring.
+//               tile (128 rows), 128-byte swizzle, and the rows' 16 block scales each (two
+//               128 x 16-byte boxes of the row-major scale arrays), into a 4-stage ring.
 //   warp 1      MMA issuer (one thread) and TMEM owner: four K = 64 block-scaled MMAs per K
 //               block into one of two 128-column FP32 accumulators.
 //   warps 2-5   epilogue: thread = output row = TMEM lane; 32 columns at a time, scaled by
 //               sg_x sg_w, rounded to bf16, stored.
-//   warps 6-9   scale factors: per K block, each of the tile's rows' 16 block scales is one
-//               16-byte load from the row-major scale arrays; every warp writes them into its own
-//               lane quarter of a 4-stage TMEM ring (32 columns a stage: X's, then W's), as the
-//               block-scaled MMA reads them: row r's four factors of a K = 64 step form the word at
-//               lane r % 32, column (step * 4 + r / 32), replicated in every lane quarter.
+//   warps 6-9   scale factors: per K block, each warp copies the stage's block scales from
+//               shared memory into its own lane quarter of a 4-stage TMEM ring (32 columns a
+//               stage: X's, then W's), as the block-scaled MMA reads them: row r's four factors of
+//               a K = 64 step form the word at lane r % 32, column (step * 4 + r / 32), replicated
+//               in every lane quarter.
 // The MMA commit of a K block frees both its shared-memory stage and its scale-factor stage.
 // All waits are bounded (a global-timer limit).
 #include <cuda.h>
@@ -49,7 +50,11 @@ constexpr int TILE_A = BM * BKB;         // 16 KB
 constexpr int TILE_B = BN * BKB;         // 16 KB
 constexpr int OFF_A = 0;
 constexpr int OFF_B = OFF_A + STAGES * TILE_A;
-constexpr int OFF_BAR = OFF_B + STAGES * TILE_B;
+constexpr int TILE_SF = 128 * 16;        // 2 KB: 128 rows x 16 block scales
+constexpr int OFF_SFX = OFF_B + STAGES * TILE_B;
+constexpr int OFF_SFW = OFF_SFX + STAGES * TILE_SF;
+constexpr int STAGE_TX = TILE_A + TILE_B + 2 * TILE_SF;
+constexpr int OFF_BAR = OFF_SFW + STAGES * TILE_SF;
 // barriers: full[STAGES] (TMA), sf_full[STAGES], empty[STAGES], acc_full[2], acc_empty[2], drain
 constexpr int B_FULL = 0, B_SFFULL = STAGES, B_EMPTY = 2 * STAGES, B_ACCF = 3 * STAGES;
 constexpr int B_ACCE = B_ACCF + 2, B_DRAIN = B_ACCE + 2, NBARS = B_DRAIN + 1;
@@ -70,8 +75,6 @@ constexpr uint32_t IDESC = idesc_mxf4_e2m1(BM, BN);
 
 struct Gemm4Args {
   int M, N, K;
-  const uint8_t* sx;        // X's block scales [M, K / 16]
-  const uint8_t* sw;        // W's block scales [N, K / 16]
   const float* sg_x;
   const float* sg_w;
   __nv_bfloat16* y;
@@ -81,6 +84,7 @@ struct Gemm4Args {
 
 __global__ void __launch_bounds__(gemm4::THREADS, 1)
     k_gemm_fp4(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
+               const __grid_constant__ CUtensorMap tm_sa, const __grid_constant__ CUtensorMap tm_sb,
                const __grid_constant__ Gemm4Args args) {
   using namespace gemm4;
   extern __shared__ uint8_t smem_raw[];
@@ -125,6 +129,8 @@ __global__ void __launch_bounds__(gemm4::THREADS, 1)
     if (lane == 0) {
       tma_prefetch_desc(&tm_a);
       tma_prefetch_desc(&tm_b);
+      tma_prefetch_desc(&tm_sa);
+      tma_prefetch_desc(&tm_sb);
       int u = 0;                                   // K blocks issued (ring position)
       bool ok = true;
       for (int t = blockIdx.x; ok && t < tiles; t += gridDim.x) {
@@ -137,9 +143,11 @@ __global__ void __launch_bounds__(gemm4::THREADS, 1)
             ok = false;
             break;
           }
-          mbar_arrive_expect_tx(BAR(B_FULL + s), TILE_A + TILE_B);
+          mbar_arrive_expect_tx(BAR(B_FULL + s), STAGE_TX);
           tma_load_2d(base_u32 + OFF_A + s * TILE_A, &tm_a, BAR(B_FULL + s), kb * BKB, m0);
           tma_load_2d(base_u32 + OFF_B + s * TILE_B, &tm_b, BAR(B_FULL + s), kb * BKB, n0);
+          tma_load_2d(base_u32 + OFF_SFX + s * TILE_SF, &tm_sa, BAR(B_FULL + s), kb * 16, m0);
+          tma_load_2d(base_u32 + OFF_SFW + s * TILE_SF, &tm_sb, BAR(B_FULL + s), kb * 16, n0);
         }
       }
       // drain: every issued load has landed before the CTA may exit (instant when healthy)
@@ -148,29 +156,24 @@ __global__ void __launch_bounds__(gemm4::THREADS, 1)
     }
   } else if (warp >= WARP_SF0) {
     // ======================= scale factors into TMEM =======================
+    // The stage's factors landed with its tiles (full barrier); the MMAs that read this TMEM
+    // stage before completed before the producer could refill the shared-memory stage.
     const int quarter = warp & 3;                  // this warp's TMEM lane quarter
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
-    const size_t row_bytes = static_cast<size_t>(args.K / 16);
     int u = 0;
     bool ok = true;
     for (int t = blockIdx.x; ok && t < tiles; t += gridDim.x) {
-      const int m0 = (t % tiles_m) * BM, n0 = (t / tiles_m) * BN;
       for (int kb = 0; kb < kblocks; ++kb, ++u) {
         const int s = u % STAGES;
-        if (u >= STAGES) {
-          ok = mbar_wait(BAR(B_EMPTY + s), ((u / STAGES) - 1) & 1, tlim, abort_flag, args.err);
-          if (!__all_sync(0xFFFFFFFFu, ok)) { ok = false; break; }
-        }
+        ok = mbar_wait(BAR(B_FULL + s), (u / STAGES) & 1, tlim, abort_flag, args.err);
+        if (!__all_sync(0xFFFFFFFFu, ok)) { ok = false; break; }
         // row group c of the tile: rows 32 c + lane; 16 factors (16 bytes) of the K block each
+        const uint32_t fx0 = base_u32 + OFF_SFX + s * TILE_SF + 16u * lane;
+        const uint32_t fw0 = base_u32 + OFF_SFW + s * TILE_SF + 16u * lane;
         uint32_t v[32];
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
-          const int rx = m0 + 32 * c + lane, rw = n0 + 32 * c + lane;
-          uint4 fx = make_uint4(0u, 0u, 0u, 0u), fw = make_uint4(0u, 0u, 0u, 0u);
-          if (rx < args.M)
-            fx = __ldg(reinterpret_cast<const uint4*>(args.sx + static_cast<size_t>(rx) * row_bytes) + kb);
-          if (rw < args.N)
-            fw = __ldg(reinterpret_cast<const uint4*>(args.sw + static_cast<size_t>(rw) * row_bytes) + kb);
+          const uint4 fx = ld_shared_v4(fx0 + 512u * c), fw = ld_shared_v4(fw0 + 512u * c);
           v[c] = fx.x; v[4 + c] = fx.y; v[8 + c] = fx.z; v[12 + c] = fx.w;
           v[16 + c] = fw.x; v[20 + c] = fw.y; v[24 + c] = fw.z; v[28 + c] = fw.w;
         }
@@ -300,6 +303,20 @@ static bool make_map_e2m1(CUtensorMap* map, const void* ptr, int rows, int K) {
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Block scales [rows, K / 16] bytes, row-major; box of 128 rows x 16 bytes (one K block's
+// factors), no swizzle; rows past the last read as zeros.
+static bool make_map_scales(CUtensorMap* map, const void* ptr, int rows, int K) {
+  Gemm4EncodeFn enc = gemm4_encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(K / 16), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(K / 16)};
+  cuuint32_t box[2] = {16u, 128u};
+  cuuint32_t estr[2] = {1u, 1u};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(ptr), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 cudaError_t launch_gemm_fp4(const uint8_t* x, const uint8_t* sx, const float* sg_x, const uint8_t* w,
                             const uint8_t* sw, const float* sg_w, void* y, int M, int N, int K,
                             int* err, uint64_t timeout_ns, int num_sms, cudaStream_t stream) {
@@ -308,15 +325,15 @@ cudaError_t launch_gemm_fp4(const uint8_t* x, const uint8_t* sx, const float* sg
   a.M = M;
   a.N = N;
   a.K = K;
-  a.sx = sx;
-  a.sw = sw;
   a.sg_x = sg_x;
   a.sg_w = sg_w;
   a.y = static_cast<__nv_bfloat16*>(y);
   a.err = err;
   a.timeout_ns = timeout_ns;
-  CUtensorMap ma, mb;
-  if (!make_map_e2m1(&ma, x, M, K) || !make_map_e2m1(&mb, w, N, K)) return cudaErrorInvalidValue;
+  CUtensorMap ma, mb, msa, msb;
+  if (!make_map_e2m1(&ma, x, M, K) || !make_map_e2m1(&mb, w, N, K) ||
+      !make_map_scales(&msa, sx, M, K) || !make_map_scales(&msb, sw, N, K))
+    return cudaErrorInvalidValue;
   static DeviceOnce configured;
   const int set = configured.get([] {
     return static_cast<int>(cudaFuncSetAttribute(k_gemm_fp4, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -325,7 +342,7 @@ cudaError_t launch_gemm_fp4(const uint8_t* x, const uint8_t* sx, const float* sg
   if (set != static_cast<int>(cudaSuccess)) return static_cast<cudaError_t>(set);
   const int tiles = ((M + gemm4::BM - 1) / gemm4::BM) * ((N + gemm4::BN - 1) / gemm4::BN);
   const int grid = tiles < num_sms ? tiles : num_sms;
-  k_gemm_fp4<<<grid, gemm4::THREADS, gemm4::ALLOC, stream>>>(ma, mb, a);
+  k_gemm_fp4<<<grid, gemm4::THREADS, gemm4::ALLOC, stream>>>(ma, mb, msa, msb, a);
   return cudaGetLastError();
 }
 
