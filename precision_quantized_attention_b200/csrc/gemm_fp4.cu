@@ -15,13 +15,13 @@
 // One persistent kernel, 320 threads, one SM per 128 x 128 output tile (m-fastest order):
 //   warp 0      TMA producer: per 256-element (128-byte) K block the X tile (128 rows) and the W
 //               tile (128 rows), 128-byte swizzle, and the rows' 16 block scales each (two
-//               128 x 16-byte boxes of the row-major scale arrays), into a 4-stage ring.
+//               128 x 16-byte boxes of the row-major scale arrays), into a 6-stage ring.
 //   warp 1      MMA issuer (one thread) and TMEM owner: four K = 64 block-scaled MMAs per K
 //               block into one of two 128-column FP32 accumulators.
 //   warps 2-5   epilogue: thread = output row = TMEM lane; 32 columns at a time, scaled by
 //               sg_x sg_w, rounded to bf16, stored.
 //   warps 6-9   scale factors: per K block, each warp copies the stage's block scales from
-//               shared memory into its own lane quarter of a 4-stage TMEM ring (32 columns a
+//               shared memory into its own lane quarter of a 6-stage TMEM ring (32 columns a
 //               stage: X's, then W's), as the block-scaled MMA reads them: row r's four factors of
 //               a K = 64 step form the word at lane r % 32, column (step * 4 + r / 32), replicated
 //               in every lane quarter.
@@ -43,7 +43,10 @@ constexpr int BM = 128;                  // output rows per tile (= TMEM lanes)
 constexpr int BN = 128;                  // output columns per tile (MMA N)
 constexpr int BK = 256;                  // K elements per stage (128 bytes of E2M1 per row)
 constexpr int BKB = BK / 2;              // bytes per row per stage
-constexpr int STAGES = 4;
+#ifndef QATTN_FP4_STAGES
+#define QATTN_FP4_STAGES 6
+#endif
+constexpr int STAGES = QATTN_FP4_STAGES;
 constexpr int THREADS = 320;
 constexpr int WARP_LOAD = 0, WARP_MMA = 1, WARP_SF0 = 6;   // warps 2-5: epilogue
 constexpr int TILE_A = BM * BKB;         // 16 KB
