@@ -35,12 +35,15 @@ FP8_PER_BF16 = 2.0          # nominal dense FP8 / BF16 tensor throughput ratio o
 FP4_PER_BF16 = 4.0          # nominal dense FP4 / BF16 ratio (9 vs 2.25 PFLOP/s)
 L2_FLUSH_BYTES = 256 << 20
 # DRAM bytes (read + write) of one launch of the attention kernel at L=8704 (B=1, H=24, D=128),
-# from ncu on the current kernel (80.30 MB read + 22.40 MB written):
-#   ncu --set full --clock-control none -k regex:k_attn_fp8_pair -s 3 -c 1 -o attn_pair \
+# from ncu on the current kernel:
+#   ncu --set full --clock-control none -k regex:k_attn_fp8_fwd -s 3 -c 1 -o attn_fwd128 \
 #       python bench.py --steps 1 --warmup 3 --no-cpu-baseline --no-e2e --no-extras
-# Set to None whenever the kernel changes, until captured again.  Other shapes of the same
-# kernel: scaled by their algorithmic bytes (Q8 + K8 + V8 + bf16 output), and so marked.
-ATTN_TRAFFIC_L8704 = 102706432
+# (80.53 MB read + 26.77 MB written).  Set to None whenever the kernel changes, until captured
+# again.  Other shapes of the same kernel: scaled by their algorithmic bytes (Q8 + K8 + V8 +
+# bf16 output), and so marked.
+ATTN_TRAFFIC_L8704 = 107305728
+# the same for the pair-of-SMs variant (--pair-kernel): 80.30 MB read + 22.40 MB written
+ATTN_TRAFFIC_L8704_PAIR = 102706432
 ATTN_TRAFFIC_SOURCE = "ncu dram__bytes_read.sum + dram__bytes_write.sum, one launch, L=8704"
 # DRAM bytes (read + write) of one Q, K, V quantize launch at L=8704 (B=1, H=24, D=128), from
 #   ncu --metrics gpu__time_duration.sum,dram__bytes_read.sum,dram__bytes_write.sum,lts__t_sector_hit_rate.pct \
@@ -49,20 +52,22 @@ ATTN_TRAFFIC_SOURCE = "ncu dram__bytes_read.sum + dram__bytes_write.sum, one lau
 # keyed by (mode, static scales); None again whenever those kernels change.
 QUANT_TRAFFIC_L8704 = {("fp8", False): 207469312, ("fp8", True): 202917120,
                        ("fp4", False): 262223104, ("fp4", True): 235917824}
-ATTN_KERNEL = {128: "k_attn_fp8_pair (cluster of two CTAs per pair of Q tiles)", 64: "k_attn_fp8_fwd<64>"}
+ATTN_KERNEL = {128: "k_attn_fp8_fwd<128> (one SM per pair of Q tiles, persistent)",
+               64: "k_attn_fp8_fwd<64>"}
+ATTN_KERNEL_PAIR = "k_attn_fp8_pair (cluster of two CTAs per pair of Q tiles; opt-in variant)"
 
 
-def attn_traffic(w):
+def attn_traffic(w, pair=False):
     """(bytes per launch, how it was obtained) for the attention kernel on workload w."""
-    if ATTN_TRAFFIC_L8704 is None or w.D != 128:
+    ref = ATTN_TRAFFIC_L8704_PAIR if pair else ATTN_TRAFFIC_L8704
+    if ref is None or w.D != 128:
         return None, "not captured for this kernel"
     tokens = sum(w.seqlens) if w.varlen else w.B * w.L
     algo = tokens * w.H * w.D * (3 + 2)            # Q8, K8, V8 read; bf16 output written
     algo_ref = 8704 * 24 * 128 * (3 + 2)
     if not w.varlen and (w.L, w.H, w.B) == (8704, 24, 1):
-        return ATTN_TRAFFIC_L8704, ATTN_TRAFFIC_SOURCE
-    return ATTN_TRAFFIC_L8704 * algo / algo_ref, (ATTN_TRAFFIC_SOURCE +
-                                                  ", scaled by this workload's algorithmic bytes")
+        return ref, ATTN_TRAFFIC_SOURCE
+    return ref * algo / algo_ref, (ATTN_TRAFFIC_SOURCE + ", scaled by this workload's algorithmic bytes")
 
 
 def quant_traffic(w, static):
@@ -206,6 +211,8 @@ def replica_workload(w, rank: int, world: int):
 def run_gpu(args):
     import precision_quantized_attention_b200 as qa
     rank, world, local = dist_setup(args.gpus)
+    if args.pair_kernel:
+        qa._lib.debug_use_pair_kernel(True)
     w = workloads.WORKLOADS[args.workload or ("edit_fp8" if args.mode == "fp8" else "edit_fp4")]
     w = replica_workload(w, rank, world)
     q, k, v = workloads.make_qkv(w)
@@ -519,7 +526,9 @@ def report(args, w, qkv, rank, world, ms, attn, quant, e2e_ms, clocks, launches,
     extra = extra or {}
     in_bytes = 3 * q.numel() * 2
     quant_bytes = quantize_bytes(w, q.numel())
-    traffic, traffic_src = attn_traffic(w)
+    pair = bool(getattr(args, "pair_kernel", False)) and w.D == 128
+    kname = ATTN_KERNEL_PAIR if pair else ATTN_KERNEL[w.D]
+    traffic, traffic_src = attn_traffic(w, pair)
     clock = clocks.summary()
     quantize = {"ms": quant, "algorithmic_bytes": quant_bytes,
                 "gbs": quant_bytes / (quant * 1e-3) / 1e9,
@@ -541,14 +550,14 @@ def report(args, w, qkv, rank, world, ms, attn, quant, e2e_ms, clocks, launches,
         x = extra["fp4"]
         w4 = x.pop("w")
         qb4 = quantize_bytes(w4, x["numel"])
-        t4, t4_src = attn_traffic(w4)
+        t4, t4_src = attn_traffic(w4, pair)
         a_tf = x["flops"] / (x["attn_ms"] * 1e-3) / 1e12
         fp4 = {"workload": bench_config(w4, world)["workload"], "steps": x["steps"],
                "ms_per_step": x["step_ms"], "value": x["flops"] / (x["step_ms"] * 1e-3) / 1e12,
                "roofline": {"bound": "tensor", "achieved": a_tf, "peak": fp8_peak,
                             "unit": "TFLOP/s", "frac": a_tf / fp8_peak, "traffic": t4,
                             "traffic_source": t4_src, "kernel_ms": x["attn_ms"],
-                            "kernel": ATTN_KERNEL[w4.D]},
+                            "kernel": kname},
                "quantize": {"ms": x["quant_ms"], "algorithmic_bytes": qb4,
                             "frac_hbm": qb4 / (x["quant_ms"] * 1e-3) / 1e9 / hbm_gbs,
                             "traffic": quant_traffic(w4, False),
@@ -573,7 +582,7 @@ def report(args, w, qkv, rank, world, ms, attn, quant, e2e_ms, clocks, launches,
         "roofline": {"bound": "tensor", "achieved": achieved_tf, "peak": fp8_peak,
                      "unit": "TFLOP/s", "frac": achieved_tf / fp8_peak,
                      "traffic": traffic, "traffic_source": traffic_src,
-                     "kernel": ATTN_KERNEL[w.D],
+                     "kernel": kname,
                      "peak_source": f"{peak_kind} bf16 burst {bf16_tf} TFLOP/s x {FP8_PER_BF16} "
                                     "(nominal FP8/BF16 ratio)",
                      "fp8_measured_tflops": extra.get("fp8_measured"),
@@ -854,6 +863,8 @@ def main():
                     help="quantize with amax values calibrated once before timing (one pass)")
     ap.add_argument("--no-extras", action="store_true",
                     help="skip the static-scale quantize, FP4-mode and measured FP8 rate timings")
+    ap.add_argument("--pair-kernel", action="store_true",
+                    help="D = 128 attention on the pair-of-SMs variant (k_attn_fp8_pair)")
     ap.add_argument("--gemm", action="store_true",
                     help="time the FP8 GEMM of the transformer block's linear layers instead")
     args = ap.parse_args()

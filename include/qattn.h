@@ -323,11 +323,20 @@ QATTN_API qattn_status qattn_debug_inject_oob(int enable);
 QATTN_API void qattn_debug_set_wait_timeout_ns(uint64_t ns);
 QATTN_API void qattn_debug_inject_missing_q(int enable);
 
-/* Test hook, not part of the method: with enable != 0 the next D = 128 attention launches copy,
+/* Kernel choice for D = 128, not part of the method: with enable != 0 the next D = 128 attention
+ * launches run the pair-of-SMs kernel (two CTAs of a cluster per pair of Q tiles, cta_group::2
+ * MMAs, three S buffers in TMEM) instead of the default one-SM kernel; enable = 0 restores the
+ * default.  Same results up to FP32 summation order; the default is the faster one on B200.
+ * qattn_forward_workspace_bytes covers both. */
+QATTN_API void qattn_debug_use_pair_kernel(int enable);
+
+/* Test hook, not part of the method: with enable != 0 the next attention launches copy,
  * for query row `row` (row index within the slab's rows: the token index for dense launches,
  * the packed token index for varlen) of slab `slab` (b * H + h; the head for varlen), the E4M3
  * codes of P of every key step s into codes_dev[s * 128 + key] (key within the step) and the
- * step's integer tile maximum (base-2 units; P(s) = e4m3(2^(S' - max) * 448)) into maxima_dev[s].
+ * integer maximum they are relative to (base-2 units; P(s) = e4m3(2^(S' - max) * 448)): the
+ * running row maximum after step s in the one-SM kernel, step s's own tile maximum in the pair
+ * kernel, into maxima_dev[s].
  * codes_dev: device, 16-byte aligned, ceil(L / 128) * 128 bytes; maxima_dev: device int32,
  * ceil(L / 128) entries; both caller-owned and written only by launches made while enabled.
  * enable = 0 turns it off (the pointers are forgotten); with it off nothing of the launches

@@ -31,6 +31,7 @@ EXPORTS = (
     "qattn_forward_workspace_bytes",
     "qattn_debug_set_wait_timeout_ns", "qattn_debug_inject_missing_q", "qattn_debug_capture_p_row",
     "qattn_debug_attention_plan", "qattn_build_info", "qattn_debug_inject_oob",
+    "qattn_debug_use_pair_kernel",
 )
 _RETURNS_STATUS = EXPORTS[:15]
 FUSED_WORKSPACE_BYTES = 256     # QATTN_FUSED_WORKSPACE_BYTES
@@ -97,6 +98,8 @@ def load() -> ctypes.CDLL:
     lib.qattn_debug_set_wait_timeout_ns.restype = None
     lib.qattn_debug_inject_missing_q.argtypes = [I]
     lib.qattn_debug_inject_missing_q.restype = None
+    lib.qattn_debug_use_pair_kernel.argtypes = [I]
+    lib.qattn_debug_use_pair_kernel.restype = None
     lib.qattn_build_info.argtypes = []
     lib.qattn_build_info.restype = I
     lib.qattn_debug_inject_oob.argtypes = [I]
@@ -368,6 +371,11 @@ def debug_inject_missing_q(enable: bool):
     load().qattn_debug_inject_missing_q(1 if enable else 0)
 
 
+def debug_use_pair_kernel(enable: bool):
+    """D = 128 attention on the pair-of-SMs kernel instead of the default one-SM kernel."""
+    load().qattn_debug_use_pair_kernel(1 if enable else 0)
+
+
 def build_info() -> int:
     """Bit 0: the loaded library is the checked build (QATTN_DEBUG=1)."""
     return int(load().qattn_build_info())
@@ -381,8 +389,9 @@ def debug_inject_oob(enable: bool):
 
 def debug_capture_p_row(enable: bool, slab: int = 0, row: int = 0, codes: torch.Tensor = None,
                         maxima: torch.Tensor = None):
-    """Test hook: the next D = 128 attention launches copy row `row` of slab `slab`'s P codes
-    (uint8 [steps * 128]) and tile maxima (int32 [steps]) into the given device tensors."""
+    """Test hook: the next attention launches copy row `row` of slab `slab`'s P codes
+    (uint8 [steps * 128]) and the integer maxima they are relative to (int32 [steps]) into the
+    given device tensors."""
     if not enable:
         _check(load().qattn_debug_capture_p_row(0, 0, 0, None, None), "qattn_debug_capture_p_row")
         return

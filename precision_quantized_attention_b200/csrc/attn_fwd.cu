@@ -104,6 +104,10 @@ struct AttnArgs {
   // slabs * rows_per_slab rows) and rows of partial results the workspace holds
   int slabs;
   long long part_rows;
+  // test hook (DebugHooks): P codes and maxima of one query row, or dbg_p == nullptr
+  uint8_t* dbg_p;
+  int* dbg_m;
+  int dbg_slab, dbg_row, dbg_steps;
 };
 
 // One unit of a CTA's work: key steps [kv0, kv1) of one pair of Q tiles.
@@ -189,7 +193,9 @@ struct TmemCols {
   static constexpr uint32_t ALLOC = USED <= 256 ? 256 : 512;
 };
 
-template <int D>
+// CAPTURE: the instance with the P-code test hook (launched only while a capture is armed); the
+// instance without it is the one every other launch runs, so the hook costs nothing there.
+template <int D, bool CAPTURE>
 __global__ void __launch_bounds__(ATTN_THREADS, 1)
     k_attn_fp8_fwd(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ AttnArgs args) {
@@ -460,6 +466,11 @@ __global__ void __launch_bounds__(ATTN_THREADS, 1)
         for (int q = 0; q < 4; ++q)
           pk[i / 4 + q] = cvt_e4m3x2(p[4 * q], p[4 * q + 1]) | (cvt_e4m3x2(p[4 * q + 2], p[4 * q + 3]) << 16);
       }
+      if constexpr (CAPTURE) {                                                  // test hook
+        if (sg.slab == args.dbg_slab && sg.seq_start + sg.q_row0 + t * BLOCK_M + r == args.dbg_row &&
+            QATTN_IN_BOUNDS(args.err, sg.kv0 + j < args.dbg_steps))
+          capture_p_codes(args.dbg_p, args.dbg_m, sg.kv0 + j, pk, m_new);
+      }
       const float rowsum = ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
       // P(j) is relative to m_new and enters O scaled by 2^(m_new - m_ref) (BMM2's scale factor),
       // so a rise of the running max leaves O alone.  Only a gap beyond 2^64, which could carry
@@ -689,14 +700,20 @@ static cudaError_t launch_attn_d(const void* q8, const void* k8, const void* v8,
   if (!make_map(&mq, q8, D, rows_per_slab, slabs) || !make_map(&mk, k8, D, rows_per_slab, slabs) ||
       !make_map(&mv, v8, D, rows_per_slab, slabs))
     return cudaErrorInvalidValue;
-  static DeviceOnce smem_attr;                  // per device and per D, set once
+  static DeviceOnce smem_attr;                  // per device and per D, set once (both instances)
   const cudaError_t ea = static_cast<cudaError_t>(smem_attr.get([] {
-    return static_cast<int>(cudaFuncSetAttribute(k_attn_fp8_fwd<D>,
-                                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                 Smem<D>::ALLOC));
+    cudaError_t e0 = cudaFuncSetAttribute(k_attn_fp8_fwd<D, false>,
+                                          cudaFuncAttributeMaxDynamicSharedMemorySize, Smem<D>::ALLOC);
+    if (e0 == cudaSuccess)
+      e0 = cudaFuncSetAttribute(k_attn_fp8_fwd<D, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                Smem<D>::ALLOC);
+    return static_cast<int>(e0);
   }));
   if (ea != cudaSuccess) return ea;
-  k_attn_fp8_fwd<D><<<grid, ATTN_THREADS, Smem<D>::ALLOC, stream>>>(mq, mk, mv, a);
+  if (a.dbg_p != nullptr)
+    k_attn_fp8_fwd<D, true><<<grid, ATTN_THREADS, Smem<D>::ALLOC, stream>>>(mq, mk, mv, a);
+  else
+    k_attn_fp8_fwd<D, false><<<grid, ATTN_THREADS, Smem<D>::ALLOC, stream>>>(mq, mk, mv, a);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess || combine_ctas == 0) return e;
   k_attn_combine<D><<<combine_ctas, COMBINE_WARPS * 32, 0, stream>>>(a);
@@ -742,8 +759,8 @@ AttnSplitPlan plan_attention_split(int B, int H, int L, int D, int num_sms) {
   return p;
 }
 
-AttnSplitPlan attention_plan(int B, int H, int L, int D, int num_sms) {
-  return plan_attention_split(B, H, L, D, D == 128 ? attention_pair_units(num_sms) : num_sms);
+AttnSplitPlan attention_plan(int B, int H, int L, int D, int num_sms, bool pair) {
+  return plan_attention_split(B, H, L, D, (D == 128 && pair) ? attention_pair_units(num_sms) : num_sms);
 }
 
 cudaError_t launch_attention(const uint8_t* q8, const uint8_t* k8, const uint8_t* v8, void* out,
@@ -769,6 +786,11 @@ cudaError_t launch_attention(const uint8_t* q8, const uint8_t* k8, const uint8_t
   a.part_o = nullptr;
   a.part_ml = nullptr;
   a.part_rows = 0;
+  a.dbg_p = dbg.p_codes;
+  a.dbg_m = dbg.p_maxima;
+  a.dbg_slab = dbg.p_slab;
+  a.dbg_row = dbg.p_row;
+  a.dbg_steps = ((varlen ? max_seqlen : L) + BLOCK_N - 1) / BLOCK_N;
   a.pairs_per_head = 0;
   a.nkv = 0;
   a.ctas = 0;
@@ -776,6 +798,7 @@ cudaError_t launch_attention(const uint8_t* q8, const uint8_t* k8, const uint8_t
   a.tail_pairs = 0;
   a.tail_w = 1;
   const int slabs = varlen ? H : B * H;
+  const bool pair = D == 128 && dbg.attn_pair != 0;   // the pair-of-SMs variant, when selected
   a.slabs = slabs;
   dim3 grid;
   int combine_ctas = 0;
@@ -783,7 +806,7 @@ cudaError_t launch_attention(const uint8_t* q8, const uint8_t* k8, const uint8_t
   if (varlen) {
     grid = dim3((max_seqlen + NQ * BLOCK_M - 1) / (NQ * BLOCK_M), H, nseq);
   } else {
-    p = attention_plan(B, H, L, D, num_sms);
+    p = attention_plan(B, H, L, D, num_sms, pair);
     if (workspace == nullptr || workspace_bytes < p.bytes) {   // no workspace: no pair is cut
       p.tail_w = p.nkv;
       p.bytes = 0;
@@ -803,7 +826,7 @@ cudaError_t launch_attention(const uint8_t* q8, const uint8_t* k8, const uint8_t
     }
     grid = dim3(p.ctas, 1, 1);
   }
-  if (D == 128) {
+  if (pair) {
     // pairs of SMs: the two Q tiles of a pair on the two CTAs of a cluster (attn_pair.cu)
     cudaError_t e = launch_attention_pair(q8, k8, v8, out, H, L, cu_seqlens, nseq, max_seqlen,
                                           a.rows_per_slab, slabs, s_q, s_k, s_v, sm_scale, err,
@@ -813,6 +836,8 @@ cudaError_t launch_attention(const uint8_t* q8, const uint8_t* k8, const uint8_t
     k_attn_combine<128><<<combine_ctas, COMBINE_WARPS * 32, 0, stream>>>(a);
     return cudaGetLastError();
   }
+  if (D == 128)
+    return launch_attn_d<128>(q8, k8, v8, a, a.rows_per_slab, slabs, grid, combine_ctas, stream);
   return launch_attn_d<64>(q8, k8, v8, a, a.rows_per_slab, slabs, grid, combine_ctas, stream);
 }
 

@@ -222,15 +222,11 @@ struct StepCursor {
 
 }  // namespace
 
-// Test hook: one row's P codes of key step `step` (word w: keys 4w..4w+3) and the step's tile
-// maximum, to the caller's buffers.
+// Test hook (see capture_p_codes), with the checked build's test of the step index.
 __device__ __forceinline__ void capture_p_row(const PairArgs& args, int step, const uint32_t (&pk)[32],
                                            float mx) {
   if (!QATTN_IN_BOUNDS(args.err, step < args.dbg_steps)) return;
-  uint4* dst = reinterpret_cast<uint4*>(args.dbg_p + static_cast<size_t>(step) * pairk::BLOCK_N);
-#pragma unroll
-  for (int i = 0; i < 8; ++i) dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
-  args.dbg_m[step] = static_cast<int>(mx);
+  capture_p_codes(args.dbg_p, args.dbg_m, step, pk, mx);
 }
 
 // Multiplies this thread's row of O (128 FP32 columns of its TMEM lane) by f, 8 columns at a

@@ -50,6 +50,7 @@ cudaError_t launch_gemm_fp8(const uint8_t* a8, const uint8_t* b8, void* y, int M
 // tile maximum into p_maxima[step].
 struct DebugHooks {
   int inject_missing_q = 0;
+  int attn_pair = 0;               // D = 128 launches run the pair-of-SMs kernel (attn_pair.cu)
   int inject_oob = 0;              // checked build only: qattn_quantize_fp8 loops one vector past n
   uint8_t* p_codes = nullptr;
   int* p_maxima = nullptr;
@@ -80,10 +81,11 @@ struct AttnSplitPlan {
 };
 AttnSplitPlan plan_attention_split(int B, int H, int L, int D, int num_sms);
 
-// Units of the persistent dense grid on the current device: SMs for D = 64 (one-SM kernel),
-// resident pair clusters for D = 128 (pair kernel); and the plan the launch uses for them.
+// Units of the persistent dense grid on the current device: SMs for the one-SM kernel,
+// resident pair clusters for the pair kernel (D = 128, when selected); and the plan the launch
+// uses for them.
 int attention_pair_units(int num_sms);
-AttnSplitPlan attention_plan(int B, int H, int L, int D, int num_sms);
+AttnSplitPlan attention_plan(int B, int H, int L, int D, int num_sms, bool pair);
 
 // The D = 128 pair kernel (attn_pair.cu): dense with `plan` (workspace may be null when the plan
 // cuts no pair), or varlen with plan == nullptr.

@@ -313,7 +313,7 @@ qattn_status qattn_forward_ws(const uint8_t* q8, const uint8_t* k8, const uint8_
   st = device_info(&d);
   if (st != QATTN_OK) return st;
   if (workspace_dev != nullptr &&
-      workspace_bytes < qattn::attention_plan(B, H, L, D, d->num_sms).bytes)
+      workspace_bytes < qattn::attention_plan(B, H, L, D, d->num_sms, g_dbg.attn_pair != 0).bytes)
     return QATTN_ERR_INVALID_ARG;
   if (p_unquantized(mode)) {
     if (static_cast<int64_t>(B) * H > 65535) return QATTN_ERR_UNSUPPORTED;
@@ -340,7 +340,10 @@ size_t qattn_forward_workspace_bytes(int B, int H, int L, int D) {
   if (B < 1 || H < 1 || L < 1 || (D != 64 && D != 128)) return 0;
   DeviceInfo* d = nullptr;
   if (device_info(&d) != QATTN_OK) return 0;
-  return qattn::attention_plan(B, H, L, D, d->num_sms).bytes;
+  // enough for either D = 128 kernel, so a workspace stays valid if the variant is switched
+  const size_t one_sm = qattn::attention_plan(B, H, L, D, d->num_sms, false).bytes;
+  const size_t pair = D == 128 ? qattn::attention_plan(B, H, L, D, d->num_sms, true).bytes : 0;
+  return one_sm > pair ? one_sm : pair;
 }
 
 qattn_status qattn_forward_varlen(const uint8_t* q8, const uint8_t* k8, const uint8_t* v8,
@@ -410,6 +413,8 @@ void qattn_debug_set_wait_timeout_ns(uint64_t ns) {
 }
 
 void qattn_debug_inject_missing_q(int enable) { g_dbg.inject_missing_q = enable ? 1 : 0; }
+
+void qattn_debug_use_pair_kernel(int enable) { g_dbg.attn_pair = enable ? 1 : 0; }
 
 int qattn_build_info(void) {
 #ifdef QATTN_CHECKED

@@ -122,4 +122,15 @@ __device__ __forceinline__ float rowmax128(const float (&s)[128]) {
   return max3f(max3f(m[0], m[1], m[2]), max3f(m[3], m[4], m[5]), fmaxf(m[6], m[7]));
 }
 
+// Test hook of the attention kernels: one row's P codes of a key step (word w: keys 4w..4w+3)
+// and the integer maximum they are relative to, to the caller's buffers (codes + 128 * step,
+// maxima + step).
+__device__ __forceinline__ void capture_p_codes(uint8_t* codes, int* maxima, int step,
+                                                const uint32_t (&pk)[32], float mx) {
+  uint4* dst = reinterpret_cast<uint4*>(codes + static_cast<size_t>(step) * 128);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+  maxima[step] = static_cast<int>(mx);
+}
+
 }  // namespace qattn

@@ -282,3 +282,47 @@ def test_p_unquantized_switch_matches_the_oracle_without_p_quantization(name, mo
     rel_p, _ = compare(quantized, want)
     print(f"{name}: error of the P codes alone (rel-L2) {rel_p:.2e}")
     assert 0.0 < rel_p < 3e-2
+
+
+# --- the pair-of-SMs variant of the D = 128 kernel (qattn_debug_use_pair_kernel) -------------
+@pytest.fixture
+def pair_kernel():
+    qa._lib.debug_use_pair_kernel(True)
+    try:
+        yield
+    finally:
+        qa._lib.debug_use_pair_kernel(False)
+
+
+@pytest.mark.parametrize("name,mode,B,H,L,D", [c for c in SMALL if c[5] == 128])
+def test_pair_kernel_small_shapes_all_rows(pair_kernel, name, mode, B, H, L, D):
+    test_small_shapes_all_rows(name, mode, B, H, L, D)
+
+
+@pytest.mark.parametrize("lens", [[1, 5, 200, 129], [513]])
+def test_pair_kernel_varlen_small_all_rows(pair_kernel, lens):
+    test_varlen_small_all_rows(lens)
+
+
+def test_pair_kernel_cut_tail_pairs_match_uncut_and_oracle(pair_kernel):
+    test_cut_tail_pairs_match_uncut_and_oracle(1, 24, 8704, 128)
+
+
+def test_pair_kernel_equals_the_one_sm_kernel_on_the_editing_workload():
+    """Both D = 128 kernels compute the same method: on edit_fp8 their outputs differ only by
+    FP32 summation order and the E4M3 subnormal-range codes of the pair kernel's per-tile
+    maxima (reading 7)."""
+    w = workloads.WORKLOADS["edit_fp8"]
+    q, k, v = workloads.make_qkv(w)
+    path = gpu_path(w, q, k, v)
+    one = path.out.float().clone()
+    qa._lib.debug_use_pair_kernel(True)
+    try:
+        path.attend()
+        assert qa.get_error() == 0
+    finally:
+        qa._lib.debug_use_pair_kernel(False)
+    two = path.out.float()
+    rel = float((two - one).norm() / one.norm())
+    print(f"pair vs one-SM kernel: rel-L2 {rel:.2e}, max-abs {float((two - one).abs().max()):.2e}")
+    assert rel < 1e-3

@@ -9,12 +9,13 @@ workload with outlier channels, rows are nearly one-hot and one such code can mo
 few percent.  This test takes the sampled row whose output is farthest from the oracle (and a few
 ordinary rows), captures every P code the kernel computes for it (qattn_debug_capture_p_row), and
 checks each against the oracle's code for that key:
-  * equal after the exact rescaling 2^(tile max - M) (the kernel quantizes P relative to its tile's
-    integer maximum, the oracle relative to the row's; E4M3 rounding commutes with powers of two
-    in the normal range), or
+  * equal after the exact rescaling 2^(max - M), max the integer maximum the kernel quantized
+    that step relative to (the running row maximum, or the tile's own maximum in the pair
+    kernel), M the oracle's row maximum (E4M3 rounding commutes with powers of two in the normal
+    range), or
   * inside the oracle's admissible range [lo, hi] of that key (an accumulation-order tie), or
   * for an oracle code in E4M3's subnormal range (below 2^-6), within one subnormal step 2^-9
-    (the kernel's finer scale rounds such values on a finer grid).
+    (a kernel scale below the row's rounds such values on a finer grid).
 Anything else would be a kernel error."""
 import numpy as np
 import pytest
@@ -60,7 +61,18 @@ def _classify(w, path, q8, k8, row, tbl):
             "subnormal": int(np.sum(sub)), "bad": np.flatnonzero(bad), "M": M}
 
 
-def test_edit_fp8_p_codes_differ_only_by_admissible_ties():
+@pytest.mark.parametrize("pair", [False, True], ids=["one_sm_kernel", "pair_kernel"])
+def test_edit_fp8_p_codes_differ_only_by_admissible_ties(pair):
+    """Both D = 128 kernels: the default one-SM kernel (codes relative to the running row
+    maximum) and the pair-of-SMs variant (codes relative to each tile's own maximum)."""
+    qa._lib.debug_use_pair_kernel(pair)
+    try:
+        _check_edit_fp8_p_codes()
+    finally:
+        qa._lib.debug_use_pair_kernel(False)
+
+
+def _check_edit_fp8_p_codes():
     w = workloads.WORKLOADS["edit_fp8"]
     q, k, v = workloads.make_qkv(w)
     path = gpu_path(w, q, k, v)
