@@ -7,9 +7,13 @@ FLOPs of BMM1 + BMM2 (4 * H * D * L^2) per second.  The L2 is flushed between st
 256 MiB write, then a 256 MiB read of another buffer, outside the timed events).  ``e2e`` repeats the measurement through the same C ABI
 with the bf16 inputs in pinned host memory: every step copies Q, K, V to the device and the
 output back.  ``--impl reference`` times the CPU oracle instead (rank 0 only) on a bounded row
-sample of the same workload.
+sample of the same workload.  Extras in the same line (skipped by ``--no-extras``): the static
+-scale quantize, FP4 mode on the same shape, the varlen FP4 batch, and the measured FP8 GEMM
+rate next to the derived peak.  ``--gemm`` prints the line of the block's linear layers instead
+(FP8 and FP4 GEMMs, the V projection with its fused E4M3 epilogue).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference] [--mode fp8|fp4]
+                    [--workload NAME] [--static-scales] [--no-extras] [--pair-kernel] [--gemm]
 Multi-GPU (launched with torchrun): every rank runs its own replica of the workload (weak
 scaling, no data-path collective); time is the max over ranks.
 """
@@ -279,6 +283,9 @@ def run_gpu(args):
         if w.name == "edit_fp8" and world == 1:
             extra["fp4"] = run_mode_extra(workloads.WORKLOADS["edit_fp4"], flush, min(args.steps, 100),
                                           args.warmup)
+            # the varlen batch of four packed sequences (FP4), the same way
+            extra["varlen_fp4"] = run_mode_extra(workloads.WORKLOADS["varlen_fp4"], flush,
+                                                 min(args.steps, 50), args.warmup)
         extra["fp8_measured"] = measured_fp8_rates(flush)
     report(args, w, (q, k, v), rank, world, ms, attn, quant, e2e_ms, clocks, launches, extra)
     barrier(world)
@@ -545,26 +552,28 @@ def report(args, w, qkv, rank, world, ms, attn, quant, e2e_ms, clocks, launches,
                               "traffic": quant_traffic(w, True),
                               "path": "static scales (qattn_quantize_qkv, one pass), the amax "
                                       "calibrated in the timed steps"}
-    fp4 = None
-    if "fp4" in extra:
-        x = extra["fp4"]
+    def mode_block(x):
+        """The JSON block of a workload timed by run_mode_extra."""
         w4 = x.pop("w")
         qb4 = quantize_bytes(w4, x["numel"])
         t4, t4_src = attn_traffic(w4, pair)
         a_tf = x["flops"] / (x["attn_ms"] * 1e-3) / 1e12
-        fp4 = {"workload": bench_config(w4, world)["workload"], "steps": x["steps"],
-               "ms_per_step": x["step_ms"], "value": x["flops"] / (x["step_ms"] * 1e-3) / 1e12,
-               "roofline": {"bound": "tensor", "achieved": a_tf, "peak": fp8_peak,
-                            "unit": "TFLOP/s", "frac": a_tf / fp8_peak, "traffic": t4,
-                            "traffic_source": t4_src, "kernel_ms": x["attn_ms"],
-                            "kernel": kname},
-               "quantize": {"ms": x["quant_ms"], "algorithmic_bytes": qb4,
-                            "frac_hbm": qb4 / (x["quant_ms"] * 1e-3) / 1e9 / hbm_gbs,
-                            "traffic": quant_traffic(w4, False),
-                            "static": {"ms": x["quant_static_ms"],
-                                       "frac_hbm": qb4 / (x["quant_static_ms"] * 1e-3) / 1e9 / hbm_gbs,
-                                       "traffic": quant_traffic(w4, True)}},
-               "fp4_direct_estimate": x.get("fp4_direct")}
+        return {"workload": bench_config(w4, world)["workload"], "steps": x["steps"],
+                "ms_per_step": x["step_ms"], "value": x["flops"] / (x["step_ms"] * 1e-3) / 1e12,
+                "roofline": {"bound": "tensor", "achieved": a_tf, "peak": fp8_peak,
+                             "unit": "TFLOP/s", "frac": a_tf / fp8_peak, "traffic": t4,
+                             "traffic_source": t4_src, "kernel_ms": x["attn_ms"],
+                             "kernel": kname},
+                "quantize": {"ms": x["quant_ms"], "algorithmic_bytes": qb4,
+                             "frac_hbm": qb4 / (x["quant_ms"] * 1e-3) / 1e9 / hbm_gbs,
+                             "traffic": quant_traffic(w4, False),
+                             "static": {"ms": x["quant_static_ms"],
+                                        "frac_hbm": qb4 / (x["quant_static_ms"] * 1e-3) / 1e9 / hbm_gbs,
+                                        "traffic": quant_traffic(w4, True)}},
+                "fp4_direct_estimate": x.get("fp4_direct")}
+
+    fp4 = mode_block(extra["fp4"]) if "fp4" in extra else None
+    varlen = mode_block(extra["varlen_fp4"]) if "varlen_fp4" in extra else None
     result = {
         "metric": "quantized attention TFLOP/s @L=8704,H=24,D=128 and % of B200 FP8 peak",
         "value": world * flops / (ms * 1e-3) / 1e12,
@@ -589,6 +598,7 @@ def report(args, w, qkv, rank, world, ms, attn, quant, e2e_ms, clocks, launches,
                      "kernel_ms": attn},
         "quantize": quantize,
         "fp4": fp4,
+        "varlen_fp4": varlen,
         "e2e": {"value": world * flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
                 "ms_per_step": e2e_ms, "h2d_bytes_per_step": in_bytes,
                 "d2h_bytes_per_step": q.numel() * 2,
