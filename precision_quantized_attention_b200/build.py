@@ -19,7 +19,8 @@ LIB = os.path.join(HERE, "libqattn.so")
 LIB_CHECKED = os.path.join(HERE, "libqattn_checked.so")
 SOURCES = ["qattn_api.cu", "quant.cu", "attn_fwd.cu", "attn_pair.cu", "attn_debug.cu", "noalloc.cu",
            "gemm_fp8.cu", "gemm_fp4.cu"]
-HEADERS = ["sm100_ptx.cuh", "softmax_sm100.cuh", "launch.h", "device_once.h", "quant_math.cuh"]
+HEADERS = ["sm100_ptx.cuh", "softmax_sm100.cuh", "launch.h", "device_once.h", "quant_math.cuh",
+           "tensor_map.h"]
 
 
 def nvcc() -> str:

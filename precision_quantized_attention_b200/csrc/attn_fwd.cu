@@ -55,6 +55,7 @@
 #include <cstdint>
 
 #include "device_once.h"
+#include "tensor_map.h"
 #include "launch.h"
 #include "sm100_ptx.cuh"
 #include "softmax_sm100.cuh"
@@ -658,26 +659,10 @@ __global__ void __launch_bounds__(COMBINE_WARPS * 32) k_attn_combine(const AttnA
 // ---------------------------------------------------------------------------------------------
 // Host side: tensor maps and launch
 // ---------------------------------------------------------------------------------------------
-using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
-                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
-                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-static EncodeTiledFn get_encode_fn() {
-  static const EncodeTiledFn fn = [] {          // initialised once, thread-safe
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
-        q != cudaDriverEntryPointSuccess)
-      return static_cast<EncodeTiledFn>(nullptr);
-    return reinterpret_cast<EncodeTiledFn>(p);
-  }();
-  return fn;
-}
 
 // 3-D map over an E4M3 tensor viewed as [slabs][rows][D]: box = one 128-row tile of one slab.
 static bool make_map(CUtensorMap* map, const void* ptr, int D, int rows, int slabs) {
-  EncodeTiledFn enc = get_encode_fn();
+  EncodeTiledFn enc = encode_tiled_fn();
   if (!enc) return false;
   cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(rows),
                         static_cast<cuuint64_t>(slabs)};

@@ -59,6 +59,7 @@
 #include <cstdint>
 
 #include "device_once.h"
+#include "tensor_map.h"
 #include "launch.h"
 #include "sm100_ptx.cuh"
 #include "softmax_sm100.cuh"
@@ -652,28 +653,12 @@ __global__ void __cluster_dims__(2, 1, 1) __maxnreg__(168)
 // ---------------------------------------------------------------------------------------------
 // Host side
 // ---------------------------------------------------------------------------------------------
-using PairEncodeFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
-                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
-                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-static PairEncodeFn pair_encode_fn() {
-  static PairEncodeFn fn = [] {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
-        q != cudaDriverEntryPointSuccess)
-      return static_cast<PairEncodeFn>(nullptr);
-    return reinterpret_cast<PairEncodeFn>(p);
-  }();
-  return fn;
-}
 
 // 3-D map over an E4M3 tensor viewed as [slabs][rows][128]: box = box_inner bytes x box_rows rows
 // of one slab, swizzle matching the inner box width (128 or 64 bytes).
 static bool pair_map(CUtensorMap* map, const void* ptr, int rows, int slabs, int box_inner,
                      int box_rows) {
-  PairEncodeFn enc = pair_encode_fn();
+  EncodeTiledFn enc = encode_tiled_fn();
   if (!enc) return false;
   constexpr int D = pairk::D;
   cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(rows),

@@ -33,6 +33,7 @@
 #include <cstdint>
 
 #include "device_once.h"
+#include "tensor_map.h"
 #include "launch.h"
 #include "sm100_ptx.cuh"
 
@@ -275,27 +276,11 @@ __global__ void __launch_bounds__(gemm4::THREADS, 1)
 // ---------------------------------------------------------------------------------------------
 // Host side
 // ---------------------------------------------------------------------------------------------
-using Gemm4EncodeFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
-                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
-                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-static Gemm4EncodeFn gemm4_encode_fn() {
-  static const Gemm4EncodeFn fn = [] {          // initialised once, thread-safe
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
-        q != cudaDriverEntryPointSuccess)
-      return static_cast<Gemm4EncodeFn>(nullptr);
-    return reinterpret_cast<Gemm4EncodeFn>(p);
-  }();
-  return fn;
-}
 
 // Packed E2M1 [rows, K / 2 bytes]; box of 128 rows x 128 bytes, 128-byte swizzle; reads past the
 // last row return zeros.
 static bool make_map_e2m1(CUtensorMap* map, const void* ptr, int rows, int K) {
-  Gemm4EncodeFn enc = gemm4_encode_fn();
+  EncodeTiledFn enc = encode_tiled_fn();
   if (!enc) return false;
   cuuint64_t dims[2] = {static_cast<cuuint64_t>(K / 2), static_cast<cuuint64_t>(rows)};
   cuuint64_t strides[1] = {static_cast<cuuint64_t>(K / 2)};
@@ -309,7 +294,7 @@ static bool make_map_e2m1(CUtensorMap* map, const void* ptr, int rows, int K) {
 // Block scales [rows, K / 16] bytes, row-major; box of 128 rows x 16 bytes (one K block's
 // factors), no swizzle; rows past the last read as zeros.
 static bool make_map_scales(CUtensorMap* map, const void* ptr, int rows, int K) {
-  Gemm4EncodeFn enc = gemm4_encode_fn();
+  EncodeTiledFn enc = encode_tiled_fn();
   if (!enc) return false;
   cuuint64_t dims[2] = {static_cast<cuuint64_t>(K / 16), static_cast<cuuint64_t>(rows)};
   cuuint64_t strides[1] = {static_cast<cuuint64_t>(K / 16)};

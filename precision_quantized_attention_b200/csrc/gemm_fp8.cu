@@ -27,6 +27,7 @@
 #include <cstdint>
 
 #include "device_once.h"
+#include "tensor_map.h"
 #include "quant_math.cuh"
 #include "launch.h"
 #include "sm100_ptx.cuh"
@@ -455,27 +456,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(gemm2::THREADS, 1)
 // ---------------------------------------------------------------------------------------------
 // Host side
 // ---------------------------------------------------------------------------------------------
-using GemmEncodeFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
-                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
-                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-static GemmEncodeFn gemm_encode_fn() {
-  static const GemmEncodeFn fn = [] {           // initialised once, thread-safe
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
-        q != cudaDriverEntryPointSuccess)
-      return static_cast<GemmEncodeFn>(nullptr);
-    return reinterpret_cast<GemmEncodeFn>(p);
-  }();
-  return fn;
-}
 
 // [rows, K] E4M3, K contiguous; box of `box_rows` rows x 128 bytes, 128-byte swizzle; reads past
 // the last row return zeros.
 static bool make_map_2d(CUtensorMap* map, const void* ptr, int rows, int K, int box_rows) {
-  GemmEncodeFn enc = gemm_encode_fn();
+  EncodeTiledFn enc = encode_tiled_fn();
   if (!enc) return false;
   cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(rows)};
   cuuint64_t strides[1] = {static_cast<cuuint64_t>(K)};
