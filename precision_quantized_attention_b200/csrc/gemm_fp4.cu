@@ -86,6 +86,22 @@ struct Gemm4Args {
   uint64_t timeout_ns;
 };
 
+// 32 FP32 accumulator columns of one row, scaled, rounded to bf16 and stored (four 16-byte
+// stores; y 16-byte aligned).
+__device__ __forceinline__ void store_bf16_32(__nv_bfloat16* y, const uint32_t (&v)[32], float scale) {
+  uint32_t packed[16];
+#pragma unroll
+  for (int e = 0; e < 16; ++e) {
+    const __nv_bfloat162 b2 = __floats2bfloat162_rn(__uint_as_float(v[2 * e]) * scale,
+                                                    __uint_as_float(v[2 * e + 1]) * scale);
+    packed[e] = *reinterpret_cast<const uint32_t*>(&b2);
+  }
+  uint4* dst = reinterpret_cast<uint4*>(y);
+#pragma unroll
+  for (int e = 0; e < 4; ++e)
+    dst[e] = make_uint4(packed[4 * e], packed[4 * e + 1], packed[4 * e + 2], packed[4 * e + 3]);
+}
+
 __global__ void __launch_bounds__(gemm4::THREADS, 1)
     k_gemm_fp4(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
                const __grid_constant__ CUtensorMap tm_sa, const __grid_constant__ CUtensorMap tm_sb,
@@ -246,19 +262,8 @@ __global__ void __launch_bounds__(gemm4::THREADS, 1)
         const size_t off = static_cast<size_t>(m) * args.N + n0 + c * 32;
         // N % 32 == 0: a 32-column chunk is all in or all out
         if (m < args.M && n0 + c * 32 < args.N &&
-            QATTN_IN_BOUNDS(args.err, off + 32 <= static_cast<size_t>(args.M) * args.N)) {
-          uint32_t packed[16];
-#pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const __nv_bfloat162 b2 = __floats2bfloat162_rn(__uint_as_float(v[2 * e]) * scale,
-                                                            __uint_as_float(v[2 * e + 1]) * scale);
-            packed[e] = *reinterpret_cast<const uint32_t*>(&b2);
-          }
-          uint4* dst = reinterpret_cast<uint4*>(args.y + off);
-#pragma unroll
-          for (int e = 0; e < 4; ++e)
-            dst[e] = make_uint4(packed[4 * e], packed[4 * e + 1], packed[4 * e + 2], packed[4 * e + 3]);
-        }
+            QATTN_IN_BOUNDS(args.err, off + 32 <= static_cast<size_t>(args.M) * args.N))
+          store_bf16_32(args.y + off, v, scale);
       }
       tc_fence_before();
       mbar_arrive(BAR(B_ACCE + ab));               // accumulator read out
@@ -274,31 +279,301 @@ __global__ void __launch_bounds__(gemm4::THREADS, 1)
 }
 
 // ---------------------------------------------------------------------------------------------
+// Pair kernel (M > 128): two SMs (a cluster of two CTAs) on one 256 x 192 output tile.
+//
+// One tcgen05.mma.cta_group::2.kind::mxf4nvf4 with M = 256, N = 192 reads 128 rows of X and 96
+// rows of W from each CTA's shared memory and leaves 128 rows x 192 columns of the FP32 tile in
+// each CTA's TMEM.  Each CTA's TMEM also holds the block scales of its own 128 rows of X and of
+// all 192 rows of W (the MMA reads W's factors of the whole N = 192 from each CTA: N / 32 = 6
+// consecutive columns per K = 64 step), in the one-SM layout.  Per K block an SM stages 28 KB
+// of operands (not 32 KB as on one SM for a third less MMA work).  TMEM per CTA: two
+// 192-column accumulators and a 3-slot factor ring of 40 columns (16 of X's factors, 24 of W's)
+// fit in the 512 columns, which is why N is 192 and not 256; the shared-memory ring has 6
+// stages, the factor ring 3 slots (slot u % 3 is refilled once the MMAs of step u - 3 completed).
+//   warp 0 (both CTAs)  TMA producer: its halves of X and W counted on the leading CTA's `full`
+//                       barrier; the block scales of its own X rows and of the tile's 192 W rows
+//                       (two boxes, no pair form) on its own `sf_data` barrier.
+//   warp 1              TMEM owner in both CTAs; in the leading CTA, one thread issues the MMAs
+//                       and commits `empty` / `acc_full` to the barriers of both CTAs.
+//   warps 2-5 (both)    epilogue of the CTA's 128 rows; each warp arrives once per tile on the
+//                       leading CTA's `acc_empty` (8 arrivals release an accumulator).
+//   warps 6-9 (both)    scale factors: once a stage's boxes landed and the factor slot is free,
+//                       copy them into the CTA's TMEM ring and arrive on the leading CTA's
+//                       `sf_full` (8 arrivals).
+// Both CTAs reach the two cluster barriers (after set-up, before the TMEM free) on every path:
+// every wait in between is bounded.
+// ---------------------------------------------------------------------------------------------
+namespace gemm4p {
+constexpr int BM = 256;                  // output rows per tile pair (128 per CTA)
+constexpr int BN = 192;                  // output columns per tile (MMA N; 96 W rows per CTA)
+constexpr int BK = 256;                  // K elements per stage (128 bytes per row)
+constexpr int BKB = BK / 2;
+constexpr int STAGES = 6;                // shared-memory ring
+constexpr int SF_SLOTS = 3;              // TMEM factor ring
+constexpr int THREADS = 320;
+constexpr int WARP_LOAD = 0, WARP_MMA = 1, WARP_SF0 = 6;   // warps 2-5: epilogue
+constexpr int ROWS_A = BM / 2, ROWS_B = BN / 2;             // operand rows per CTA
+constexpr int TILE_A = ROWS_A * BKB;     // 16 KB
+constexpr int TILE_B = ROWS_B * BKB;     // 12 KB
+constexpr int TILE_SFA = ROWS_A * 16;    // 2 KB: this CTA's X rows' factors of the K block
+constexpr int TILE_SFB = BN * 16;        // 3 KB: all of the tile's W rows' factors
+constexpr int OFF_A = 0;
+constexpr int OFF_B = OFF_A + STAGES * TILE_A;
+constexpr int OFF_SFA = OFF_B + STAGES * TILE_B;
+constexpr int OFF_SFB = OFF_SFA + STAGES * TILE_SFA;
+constexpr int OFF_BAR = OFF_SFB + STAGES * TILE_SFB;
+constexpr int B_FULL = 0, B_SFDATA = STAGES, B_SFFULL = 2 * STAGES, B_EMPTY = 3 * STAGES;
+constexpr int B_ACCF = 4 * STAGES, B_ACCE = B_ACCF + 2, B_DRAIN = B_ACCE + 2, NBARS = B_DRAIN + 1;
+constexpr int OFF_TMEM = OFF_BAR + 8 * NBARS;
+constexpr int OFF_ABORT = OFF_TMEM + 4;
+constexpr int BYTES = OFF_ABORT + 4;
+constexpr int ALLOC = BYTES + 1024;
+static_assert(TILE_A % 1024 == 0 && TILE_B % 1024 == 0 && OFF_SFA % 1024 == 0, "alignment");
+static_assert(TILE_SFB % 128 == 0, "scale boxes stay 128-byte aligned");
+static_assert(ALLOC <= 227 * 1024, "shared memory per CTA");
+// factor slot f at SF0 + 40 f: X's factors of step kk in column kk * 4 + c (c < 4), W's in
+// column 16 + kk * 6 + c (c < 6), c = row / 32
+constexpr uint32_t SF0 = 2 * BN;
+constexpr uint32_t SF_COLS = 40;
+constexpr uint32_t TMEM_COLS = 512;
+static_assert(SF0 + SF_SLOTS * SF_COLS <= TMEM_COLS, "TMEM budget");
+constexpr uint32_t STAGE_TX = 2u * (TILE_A + TILE_B);     // operand bytes of both CTAs per stage
+constexpr uint32_t IDESC = idesc_mxf4_e2m1(BM, BN);
+}  // namespace gemm4p
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(gemm4p::THREADS, 1)
+    k_gemm_fp4_pair(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
+                    const __grid_constant__ CUtensorMap tm_sa, const __grid_constant__ CUtensorMap tm_sb,
+                    const __grid_constant__ Gemm4Args args) {
+  using namespace gemm4p;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_u32 = smem_u32(smem_raw);
+  const uint32_t base_u32 = (raw_u32 + 1023u) & ~1023u;   // the same offset in both CTAs
+  uint8_t* base = smem_raw + (base_u32 - raw_u32);
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();                  // 0 leads the pair
+  const bool leader = rank == 0;
+  const int pair = static_cast<int>(blockIdx.x >> 1), npairs = static_cast<int>(gridDim.x >> 1);
+
+  const int tiles_m = (args.M + BM - 1) / BM;
+  const int tiles = tiles_m * ((args.N + BN - 1) / BN);   // the host launches <= tiles pairs
+  const int kblocks = args.K / BK;
+
+  const uint32_t bar0 = base_u32 + OFF_BAR;
+  auto BAR = [&](int i) { return bar0 + 8u * static_cast<uint32_t>(i); };
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(base + OFF_ABORT);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base + OFF_TMEM);
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < STAGES; ++i) {
+      mbar_init(BAR(B_FULL + i), 1);
+      mbar_init(BAR(B_SFDATA + i), 1);
+      mbar_init(BAR(B_SFFULL + i), 8);             // 4 factor warps x 2 CTAs (leading CTA's)
+      mbar_init(BAR(B_EMPTY + i), 1);
+    }
+    for (int b = 0; b < 2; ++b) { mbar_init(BAR(B_ACCF + b), 1); mbar_init(BAR(B_ACCE + b), 8); }
+    mbar_init(BAR(B_DRAIN), 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == WARP_MMA) {
+    tmem_alloc_pair(base_u32 + OFF_TMEM, TMEM_COLS);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  cluster_sync();                      // barriers of both CTAs initialised, TMEM allocated
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint64_t tlim = args.timeout_ns;
+
+  if (warp == WARP_LOAD) {
+    // ======================= TMA producer (both CTAs) =======================
+    if (lane == 0) {
+      tma_prefetch_desc(&tm_a);
+      tma_prefetch_desc(&tm_b);
+      tma_prefetch_desc(&tm_sa);
+      tma_prefetch_desc(&tm_sb);
+      int u = 0;
+      bool ok = true;
+      for (int t = pair; ok && t < tiles; t += npairs) {
+        const int m0 = (t % tiles_m) * BM + static_cast<int>(rank) * ROWS_A;
+        const int n0 = (t / tiles_m) * BN + static_cast<int>(rank) * ROWS_B;
+        (void)QATTN_IN_BOUNDS(args.err, (t % tiles_m) * BM < args.M && (t / tiles_m) * BN < args.N);
+        for (int kb = 0; kb < kblocks; ++kb, ++u) {
+          const int s = u % STAGES;
+          if (u >= STAGES &&
+              !mbar_wait(BAR(B_EMPTY + s), ((u / STAGES) - 1) & 1, tlim, abort_flag, args.err)) {
+            ok = false;
+            break;
+          }
+          if (leader) mbar_arrive_expect_tx(BAR(B_FULL + s), STAGE_TX);
+          const uint32_t full_lead = mapa_shared(BAR(B_FULL + s), 0);
+          tma_load_2d_pair(base_u32 + OFF_A + s * TILE_A, &tm_a, full_lead, kb * BKB, m0);
+          tma_load_2d_pair(base_u32 + OFF_B + s * TILE_B, &tm_b, full_lead, kb * BKB, n0);
+          mbar_arrive_expect_tx(BAR(B_SFDATA + s), TILE_SFA + TILE_SFB);
+          tma_load_2d(base_u32 + OFF_SFA + s * TILE_SFA, &tm_sa, BAR(B_SFDATA + s), kb * 16, m0);
+          tma_load_2d(base_u32 + OFF_SFB + s * TILE_SFB, &tm_sb, BAR(B_SFDATA + s), kb * 16,
+                      (t / tiles_m) * BN);
+        }
+      }
+      // the MMAs have released every stage this CTA filled: its loads have landed and no
+      // commit from the leading CTA is still on its way here (instant when healthy)
+      for (int j = u - 1; j >= 0 && j >= u - STAGES; --j) {
+        mbar_drain(BAR(B_EMPTY + j % STAGES), (j / STAGES) & 1, tlim);
+        mbar_drain(BAR(B_SFDATA + j % STAGES), (j / STAGES) & 1, tlim);
+      }
+    }
+  } else if (warp >= WARP_SF0) {
+    // ======================= scale factors into TMEM (both CTAs) =======================
+    const int quarter = warp & 3;
+    const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+    int u = 0;
+    bool ok = true;
+    for (int t = pair; ok && t < tiles; t += npairs) {
+      for (int kb = 0; kb < kblocks; ++kb, ++u) {
+        const int s = u % STAGES, f = u % SF_SLOTS;
+        ok = mbar_wait(BAR(B_SFDATA + s), (u / STAGES) & 1, tlim, abort_flag, args.err);
+        // factor slot f was last read by the MMAs of step u - SF_SLOTS: their commit arrived on
+        // that step's `empty` barrier (in both CTAs)
+        if (ok && u >= SF_SLOTS) {
+          const int v = u - SF_SLOTS;
+          ok = mbar_wait(BAR(B_EMPTY + v % STAGES), (v / STAGES) & 1, tlim, abort_flag, args.err);
+        }
+        if (!__all_sync(0xFFFFFFFFu, ok)) { ok = false; break; }
+        // row group c: rows 32 c + lane of this CTA's X rows (c < 4) and of the W rows (c < 6)
+        const uint32_t fa0 = base_u32 + OFF_SFA + s * TILE_SFA + 16u * lane;
+        const uint32_t fb0 = base_u32 + OFF_SFB + s * TILE_SFB + 16u * lane;
+        uint32_t va[32], vb[8];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const uint4 fa = ld_shared_v4(fa0 + 512u * c);
+          va[c] = fa.x; va[4 + c] = fa.y; va[8 + c] = fa.z; va[12 + c] = fa.w;
+        }
+        // W: column 16 + kk * 6 + c of the slot, i.e. va[16 + ...] for the first 16 and vb after
+        uint32_t w[24];
+#pragma unroll
+        for (int c = 0; c < 6; ++c) {
+          const uint4 fb = ld_shared_v4(fb0 + 512u * c);
+          w[c] = fb.x; w[6 + c] = fb.y; w[12 + c] = fb.z; w[18 + c] = fb.w;
+        }
+#pragma unroll
+        for (int i = 0; i < 16; ++i) va[16 + i] = w[i];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) vb[i] = w[16 + i];
+        const uint32_t slot = tmem + lane_off + SF0 + static_cast<uint32_t>(f) * SF_COLS;
+        tmem_st32(slot, va);
+        tmem_st8(slot + 32, vb);
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(mapa_shared(BAR(B_SFFULL + s), 0));
+      }
+    }
+  } else if (warp == WARP_MMA) {
+    // ======================= MMA issuer (leading CTA) =======================
+    if (leader && lane == 0) {
+      const uint32_t peer = rank ^ 1u;
+      int u = 0, i = 0;
+      bool ok = true;
+      for (int t = pair; ok && t < tiles; t += npairs, ++i) {
+        const int ab = i & 1;
+        if (i >= 2)
+          ok = mbar_wait(BAR(B_ACCE + ab), ((i >> 1) - 1) & 1, tlim, abort_flag, args.err);
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t acc = tmem + static_cast<uint32_t>(ab * BN);
+        for (int kb = 0; kb < kblocks; ++kb, ++u) {
+          const int s = u % STAGES;
+          ok = mbar_wait(BAR(B_FULL + s), (u / STAGES) & 1, tlim, abort_flag, args.err) &&
+               mbar_wait(BAR(B_SFFULL + s), (u / STAGES) & 1, tlim, abort_flag, args.err);
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t a_s = base_u32 + OFF_A + s * TILE_A;
+          const uint32_t b_s = base_u32 + OFF_B + s * TILE_B;
+          const uint32_t sf = tmem + SF0 + static_cast<uint32_t>(u % SF_SLOTS) * SF_COLS;
+#pragma unroll
+          for (int kk = 0; kk < BK / 64; ++kk) {
+            const uint64_t da = smem_desc(a_s + kk * 32, 16, 1024, 2u);
+            const uint64_t db = smem_desc(b_s + kk * 32, 16, 1024, 2u);
+            mma_mxf4_ss_pair(acc, da, db, IDESC, sf + kk * 4, sf + 16 + kk * 6,
+                             (kb > 0 || kk > 0) ? 1u : 0u);
+          }
+          mma_commit_pair(BAR(B_EMPTY + s));                      // stage free in both CTAs
+          mma_commit_pair(mapa_shared(BAR(B_EMPTY + s), peer));
+        }
+        if (ok) {
+          mma_commit_pair(BAR(B_ACCF + ab));                      // accumulator complete
+          mma_commit_pair(mapa_shared(BAR(B_ACCF + ab), peer));
+        }
+      }
+      mma_commit_pair(BAR(B_DRAIN));
+      mbar_drain(BAR(B_DRAIN), 0, tlim);
+    }
+  } else {
+    // ======================= epilogue warps (both CTAs) =======================
+    const int quarter = warp & 3;
+    const int r = quarter * 32 + lane;
+    const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+    const float scale = __ldg(args.sg_x) * __ldg(args.sg_w);
+    int i = 0;
+    for (int t = pair; t < tiles; t += npairs, ++i) {
+      const int ab = i & 1;
+      const bool ok = mbar_wait(BAR(B_ACCF + ab), (i >> 1) & 1, tlim, abort_flag, args.err);
+      if (!__all_sync(0xFFFFFFFFu, ok)) break;
+      tc_fence_after();
+      const int m = (t % tiles_m) * BM + static_cast<int>(rank) * ROWS_A + r;
+      const int n0 = (t / tiles_m) * BN;
+      const uint32_t acc = tmem + lane_off + static_cast<uint32_t>(ab * BN);
+#pragma unroll 1
+      for (int c = 0; c < BN / 32; ++c) {
+        uint32_t v[32];
+        tmem_ld32(acc + c * 32, v);
+        tmem_wait_ld();
+        const size_t off = static_cast<size_t>(m) * args.N + n0 + c * 32;
+        if (m < args.M && n0 + c * 32 < args.N &&
+            QATTN_IN_BOUNDS(args.err, off + 32 <= static_cast<size_t>(args.M) * args.N))
+          store_bf16_32(args.y + off, v, scale);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(mapa_shared(BAR(B_ACCE + ab), 0));   // read out
+    }
+  }
+
+  tc_fence_before();
+  cluster_sync();                      // no MMA, load or arrival of either CTA is outstanding
+  if (warp == WARP_MMA) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem, TMEM_COLS);
+  }
+}
+
+// ---------------------------------------------------------------------------------------------
 // Host side
 // ---------------------------------------------------------------------------------------------
 
-// Packed E2M1 [rows, K / 2 bytes]; box of 128 rows x 128 bytes, 128-byte swizzle; reads past the
-// last row return zeros.
-static bool make_map_e2m1(CUtensorMap* map, const void* ptr, int rows, int K) {
+// Packed E2M1 [rows, K / 2 bytes]; box of `box_rows` rows x 128 bytes, 128-byte swizzle; reads
+// past the last row return zeros.
+static bool make_map_e2m1(CUtensorMap* map, const void* ptr, int rows, int K, int box_rows) {
   EncodeTiledFn enc = encode_tiled_fn();
   if (!enc) return false;
   cuuint64_t dims[2] = {static_cast<cuuint64_t>(K / 2), static_cast<cuuint64_t>(rows)};
   cuuint64_t strides[1] = {static_cast<cuuint64_t>(K / 2)};
-  cuuint32_t box[2] = {static_cast<cuuint32_t>(gemm4::BKB), static_cast<cuuint32_t>(gemm4::BM)};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(gemm4::BKB), static_cast<cuuint32_t>(box_rows)};
   cuuint32_t estr[2] = {1u, 1u};
   return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(ptr), dims, strides, box,
              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// Block scales [rows, K / 16] bytes, row-major; box of 128 rows x 16 bytes (one K block's
+// Block scales [rows, K / 16] bytes, row-major; box of `box_rows` rows x 16 bytes (one K block's
 // factors), no swizzle; rows past the last read as zeros.
-static bool make_map_scales(CUtensorMap* map, const void* ptr, int rows, int K) {
+static bool make_map_scales(CUtensorMap* map, const void* ptr, int rows, int K, int box_rows) {
   EncodeTiledFn enc = encode_tiled_fn();
   if (!enc) return false;
   cuuint64_t dims[2] = {static_cast<cuuint64_t>(K / 16), static_cast<cuuint64_t>(rows)};
   cuuint64_t strides[1] = {static_cast<cuuint64_t>(K / 16)};
-  cuuint32_t box[2] = {16u, 128u};
+  cuuint32_t box[2] = {16u, static_cast<cuuint32_t>(box_rows)};
   cuuint32_t estr[2] = {1u, 1u};
   return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(ptr), dims, strides, box,
              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
@@ -308,7 +583,6 @@ static bool make_map_scales(CUtensorMap* map, const void* ptr, int rows, int K) 
 cudaError_t launch_gemm_fp4(const uint8_t* x, const uint8_t* sx, const float* sg_x, const uint8_t* w,
                             const uint8_t* sw, const float* sg_w, void* y, int M, int N, int K,
                             int* err, uint64_t timeout_ns, int num_sms, cudaStream_t stream) {
-  static_assert(gemm4::BM == gemm4::BN, "one box shape serves both operands");
   Gemm4Args a;
   a.M = M;
   a.N = N;
@@ -319,8 +593,38 @@ cudaError_t launch_gemm_fp4(const uint8_t* x, const uint8_t* sx, const float* sg
   a.err = err;
   a.timeout_ns = timeout_ns;
   CUtensorMap ma, mb, msa, msb;
-  if (!make_map_e2m1(&ma, x, M, K) || !make_map_e2m1(&mb, w, N, K) ||
-      !make_map_scales(&msa, sx, M, K) || !make_map_scales(&msb, sw, N, K))
+  if (M > gemm4::BM && num_sms >= 2) {
+    // pairs of SMs on 256 x 192 tiles
+    using namespace gemm4p;
+    if (!make_map_e2m1(&ma, x, M, K, ROWS_A) || !make_map_e2m1(&mb, w, N, K, ROWS_B) ||
+        !make_map_scales(&msa, sx, M, K, ROWS_A) || !make_map_scales(&msb, sw, N, K, BN))
+      return cudaErrorInvalidValue;
+    static DeviceOnce configured_pair;
+    const int set = configured_pair.get([] {
+      return static_cast<int>(cudaFuncSetAttribute(k_gemm_fp4_pair,
+                                                   cudaFuncAttributeMaxDynamicSharedMemorySize, ALLOC));
+    });
+    if (set != static_cast<int>(cudaSuccess)) return static_cast<cudaError_t>(set);
+    static DeviceOnce resident_pairs;
+    const int resident = resident_pairs.get([num_sms] {
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3(static_cast<unsigned>(num_sms & ~1));
+      cfg.blockDim = dim3(THREADS);
+      cfg.dynamicSmemBytes = ALLOC;
+      int n = 0;
+      if (cudaOccupancyMaxActiveClusters(&n, k_gemm_fp4_pair, &cfg) != cudaSuccess || n <= 0) {
+        cudaGetLastError();
+        n = num_sms / 2;
+      }
+      return n;
+    });
+    const int tiles = ((M + BM - 1) / BM) * ((N + BN - 1) / BN);
+    const int pairs = tiles < resident ? tiles : resident;
+    k_gemm_fp4_pair<<<2 * pairs, THREADS, ALLOC, stream>>>(ma, mb, msa, msb, a);
+    return cudaGetLastError();
+  }
+  if (!make_map_e2m1(&ma, x, M, K, gemm4::BM) || !make_map_e2m1(&mb, w, N, K, gemm4::BN) ||
+      !make_map_scales(&msa, sx, M, K, gemm4::BM) || !make_map_scales(&msb, sw, N, K, gemm4::BN))
     return cudaErrorInvalidValue;
   static DeviceOnce configured;
   const int set = configured.get([] {

@@ -319,6 +319,21 @@ __device__ __forceinline__ void mma_mxf4_ss(uint32_t d_tmem, uint64_t a_desc, ui
       : "memory");
 }
 
+// The same on a pair of SMs (cta_group::2, M = 256): each CTA's shared memory holds its 128 rows
+// of A and its half of B, and each CTA's TMEM the factors of its own rows of A and of its half
+// of B, at the same addresses in both CTAs.
+__device__ __forceinline__ void mma_mxf4_ss_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                                 uint32_t idesc, uint32_t sfa_tmem, uint32_t sfb_tmem,
+                                                 uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %6, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%4], [%5], p;\n\t}" ::"r"(
+          d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(sfa_tmem), "r"(sfb_tmem), "r"(accumulate)
+      : "memory");
+}
+
 // Block-scaled, A from tensor memory (kind::mxf8f6f4, E8M0 scale factors, one per 32 K
 // elements; A's row m in lane m, element k in column k/4, byte k%4), one issuing thread:
 // D[tmem] (+)= (A[tmem] * SFA) * (B[smem desc] * SFB).  sfa_tmem / sfb_tmem address 4-column
