@@ -805,7 +805,8 @@ def fp4_gemm_rates(flush, steps, warmup):
         per_shape[name] = {"M": M, "N": N, "K": K, "ms": ms, "tflops": flops / (ms * 1e-3) / 1e12}
         flops_sum += flops
         ms_sum += ms
-    return {"kernel": "k_gemm_fp4 (kind::mxf4nvf4, 128 x 128 tiles, one SM each)",
+    return {"kernel": "k_gemm_fp4_pair (kind::mxf4nvf4, 256 x 192 tiles on pairs of SMs; "
+                      "k_gemm_fp4 for M <= 128)",
             "value": flops_sum / (ms_sum * 1e-3) / 1e12, "unit": "TFLOP/s", "ms": ms_sum,
             "per_shape": per_shape, "gpu_launches": len(GEMM_SHAPES) * steps}
 
