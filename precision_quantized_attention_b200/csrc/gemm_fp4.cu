@@ -304,12 +304,15 @@ __global__ void __launch_bounds__(gemm4::THREADS, 1)
 // every wait in between is bounded.
 // ---------------------------------------------------------------------------------------------
 namespace gemm4p {
+#ifndef QATTN_FP4_PAIR_N
+#define QATTN_FP4_PAIR_N 192
+#endif
 constexpr int BM = 256;                  // output rows per tile pair (128 per CTA)
-constexpr int BN = 192;                  // output columns per tile (MMA N; 96 W rows per CTA)
+constexpr int BN = QATTN_FP4_PAIR_N;     // output columns per tile (MMA N; BN / 2 W rows per CTA)
 constexpr int BK = 256;                  // K elements per stage (128 bytes per row)
 constexpr int BKB = BK / 2;
 constexpr int STAGES = 6;                // shared-memory ring
-constexpr int SF_SLOTS = 3;              // TMEM factor ring
+constexpr int GW = BN / 32;              // W row groups per K = 64 step (TMEM columns of W's factors)
 constexpr int THREADS = 320;
 constexpr int WARP_LOAD = 0, WARP_MMA = 1, WARP_SF0 = 6;   // warps 2-5: epilogue
 constexpr int ROWS_A = BM / 2, ROWS_B = BN / 2;             // operand rows per CTA
@@ -331,12 +334,15 @@ constexpr int ALLOC = BYTES + 1024;
 static_assert(TILE_A % 1024 == 0 && TILE_B % 1024 == 0 && OFF_SFA % 1024 == 0, "alignment");
 static_assert(TILE_SFB % 128 == 0, "scale boxes stay 128-byte aligned");
 static_assert(ALLOC <= 227 * 1024, "shared memory per CTA");
-// factor slot f at SF0 + 40 f: X's factors of step kk in column kk * 4 + c (c < 4), W's in
-// column 16 + kk * 6 + c (c < 6), c = row / 32
+// factor slot f at SF0 + SF_COLS f: X's factors of step kk in column kk * 4 + c (c < 4), W's in
+// column 16 + kk * GW + c (c < GW), c = row / 32
 constexpr uint32_t SF0 = 2 * BN;
-constexpr uint32_t SF_COLS = 40;
+constexpr uint32_t SF_COLS = 16 + 4 * GW;
 constexpr uint32_t TMEM_COLS = 512;
-static_assert(SF0 + SF_SLOTS * SF_COLS <= TMEM_COLS, "TMEM budget");
+constexpr int SF_SLOTS = (TMEM_COLS - SF0) / SF_COLS < STAGES ? (TMEM_COLS - SF0) / SF_COLS : STAGES;
+static_assert(SF_SLOTS >= 2 && SF0 + SF_SLOTS * SF_COLS <= TMEM_COLS, "TMEM budget");
+static_assert(BN % 64 == 0 && BN <= 256, "W rows per CTA: whole 32-row groups");
+static_assert(SF_COLS == 32 || SF_COLS == 40, "a slot is written with one 32-column store (+ 8)");
 constexpr uint32_t STAGE_TX = 2u * (TILE_A + TILE_B);     // operand bytes of both CTAs per stage
 constexpr uint32_t IDESC = idesc_mxf4_e2m1(BM, BN);
 }  // namespace gemm4p
@@ -440,29 +446,23 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(gemm4p::THREADS, 1)
           ok = mbar_wait(BAR(B_EMPTY + v % STAGES), (v / STAGES) & 1, tlim, abort_flag, args.err);
         }
         if (!__all_sync(0xFFFFFFFFu, ok)) { ok = false; break; }
-        // row group c: rows 32 c + lane of this CTA's X rows (c < 4) and of the W rows (c < 6)
+        // row group c: rows 32 c + lane of this CTA's X rows (c < 4) and of the W rows (c < GW)
         const uint32_t fa0 = base_u32 + OFF_SFA + s * TILE_SFA + 16u * lane;
         const uint32_t fb0 = base_u32 + OFF_SFB + s * TILE_SFB + 16u * lane;
-        uint32_t va[32], vb[8];
+        uint32_t v[40];                            // the slot's columns, in order (SF_COLS used)
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
           const uint4 fa = ld_shared_v4(fa0 + 512u * c);
-          va[c] = fa.x; va[4 + c] = fa.y; va[8 + c] = fa.z; va[12 + c] = fa.w;
+          v[c] = fa.x; v[4 + c] = fa.y; v[8 + c] = fa.z; v[12 + c] = fa.w;
         }
-        // W: column 16 + kk * 6 + c of the slot, i.e. va[16 + ...] for the first 16 and vb after
-        uint32_t w[24];
 #pragma unroll
-        for (int c = 0; c < 6; ++c) {
+        for (int c = 0; c < GW; ++c) {
           const uint4 fb = ld_shared_v4(fb0 + 512u * c);
-          w[c] = fb.x; w[6 + c] = fb.y; w[12 + c] = fb.z; w[18 + c] = fb.w;
+          v[16 + c] = fb.x; v[16 + GW + c] = fb.y; v[16 + 2 * GW + c] = fb.z; v[16 + 3 * GW + c] = fb.w;
         }
-#pragma unroll
-        for (int i = 0; i < 16; ++i) va[16 + i] = w[i];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) vb[i] = w[16 + i];
         const uint32_t slot = tmem + lane_off + SF0 + static_cast<uint32_t>(f) * SF_COLS;
-        tmem_st32(slot, va);
-        tmem_st8(slot + 32, vb);
+        tmem_st32(slot, *reinterpret_cast<const uint32_t(*)[32]>(v));
+        if constexpr (SF_COLS > 32) tmem_st8(slot + 32, *reinterpret_cast<const uint32_t(*)[8]>(v + 32));
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
@@ -495,7 +495,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(gemm4p::THREADS, 1)
           for (int kk = 0; kk < BK / 64; ++kk) {
             const uint64_t da = smem_desc(a_s + kk * 32, 16, 1024, 2u);
             const uint64_t db = smem_desc(b_s + kk * 32, 16, 1024, 2u);
-            mma_mxf4_ss_pair(acc, da, db, IDESC, sf + kk * 4, sf + 16 + kk * 6,
+            mma_mxf4_ss_pair(acc, da, db, IDESC, sf + kk * 4, sf + 16 + kk * GW,
                              (kb > 0 || kk > 0) ? 1u : 0u);
           }
           mma_commit_pair(BAR(B_EMPTY + s));                      // stage free in both CTAs
