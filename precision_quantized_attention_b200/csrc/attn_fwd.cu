@@ -1,4 +1,6 @@
-// attn_fwd.cu -- fused quantized attention forward for sm_100a (TMA + tcgen05 + TMEM).
+// attn_fwd.cu -- fused quantized attention forward for sm_100a (TMA + tcgen05 + TMEM): the
+// kernel of every launch (D = 64 and 128) unless the pair-of-SMs variant (attn_pair.cu) is
+// selected for D = 128; the persistent schedule, the combine of cut pairs and the launch.
 //
 // Method: NVIDIA developer blog "Optimizing FLUX.1 Kontext for Image Editing with Low-Precision
 // Quantization", section "Workflow and quantization" and Fig. 4:

@@ -1,5 +1,8 @@
 // attn_pair.cu -- fused quantized attention forward for D = 128 on pairs of SMs (sm_100a:
-// cluster of two CTAs, tcgen05.mma.cta_group::2, TMA, TMEM).
+// cluster of two CTAs, tcgen05.mma.cta_group::2, TMA, TMEM).  A variant of the one-SM kernel
+// of attn_fwd.cu, selected with qattn_debug_use_pair_kernel; on B200 it measures about 6 %
+// slower than that kernel at L = 8704 (its extra S buffers do not pay for the cross-CTA
+// handshakes), so the one-SM kernel is the default.
 //
 // Method: NVIDIA developer blog "Optimizing FLUX.1 Kontext for Image Editing with Low-Precision
 // Quantization", section "Workflow and quantization" and Fig. 4:
