@@ -11,19 +11,24 @@
  *   3. softmax in FP32, unquantized;
  *   4. P requantized to per-tensor FP8 (scale 1/448), BMM2 = P V in FP8.
  * Scales come from max-calibration of the tensor in hand (the blog's post-training
- * calibration step reduced to one tensor).
+ * calibration step reduced to one tensor), or are given (static scales, qattn_quantize_qkv).
+ * The block's linear layers around the attention (the blog quantizes them with the same
+ * schemes) are here too: qattn_gemm_fp8 / qattn_gemm_fp8_e4m3 (per-tensor FP8) and
+ * qattn_gemm_fp4 (per-block FP4).
  *
  * Conventions for every entry point:
  *   - Pointers named *_dev or tensor data are DEVICE pointers on the current CUDA device; the
  *     caller owns and allocates every buffer.  The library keeps no state besides one device
- *     error word per device and cached kernel attributes.
+ *     error word per device, cached kernel attributes, the 256-byte static workspace of
+ *     qattn_calibrate_quantize_fp8_noalloc and the settings of the qattn_debug_* hooks.
  *   - Work is enqueued on `stream` (0 = legacy default stream) and is asynchronous: scales and
  *     amax stay in device memory, nothing synchronizes with the host.  qattn_get_error() is the
  *     only call that synchronizes.
  *   - Argument errors are detected on the host before anything is launched and returned as
  *     QATTN_ERR_INVALID_ARG / QATTN_ERR_UNSUPPORTED; launch failures as QATTN_ERR_CUDA.  Errors
- *     found on the device (non-finite input, a timed-out wait) are recorded in the device
- *     error word and reported by qattn_get_error().
+ *     found on the device (non-finite input, a timed-out wait, and in the checked build an
+ *     index outside its buffer) are recorded in the device error word and reported by
+ *     qattn_get_error().
  *   - Tensors are contiguous.  bf16 inputs are 16-byte aligned; E4M3 code buffers are 16-byte
  *     aligned (the attention kernel reads them with TMA).
  *   - Only sm_100 devices are supported (QATTN_ERR_UNSUPPORTED otherwise).

@@ -7,6 +7,7 @@
 // with Low-Precision Quantization", "Workflow and quantization", third SDPA bullet: softmax in
 // FP32, no quantization at that stage).
 #pragma once
+#include <cuda_runtime.h>
 #include <cstdint>
 
 namespace qattn {
